@@ -1,0 +1,118 @@
+"""Planted mistakes: each plausible slip in the oracle must fail at least one pin.
+
+Every case swaps one oracle function (on the CPU, through monkeypatch) for a
+copy with a single deliberate error -- an off-by-one window, a dropped or
+swapped term, a wrong tie rule, a missing scale -- and checks that the named
+pin test then fails.  This is what makes the pins a check on the oracle and
+not a restatement of it.
+"""
+import numpy as np
+import pytest
+
+import test_oracle_attention as TA
+import test_oracle_decode as TD
+import test_oracle_selection as TS
+from oracle import attention as A
+from oracle import decode as D
+from oracle import selection as Sel
+
+_kept = A.kept_mask
+_bounds = Sel.logical_bounds
+_masked = A.masked_attention
+
+
+def kept_window_off_by_one(rows, S, streaming, sink, local, tm):
+    i = np.asarray(rows)[:, None]
+    j = np.arange(S)[None, :]
+    if streaming:
+        return (j <= i) & ((j < sink) | (i - j <= local))
+    return _kept(rows, S, streaming, sink, local, tm)
+
+
+def kept_sink_inclusive(rows, S, streaming, sink, local, tm):
+    i = np.asarray(rows)[:, None]
+    j = np.arange(S)[None, :]
+    if streaming:
+        return (j <= i) & ((j <= sink) | (i - j < local))
+    return _kept(rows, S, streaming, sink, local, tm)
+
+
+def kept_mask_transposed(rows, S, streaming, sink, local, tm):
+    i = np.asarray(rows)[:, None]
+    j = np.arange(S)[None, :]
+    if not streaming and tm is not None:
+        return (j <= i) & (np.asarray(tm)[j // 64, i // 64] != 0)
+    return _kept(rows, S, streaming, sink, local, tm)
+
+
+def bounds_kmax_only(q, stats, page_table, seq_len, b, h, G):
+    st = np.array(stats, dtype=np.float64)
+    st[..., 0, :] = st[..., 1, :]
+    return _bounds(q, st, page_table, seq_len, b, h, G)
+
+
+def bounds_min_instead_of_max(q, stats, page_table, seq_len, b, h, G):
+    q = np.asarray(q, dtype=np.float64)
+    out = _bounds(q, stats, page_table, seq_len, b, h, G)
+    kvh = h // G
+    for i in range(out.shape[0]):
+        for l in range(4):
+            if np.isfinite(out[i, l]):
+                s = stats[page_table[b][i], kvh, l]
+                out[i, l] = np.minimum(q[b, h] * s[1], q[b, h] * s[0]).sum()
+    return out
+
+
+def topk_ties_high(scores_row, k):
+    s = np.asarray(scores_row, dtype=np.float64)
+    order = np.lexsort((-np.arange(len(s)), -s))
+    return np.sort(order[:k]), np.inf
+
+
+def token_set_drops_current(seq_len, streaming, sink, local, pages=None):
+    t = _token_set(seq_len, streaming, sink, local, pages)
+    return t[t < seq_len - 1]
+
+
+def masked_no_scale(q, k, v, head_kind, sink, local, block_mask=None, scale=None, rows=None, row_chunk=256):
+    return _masked(q, k, v, head_kind, sink, local, block_mask, 1.0, rows, row_chunk)
+
+
+def page_stats_ignores_length(k_pages, page_table, seq_lens, head_kind, first_logical_page=0, stats=None):
+    full = [64 * ((int(L) + 63) // 64) for L in seq_lens]
+    return _stats(k_pages, page_table, full, head_kind, first_logical_page, stats)
+
+
+_stats = Sel.page_stats
+_token_set = D.token_set
+
+
+CASES = [
+    ("window off by one", A, "kept_mask", kept_window_off_by_one,
+     lambda: TA.test_streaming_equals_sdpa_with_lambda_mask(0, 64)),
+    ("sink inclusive", A, "kept_mask", kept_sink_inclusive,
+     lambda: TA.test_streaming_equals_sdpa_with_lambda_mask(3, 1)),
+    ("block mask transposed", A, "kept_mask", kept_mask_transposed,
+     TA.test_block_mask_equals_sdpa_with_expanded_mask),
+    ("no softmax scale", A, "masked_attention", masked_no_scale,
+     lambda: TA.test_all_tiles_kept_equals_dense_causal(2)),
+    ("bound drops kmin", Sel, "logical_bounds", bounds_kmax_only,
+     lambda: TS.test_bound_dominates_every_dot_product(1)),
+    ("bound takes min", Sel, "logical_bounds", bounds_min_instead_of_max,
+     TS.test_bound_hand_example),
+    ("ties to higher index", Sel, "topk_pages", topk_ties_high,
+     lambda: TS.test_topk_brute_force_with_ties(0)),
+    ("decode drops current token", D, "token_set", token_set_drops_current,
+     lambda: TD.test_full_budget_equals_dense_decode(None)),
+    ("stats ignore sequence length", Sel, "page_stats", page_stats_ignores_length,
+     TS.test_stats_closed_form_on_contiguous_keys),
+]
+
+
+@pytest.mark.parametrize("name,mod,attr,bad,pin", CASES, ids=[c[0] for c in CASES])
+def test_planted_mistake_is_caught(monkeypatch, name, mod, attr, bad, pin):
+    monkeypatch.setattr(mod, attr, bad)
+    if mod is Sel and attr == "page_stats":
+        monkeypatch.setattr(TS.Sel, attr, bad)
+    with pytest.raises(AssertionError):
+        pin()
