@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark of the unified sparse-attention hot path on B200.
+
+One step = one pass of the whole path on one GPU:
+  * prefill: kept-tile lists + block-sparse causal attention at 128K tokens
+    (Llama-3-8B layer shape, 4 streaming KV heads with sink 64 + local 256, 4
+    dense KV heads with a seeded vertical-slash block mask at ~30 % tile density);
+  * decode: incremental page-summary refresh of the newest logical page, then
+    one sparse decode step -- bound scoring, top-k pages, split-KV paged
+    attention and LSE merge -- for 4 sequences of 262,144 tokens (Llama-2-7B MHA
+    shape, 16 dense + 16 streaming KV heads, budget 8,192 tokens).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Prints ONE JSON line on rank 0.  Multi-GPU runs are independent replicas
+(the path has no exchange step); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "prefill attn ms & kept-tile TFLOPS at 128K; decode attn µs/step & HBM GB/s"
+PREFILL_WL = "llama3_8b_prefill_128k_vslash"
+DECODE_WL = "llama2_7b_mha"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sust=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------------ workload
+
+def kept_tile_counts(w, bm, kind):
+    """Kept 64x64 tiles per KV head (dense: causal tiles the mask keeps; streaming:
+    tiles meeting the Lambda support).  Pure bookkeeping for the FLOP count."""
+    n = w.S // 64
+    qt = torch.arange(n, device=bm.device if bm is not None else "cpu")[:, None]
+    kt = torch.arange(n, device=qt.device)[None, :]
+    causal = kt <= qt
+    counts = []
+    for g in range(w.Hkv):
+        if kind[g]:
+            mind = torch.clamp(64 * qt - 64 * kt - 63, min=0)
+            keep = causal & ((64 * kt < w.sink) | (mind < w.local))
+        elif bm is not None:
+            keep = causal & (bm[0, g] != 0)
+        else:
+            keep = causal
+        counts.append(int(keep.sum()))
+    return counts
+
+
+def decode_bytes(w, kind, k_pages_per_seq, d):
+    """Bytes the decode step must read/write (algorithmic, not what a kernel happens to touch)."""
+    n_dense = sum(1 for x in kind if x == 0)
+    n_stream = len(kind) - n_dense
+    n_pages = (w.ctx + 63) // 64
+    stats = w.dec_B * n_dense * n_pages * 4 * 2 * d * 2
+    sel = w.dec_B * n_dense * k_pages_per_seq * 64 * d * 2 * 2
+    stream_tok = min(w.ctx, w.sink + w.local)
+    stream = w.dec_B * n_stream * stream_tok * d * 2 * 2
+    q_out = 2 * w.dec_B * w.Hq * d * 2
+    table = w.dec_B * n_pages * 4
+    return dict(stats=stats, selected=sel, streaming=stream, q_out=q_out, table=table,
+                total=stats + sel + stream + q_out + table)
+
+
+class Setup:
+    def __init__(self, device):
+        self.dev = device
+        self.wp = W.WORKLOADS[PREFILL_WL]
+        self.wd = W.WORKLOADS[DECODE_WL]
+        wp, wd = self.wp, self.wd
+        self.kind_p = W.head_kind(wp)
+        self.kind_d = W.head_kind(wd)
+        self.q, self.k, self.v = W.prefill_inputs(wp, device=device)
+        self.bm = W.block_mask(wp, device=device)
+        self.hk_p = self.kind_p.to(device)
+        self.tiles = kept_tile_counts(wp, self.bm, self.kind_p.tolist())
+        G = wp.Hq // wp.Hkv
+        self.prefill_flops = sum(self.tiles) * G * 4 * 64 * 64 * wp.d
+        pc = W.decode_cache(wd, device=device)
+        self.kp, self.vp = pc.k_pages, pc.v_pages
+        self.pt, self.sl = pc.page_table.to(device), pc.seq_lens.to(device)
+        self.hk_d = self.kind_d.to(device)
+        self.qd = W.decode_query(wd, device=device)
+        self.k_sel = min(wd.token_budget // 64, (wd.ctx + 63) // 64)
+        self.dbytes = decode_bytes(wd, self.kind_d.tolist(), self.k_sel, wd.d)
+        self.last_lp = (wd.ctx - 1) // 16
+
+
+# -------------------------------------------------------------------- timing
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.flush()
+        rows = [r.split(", ") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, reasons, smax = [], set(), None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+                for nme, val in zip(names, r[5:9]):
+                    if val.strip().lower() == "active":
+                        reasons.add(nme)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def flush_l2(buf):
+    buf.add_(1.0)
+
+
+def time_loop(fn, steps, warmup, stream, scratch, events_per_step=1):
+    """Warm up, then time `steps` calls with CUDA events on `stream`, flushing L2 between calls."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush_l2(scratch)
+        starts[i].record(stream)
+        fn()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_prefill_sample(setup, seconds=10.0, seed=0):
+    """Time the fp64 oracle on sampled query rows of the prefill workload.
+    Returns (rate in kept-tile TFLOP/s equivalent, rows, seconds)."""
+    from oracle import attention as OA
+    wp = setup.wp
+    rng = np.random.default_rng(seed)
+    kind = setup.kind_p.tolist()
+    k = setup.k.float().cpu().numpy()
+    v = setup.v.float().cpu().numpy()
+    bm = setup.bm.cpu().numpy()
+    n = wp.S // 64
+    tiles_per_row = np.zeros((wp.Hkv, n), np.int64)
+    for g in range(wp.Hkv):
+        keep = OA.tile_kept(wp.S, bool(kind[g]), wp.sink, wp.local, None if kind[g] else bm[0, g])
+        tiles_per_row[g] = keep.sum(axis=1)
+    G = wp.Hq // wp.Hkv
+    done_rows, flops, t_used = 0, 0.0, 0.0
+    while t_used < seconds:
+        rows = np.sort(rng.choice(wp.S, size=4, replace=False))
+        qr = setup.q[:, torch.from_numpy(rows).to(setup.q.device)].float().cpu().numpy()
+        t0 = time.perf_counter()
+        OA.masked_attention(qr, k, v, kind, wp.sink, wp.local, bm, rows=rows, q_at_rows=True)
+        t_used += time.perf_counter() - t0
+        done_rows += len(rows)
+        flops += sum(int(tiles_per_row[g, r // 64]) * G * 4 * 64 * wp.d for g in range(wp.Hkv) for r in rows)
+    return flops / t_used / 1e12, done_rows, t_used
+
+
+def cpu_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+# ---------------------------------------------------------------------- main
+
+def run_reference(args, rank, world):
+    """Reference arm: the CPU oracle as it stands, on bounded samples of the same workload."""
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    setup = Setup(dev)
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup):
+        oracle_prefill_sample(setup, seconds=per_step / 4, seed=100 + i)
+    rates, secs, rows = [], 0.0, 0
+    for i in range(args.steps):
+        r, nr, t = oracle_prefill_sample(setup, seconds=per_step, seed=i)
+        rates.append(r)
+        secs += t
+        rows += nr
+    value = float(np.mean(rates))
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(1, args.steps) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": PREFILL_WL, "seq_len": setup.wp.S, "kind": "oracle on sampled rows"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} query rows x {setup.wp.Hq} heads of the 128K prefill, "
+                                   f"{secs:.1f} s of fp64 NumPy"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    import unified_sparse_attention_b200 as U
+    U.load_library()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    setup = Setup(dev)
+    wp, wd = setup.wp, setup.wd
+    pk = peaks()
+
+    out_p = torch.empty_like(setup.q)
+    ws_p = torch.empty(U.lserve_prefill_workspace_size(wp.B, wp.S, wp.Hq, wp.Hkv, wp.d), dtype=torch.uint8,
+                       device=dev)
+    stats = U.lserve_update_page_stats(setup.kp, setup.pt, setup.sl, setup.hk_d)
+    dargs = (setup.qd, setup.kp, setup.vp, setup.pt, setup.sl, stats, setup.hk_d, wd.sink, wd.local,
+             wd.token_budget)
+    ws_d = torch.empty(U.lserve_decode_workspace_size(*dargs), dtype=torch.uint8, device=dev)
+    out_d = torch.empty_like(setup.qd)
+    n = wp.S // 64
+    ws_t = torch.empty_like(ws_p)
+
+    def prefill():
+        U.lserve_prefill(setup.q, setup.k, setup.v, setup.hk_p, wp.sink, wp.local, setup.bm, out=out_p,
+                         workspace=ws_p)
+
+    def tile_lists():
+        U.lserve_prefill_tile_lists(wp.B, wp.S, wp.Hq, wp.Hkv, wp.d, setup.hk_p, wp.sink, wp.local, setup.bm)
+
+    def decode():
+        U.lserve_update_page_stats(setup.kp, setup.pt, setup.sl, setup.hk_d, stats=stats,
+                                   first_logical_page=setup.last_lp)
+        U.lserve_decode(*dargs, out=out_d, workspace=ws_d)
+
+    def decode_only():
+        U.lserve_decode(*dargs, out=out_d, workspace=ws_d)
+
+    def step():
+        prefill()
+        decode()
+
+    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    # component timings (same launches, timed separately)
+    t_tiles = time_loop(tile_lists, max(3, args.steps // 2), 2, stream, scratch)
+    t_prefill = time_loop(prefill, args.steps, args.warmup, stream, scratch)
+    t_decode = time_loop(decode_only, args.steps, args.warmup, stream, scratch)
+
+    # the timed steps
+    clocks = Clocks(local_rank)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_step = time_loop(step, args.steps, 0, stream, scratch)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    assert U.lserve_get_device_status() == 0, "kernel reported an error"
+
+    ms_step = float(np.mean(t_step))
+    ms_prefill = float(np.median(t_prefill))
+    ms_tiles = float(np.median(t_tiles))
+    ms_attn = max(1e-6, ms_prefill - ms_tiles)
+    us_decode = float(np.median(t_decode)) * 1e3
+    if dist is not None:
+        t = torch.tensor([ms_step, ms_prefill, us_decode], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, ms_prefill, us_decode = t.tolist()
+
+    tflops_prefill = setup.prefill_flops / (ms_prefill * 1e-3) / 1e12
+    tflops_attn = setup.prefill_flops / (ms_attn * 1e-3) / 1e12
+    gbps_decode = setup.dbytes["total"] / (us_decode * 1e-6) / 1e9
+    value = world * setup.prefill_flops / (ms_prefill * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (setup.q, setup.k, setup.v))
+        hbm_ = setup.bm.cpu().pin_memory()
+        hqd = setup.qd.cpu().pin_memory()
+        ho = torch.empty(setup.q.shape, dtype=torch.bfloat16).pin_memory()
+        hod = torch.empty(setup.qd.shape, dtype=torch.bfloat16).pin_memory()
+        dq, dk, dv, dbm, dqd = (torch.empty_like(t) for t in (setup.q, setup.k, setup.v, setup.bm, setup.qd))
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dbm.copy_(hbm_, non_blocking=True)
+            dqd.copy_(hqd, non_blocking=True)
+            U.lserve_prefill(dq, dk, dv, setup.hk_p, wp.sink, wp.local, dbm, out=out_p, workspace=ws_p)
+            U.lserve_update_page_stats(setup.kp, setup.pt, setup.sl, setup.hk_d, stats=stats,
+                                       first_logical_page=setup.last_lp)
+            U.lserve_decode(dqd, *dargs[1:], out=out_d, workspace=ws_d)
+            ho.copy_(out_p, non_blocking=True)
+            hod.copy_(out_d, non_blocking=True)
+
+        t_e2e = time_loop(e2e_step, max(3, args.steps // 2), 2, stream, scratch)
+        ms_e2e = float(np.mean(t_e2e))
+        if dist is not None:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = t.item()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hbm_, hqd))
+        d2h = ho.numel() * 2 + hod.numel() * 2
+        e2e = {"value": world * setup.prefill_flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "note": "prefill TFLOP/s over the whole step (prefill + decode) incl. H2D of q,k,v,mask,"
+                       "decode q and D2H of both outputs; the KV page pool stays resident"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, rows, secs = oracle_prefill_sample(setup, seconds=10.0)
+        cpu = {"value": rate, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{rows} query rows x {wp.Hq} heads of the 128K prefill ({secs:.1f} s fp64 NumPy), "
+                         f"rate scaled by each row's kept-tile FLOPs"}
+
+    launches_per_step = 4 + 1 + 4   # tile count/scan/fill + attention; stats refresh; score/top-k/decode/merge
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{PREFILL_WL} prefill (B1 S131072 Hq32 Hkv8 d128, vertical-slash mask "
+                               f"{sum(setup.tiles[g] for g in range(wp.Hkv) if setup.kind_p[g] == 0) / (4 * n * (n + 1) / 2):.3f}"
+                               f" density) + {DECODE_WL} decode (B4 ctx262144 Hq32 Hkv32 d128, budget 8192)",
+                   "l2": "flushed between steps (write of 252 MB)", "parallelism": f"replicas x{world}"},
+        "prefill_ms": ms_prefill, "prefill_attention_ms": ms_attn, "tile_lists_ms": ms_tiles,
+        "prefill_tflops": tflops_prefill, "kept_tile_tflop": setup.prefill_flops / 1e12,
+        "decode_us_per_step": us_decode, "decode_GBps": gbps_decode, "decode_bytes": setup.dbytes,
+        "roofline": {"bound": "tensor", "kernel": "prefill attention", "achieved": tflops_attn,
+                     "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tflops_attn / pk["bf16"],
+                     "traffic": None, "peak_source": pk["source"] + " bf16 burst",
+                     "achieved_note": "kept-tile FLOPs / (lserve_prefill - tile-list build) time"},
+        "roofline_decode": {"bound": "hbm", "kernel": "decode (score + top-k + paged attention + merge)",
+                            "achieved": gbps_decode, "peak": pk["hbm"], "unit": "GB/s",
+                            "frac": gbps_decode / pk["hbm"], "traffic": None, "peak_source": pk["source"]},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

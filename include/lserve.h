@@ -1,0 +1,234 @@
+/*
+ * lserve.h -- C ABI of the unified block-sparse attention library (liblserve.so).
+ *
+ * One library serves both phases of LServe-style unified sparse attention
+ * (mlsanity, "LServe: Efficient Long-sequence LLM Serving with Unified Sparse
+ * Attention", Abstract: structured sparsity for prefilling and decoding in one
+ * framework, computations on less important tokens skipped block-wise):
+ *
+ *   prefill  causal flash attention that skips whole 64x64 KV tiles; dense KV
+ *            heads keep every causal tile (optionally ANDed with a block mask),
+ *            streaming KV heads keep only the Lambda support (sink tokens plus a
+ *            local window)  -- LServe + SampleAttention blog post, "LServe -
+ *            Prefill Phase", Fig. 1(a)/(b);
+ *   decode   per-logical-page key min/max summaries, an upper-bound page score,
+ *            the max over the logical pages of each physical page, top-k pages
+ *            within a token budget, then split-KV paged attention over only those
+ *            pages and a log-sum-exp merge -- same blog post, "LServe - Decode
+ *            Phase", Fig. 2; the summary/bound follow Quest (listed under
+ *            "Builds on" on the mlsanity LServe page).
+ *
+ * Conventions (all entry points):
+ *   - Every tensor pointer is DEVICE memory owned by the caller; the library
+ *     never allocates, frees or keeps a pointer past the call.  Workspaces are
+ *     caller-provided; query their size with the *_workspace_size functions.
+ *     Workspace contents on entry are ignored; on return they are undefined.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous on that stream; none synchronises the host except
+ *     lserve_get_device_status.
+ *   - Argument errors are detected on the host and returned before anything is
+ *     launched.  Launch failures return LSERVE_ERR_CUDA.  Errors found by the
+ *     kernels themselves (an out-of-range page id, a bounded wait that ran out)
+ *     are recorded in a per-device status word, read by lserve_get_device_status.
+ *   - bf16 means IEEE bfloat16 stored as uint16; all tensors are dense,
+ *     row-major, in the layout given (last index fastest), 16-byte aligned.
+ *   - Supported: head_dim d in {64, 128}; Hq a multiple of Hkv; physical page
+ *     64 tokens, logical page 16 tokens, prefill tile 64x64.  Anything else
+ *     returns LSERVE_ERR_UNSUPPORTED.  There is no fallback path.
+ *   - No exception crosses the ABI.  The library keeps no state between calls
+ *     except the device status word and the thread-local error string.
+ */
+#ifndef LSERVE_H_
+#define LSERVE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lserve_status {
+  LSERVE_OK = 0,
+  LSERVE_ERR_INVALID_ARG = 1,     /* null pointer, negative size, bad sink/local/budget   */
+  LSERVE_ERR_UNSUPPORTED = 2,     /* shape outside the supported set (see above)          */
+  LSERVE_ERR_WORKSPACE = 3,       /* workspace pointer null/misaligned or too small       */
+  LSERVE_ERR_CUDA = 4,            /* a CUDA runtime call or kernel launch failed          */
+  LSERVE_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait ran out (device status)      */
+  LSERVE_ERR_DEVICE_BOUNDS = 6    /* a kernel met an out-of-range index (device status)   */
+} lserve_status;
+
+#define LSERVE_PAGE 64            /* tokens per physical KV page                          */
+#define LSERVE_LOGICAL_PAGE 16    /* tokens per logical page (granularity of the summary) */
+#define LSERVE_TILE 64            /* prefill tile: 64 query rows x 64 keys                */
+
+/* Head kinds (uint8 per KV head). */
+#define LSERVE_HEAD_DENSE 0       /* retrieval head: all causal tiles / top-k pages       */
+#define LSERVE_HEAD_STREAMING 1   /* streaming head: Lambda support (sink + local window) */
+
+/* ------------------------------------------------------------------ prefill */
+
+typedef struct lserve_shape {
+  int32_t B;      /* batch                                                         */
+  int32_t S;      /* sequence length, a positive multiple of 64                    */
+  int32_t Hq;     /* query heads                                                   */
+  int32_t Hkv;    /* KV heads; query head h reads KV head h / (Hq / Hkv)           */
+  int32_t d;      /* head dim, 64 or 128                                           */
+  float scale;    /* softmax scale; <= 0 selects 1/sqrt(d)                         */
+} lserve_shape;
+
+/*
+ * Bytes of workspace lserve_prefill needs for `shape` (0 on an invalid shape).
+ * It holds the kept-tile lists (CSR), the longest-first work order and
+ * counters; it is sized for the worst case (every causal tile kept).
+ */
+size_t lserve_prefill_workspace_size(const lserve_shape* shape);
+
+/*
+ * Block-sparse causal prefill attention.
+ *
+ * Kept set of query row i (token position within its sequence) for query head
+ * h, KV head g = h / (Hq/Hkv):
+ *   dense g      (head_kind[g] == 0):  { j <= i : block_mask[b,g,i/64,j/64] != 0 }
+ *                                       (every j <= i when block_mask == NULL)
+ *   streaming g  (head_kind[g] == 1):  { j <= i : j < sink  or  i - j < local }
+ * out[b,i,h,:] = sum_j softmax_j(scale * q.k_j) v_j over the kept set; a row
+ * whose kept set is empty gets out = 0 and lse = -inf.  A 64x64 tile with no
+ * kept element is never read (whole-tile skipping, blog "LServe - Prefill
+ * Phase", Fig. 1(a)); elements inside kept tiles are masked exactly.
+ *
+ *   q          bf16 [B, S, Hq, d]
+ *   k, v       bf16 [B, S, Hkv, d]
+ *   head_kind  uint8 [Hkv]                    (device)
+ *   sink,local >= 0 tokens                    (used by streaming heads only)
+ *   block_mask uint8 [B, Hkv, S/64, S/64] or NULL; read for dense heads only,
+ *              ANDed with causality (entries above the diagonal are ignored)
+ *   out        bf16 [B, S, Hq, d]             (written)
+ *   lse        fp32 [B, Hq, S] or NULL        (natural-log LSE of the kept logits)
+ *   workspace  >= lserve_prefill_workspace_size(shape) bytes, 256-byte aligned
+ */
+lserve_status lserve_prefill(const lserve_shape* shape, const void* q, const void* k,
+                             const void* v, const uint8_t* head_kind, int32_t sink,
+                             int32_t local, const uint8_t* block_mask, void* out,
+                             float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The tile-list step of lserve_prefill on its own, for inspection: the kept
+ * KV tiles of every (b, kvh, qt) row as a CSR.  Row r = (b*Hkv + kvh)*(S/64) + qt.
+ *   row_offsets int32 [B*Hkv*(S/64) + 1]      (written; row_offsets[0] = 0)
+ *   tile_cols   uint16 [max_nnz]              (written; kt ascending within a row)
+ *   max_nnz     capacity of tile_cols; B*Hkv*n*(n+1)/2 with n = S/64 always fits.
+ *               If the kept tiles exceed it the call records LSERVE_ERR_DEVICE_BOUNDS
+ *               in the device status and writes nothing past the capacity.
+ * Same tile rule as lserve_prefill: dense rows keep kt <= qt (ANDed with the
+ * block mask); streaming rows keep kt <= qt with 64*kt < sink or
+ * max(64*qt - 64*kt - 63, 0) < local.
+ */
+lserve_status lserve_prefill_tile_lists(const lserve_shape* shape, const uint8_t* head_kind,
+                                        int32_t sink, int32_t local,
+                                        const uint8_t* block_mask, int32_t* row_offsets,
+                                        uint16_t* tile_cols, int64_t max_nnz,
+                                        void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------- page summaries */
+
+/*
+ * Per-logical-page key summaries for the decode selector (blog "LServe - Decode
+ * Phase": every page scored from a summary vector; Quest min/max summary).
+ *
+ * For every sequence b, every physical page i < ceil(seq_lens[b]/64) of its
+ * page table, every DENSE KV head g and every logical page l in 0..3 whose
+ * sequence-wide index 4*i + l >= first_logical_page:
+ *   stats[p,g,l,0,c] = min over the valid tokens t (t < seq_lens[b]) of the
+ *                      logical page of k[t,g,c];  stats[p,g,l,1,c] = max.
+ *   A logical page without a valid token gets min = +inf, max = -inf.
+ * p = page_table[b*maxP + i].  Min/max of bf16 values are exact: results are
+ * bit-identical to any correct implementation.  Streaming heads and pages not
+ * reached are left untouched.
+ *
+ *   k_pages     bf16 [num_pages, Hkv, 64, d]
+ *   page_table  int32 [B, maxP]; entries must lie in [0, num_pages)
+ *               (an entry outside records LSERVE_ERR_DEVICE_BOUNDS and is skipped)
+ *   seq_lens    int32 [B], 0 <= seq_lens[b] <= 64*maxP (device)
+ *   first_logical_page  0 = full rebuild; > 0 = refresh only logical pages at or
+ *               past this index (after appending tokens)
+ *   head_kind   uint8 [Hkv] (device)
+ *   stats       bf16 [num_pages, Hkv, 4, 2, d] (written)
+ */
+lserve_status lserve_update_page_stats(int32_t B, int32_t Hkv, int32_t d, int32_t num_pages,
+                                       const void* k_pages, const int32_t* page_table,
+                                       int32_t maxP, const int32_t* seq_lens,
+                                       int32_t first_logical_page, const uint8_t* head_kind,
+                                       void* stats, void* stream);
+
+/* ------------------------------------------------------------------- decode */
+
+typedef struct lserve_decode_args {
+  int32_t B, Hq, Hkv, d;
+  int32_t num_pages;          /* physical pages in the pool                              */
+  int32_t maxP;               /* row length of page_table                                */
+  const void* q;              /* bf16 [B, Hq, d]: one query token per sequence            */
+  const void* k_pages;        /* bf16 [num_pages, Hkv, 64, d]                            */
+  const void* v_pages;        /* bf16 [num_pages, Hkv, 64, d]                            */
+  const int32_t* page_table;  /* int32 [B, maxP]                                         */
+  const int32_t* seq_lens;    /* int32 [B]: tokens in the cache, the query's own included */
+  const void* stats;          /* bf16 [num_pages, Hkv, 4, 2, d] from lserve_update_page_stats */
+  const uint8_t* head_kind;   /* uint8 [Hkv]                                             */
+  int32_t sink, local;        /* streaming heads: tokens t < sink or t >= seq_len - local */
+  int32_t token_budget;       /* dense heads keep k = min(budget/64, n_pages) pages; >= 64 */
+  float scale;                /* <= 0 selects 1/sqrt(d)                                  */
+} lserve_decode_args;
+
+/* Capacity (pages) of one selection row: max(min(budget/64, maxP), streaming pages). */
+int32_t lserve_decode_max_selected(const lserve_decode_args* args);
+
+/* Bytes of workspace lserve_decode needs (page scores, selection, split partials). */
+size_t lserve_decode_workspace_size(const lserve_decode_args* args);
+
+/*
+ * One sparse decode step for B sequences.
+ *
+ * Dense KV head g of sequence b (n = ceil(seq_len/64) pages):
+ *   bound of query head h on logical page l:  s_h(l) = sum_c max(q_h,c*kmax_c, q_h,c*kmin_c)
+ *   group score    s(l) = max over the Hq/Hkv query heads of g of s_h(l)
+ *   page score     max of s(l) over the logical pages holding a valid token
+ *   selection      the k = min(token_budget/64, n) highest-scoring pages, ties to
+ *                  the lower page index, listed in ascending page order
+ *   attention      softmax(scale * q.k_t) over every valid token t of the
+ *                  selected pages, computed split-KV and merged by log-sum-exp.
+ * Streaming KV head: the pages holding tokens [0, sink) and
+ * [seq_len - local, seq_len), attending to exactly those tokens.
+ * The query is at position seq_len - 1 (its own key/value are in the cache).
+ *
+ *   out      bf16 [B, Hq, d] (written)
+ *   lse      fp32 [B, Hq] or NULL
+ *   sel_out  int32 [B, Hkv, lserve_decode_max_selected(args)] or NULL: selected
+ *            page indices (within the sequence, ascending; unused slots -1)
+ *   sel_n    int32 [B, Hkv] or NULL: number of selected pages
+ *   workspace >= lserve_decode_workspace_size(args) bytes, 256-byte aligned
+ */
+lserve_status lserve_decode(const lserve_decode_args* args, void* out, float* lse,
+                            int32_t* sel_out, int32_t* sel_n, void* workspace,
+                            size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ status */
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status
+ * word: LSERVE_OK, LSERVE_ERR_DEVICE_TIMEOUT or LSERVE_ERR_DEVICE_BOUNDS (the
+ * first error recorded since the last read), or LSERVE_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+lserve_status lserve_get_device_status(void* stream);
+
+/* Message of the last error returned on the calling thread ("" if none). */
+const char* lserve_last_error_string(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* lserve_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSERVE_H_ */

@@ -44,7 +44,7 @@ def kept_mask(rows: np.ndarray, S: int, streaming: bool, sink: int, local: int,
 
 
 def masked_attention(q, k, v, head_kind, sink, local, block_mask=None, scale=None,
-                     rows=None, row_chunk=256):
+                     rows=None, row_chunk=256, q_at_rows=False):
     """Exact masked attention in float64.
 
     q : [B, S, Hq, d]; k, v : [B, S, Hkv, d] (any float dtype, up-cast to f64)
@@ -52,13 +52,15 @@ def masked_attention(q, k, v, head_kind, sink, local, block_mask=None, scale=Non
     block_mask : [B, Hkv, S/64, S/64] or None
     rows : optional 1-D array of query positions to evaluate (all when None);
            rows are independent, so a sampled row is an exact row.
+    q_at_rows : q is given only at ``rows`` ([B, R, Hq, d]) instead of [B, S, Hq, d].
 
     Returns (out [B, R, Hq, d], lse [B, Hq, R]) with R = len(rows).
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
-    B, S, Hq, d = q.shape
+    B, _, Hq, d = q.shape
+    S = k.shape[1]
     Hkv = k.shape[2]
     G = Hq // Hkv
     scale = 1.0 / np.sqrt(d) if scale is None or scale <= 0 else float(scale)
@@ -76,7 +78,8 @@ def masked_attention(q, k, v, head_kind, sink, local, block_mask=None, scale=Non
             for c0 in range(0, R, row_chunk):
                 r = rows[c0:c0 + row_chunk]
                 keep = kept_mask(r, S, streaming, sink, local, tm)
-                logits = scale * (q[b, r, h, :] @ K.T)
+                qr = q[b, c0:c0 + len(r), h, :] if q_at_rows else q[b, r, h, :]
+                logits = scale * (qr @ K.T)
                 logits = np.where(keep, logits, -np.inf)
                 m = logits.max(axis=1, keepdims=True)
                 has = np.isfinite(m[:, 0])

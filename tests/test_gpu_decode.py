@@ -1,0 +1,139 @@
+"""GPU parity of the decode path (page summaries, bound scores, top-k, split-KV
+paged attention + LSE merge) against the oracle, through the C ABI."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import decode as OD
+from oracle import selection as OS
+from parity import assert_attn_close, assert_lse_close, check_selection, f64
+
+pytestmark = pytest.mark.gpu
+
+U = pytest.importorskip("unified_sparse_attention_b200")
+
+
+def make(w, B, ctx, lens=None, NP=None):
+    pc = W.decode_cache(w, B=B, ctx=ctx, seq_lens=lens, NP=NP)
+    q = W.decode_query(w, B=B)
+    return pc, q
+
+
+def run_decode(w, B, ctx, budget, sink, local, lens=None, kind=None, NP=None):
+    dev = "cuda"
+    pc, q = make(w, B, ctx, lens, NP)
+    kind = W.head_kind(w).tolist() if kind is None else kind
+    hk = torch.tensor(kind, dtype=torch.uint8)
+    kp, vp = pc.k_pages.to(dev), pc.v_pages.to(dev)
+    pt, sl = pc.page_table.to(dev), pc.seq_lens.to(dev)
+    stats = U.lserve_update_page_stats(kp, pt, sl, hk.to(dev))
+    lse = torch.empty(B, w.Hq, dtype=torch.float32, device=dev)
+    out, _, sel, sel_n = U.lserve_decode(q.to(dev), kp, vp, pt, sl, stats, hk.to(dev), sink, local, budget,
+                                         lse=lse, return_selection=True)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+    # oracle on the same bf16 inputs
+    kp64, vp64, pt_np, L = f64(pc.k_pages), f64(pc.v_pages), pc.page_table.numpy(), pc.seq_lens.numpy()
+    st_ref = OS.page_stats(kp64, pt_np, L, kind)
+    np.testing.assert_array_equal(f64(stats), st_ref)          # bit-exact summaries
+    q64 = f64(q)
+    sel_ref, margin, scores = OS.select(q64, st_ref, pt_np, L, kind, budget, sink, local)
+    sel_np, seln_np = sel.cpu().numpy(), sel_n.cpu().numpy()
+    gpu_sel, ties = {}, 0
+    for b in range(B):
+        for g in range(w.Hkv):
+            row = sel_np[b, g, : seln_np[b, g]]
+            gpu_sel[(b, g)] = row
+            if kind[g]:
+                assert list(row) == list(sel_ref[(b, g)])
+            else:
+                n = OS.n_pages(L[b])
+                ties += check_selection(row, OS.budget_pages(budget, L[b]), scores[b, g, :n])
+            assert np.all(sel_np[b, g, seln_np[b, g]:] == -1)
+    ref_out, ref_lse = OD.decode_attention(q64, kp64, vp64, pt_np, L, kind, gpu_sel, sink, local)
+    assert_attn_close(f64(out), ref_out, "decode out")
+    assert_lse_close(f64(lse), ref_lse, "decode lse")
+    return dict(pc=pc, q=q, out=out, sel=gpu_sel, stats=stats, kind=kind, ties=ties)
+
+
+def test_tiny_workload_exact_config():
+    w = W.WORKLOADS["tiny"]
+    r = run_decode(w, 1, w.ctx, w.token_budget, w.sink, w.local)
+    dense = [g for g in range(w.Hkv) if r["kind"][g] == 0]
+    assert all(len(r["sel"][(0, g)]) == 4 for g in dense)
+
+
+@pytest.mark.parametrize("G,d", [(1, 128), (2, 64), (4, 128), (8, 128)])
+def test_ragged_batch(G, d):
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2 * G, Hkv=2, d=d, dec_anchors=16)
+    run_decode(w, 3, 1000, 512, 64, 100, lens=[1000, 333, 65], kind=[0, 1])
+
+
+def test_more_heads_and_pages():
+    w = dataclasses.replace(W.WORKLOADS["llama3_8b_decode_b16_64k"], dec_anchors=32)
+    run_decode(w, 2, 8192 + 77, 1024, 64, 256)
+
+
+def test_budget_covers_context_equals_dense():
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=4, Hkv=2, d=128)
+    r = run_decode(w, 2, 700, 1 << 20, 64, 256, kind=[0, 0])
+    for b in range(2):
+        assert list(r["sel"][(b, 0)]) == list(range(11))
+
+
+def test_single_token_and_empty_sequence():
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=4, Hkv=2, d=64)
+    run_decode(w, 3, 130, 128, 0, 1, lens=[1, 130, 0], kind=[0, 1])
+
+
+def test_unselected_pages_are_never_read():
+    """Poison every pool row outside the attended token sets: the output is unchanged."""
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=8, Hkv=2, d=128, dec_anchors=8)
+    r = run_decode(w, 2, 1500, 256, 64, 100, lens=[1500, 1210], kind=[0, 1])
+    pc, q, kind = r["pc"], r["q"], r["kind"]
+    kp, vp = pc.k_pages.clone(), pc.v_pages.clone()
+    L = pc.seq_lens.tolist()
+    for b in range(2):
+        for g in range(2):
+            toks = set(OD.token_set(L[b], bool(kind[g]), 64, 100, None if kind[g] else r["sel"][(b, g)]).tolist())
+            for i in range(OS.n_pages(L[b])):
+                p = int(pc.page_table[b, i])
+                for row in range(64):
+                    if i * 64 + row not in toks:
+                        kp[p, g, row] = float("nan")
+                        vp[p, g, row] = float("nan")
+    dev = "cuda"
+    out2 = U.lserve_decode(q.to(dev), kp.to(dev), vp.to(dev), pc.page_table.to(dev), pc.seq_lens.to(dev),
+                           r["stats"], torch.tensor(kind, dtype=torch.uint8, device=dev), 64, 100, 256)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, r["out"])
+
+
+def test_incremental_page_stats():
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=4, Hkv=2, d=128)
+    pc = W.decode_cache(w, B=1, ctx=1000)
+    dev = "cuda"
+    hk = torch.tensor([0, 0], dtype=torch.uint8, device=dev)
+    kp, pt = pc.k_pages.to(dev), pc.page_table.to(dev)
+    full = U.lserve_update_page_stats(kp, pt, pc.seq_lens.to(dev), hk)
+    stale = full.clone()
+    stale[pc.page_table[0, 10:].long().to(dev)] = 0
+    U.lserve_update_page_stats(kp, pt, pc.seq_lens.to(dev), hk, stats=stale, first_logical_page=40)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.nan_to_num(stale.float(), nan=7.0), torch.nan_to_num(full.float(), nan=7.0))
+
+
+def test_out_of_range_page_id_is_reported_not_read():
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2, Hkv=1, d=64)
+    pc = W.decode_cache(w, B=1, ctx=256, NP=4)
+    pt = pc.page_table.clone()
+    pt[0, 2] = 1 << 20                       # outside the pool
+    dev = "cuda"
+    U.lserve_get_device_status()
+    U.lserve_update_page_stats(pc.k_pages.to(dev), pt.to(dev), pc.seq_lens.to(dev),
+                               torch.zeros(1, dtype=torch.uint8, device=dev))
+    assert U.lserve_get_device_status() == 6
+    assert U.lserve_get_device_status() == 0   # read clears it

@@ -1,0 +1,121 @@
+"""GPU parity of block-sparse prefill (tile lists + attention) against the oracle.
+
+All calls go through the C ABI (ctypes binding).  Inputs come from the seeded
+generators and are handed unchanged to both sides.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import attention as OA
+from parity import assert_attn_close, assert_lse_close, f64
+
+pytestmark = pytest.mark.gpu
+
+U = pytest.importorskip("unified_sparse_attention_b200")
+
+
+def run_case(w, S, kind, sink, local, mask_fill=None, B=None, seed_mask=True):
+    dev = "cuda"
+    q, k, v = W.prefill_inputs(w, S=S, B=B)
+    hk = torch.tensor(kind, dtype=torch.uint8)
+    bm = None
+    if mask_fill is not None:
+        ww = dataclasses.replace(w, mask_columns=2, mask_band=2)
+        bm = W.block_mask(ww, S=S, fill=mask_fill, B=q.shape[0])
+    out, lse = U.lserve_prefill(q.to(dev), k.to(dev), v.to(dev), hk.to(dev), sink, local,
+                                None if bm is None else bm.to(dev), return_lse=True)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+    ref, ref_lse = OA.masked_attention(f64(q), f64(k), f64(v), kind, sink, local,
+                                       None if bm is None else bm.numpy())
+    assert_attn_close(f64(out), ref, "prefill out")
+    assert_lse_close(f64(lse), ref_lse, "prefill lse")
+    return q, k, v, hk, bm, out
+
+
+def test_tiny_workload_exact_config():
+    w = W.WORKLOADS["tiny"]
+    run_case(w, w.S, W.head_kind(w).tolist(), w.sink, w.local)
+
+
+@pytest.mark.parametrize("sink,local", [(64, 256), (70, 130), (0, 1), (1, 0), (200, 64)])
+def test_gqa4_d128_block_mask(sink, local):
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=8, Hkv=2, d=128)
+    run_case(w, 1024, [0, 1], sink, local, mask_fill=0.4)
+
+
+def test_mha_d128_batch2():
+    w = dataclasses.replace(W.WORKLOADS["tiny"], B=2, Hq=4, Hkv=4, d=128)
+    run_case(w, 512, [0, 1, 1, 0], 64, 256, B=2)
+
+
+def test_gqa8_d64_masks():
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=16, Hkv=2, d=64)
+    run_case(w, 640, [1, 0], 0, 100, mask_fill=0.3)
+
+
+def test_single_tile_and_empty_rows():
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2, Hkv=2, d=128)
+    run_case(w, 64, [0, 1], 0, 0)          # streaming head: sink=0, local=0 -> every row empty
+    w2 = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2, Hkv=1, d=64)
+    q, k, v = W.prefill_inputs(w2, S=256)
+    bm = torch.zeros(1, 1, 4, 4, dtype=torch.uint8)
+    bm[0, 0, 2, 0] = 1                      # q-tile 2 keeps only kt=0; tiles 0, 1, 3 keep nothing
+    dev = "cuda"
+    out, lse = U.lserve_prefill(q.to(dev), k.to(dev), v.to(dev), torch.zeros(1, dtype=torch.uint8, device=dev),
+                                0, 0, bm.to(dev), return_lse=True)
+    ref, ref_lse = OA.masked_attention(f64(q), f64(k), f64(v), [0], 0, 0, bm.numpy())
+    assert_attn_close(f64(out), ref, "empty rows")
+    assert_lse_close(f64(lse), ref_lse, "empty rows lse")
+
+
+@pytest.mark.parametrize("mask_fill", [None, 0.35])
+def test_tile_lists_bit_exact(mask_fill):
+    w = dataclasses.replace(W.WORKLOADS["tiny"], B=2, Hq=8, Hkv=4, d=128, mask_columns=3, mask_band=2)
+    S = 1472   # 23 tiles
+    kind = [0, 1, 0, 1]
+    bm = W.block_mask(w, S=S, fill=mask_fill, B=2) if mask_fill is not None else None
+    hk = torch.tensor(kind, dtype=torch.uint8, device="cuda")
+    off, cols = U.lserve_prefill_tile_lists(2, S, 8, 4, 128, hk, 70, 190,
+                                            None if bm is None else bm.cuda())
+    torch.cuda.synchronize()
+    ref_off, ref_cols = OA.tile_lists(2, S, kind, 70, 190, None if bm is None else bm.numpy())
+    np.testing.assert_array_equal(off.cpu().numpy(), ref_off)
+    got = cols.cpu().numpy().view(np.uint16)[: ref_off[-1]].astype(np.int64)
+    np.testing.assert_array_equal(got, ref_cols)
+
+
+def test_skipped_tiles_are_never_read():
+    """Poison (NaN) every KV tile the last query tile does not keep: its rows are unchanged."""
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=4, Hkv=2, d=128, mask_columns=1, mask_band=1)
+    S, kind, sink, local = 1024, [0, 1], 64, 200
+    q, k, v = W.prefill_inputs(w, S=S)
+    bm = W.block_mask(w, S=S, fill=0.3)
+    dev = "cuda"
+    hk = torch.tensor(kind, dtype=torch.uint8, device=dev)
+    clean = U.lserve_prefill(q.to(dev), k.to(dev), v.to(dev), hk, sink, local, bm.to(dev))
+    k2, v2 = k.clone(), v.clone()
+    nq = S // 64
+    for g in range(2):
+        kept = OA.tile_kept(S, bool(kind[g]), sink, local, None if kind[g] else bm[0, g].numpy())[nq - 1]
+        for kt in np.nonzero(~kept)[0]:
+            k2[0, kt * 64:(kt + 1) * 64, g] = float("nan")
+            v2[0, kt * 64:(kt + 1) * 64, g] = float("nan")
+    pois = U.lserve_prefill(q.to(dev), k2.to(dev), v2.to(dev), hk, sink, local, bm.to(dev))
+    torch.cuda.synchronize()
+    last = slice(S - 64, S)
+    assert torch.equal(clean[:, last], pois[:, last])
+    assert torch.isfinite(pois[:, last].float()).all()
+
+
+def test_repeated_calls_are_deterministic():
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=8, Hkv=2, d=128)
+    q, k, v = (t.cuda() for t in W.prefill_inputs(w, S=512))
+    hk = torch.tensor([0, 1], dtype=torch.uint8, device="cuda")
+    a = U.lserve_prefill(q, k, v, hk, 64, 256)
+    b = U.lserve_prefill(q, k, v, hk, 64, 256)
+    assert torch.equal(a, b)

@@ -240,3 +240,13 @@ def test_tile_counts_tiny_workload():
 def test_tile_counts_closed_form_dense():
     for n in (1, 2, 7, 33):
         assert A.tile_kept(64 * n, False, 0, 0).sum() == n * (n + 1) // 2
+
+
+def test_q_at_rows_matches_full_q():
+    q, k, v = rand_qkv(1, 192, 2, 1, 8, 31)
+    kind = np.array([1], np.uint8)
+    rows = np.array([3, 64, 191])
+    o, lse = A.masked_attention(q, k, v, kind, 5, 20, rows=rows)
+    o2, lse2 = A.masked_attention(q[:, rows], k, v, kind, 5, 20, rows=rows, q_at_rows=True, row_chunk=2)
+    np.testing.assert_allclose(o, o2, atol=1e-14, rtol=0)
+    np.testing.assert_allclose(lse, lse2, atol=1e-14, rtol=0)

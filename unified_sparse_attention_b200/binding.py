@@ -1,0 +1,291 @@
+"""ctypes binding of liblserve.so: the C ABI's entry points under the same names.
+
+Argument marshalling only.  Tensors must already live on the CUDA device in the
+dtype and layout ``include/lserve.h`` gives; nothing here computes any part of
+the method, and a missing library or device raises instead of falling back.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+LSERVE_HEAD_DENSE = 0
+LSERVE_HEAD_STREAMING = 1
+PAGE = 64
+
+STATUS = {
+    0: "LSERVE_OK",
+    1: "LSERVE_ERR_INVALID_ARG",
+    2: "LSERVE_ERR_UNSUPPORTED",
+    3: "LSERVE_ERR_WORKSPACE",
+    4: "LSERVE_ERR_CUDA",
+    5: "LSERVE_ERR_DEVICE_TIMEOUT",
+    6: "LSERVE_ERR_DEVICE_BOUNDS",
+}
+
+# Every symbol include/lserve.h declares.
+EXPORTED_SYMBOLS = (
+    "lserve_prefill_workspace_size",
+    "lserve_prefill",
+    "lserve_prefill_tile_lists",
+    "lserve_update_page_stats",
+    "lserve_decode_max_selected",
+    "lserve_decode_workspace_size",
+    "lserve_decode",
+    "lserve_get_device_status",
+    "lserve_last_error_string",
+    "lserve_version",
+)
+
+
+class LServeError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("S", ctypes.c_int32), ("Hq", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class DecodeArgs(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("maxP", ctypes.c_int32),
+                ("q", ctypes.c_void_p), ("k_pages", ctypes.c_void_p), ("v_pages", ctypes.c_void_p),
+                ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p), ("stats", ctypes.c_void_p),
+                ("head_kind", ctypes.c_void_p), ("sink", ctypes.c_int32), ("local", ctypes.c_int32),
+                ("token_budget", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return os.environ.get("LSERVE_LIBRARY", os.path.join(_HERE, "liblserve.so"))
+
+
+def load_library():
+    """Load liblserve.so once (raises OSError with the path when it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise OSError(f"liblserve.so not found at {path}; build it with "
+                      f"`python -m unified_sparse_attention_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    sig = {
+        "lserve_prefill_workspace_size": (sz, [ctypes.POINTER(Shape)]),
+        "lserve_prefill": (i32, [ctypes.POINTER(Shape), vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
+        "lserve_prefill_tile_lists": (i32, [ctypes.POINTER(Shape), vp, i32, i32, vp, vp, vp, ctypes.c_int64,
+                                            vp, sz, vp]),
+        "lserve_update_page_stats": (i32, [i32, i32, i32, i32, vp, vp, i32, vp, i32, vp, vp, vp]),
+        "lserve_decode_max_selected": (i32, [ctypes.POINTER(DecodeArgs)]),
+        "lserve_decode_workspace_size": (sz, [ctypes.POINTER(DecodeArgs)]),
+        "lserve_decode": (i32, [ctypes.POINTER(DecodeArgs), vp, vp, vp, vp, vp, sz, vp]),
+        "lserve_get_device_status": (i32, [vp]),
+        "lserve_last_error_string": (ctypes.c_char_p, []),
+        "lserve_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def lserve_last_error_string() -> str:
+    return load_library().lserve_last_error_string().decode()
+
+
+def lserve_version() -> str:
+    return load_library().lserve_version().decode()
+
+
+def _check(status: int):
+    if status != 0:
+        raise LServeError(status, lserve_last_error_string())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    if workspace is not None:
+        return workspace
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------- prefill
+
+def _shape(q, k, scale):
+    B, S, Hq, d = q.shape
+    return Shape(B, S, Hq, k.shape[2], d, float(scale))
+
+
+def lserve_prefill_workspace_size(B: int, S: int, Hq: int, Hkv: int, d: int) -> int:
+    return int(load_library().lserve_prefill_workspace_size(ctypes.byref(Shape(B, S, Hq, Hkv, d, 0.0))))
+
+
+def lserve_prefill(q, k, v, head_kind, sink: int, local: int, block_mask=None, out=None, lse=None,
+                   scale: float = 0.0, workspace=None, stream=None, return_lse: bool = False):
+    """Block-sparse causal prefill; see include/lserve.h.  Returns out (and lse)."""
+    lib = load_library()
+    _dev(q, "q", torch.bfloat16)
+    B, S, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _dev(k, "k", torch.bfloat16, (B, S, Hkv, d))
+    _dev(v, "v", torch.bfloat16, (B, S, Hkv, d))
+    _dev(head_kind, "head_kind", torch.uint8, (Hkv,))
+    if block_mask is not None:
+        _dev(block_mask, "block_mask", torch.uint8, (B, Hkv, S // PAGE, S // PAGE))
+    out = torch.empty_like(q) if out is None else _dev(out, "out", torch.bfloat16, q.shape)
+    if lse is None and return_lse:
+        lse = torch.empty(B, Hq, S, dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _dev(lse, "lse", torch.float32, (B, Hq, S))
+    shape = _shape(q, k, scale)
+    need = int(lib.lserve_prefill_workspace_size(ctypes.byref(shape)))
+    ws = _workspace(need, q.device, workspace)
+    _check(lib.lserve_prefill(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(head_kind), int(sink),
+                              int(local), _ptr(block_mask), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                              _stream(stream)))
+    return (out, lse) if (return_lse or lse is not None) else out
+
+
+def lserve_prefill_tile_lists(B, S, Hq, Hkv, d, head_kind, sink, local, block_mask=None, stream=None):
+    """Kept-tile CSR (row_offsets int32[R+1], tile_cols uint16[nnz]) on the device."""
+    lib = load_library()
+    _dev(head_kind, "head_kind", torch.uint8, (Hkv,))
+    n = S // PAGE
+    if block_mask is not None:
+        _dev(block_mask, "block_mask", torch.uint8, (B, Hkv, n, n))
+    dev = head_kind.device
+    R = B * Hkv * n
+    max_nnz = R * (n + 1) // 2
+    offsets = torch.empty(R + 1, dtype=torch.int32, device=dev)
+    cols = torch.empty(max(max_nnz, 1), dtype=torch.int16, device=dev)
+    shape = Shape(B, S, Hq, Hkv, d, 0.0)
+    ws = _workspace(lib.lserve_prefill_workspace_size(ctypes.byref(shape)), dev, None)
+    _check(lib.lserve_prefill_tile_lists(ctypes.byref(shape), _ptr(head_kind), int(sink), int(local),
+                                         _ptr(block_mask), _ptr(offsets), _ptr(cols), max_nnz, _ptr(ws),
+                                         ws.numel(), _stream(stream)))
+    return offsets, cols
+
+
+# ------------------------------------------------------------ page stats
+
+def lserve_update_page_stats(k_pages, page_table, seq_lens, head_kind, stats=None, first_logical_page: int = 0,
+                             stream=None):
+    """Per-logical-page key min/max; returns stats bf16[NP, Hkv, 4, 2, d]."""
+    lib = load_library()
+    _dev(k_pages, "k_pages", torch.bfloat16)
+    NP, Hkv, P, d = k_pages.shape
+    if P != PAGE:
+        raise ValueError("k_pages must have 64-token pages")
+    _dev(page_table, "page_table", torch.int32)
+    B, maxP = page_table.shape
+    _dev(seq_lens, "seq_lens", torch.int32, (B,))
+    _dev(head_kind, "head_kind", torch.uint8, (Hkv,))
+    if stats is None:
+        stats = torch.full((NP, Hkv, 4, 2, d), float("nan"), dtype=torch.bfloat16, device=k_pages.device)
+    _dev(stats, "stats", torch.bfloat16, (NP, Hkv, 4, 2, d))
+    _check(lib.lserve_update_page_stats(B, Hkv, d, NP, _ptr(k_pages), _ptr(page_table), maxP, _ptr(seq_lens),
+                                        int(first_logical_page), _ptr(head_kind), _ptr(stats), _stream(stream)))
+    return stats
+
+
+# ----------------------------------------------------------------- decode
+
+def _decode_args(q, k_pages, v_pages, page_table, seq_lens, stats, head_kind, sink, local, token_budget, scale):
+    _dev(q, "q", torch.bfloat16)
+    B, Hq, d = q.shape
+    _dev(k_pages, "k_pages", torch.bfloat16)
+    NP, Hkv, P, d2 = k_pages.shape
+    if P != PAGE or d2 != d:
+        raise ValueError("k_pages must be [NP, Hkv, 64, d]")
+    _dev(v_pages, "v_pages", torch.bfloat16, k_pages.shape)
+    _dev(page_table, "page_table", torch.int32)
+    if page_table.shape[0] != B:
+        raise ValueError("page_table must be [B, maxP]")
+    _dev(seq_lens, "seq_lens", torch.int32, (B,))
+    _dev(stats, "stats", torch.bfloat16, (NP, Hkv, 4, 2, d))
+    _dev(head_kind, "head_kind", torch.uint8, (Hkv,))
+    return DecodeArgs(B, Hq, Hkv, d, NP, page_table.shape[1], q.data_ptr(), k_pages.data_ptr(),
+                      v_pages.data_ptr(), page_table.data_ptr(), seq_lens.data_ptr(), stats.data_ptr(),
+                      head_kind.data_ptr(), int(sink), int(local), int(token_budget), float(scale))
+
+
+def lserve_decode_max_selected(B, Hq, Hkv, d, num_pages, maxP, sink, local, token_budget) -> int:
+    a = DecodeArgs(B, Hq, Hkv, d, num_pages, maxP, None, None, None, None, None, None, None, sink, local,
+                   token_budget, 0.0)
+    return int(load_library().lserve_decode_max_selected(ctypes.byref(a)))
+
+
+def lserve_decode_workspace_size(q, k_pages, v_pages, page_table, seq_lens, stats, head_kind, sink, local,
+                                 token_budget, scale=0.0) -> int:
+    a = _decode_args(q, k_pages, v_pages, page_table, seq_lens, stats, head_kind, sink, local, token_budget, scale)
+    return int(load_library().lserve_decode_workspace_size(ctypes.byref(a)))
+
+
+def lserve_decode(q, k_pages, v_pages, page_table, seq_lens, stats, head_kind, sink: int, local: int,
+                  token_budget: int, scale: float = 0.0, out=None, lse=None, sel_out=None, sel_n=None,
+                  workspace=None, stream=None, return_selection: bool = False):
+    """One sparse decode step; see include/lserve.h.  Returns out (and lse, sel, sel_n)."""
+    lib = load_library()
+    a = _decode_args(q, k_pages, v_pages, page_table, seq_lens, stats, head_kind, sink, local, token_budget, scale)
+    B, Hq, d = q.shape
+    Hkv = a.Hkv
+    out = torch.empty_like(q) if out is None else _dev(out, "out", torch.bfloat16, q.shape)
+    if lse is not None:
+        _dev(lse, "lse", torch.float32, (B, Hq))
+    kcap = int(lib.lserve_decode_max_selected(ctypes.byref(a)))
+    if return_selection and sel_out is None:
+        sel_out = torch.empty(B, Hkv, kcap, dtype=torch.int32, device=q.device)
+        sel_n = torch.empty(B, Hkv, dtype=torch.int32, device=q.device) if sel_n is None else sel_n
+    if sel_out is not None:
+        _dev(sel_out, "sel_out", torch.int32, (B, Hkv, kcap))
+    if sel_n is not None:
+        _dev(sel_n, "sel_n", torch.int32, (B, Hkv))
+    need = int(lib.lserve_decode_workspace_size(ctypes.byref(a)))
+    if need == 0:   # invalid arguments: let the library report which
+        _check(lib.lserve_decode(ctypes.byref(a), _ptr(out), None, None, None, None, 0, _stream(stream)))
+    ws = _workspace(need, q.device, workspace)
+    _check(lib.lserve_decode(ctypes.byref(a), _ptr(out), _ptr(lse), _ptr(sel_out), _ptr(sel_n), _ptr(ws),
+                             ws.numel(), _stream(stream)))
+    if return_selection:
+        return out, lse, sel_out, sel_n
+    return out
+
+
+def lserve_get_device_status(stream=None) -> int:
+    """Synchronise, read and clear the device status word (0 = OK)."""
+    return int(load_library().lserve_get_device_status(_stream(stream)))

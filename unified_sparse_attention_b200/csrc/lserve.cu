@@ -1,0 +1,430 @@
+// lserve.cu -- the C ABI of liblserve.so (declared in include/lserve.h).
+//
+// Host side only: argument validation (before any launch), workspace carving,
+// TMA descriptor encoding and kernel launches on the caller's stream.  All
+// arithmetic of the method runs in the kernels included below.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "page_stats.cuh"
+#include "prefill_mma.cuh"
+#include "select.cuh"
+#include "tile_lists.cuh"
+
+using namespace lserve;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+lserve_status fail(lserve_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+lserve_status ok() {
+  g_err[0] = '\0';
+  return LSERVE_OK;
+}
+
+lserve_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(LSERVE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return LSERVE_OK;
+}
+
+unsigned long long wait_timeout_ns() {
+  static unsigned long long v = [] {
+    const char* s = getenv("LSERVE_WAIT_TIMEOUT_NS");
+    unsigned long long t = s ? strtoull(s, nullptr, 10) : 0ull;
+    return t ? t : 2000000000ull;   // 2 s
+  }();
+  return v;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+template <typename K>
+void ensure_smem(K* kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.insert(key).second)
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// ---------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// 2-D bf16 view [rows, inner] (row stride = inner elements), box 64 x 64, 128B swizzle.
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 view [tokens, heads, D], box (64 channels, 1 head, 64 tokens), 128B swizzle.
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t D, uint64_t H, uint64_t T) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {D, H, T};
+  cuuint64_t strides[2] = {D * 2, H * D * 2};
+  cuuint32_t box[3] = {64, 1, 64};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- workspace
+struct Carver {
+  uintptr_t base, cur;
+  explicit Carver(void* p) : base(reinterpret_cast<uintptr_t>(p)), cur(reinterpret_cast<uintptr_t>(p)) {}
+  template <typename T>
+  T* take(size_t count) {
+    cur = (cur + 255) & ~uintptr_t(255);
+    T* p = reinterpret_cast<T*>(cur);
+    cur += count * sizeof(T);
+    return p;
+  }
+  size_t used() const { return cur - base + 256; }
+};
+
+// ---------------------------------------------------------------- prefill
+struct PrefillWs {
+  int* counts;
+  int* offsets;
+  int* order;
+  int* hist;     // [nQT + 1]
+  int* fill;     // [nQT + 1]  (contiguous with hist: one memset clears both)
+  int* bucket;   // [nQT + 1]
+  int* overflow;
+  uint16_t* cols;
+  long long max_nnz;
+};
+
+bool shape_valid(const lserve_shape* s) {
+  return s && s->B > 0 && s->S > 0 && s->Hq > 0 && s->Hkv > 0 && s->d > 0 && s->Hq % s->Hkv == 0;
+}
+
+PrefillWs carve_prefill(const lserve_shape* s, void* ws, size_t* bytes) {
+  const long long nQT = s->S / kTile;
+  const long long R = static_cast<long long>(s->B) * s->Hkv * nQT;
+  Carver c(ws);
+  PrefillWs w;
+  w.counts = c.take<int>(R);
+  w.offsets = c.take<int>(R + 1);
+  w.order = c.take<int>(R);
+  w.hist = c.take<int>(2 * (nQT + 1));
+  w.fill = w.hist + (nQT + 1);
+  w.bucket = c.take<int>(nQT + 1);
+  w.overflow = c.take<int>(1);
+  w.max_nnz = R * (nQT + 1) / 2;
+  w.cols = c.take<uint16_t>(w.max_nnz);
+  if (bytes) *bytes = c.used();
+  return w;
+}
+
+lserve_status validate_prefill(const lserve_shape* s, int sink, int local) {
+  if (!shape_valid(s)) return fail(LSERVE_ERR_INVALID_ARG, "prefill: invalid shape");
+  if (s->d != 64 && s->d != 128) return fail(LSERVE_ERR_UNSUPPORTED, "prefill: head dim %d not in {64,128}", s->d);
+  if (s->S % kTile) return fail(LSERVE_ERR_UNSUPPORTED, "prefill: S=%d is not a multiple of 64", s->S);
+  if (s->S / kTile > 65535) return fail(LSERVE_ERR_UNSUPPORTED, "prefill: S=%d too long", s->S);
+  if (static_cast<long long>(s->B) * s->S > (1ll << 31) - 1)
+    return fail(LSERVE_ERR_UNSUPPORTED, "prefill: B*S too large");
+  if (sink < 0 || local < 0) return fail(LSERVE_ERR_INVALID_ARG, "prefill: sink/local must be >= 0");
+  const long long R = static_cast<long long>(s->B) * s->Hkv * (s->S / kTile);
+  if (R * (s->S / kTile + 1) / 2 > (1ll << 31) - 1) return fail(LSERVE_ERR_UNSUPPORTED, "prefill: too many tiles");
+  return LSERVE_OK;
+}
+
+lserve_status launch_tile_lists(const lserve_shape* s, const uint8_t* head_kind, int sink, int local,
+                                const uint8_t* block_mask, const PrefillWs& w, int* offsets, uint16_t* cols,
+                                long long max_nnz, int* order, cudaStream_t st) {
+  const int nQT = s->S / kTile;
+  const int R = s->B * s->Hkv * nQT;
+  TileListParams P{s->B, s->Hkv, nQT, sink, local, head_kind, block_mask};
+  if (cudaMemsetAsync(w.hist, 0, sizeof(int) * 2 * (nQT + 1), st) != cudaSuccess)
+    return fail(LSERVE_ERR_CUDA, "prefill: memset failed");
+  const int blocks = (R + 7) / 8;
+  tile_count_kernel<<<blocks, 256, 0, st>>>(P, w.counts, w.hist);
+  tile_scan_kernel<<<1, 1024, 0, st>>>(w.counts, R, offsets, w.hist, nQT + 1, w.bucket, max_nnz, w.overflow);
+  tile_fill_kernel<<<blocks, 256, 0, st>>>(P, offsets, w.counts, cols, w.bucket, w.fill, order, w.overflow);
+  return check_launch("tile lists");
+}
+
+template <int D>
+lserve_status launch_prefill_mma(const lserve_shape* s, const void* q, const void* k, const void* v,
+                                 const PrefillArgs& A, int n_rows, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  const uint64_t T = static_cast<uint64_t>(s->B) * s->S;
+  if (!make_map_3d(&tq, q, D, s->Hq, T) || !make_map_3d(&tk, k, D, s->Hkv, T) || !make_map_3d(&tv, v, D, s->Hkv, T))
+    return fail(LSERVE_ERR_CUDA, "prefill: cuTensorMapEncodeTiled failed");
+  ensure_smem(prefill_mma_kernel<D>, PrefillCfg<D>::kSmemBytes);
+  const long long grid = static_cast<long long>(n_rows) * A.G;
+  prefill_mma_kernel<D><<<static_cast<unsigned>(grid), kPrefillThreads, PrefillCfg<D>::kSmemBytes, st>>>(tq, tk, tv,
+                                                                                                      A);
+  return check_launch("prefill attention");
+}
+
+// ----------------------------------------------------------------- decode
+struct DecodePlan {
+  int kcap, budget_pages, pps, nsplit, G, ppb;
+  float* scores;
+  int32_t* sel;
+  int32_t* sel_n;
+  float* part_o;
+  float* part_lse;
+  size_t bytes;
+};
+
+int streaming_page_bound(int sink, int local) {
+  return (sink + kPage - 1) / kPage + (local + kPage - 1) / kPage + 1;
+}
+
+lserve_status validate_decode(const lserve_decode_args* a) {
+  if (!a) return fail(LSERVE_ERR_INVALID_ARG, "decode: null args");
+  if (a->B <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->d <= 0 || a->Hq % a->Hkv || a->num_pages <= 0 || a->maxP <= 0)
+    return fail(LSERVE_ERR_INVALID_ARG, "decode: invalid shape");
+  if (a->d != 64 && a->d != 128) return fail(LSERVE_ERR_UNSUPPORTED, "decode: head dim %d not in {64,128}", a->d);
+  if (a->Hkv > 256) return fail(LSERVE_ERR_UNSUPPORTED, "decode: more than 256 KV heads");
+  const int G = a->Hq / a->Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return fail(LSERVE_ERR_UNSUPPORTED, "decode: Hq/Hkv=%d not in {1,2,4,8}", G);
+  if (a->token_budget < kPage) return fail(LSERVE_ERR_INVALID_ARG, "decode: token_budget must be >= 64");
+  if (a->sink < 0 || a->local < 0) return fail(LSERVE_ERR_INVALID_ARG, "decode: sink/local must be >= 0");
+  if (static_cast<long long>(a->num_pages) * a->Hkv * kPage > (1ll << 31) - 1)
+    return fail(LSERVE_ERR_UNSUPPORTED, "decode: page pool too large for 32-bit TMA coordinates");
+  if (!a->q || !a->k_pages || !a->v_pages || !a->page_table || !a->seq_lens || !a->stats || !a->head_kind)
+    return fail(LSERVE_ERR_INVALID_ARG, "decode: null tensor pointer");
+  if (!aligned16(a->q) || !aligned16(a->k_pages) || !aligned16(a->v_pages) || !aligned16(a->stats))
+    return fail(LSERVE_ERR_INVALID_ARG, "decode: tensors must be 16-byte aligned");
+  return LSERVE_OK;
+}
+
+DecodePlan plan_decode(const lserve_decode_args* a, void* ws) {
+  DecodePlan p{};
+  p.G = a->Hq / a->Hkv;
+  p.budget_pages = a->token_budget / kPage;
+  const int dense_cap = std::min(p.budget_pages, a->maxP);
+  p.kcap = std::max(1, std::max(dense_cap, std::min(streaming_page_bound(a->sink, a->local), a->maxP)));
+  // split-KV: aim for ~8 CTAs per SM over the dense selections
+  const long long total = static_cast<long long>(a->B) * a->Hkv * p.kcap;
+  long long pps = (total + 8 * 148 - 1) / (8 * 148);
+  p.pps = static_cast<int>(std::max(2ll, std::min<long long>(pps, 64)));
+  p.nsplit = (p.kcap + p.pps - 1) / p.pps;
+  // scoring: aim for >= ~4 CTAs per SM
+  const long long pages = static_cast<long long>(a->B) * a->maxP;
+  long long ppb = pages / (4 * 148);
+  p.ppb = static_cast<int>(std::max(4ll, std::min<long long>(ppb, 64)));
+  Carver c(ws);
+  const long long units = static_cast<long long>(a->B) * a->Hkv;
+  p.scores = c.take<float>(units * a->maxP);
+  p.sel = c.take<int32_t>(units * p.kcap);
+  p.sel_n = c.take<int32_t>(units);
+  p.part_o = c.take<float>(units * p.nsplit * p.G * a->d);
+  p.part_lse = c.take<float>(units * p.nsplit * p.G);
+  p.bytes = c.used();
+  return p;
+}
+
+template <int D, int G>
+void launch_score(const lserve_decode_args* a, const DecodePlan& p, cudaStream_t st) {
+  dim3 grid((a->maxP + p.ppb - 1) / p.ppb, a->B);
+  score_pages_kernel<D, G><<<grid, 256, 0, st>>>(static_cast<const bf16*>(a->q), static_cast<const bf16*>(a->stats),
+                                                 a->page_table, a->maxP, a->seq_lens, a->head_kind, a->Hkv,
+                                                 a->num_pages, p.ppb, p.scores);
+}
+
+template <int D>
+lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, int32_t* sel, int32_t* sel_n,
+                              void* out, float* lse, cudaStream_t st) {
+  switch (p.G) {
+    case 1: launch_score<D, 1>(a, p, st); break;
+    case 2: launch_score<D, 2>(a, p, st); break;
+    case 4: launch_score<D, 4>(a, p, st); break;
+    default: launch_score<D, 8>(a, p, st); break;
+  }
+  ensure_smem(topk_pages_kernel, kTopkSmemKeys * static_cast<int>(sizeof(uint32_t)));
+  const int topk_smem = std::min(a->maxP, kTopkSmemKeys) * static_cast<int>(sizeof(uint32_t));
+  topk_pages_kernel<<<a->B * a->Hkv, kTopkThreads, topk_smem, st>>>(p.scores, a->maxP, a->seq_lens, a->head_kind,
+                                                                     a->Hkv, p.budget_pages, a->sink, a->local, sel,
+                                                                     sel_n, p.kcap);
+  CUtensorMap tk, tv;
+  const uint64_t rows = static_cast<uint64_t>(a->num_pages) * a->Hkv * kPage;
+  if (!make_map_2d(&tk, a->k_pages, D, rows) || !make_map_2d(&tv, a->v_pages, D, rows))
+    return fail(LSERVE_ERR_CUDA, "decode: cuTensorMapEncodeTiled failed");
+  ensure_smem(paged_decode_kernel<D>, DecodeCfg<D>::kSmemBytes);
+  const float scale = a->scale > 0.f ? a->scale : 1.f / std::sqrt(static_cast<float>(D));
+  dim3 grid(p.nsplit, a->B * a->Hkv);
+  paged_decode_kernel<D><<<grid, kDecodeThreads, DecodeCfg<D>::kSmemBytes, st>>>(
+      tk, tv, static_cast<const bf16*>(a->q), a->page_table, a->maxP, a->seq_lens, a->head_kind, sel, sel_n, p.kcap,
+      p.pps, p.nsplit, a->Hkv, p.G, a->num_pages, a->sink, a->local, scale * 1.4426950408889634f, wait_timeout_ns(),
+      p.part_o, p.part_lse);
+  lse_merge_kernel<D><<<a->B * a->Hq, D, 0, st>>>(p.part_o, p.part_lse, sel_n, p.kcap, p.pps, p.nsplit, a->Hkv, p.G,
+                                                  static_cast<bf16*>(out), lse);
+  return check_launch("decode");
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* lserve_version(void) { return "0.1.0"; }
+
+const char* lserve_last_error_string(void) { return g_err; }
+
+size_t lserve_prefill_workspace_size(const lserve_shape* shape) {
+  if (!shape_valid(shape) || shape->S % kTile) return 0;
+  size_t bytes = 0;
+  carve_prefill(shape, nullptr, &bytes);
+  return bytes;
+}
+
+lserve_status lserve_prefill_tile_lists(const lserve_shape* shape, const uint8_t* head_kind, int32_t sink,
+                                        int32_t local, const uint8_t* block_mask, int32_t* row_offsets,
+                                        uint16_t* tile_cols, int64_t max_nnz, void* workspace, size_t ws_bytes,
+                                        void* stream) {
+  lserve_status s = validate_prefill(shape, sink, local);
+  if (s != LSERVE_OK) return s;
+  if (!head_kind || !row_offsets || !tile_cols || max_nnz < 0)
+    return fail(LSERVE_ERR_INVALID_ARG, "tile lists: null pointer or negative capacity");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      ws_bytes < lserve_prefill_workspace_size(shape))
+    return fail(LSERVE_ERR_WORKSPACE, "tile lists: workspace missing, misaligned or smaller than %zu bytes",
+                lserve_prefill_workspace_size(shape));
+  PrefillWs w = carve_prefill(shape, workspace, nullptr);
+  s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, row_offsets, tile_cols, max_nnz, nullptr,
+                        static_cast<cudaStream_t>(stream));
+  return s == LSERVE_OK ? ok() : s;
+}
+
+lserve_status lserve_prefill(const lserve_shape* shape, const void* q, const void* k, const void* v,
+                             const uint8_t* head_kind, int32_t sink, int32_t local, const uint8_t* block_mask,
+                             void* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  lserve_status s = validate_prefill(shape, sink, local);
+  if (s != LSERVE_OK) return s;
+  if (!q || !k || !v || !head_kind || !out) return fail(LSERVE_ERR_INVALID_ARG, "prefill: null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(LSERVE_ERR_INVALID_ARG, "prefill: q/k/v/out must be 16-byte aligned");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      ws_bytes < lserve_prefill_workspace_size(shape))
+    return fail(LSERVE_ERR_WORKSPACE, "prefill: workspace missing, misaligned or smaller than %zu bytes",
+                lserve_prefill_workspace_size(shape));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  PrefillWs w = carve_prefill(shape, workspace, nullptr);
+  s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz, w.order, st);
+  if (s != LSERVE_OK) return s;
+  const float scale = shape->scale > 0.f ? shape->scale : 1.f / std::sqrt(static_cast<float>(shape->d));
+  PrefillArgs A{w.offsets, w.cols, w.order, head_kind, static_cast<bf16*>(out), lse, shape->Hq / shape->Hkv,
+                shape->Hkv, shape->S / kTile, shape->S, sink, local, scale * 1.4426950408889634f, wait_timeout_ns()};
+  const int n_rows = shape->B * shape->Hkv * (shape->S / kTile);
+  s = shape->d == 128 ? launch_prefill_mma<128>(shape, q, k, v, A, n_rows, st)
+                      : launch_prefill_mma<64>(shape, q, k, v, A, n_rows, st);
+  return s == LSERVE_OK ? ok() : s;
+}
+
+lserve_status lserve_update_page_stats(int32_t B, int32_t Hkv, int32_t d, int32_t num_pages, const void* k_pages,
+                                       const int32_t* page_table, int32_t maxP, const int32_t* seq_lens,
+                                       int32_t first_logical_page, const uint8_t* head_kind, void* stats,
+                                       void* stream) {
+  if (B <= 0 || Hkv <= 0 || num_pages <= 0 || maxP <= 0 || first_logical_page < 0)
+    return fail(LSERVE_ERR_INVALID_ARG, "page stats: invalid sizes");
+  if (d != 64 && d != 128) return fail(LSERVE_ERR_UNSUPPORTED, "page stats: head dim %d not in {64,128}", d);
+  if (!k_pages || !page_table || !seq_lens || !head_kind || !stats)
+    return fail(LSERVE_ERR_INVALID_ARG, "page stats: null pointer");
+  if (!aligned16(k_pages) || !aligned16(stats))
+    return fail(LSERVE_ERR_INVALID_ARG, "page stats: k_pages/stats must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long units = static_cast<long long>(maxP) * Hkv;
+  dim3 grid(static_cast<unsigned>((units + 7) / 8), B);
+  if (d == 128)
+    page_stats_kernel<128><<<grid, 256, 0, st>>>(static_cast<const bf16*>(k_pages), page_table, maxP, seq_lens,
+                                                 first_logical_page, head_kind, Hkv, num_pages,
+                                                 static_cast<bf16*>(stats));
+  else
+    page_stats_kernel<64><<<grid, 256, 0, st>>>(static_cast<const bf16*>(k_pages), page_table, maxP, seq_lens,
+                                                first_logical_page, head_kind, Hkv, num_pages,
+                                                static_cast<bf16*>(stats));
+  lserve_status s = check_launch("page stats");
+  return s == LSERVE_OK ? ok() : s;
+}
+
+int32_t lserve_decode_max_selected(const lserve_decode_args* args) {
+  if (!args || args->maxP <= 0 || args->token_budget < kPage) return 0;
+  return std::max(1, std::max(std::min(args->token_budget / kPage, args->maxP),
+                              std::min(streaming_page_bound(args->sink, args->local), args->maxP)));
+}
+
+size_t lserve_decode_workspace_size(const lserve_decode_args* args) {
+  if (validate_decode(args) != LSERVE_OK) return 0;
+  return plan_decode(args, nullptr).bytes;
+}
+
+lserve_status lserve_decode(const lserve_decode_args* args, void* out, float* lse, int32_t* sel_out,
+                            int32_t* sel_n, void* workspace, size_t ws_bytes, void* stream) {
+  lserve_status s = validate_decode(args);
+  if (s != LSERVE_OK) return s;
+  if (!out || !aligned16(out)) return fail(LSERVE_ERR_INVALID_ARG, "decode: out must be non-null and 16-byte aligned");
+  const size_t need = plan_decode(args, nullptr).bytes;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < need)
+    return fail(LSERVE_ERR_WORKSPACE, "decode: workspace missing, misaligned or smaller than %zu bytes", need);
+  DecodePlan p = plan_decode(args, workspace);
+  int32_t* sel = sel_out ? sel_out : p.sel;
+  int32_t* seln = sel_n ? sel_n : p.sel_n;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = args->d == 128 ? launch_decode_d<128>(args, p, sel, seln, out, lse, st)
+                     : launch_decode_d<64>(args, p, sel, seln, out, lse, st);
+  return s == LSERVE_OK ? ok() : s;
+}
+
+lserve_status lserve_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(LSERVE_ERR_CUDA, "device status: stream synchronisation failed: %s",
+                cudaGetErrorString(cudaGetLastError()));
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess)
+    return fail(LSERVE_ERR_CUDA, "device status: read failed");
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess)
+    return fail(LSERVE_ERR_CUDA, "device status: clear failed");
+  if (v == 0) return ok();
+  return fail(static_cast<lserve_status>(v), "kernel reported %s",
+              v == LSERVE_ERR_DEVICE_TIMEOUT ? "a bounded wait that ran out" : "an out-of-range index");
+}
+
+}  // extern "C"

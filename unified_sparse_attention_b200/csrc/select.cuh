@@ -1,0 +1,293 @@
+// select.cuh -- query-aware hierarchical page selection for decode.
+//
+// LServe + SampleAttention blog post, "LServe - Decode Phase" and Fig. 2: score
+// every page from its summary, keep the top-k, then attend inside those pages
+// only; mlsanity LServe page, Abstract: a hierarchical KV page selection policy
+// by query-centric similarity, with a constant number of pages kept.
+//
+// score_pages_kernel  (HBM-bound stream over the summaries)
+//   bound of query head h on logical page l:  sum_c max(q_hc * kmax_c, q_hc * kmin_c)
+//   group score: max over the G query heads of the KV head; page score: max over
+//   the page's logical pages that hold a valid token.  One warp per physical
+//   page: lane = (logical page l = lane/8, 16 (d=128) or 8 (d=64) channels),
+//   four 16-byte loads per lane, fp32 products (exact for bf16 operands) and a
+//   3-step shuffle sum per head, then shuffle max over heads and logical pages.
+//
+// topk_pages_kernel  (latency-bound, one CTA per (sequence, KV head))
+//   k = min(budget/64, n_pages) pages by 4-pass 8-bit radix select on the
+//   order-preserving uint32 image of the fp32 scores, ties to the lower page
+//   index, emitted in ascending page order by a block-wide scan.  Streaming
+//   heads get their fixed sink + local page list from the same kernel.
+#pragma once
+
+#include "common.cuh"
+
+namespace lserve {
+
+// ------------------------------------------------------------------ scoring
+template <int D, int G>
+__global__ void __launch_bounds__(256) score_pages_kernel(
+    const bf16* __restrict__ q, const bf16* __restrict__ stats, const int32_t* __restrict__ page_table, int maxP,
+    const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind, int Hkv, int num_pages,
+    int pages_per_block, float* __restrict__ scores) {
+  constexpr int CPL = D / 8;   // channels per lane
+  __shared__ int s_dense[256];
+  __shared__ int s_ndense;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int b = blockIdx.y;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int g = 0; g < Hkv; ++g)
+      if (head_kind[g] == LSERVE_HEAD_DENSE) s_dense[n++] = g;
+    s_ndense = n;
+  }
+  __syncthreads();
+  const int L = seq_lens[b];
+  const int n_pages = min(maxP, (L + kPage - 1) / kPage);
+  const int i0 = blockIdx.x * pages_per_block;
+  const int i1 = min(i0 + pages_per_block, n_pages);
+  if (i0 >= i1) return;
+  const int npg = i1 - i0;
+  const int units = s_ndense * npg;
+  const int l = lane >> 3;           // logical page of this lane
+  const int c0 = (lane & 7) * CPL;   // first channel of this lane
+  const float ninf = kNegInf;
+
+  int cur_g = -1;
+  float qf[G][CPL];
+  for (int u = warp; u < units; u += nwarps) {
+    const int g = s_dense[u / npg];
+    const int i = i0 + u % npg;
+    if (g != cur_g) {
+      cur_g = g;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const bf16* qp = q + (static_cast<long>(b) * Hkv * G + g * G + h) * D + c0;
+#pragma unroll
+        for (int c = 0; c < CPL; c += 8) {
+          uint4 v = __ldg(reinterpret_cast<const uint4*>(qp + c));
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            qf[h][c + 2 * e] = bf16_lo(w[e]);
+            qf[h][c + 2 * e + 1] = bf16_hi(w[e]);
+          }
+        }
+      }
+    }
+    const int p = page_table[static_cast<long>(b) * maxP + i];
+    float s = ninf;
+    if (p >= 0 && p < num_pages) {
+      const bf16* sp = stats + ((static_cast<long>(p) * Hkv + g) * kNL + l) * 2 * D + c0;
+      uint4 mn[CPL / 8], mx[CPL / 8];
+#pragma unroll
+      for (int c = 0; c < CPL / 8; ++c) {
+        mn[c] = __ldg(reinterpret_cast<const uint4*>(sp + c * 8));
+        mx[c] = __ldg(reinterpret_cast<const uint4*>(sp + D + c * 8));
+      }
+      float best = ninf;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL / 8; ++c) {
+          const uint32_t* a = reinterpret_cast<const uint32_t*>(&mn[c]);
+          const uint32_t* z = reinterpret_cast<const uint32_t*>(&mx[c]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float q0 = qf[h][c * 8 + 2 * e], q1 = qf[h][c * 8 + 2 * e + 1];
+            acc += fmaxf(q0 * bf16_lo(z[e]), q0 * bf16_lo(a[e]));
+            acc += fmaxf(q1 * bf16_hi(z[e]), q1 * bf16_hi(a[e]));
+          }
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        best = fmaxf(best, acc);
+      }
+      // logical pages without a valid token do not count
+      s = (i * kPage + l * kLogical < L) ? best : ninf;
+    } else if (lane == 0) {
+      report(LSERVE_ERR_DEVICE_BOUNDS);
+    }
+    s = fmaxf(s, __shfl_xor_sync(0xffffffffu, s, 8));
+    s = fmaxf(s, __shfl_xor_sync(0xffffffffu, s, 16));
+    if (lane == 0) scores[(static_cast<long>(b) * Hkv + g) * maxP + i] = s;
+  }
+}
+
+// -------------------------------------------------------------------- top-k
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Block-wide exclusive scan of one int per thread; returns the prefix, writes
+// the block total to *total.  Needs blockDim.x/32 ints of scratch.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < nw) scratch[lane] = w;
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? scratch[warp - 1] : 0) + x - v;
+  *total = scratch[nw - 1];
+  __syncthreads();
+  return before;
+}
+
+constexpr int kTopkThreads = 1024;
+constexpr int kTopkSmemKeys = 16384;   // scores cached in shared memory up to this many pages
+
+__global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
+    const float* __restrict__ scores, int maxP, const int32_t* __restrict__ seq_lens,
+    const uint8_t* __restrict__ head_kind, int Hkv, int budget_pages, int sink, int local,
+    int32_t* __restrict__ sel, int32_t* __restrict__ sel_n, int kcap) {
+  extern __shared__ uint32_t s_keys[];
+  __shared__ int s_hist[256];
+  __shared__ int s_scan[32];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_remaining;
+  const int unit = blockIdx.x;   // b * Hkv + g
+  const int b = unit / Hkv, g = unit % Hkv;
+  const int L = max(0, seq_lens[b]);
+  int n = (L + kPage - 1) / kPage;
+  if (n > maxP) {   // sequence longer than its page-table row
+    if (threadIdx.x == 0) report(LSERVE_ERR_DEVICE_BOUNDS);
+    n = maxP;
+  }
+  int32_t* row = sel + static_cast<long>(unit) * kcap;
+  const int tid = threadIdx.x;
+
+  if (head_kind[g] != LSERVE_HEAD_DENSE) {
+    // pages holding a token of [0, sink) or [L - local, L)
+    const int n_sink = (min(sink, L) + kPage - 1) / kPage;
+    const int w0 = local > 0 ? max(0, L - local) / kPage : n;   // first window page
+    const int w1 = local > 0 ? (L - 1) / kPage + 1 : n;         // one past the last
+    const int a = min(n_sink, n), bb = max(w0, a);
+    int cnt = L > 0 ? a + max(0, min(w1, n) - bb) : 0;
+    if (cnt > kcap) {
+      if (tid == 0) report(LSERVE_ERR_DEVICE_BOUNDS);
+      cnt = kcap;
+    }
+    for (int j = tid; j < kcap; j += blockDim.x) {
+      int v = -1;
+      if (j < a) v = j;
+      else if (j < cnt) v = bb + (j - a);
+      row[j] = v;
+    }
+    if (tid == 0 && sel_n) sel_n[unit] = cnt;
+    return;
+  }
+
+  const int k = min(budget_pages, n);
+  if (k >= n) {
+    for (int j = tid; j < kcap; j += blockDim.x) row[j] = j < n ? j : -1;
+    if (tid == 0 && sel_n) sel_n[unit] = n;
+    return;
+  }
+  const float* srow = scores + static_cast<long>(unit) * maxP;
+  const bool cached = n <= kTopkSmemKeys;
+  if (cached)
+    for (int j = tid; j < n; j += blockDim.x) s_keys[j] = order_key(srow[j]);
+  if (tid == 0) {
+    s_prefix = 0;
+    s_remaining = k;
+  }
+  __syncthreads();
+  auto key_at = [&](int j) -> uint32_t { return cached ? s_keys[j] : order_key(srow[j]); };
+
+  uint32_t prefix = 0, mask = 0;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int j = tid; j < 256; j += blockDim.x) s_hist[j] = 0;
+    __syncthreads();
+    for (int j = tid; j < n; j += blockDim.x) {
+      const uint32_t kk = key_at(j);
+      if ((kk & mask) == prefix) atomicAdd(&s_hist[(kk >> shift) & 255], 1);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane t owns digits 8t..8t+7; find the digit holding the remaining-th largest
+      int c[8], sum = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        c[e] = s_hist[tid * 8 + e];
+        sum += c[e];
+      }
+      // inclusive suffix sum over lanes (sum of lanes >= tid)
+      int suf = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_down_sync(0xffffffffu, suf, o);
+        if (tid + o < 32) suf += y;
+      }
+      const int above = suf - sum;   // keys with a higher digit
+      const int rem = s_remaining;
+      if (above < rem && rem <= suf) {   // exactly one lane
+        int acc = above, digit = tid * 8;
+        for (int e = 7; e >= 0; --e) {
+          if (acc + c[e] >= rem) {
+            digit = tid * 8 + e;
+            break;
+          }
+          acc += c[e];
+        }
+        s_prefix = prefix | (static_cast<uint32_t>(digit) << shift);
+        s_remaining = rem - acc;
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    mask |= 255u << shift;
+  }
+  const uint32_t T = prefix;        // key of the k-th largest score
+  const int take_eq = s_remaining;  // how many keys equal to T are taken (lowest indices)
+
+  // ascending emission: each thread owns a contiguous run of indices
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int j0 = min(n, tid * per), j1 = min(n, j0 + per);
+  int n_eq = 0;
+  for (int j = j0; j < j1; ++j) n_eq += key_at(j) == T;
+  int tot;
+  int eq_before = block_exclusive_scan(n_eq, s_scan, &tot);
+  int n_sel = 0;
+  {
+    int e = eq_before;
+    for (int j = j0; j < j1; ++j) {
+      const uint32_t kk = key_at(j);
+      if (kk > T) ++n_sel;
+      else if (kk == T) n_sel += (e++ < take_eq);
+    }
+  }
+  int sel_before = block_exclusive_scan(n_sel, s_scan, &tot);
+  {
+    int e = eq_before, pos = sel_before;
+    for (int j = j0; j < j1; ++j) {
+      const uint32_t kk = key_at(j);
+      bool take = kk > T;
+      if (kk == T) take = (e++ < take_eq);
+      if (take && pos < kcap) row[pos++] = j;
+    }
+  }
+  for (int j = k + tid; j < kcap; j += blockDim.x) row[j] = -1;
+  if (tid == 0 && sel_n) sel_n[unit] = k;
+}
+
+}  // namespace lserve

@@ -1,0 +1,154 @@
+// tile_lists.cuh -- device-built kept-tile lists for block-sparse prefill.
+//
+// LServe + SampleAttention blog post, "LServe - Prefill Phase", Fig. 1: every KV
+// block is fully computed or fully skipped at the kernel's tile granularity;
+// dense heads walk the causal tiles (optionally thinned by a block mask),
+// streaming heads only the tiles that meet the Lambda support.
+//
+// Row r = (b * Hkv + g) * nQT + qt owns the ascending list of kept KV tiles kt:
+//   dense      kt <= qt  and (no mask or block_mask[b, g, qt, kt] != 0)
+//   streaming  kt <= qt  and (64 kt < sink  or  max(64 qt - 64 kt - 63, 0) < local)
+// Built in three launches, all on device, no host round trip:
+//   tile_count_kernel  one warp per row: count kept tiles (4 mask bytes per lane
+//                      per step), histogram of row lengths
+//   tile_scan_kernel   one CTA: CSR offsets (exclusive scan of the counts) and the
+//                      start of every row-length bucket in longest-first order
+//   tile_fill_kernel   one warp per row: ballot-ordered compaction of kt into the
+//                      CSR, and the row's slot in the longest-first work order
+#pragma once
+
+#include "common.cuh"
+
+namespace lserve {
+
+struct TileListParams {
+  int B, Hkv, nQT, sink, local;
+  const uint8_t* head_kind;
+  const uint8_t* block_mask;   // [B, Hkv, nQT, nQT] or null
+};
+
+__device__ __forceinline__ bool tile_keep(const TileListParams& P, bool streaming, const uint8_t* mrow, int qt,
+                                          int kt) {
+  if (kt > qt) return false;
+  if (streaming) {
+    const int mind = max(kTile * (qt - kt) - (kTile - 1), 0);
+    return kTile * kt < P.sink || mind < P.local;
+  }
+  return mrow == nullptr || mrow[kt] != 0;
+}
+
+// Calls f(kt, keep) for kt = 0..qt in ascending order, 32 lanes x 4 tiles per step.
+template <typename F>
+__device__ __forceinline__ void tile_row_walk(const TileListParams& P, int r, F&& f) {
+  const int qt = r % P.nQT;
+  const int bg = r / P.nQT;
+  const int g = bg % P.Hkv;
+  const bool streaming = P.head_kind[g] != LSERVE_HEAD_DENSE;
+  const uint8_t* mrow = (!streaming && P.block_mask) ? P.block_mask + (static_cast<long>(bg) * P.nQT + qt) * P.nQT
+                                                     : nullptr;
+  const int lane = threadIdx.x & 31;
+  for (int base = 0; base <= qt; base += 128) {
+    const int kt0 = base + lane * 4;
+    bool k4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) k4[e] = tile_keep(P, streaming, mrow, qt, kt0 + e);
+    f(base, kt0, k4);
+  }
+}
+
+__global__ void __launch_bounds__(256) tile_count_kernel(TileListParams P, int* __restrict__ counts,
+                                                         int* __restrict__ hist) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int R = P.B * P.Hkv * P.nQT;
+  if (r >= R) return;
+  int cnt = 0;
+  tile_row_walk(P, r, [&](int, int, const bool (&k4)[4]) { cnt += k4[0] + k4[1] + k4[2] + k4[3]; });
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if ((threadIdx.x & 31) == 0) {
+    counts[r] = cnt;
+    atomicAdd(&hist[cnt], 1);
+  }
+}
+
+// One CTA of 1024 threads.  offsets[r] = sum_{r' < r} counts[r']; bucket[c] =
+// number of rows with more than c kept tiles (start of bucket c in the order).
+__global__ void __launch_bounds__(1024) tile_scan_kernel(const int* __restrict__ counts, int R,
+                                                         int* __restrict__ offsets, const int* __restrict__ hist,
+                                                         int nbucket, int* __restrict__ bucket,
+                                                         long long max_nnz, int* __restrict__ overflow) {
+  __shared__ int s_warp[32];
+  __shared__ long long s_carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
+  for (int base = 0; base < R; base += 1024) {
+    const int r = base + tid;
+    const int v = r < R ? counts[r] : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = s_warp[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      s_warp[lane] = w;
+    }
+    __syncthreads();
+    const long long carry = s_carry;
+    const long long excl = carry + (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
+    if (r < R) offsets[r] = static_cast<int>(excl);
+    __syncthreads();
+    if (tid == 1023) s_carry = carry + s_warp[31];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    offsets[R] = static_cast<int>(s_carry);
+    *overflow = s_carry > max_nnz;
+    if (s_carry > max_nnz) report(LSERVE_ERR_DEVICE_BOUNDS);
+    int above = 0;   // rows with more kept tiles than c
+    for (int c = nbucket - 1; c >= 0; --c) {
+      bucket[c] = above;
+      above += hist[c];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) tile_fill_kernel(TileListParams P, const int* __restrict__ offsets,
+                                                        const int* __restrict__ counts, uint16_t* __restrict__ cols,
+                                                        const int* __restrict__ bucket, int* __restrict__ fill,
+                                                        int* __restrict__ order, const int* __restrict__ overflow) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int R = P.B * P.Hkv * P.nQT;
+  if (r >= R || *overflow) return;
+  const int lane = threadIdx.x & 31;
+  int pos = offsets[r];
+  tile_row_walk(P, r, [&](int, int kt0, const bool (&k4)[4]) {
+    const int c = k4[0] + k4[1] + k4[2] + k4[3];
+    int x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    int w = pos + x - c;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (k4[e]) cols[w++] = static_cast<uint16_t>(kt0 + e);
+    pos += __shfl_sync(0xffffffffu, x, 31);
+  });
+  if (lane == 0 && order) {
+    const int cnt = counts[r];
+    order[bucket[cnt] + atomicAdd(&fill[cnt], 1)] = r;
+  }
+}
+
+}  // namespace lserve
