@@ -36,7 +36,8 @@
  *     64 tokens, logical page 16 tokens, prefill tile 64x64.  Anything else
  *     returns LSERVE_ERR_UNSUPPORTED.  There is no fallback path.
  *   - No exception crosses the ABI.  The library keeps no state between calls
- *     except the device status word and the thread-local error string.
+ *     except the device status word, the thread-local error string and the
+ *     fixed scratch array of lserve_decode_noalloc.
  */
 #ifndef LSERVE_H_
 #define LSERVE_H_
@@ -210,6 +211,37 @@ size_t lserve_decode_workspace_size(const lserve_decode_args* args);
 lserve_status lserve_decode(const lserve_decode_args* args, void* out, float* lse,
                             int32_t* sel_out, int32_t* sel_n, void* workspace,
                             size_t ws_bytes, void* stream);
+
+/*
+ * lserve_decode_noalloc -- lserve_decode for callers that cannot allocate.
+ *
+ * The paper has no counterpart to this entry point; it exists for deployment.
+ * Some callers must not allocate device memory at all once they are running:
+ * serving loops that fix their memory budget at start-up and keep the
+ * allocator (and its implicit synchronisation) off the per-token path, and
+ * plugin hosts that own every device allocation and hand a kernel library only
+ * its input and output buffers.  Such callers cannot provide the workspace
+ * lserve_decode needs.  This variant computes exactly what lserve_decode
+ * computes, with the same arguments except the workspace, and takes its
+ * scratch (page scores, selections, split partials) from a fixed array of
+ * LSERVE_NOALLOC_SCRATCH_BYTES that is part of the library image on every
+ * device that loads it, held until the process exits.  It calls no cudaMalloc,
+ * cudaFree or any other allocating routine.
+ *
+ *   - The first call on a device looks up that array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - A batch whose scratch need (lserve_decode_workspace_size) exceeds
+ *     LSERVE_NOALLOC_SCRATCH_BYTES is rejected with LSERVE_ERR_WORKSPACE and
+ *     nothing is launched.
+ *   - All calls on a device share the one array and it keeps whatever the last
+ *     call left in it (nothing in it needs to start at zero).  Calls whose
+ *     kernels overlap on the GPU -- on different streams, or from different
+ *     host threads -- race on it; serialise them on one stream.
+ */
+#define LSERVE_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB per device */
+lserve_status lserve_decode_noalloc(const lserve_decode_args* args, void* out, float* lse,
+                                    int32_t* sel_out, int32_t* sel_n, void* stream);
 
 /* ------------------------------------------------------------------ status */
 

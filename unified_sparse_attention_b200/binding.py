@@ -37,6 +37,7 @@ EXPORTED_SYMBOLS = (
     "lserve_decode_max_selected",
     "lserve_decode_workspace_size",
     "lserve_decode",
+    "lserve_decode_noalloc",
     "lserve_get_device_status",
     "lserve_last_error_string",
     "lserve_version",
@@ -90,6 +91,7 @@ def load_library():
         "lserve_decode_max_selected": (i32, [ctypes.POINTER(DecodeArgs)]),
         "lserve_decode_workspace_size": (sz, [ctypes.POINTER(DecodeArgs)]),
         "lserve_decode": (i32, [ctypes.POINTER(DecodeArgs), vp, vp, vp, vp, vp, sz, vp]),
+        "lserve_decode_noalloc": (i32, [ctypes.POINTER(DecodeArgs), vp, vp, vp, vp, vp]),
         "lserve_get_device_status": (i32, [vp]),
         "lserve_last_error_string": (ctypes.c_char_p, []),
         "lserve_version": (ctypes.c_char_p, []),
@@ -283,6 +285,35 @@ def lserve_decode(q, k_pages, v_pages, page_table, seq_lens, stats, head_kind, s
                              ws.numel(), _stream(stream)))
     if return_selection:
         return out, lse, sel_out, sel_n
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def lserve_decode_noalloc(q, k_pages, v_pages, page_table, seq_lens, stats, head_kind, sink: int, local: int,
+                          token_budget: int, out, scale: float = 0.0, lse=None, sel_out=None, sel_n=None,
+                          stream=None):
+    """lserve_decode without a workspace, for callers that may not allocate device memory.
+
+    The library takes its scratch from a fixed per-device array of
+    NOALLOC_SCRATCH_BYTES.  ``out`` (and any of lse / sel_out / sel_n) must be
+    provided by the caller; this wrapper allocates nothing.  Calls that overlap
+    on the GPU share that array and race; keep them on one stream.
+    """
+    lib = load_library()
+    a = _decode_args(q, k_pages, v_pages, page_table, seq_lens, stats, head_kind, sink, local, token_budget, scale)
+    B, Hq, d = q.shape
+    _dev(out, "out", torch.bfloat16, q.shape)
+    if lse is not None:
+        _dev(lse, "lse", torch.float32, (B, Hq))
+    kcap = int(lib.lserve_decode_max_selected(ctypes.byref(a)))
+    if sel_out is not None:
+        _dev(sel_out, "sel_out", torch.int32, (B, a.Hkv, kcap))
+    if sel_n is not None:
+        _dev(sel_n, "sel_n", torch.int32, (B, a.Hkv))
+    _check(lib.lserve_decode_noalloc(ctypes.byref(a), _ptr(out), _ptr(lse), _ptr(sel_out), _ptr(sel_n),
+                                     _stream(stream)))
     return out
 
 

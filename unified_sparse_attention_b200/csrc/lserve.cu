@@ -301,6 +301,38 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
 
 }  // namespace
 
+// ------------------------------------------------- decode without a workspace
+// Scratch for lserve_decode_noalloc: one fixed array per device, part of the
+// module image, so that callers who may not allocate device memory still get
+// the decode step.  Its size is LSERVE_NOALLOC_SCRATCH_BYTES; the array lives
+// (and holds its memory) for as long as the library stays loaded on a device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LSERVE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device.  Host code only
+// sees a host-side stand-in under that name, so the address must be asked for
+// once per device (with that device current) and cached.
+lserve_status noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return fail(LSERVE_ERR_CUDA, "decode_noalloc: no usable current device");
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(LSERVE_ERR_CUDA, "decode_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return LSERVE_OK;
+}
+
+}  // namespace
+
 // =================================================================== C ABI
 extern "C" {
 
@@ -404,6 +436,31 @@ lserve_status lserve_decode(const lserve_decode_args* args, void* out, float* ls
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < need)
     return fail(LSERVE_ERR_WORKSPACE, "decode: workspace missing, misaligned or smaller than %zu bytes", need);
   DecodePlan p = plan_decode(args, workspace);
+  int32_t* sel = sel_out ? sel_out : p.sel;
+  int32_t* seln = sel_n ? sel_n : p.sel_n;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = args->d == 128 ? launch_decode_d<128>(args, p, sel, seln, out, lse, st)
+                     : launch_decode_d<64>(args, p, sel, seln, out, lse, st);
+  return s == LSERVE_OK ? ok() : s;
+}
+
+lserve_status lserve_decode_noalloc(const lserve_decode_args* args, void* out, float* lse, int32_t* sel_out,
+                                    int32_t* sel_n, void* stream) {
+  lserve_status s = validate_decode(args);
+  if (s != LSERVE_OK) return s;
+  if (!out || !aligned16(out)) return fail(LSERVE_ERR_INVALID_ARG, "decode: out must be non-null and 16-byte aligned");
+  const size_t need = plan_decode(args, nullptr).bytes;
+  if (need > LSERVE_NOALLOC_SCRATCH_BYTES)
+    return fail(LSERVE_ERR_WORKSPACE,
+                "decode_noalloc: this batch needs %zu bytes of scratch but the built-in array holds %zu; "
+                "split the batch or call lserve_decode with a workspace",
+                need, static_cast<size_t>(LSERVE_NOALLOC_SCRATCH_BYTES));
+  void* scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != LSERVE_OK) return s;
+  // Every buffer carved here is fully written by the kernels before it is read,
+  // so the previous call's leftovers need no clearing.
+  DecodePlan p = plan_decode(args, scratch);
   int32_t* sel = sel_out ? sel_out : p.sel;
   int32_t* seln = sel_n ? sel_n : p.sel_n;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
