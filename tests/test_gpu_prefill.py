@@ -18,6 +18,16 @@ pytestmark = pytest.mark.gpu
 U = pytest.importorskip("unified_sparse_attention_b200")
 
 
+@pytest.fixture(params=["tc", "mma"], autouse=True)
+def impl(request, monkeypatch):
+    """Run every case on the tcgen05 kernel (default) and on the mma.sync kernel."""
+    if request.param == "mma":
+        monkeypatch.setenv("LSERVE_PREFILL_IMPL", "mma")
+    else:
+        monkeypatch.delenv("LSERVE_PREFILL_IMPL", raising=False)
+    return request.param
+
+
 def run_case(w, S, kind, sink, local, mask_fill=None, B=None, seed_mask=True):
     dev = "cuda"
     q, k, v = W.prefill_inputs(w, S=S, B=B)
@@ -119,3 +129,15 @@ def test_repeated_calls_are_deterministic():
     a = U.lserve_prefill(q, k, v, hk, 64, 256)
     b = U.lserve_prefill(q, k, v, hk, 64, 256)
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("G,S", [(1, 960), (2, 512), (8, 384)])
+def test_gqa_ratios_and_odd_tile_count(G, S):
+    """G = 1 pairs query tiles (odd tile count leaves a half pair); G = 8 splits heads."""
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2 * G, Hkv=2, d=128)
+    run_case(w, S, [0, 1], 64, 150, mask_fill=0.5)
+
+
+def test_d64_mha_pairs_with_mask():
+    w = dataclasses.replace(W.WORKLOADS["tiny"], B=2, Hq=2, Hkv=2, d=64)
+    run_case(w, 832, [0, 1], 32, 97, mask_fill=0.3, B=2)

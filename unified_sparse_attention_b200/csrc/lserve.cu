@@ -18,6 +18,7 @@
 #include "decode.cuh"
 #include "page_stats.cuh"
 #include "prefill_mma.cuh"
+#include "prefill_tc.cuh"
 #include "select.cuh"
 #include "tile_lists.cuh"
 
@@ -173,10 +174,11 @@ lserve_status validate_prefill(const lserve_shape* s, int sink, int local) {
 
 lserve_status launch_tile_lists(const lserve_shape* s, const uint8_t* head_kind, int sink, int local,
                                 const uint8_t* block_mask, const PrefillWs& w, int* offsets, uint16_t* cols,
-                                long long max_nnz, int* order, cudaStream_t st) {
+                                long long max_nnz, int* order, cudaStream_t st, int qg = 1) {
   const int nQT = s->S / kTile;
-  const int R = s->B * s->Hkv * nQT;
-  TileListParams P{s->B, s->Hkv, nQT, sink, local, head_kind, block_mask};
+  const int nRow = (nQT + qg - 1) / qg;
+  const int R = s->B * s->Hkv * nRow;
+  TileListParams P{s->B, s->Hkv, nQT, sink, local, head_kind, block_mask, qg, nRow};
   if (cudaMemsetAsync(w.hist, 0, sizeof(int) * 2 * (nQT + 1), st) != cudaSuccess)
     return fail(LSERVE_ERR_CUDA, "prefill: memset failed");
   const int blocks = (R + 7) / 8;
@@ -198,6 +200,39 @@ lserve_status launch_prefill_mma(const lserve_shape* s, const void* q, const voi
   prefill_mma_kernel<D><<<static_cast<unsigned>(grid), kPrefillThreads, PrefillCfg<D>::kSmemBytes, st>>>(tq, tk, tv,
                                                                                                       A);
   return check_launch("prefill attention");
+}
+
+// tcgen05 path: work-item shape from the GQA ratio (see prefill_tc.cuh).
+struct TcPlan {
+  int QG, HG, NM;
+};
+
+bool tc_plan(int G, TcPlan* p) {
+  if (G % 4 == 0) *p = {1, 4, 2};
+  else if (G == 2) *p = {1, 2, 1};
+  else if (G == 1) *p = {2, 1, 1};
+  else return false;
+  return true;
+}
+
+template <int D, int NM>
+lserve_status launch_prefill_tc(const lserve_shape* s, const void* q, const void* k, const void* v,
+                                const tc::TcArgs& T, int n_rows, cudaStream_t st) {
+  using C = tc::Cfg<D, NM>;
+  CUtensorMap tq, tk, tv;
+  const uint64_t Tn = static_cast<uint64_t>(s->B) * s->S;
+  if (!make_map_3d(&tq, q, D, s->Hq, Tn) || !make_map_3d(&tk, k, D, s->Hkv, Tn) ||
+      !make_map_3d(&tv, v, D, s->Hkv, Tn))
+    return fail(LSERVE_ERR_CUDA, "prefill: cuTensorMapEncodeTiled failed");
+  ensure_smem(tc::prefill_tc_kernel<D, NM>, C::kSmem);
+  const long long grid = static_cast<long long>(n_rows) * T.hsplit;
+  tc::prefill_tc_kernel<D, NM><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, st>>>(tq, tk, tv, T);
+  return check_launch("prefill attention (tcgen05)");
+}
+
+bool use_legacy_prefill() {
+  const char* e = getenv("LSERVE_PREFILL_IMPL");
+  return e && strcmp(e, "mma") == 0;
 }
 
 // ----------------------------------------------------------------- decode
@@ -379,12 +414,30 @@ lserve_status lserve_prefill(const lserve_shape* shape, const void* q, const voi
                 lserve_prefill_workspace_size(shape));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   PrefillWs w = carve_prefill(shape, workspace, nullptr);
+  const int G = shape->Hq / shape->Hkv;
+  const int nQT = shape->S / kTile;
+  const float scale = shape->scale > 0.f ? shape->scale : 1.f / std::sqrt(static_cast<float>(shape->d));
+  PrefillArgs A{w.offsets, w.cols, w.order, head_kind, static_cast<bf16*>(out), lse, G,
+                shape->Hkv, nQT, shape->S, sink, local, scale * 1.4426950408889634f, wait_timeout_ns()};
+  TcPlan tp;
+  if (!use_legacy_prefill() && tc_plan(G, &tp)) {
+    s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz, w.order, st,
+                          tp.QG);
+    if (s != LSERVE_OK) return s;
+    const int nRow = (nQT + tp.QG - 1) / tp.QG;
+    tc::TcArgs T{A, block_mask, tp.QG, tp.HG, nRow, G / tp.HG};
+    const int n_rows = shape->B * shape->Hkv * nRow;
+    if (shape->d == 128)
+      s = tp.NM == 2 ? launch_prefill_tc<128, 2>(shape, q, k, v, T, n_rows, st)
+                     : launch_prefill_tc<128, 1>(shape, q, k, v, T, n_rows, st);
+    else
+      s = tp.NM == 2 ? launch_prefill_tc<64, 2>(shape, q, k, v, T, n_rows, st)
+                     : launch_prefill_tc<64, 1>(shape, q, k, v, T, n_rows, st);
+    return s == LSERVE_OK ? ok() : s;
+  }
   s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz, w.order, st);
   if (s != LSERVE_OK) return s;
-  const float scale = shape->scale > 0.f ? shape->scale : 1.f / std::sqrt(static_cast<float>(shape->d));
-  PrefillArgs A{w.offsets, w.cols, w.order, head_kind, static_cast<bf16*>(out), lse, shape->Hq / shape->Hkv,
-                shape->Hkv, shape->S / kTile, shape->S, sink, local, scale * 1.4426950408889634f, wait_timeout_ns()};
-  const int n_rows = shape->B * shape->Hkv * (shape->S / kTile);
+  const int n_rows = shape->B * shape->Hkv * nQT;
   s = shape->d == 128 ? launch_prefill_mma<128>(shape, q, k, v, A, n_rows, st)
                       : launch_prefill_mma<64>(shape, q, k, v, A, n_rows, st);
   return s == LSERVE_OK ? ok() : s;

@@ -25,6 +25,8 @@ struct TileListParams {
   int B, Hkv, nQT, sink, local;
   const uint8_t* head_kind;
   const uint8_t* block_mask;   // [B, Hkv, nQT, nQT] or null
+  int qg = 1;                  // query tiles per row (a row keeps the union of their lists)
+  int nRow = 0;                // rows per (b, kvh) = ceil(nQT / qg)
 };
 
 __device__ __forceinline__ bool tile_keep(const TileListParams& P, bool streaming, const uint8_t* mrow, int qt,
@@ -37,21 +39,30 @@ __device__ __forceinline__ bool tile_keep(const TileListParams& P, bool streamin
   return mrow == nullptr || mrow[kt] != 0;
 }
 
-// Calls f(kt, keep) for kt = 0..qt in ascending order, 32 lanes x 4 tiles per step.
+// Calls f(base, kt0, keep[4]) for kt = 0..(last query tile of the row) in
+// ascending order, 32 lanes x 4 tiles per step.  A row of qg query tiles keeps
+// the union of their tiles.
 template <typename F>
 __device__ __forceinline__ void tile_row_walk(const TileListParams& P, int r, F&& f) {
-  const int qt = r % P.nQT;
-  const int bg = r / P.nQT;
+  const int qgi = r % P.nRow;
+  const int bg = r / P.nRow;
   const int g = bg % P.Hkv;
+  const int qt_lo = qgi * P.qg;
+  const int qt_hi = min(P.nQT - 1, qt_lo + P.qg - 1);
   const bool streaming = P.head_kind[g] != LSERVE_HEAD_DENSE;
-  const uint8_t* mrow = (!streaming && P.block_mask) ? P.block_mask + (static_cast<long>(bg) * P.nQT + qt) * P.nQT
-                                                     : nullptr;
+  const uint8_t* mbase = (!streaming && P.block_mask) ? P.block_mask + static_cast<long>(bg) * P.nQT * P.nQT
+                                                      : nullptr;
   const int lane = threadIdx.x & 31;
-  for (int base = 0; base <= qt; base += 128) {
+  for (int base = 0; base <= qt_hi; base += 128) {
     const int kt0 = base + lane * 4;
     bool k4[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) k4[e] = tile_keep(P, streaming, mrow, qt, kt0 + e);
+    for (int e = 0; e < 4; ++e) {
+      bool keep = false;
+      for (int qt = qt_lo; qt <= qt_hi; ++qt)
+        keep |= tile_keep(P, streaming, mbase ? mbase + static_cast<long>(qt) * P.nQT : nullptr, qt, kt0 + e);
+      k4[e] = keep;
+    }
     f(base, kt0, k4);
   }
 }
@@ -59,7 +70,7 @@ __device__ __forceinline__ void tile_row_walk(const TileListParams& P, int r, F&
 __global__ void __launch_bounds__(256) tile_count_kernel(TileListParams P, int* __restrict__ counts,
                                                          int* __restrict__ hist) {
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int R = P.B * P.Hkv * P.nQT;
+  const int R = P.B * P.Hkv * P.nRow;
   if (r >= R) return;
   int cnt = 0;
   tile_row_walk(P, r, [&](int, int, const bool (&k4)[4]) { cnt += k4[0] + k4[1] + k4[2] + k4[3]; });
@@ -127,7 +138,7 @@ __global__ void __launch_bounds__(256) tile_fill_kernel(TileListParams P, const 
                                                         const int* __restrict__ bucket, int* __restrict__ fill,
                                                         int* __restrict__ order, const int* __restrict__ overflow) {
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int R = P.B * P.Hkv * P.nQT;
+  const int R = P.B * P.Hkv * P.nRow;
   if (r >= R || *overflow) return;
   const int lane = threadIdx.x & 31;
   int pos = offsets[r];
