@@ -63,11 +63,11 @@ def kept_tile_counts(w, bm, kind):
         if kind[g]:
             mind = torch.clamp(64 * qt - 64 * kt - 63, min=0)
             keep = causal & ((64 * kt < w.sink) | (mind < w.local))
+            counts.append(int(keep.sum()) * w.B)
         elif bm is not None:
-            keep = causal & (bm[0, g] != 0)
+            counts.append(sum(int((causal & (bm[b, g] != 0)).sum()) for b in range(w.B)))
         else:
-            keep = causal
-        counts.append(int(keep.sum()))
+            counts.append(int(causal.sum()) * w.B)
     return counts
 
 
@@ -87,10 +87,11 @@ def decode_bytes(w, kind, k_pages_per_seq, d):
 
 
 class Setup:
-    def __init__(self, device):
+    def __init__(self, device, prefill_wl=PREFILL_WL, decode_wl=DECODE_WL):
         self.dev = device
-        self.wp = W.WORKLOADS[PREFILL_WL]
-        self.wd = W.WORKLOADS[DECODE_WL]
+        self.prefill_wl, self.decode_wl = prefill_wl, decode_wl
+        self.wp = W.WORKLOADS[prefill_wl]
+        self.wd = W.WORKLOADS[decode_wl]
         wp, wd = self.wp, self.wd
         self.kind_p = W.head_kind(wp)
         self.kind_d = W.head_kind(wd)
@@ -226,7 +227,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    setup = Setup(dev)
+    setup = Setup(dev, args.prefill_wl, args.decode_wl)
     per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup):
         oracle_prefill_sample(setup, seconds=per_step / 4, seed=100 + i)
@@ -242,7 +243,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(1, args.steps) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": PREFILL_WL, "seq_len": setup.wp.S, "kind": "oracle on sampled rows"},
+        "config": {"workload": setup.wp.name, "seq_len": setup.wp.S, "kind": "oracle on sampled rows"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"{rows} query rows x {setup.wp.Hq} heads of the 128K prefill, "
                                    f"{secs:.1f} s of fp64 NumPy"},
@@ -259,6 +260,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--prefill-wl", default=PREFILL_WL, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--decode-wl", default=DECODE_WL, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--no-legacy", action="store_true", help="skip timing the mma.sync prefill kernel")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -284,7 +288,7 @@ def main():
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    setup = Setup(dev)
+    setup = Setup(dev, args.prefill_wl, args.decode_wl)
     wp, wd = setup.wp, setup.wd
     pk = peaks()
 
@@ -323,6 +327,11 @@ def main():
     t_tiles = time_loop(tile_lists, max(3, args.steps // 2), 2, stream, scratch)
     t_prefill = time_loop(prefill, args.steps, args.warmup, stream, scratch)
     t_decode = time_loop(decode_only, args.steps, args.warmup, stream, scratch)
+    ms_legacy = None
+    if not args.no_legacy:   # the mma.sync kernel on the same call, for comparison only
+        os.environ["LSERVE_PREFILL_IMPL"] = "mma"
+        ms_legacy = float(np.median(time_loop(prefill, max(2, args.steps // 2), 2, stream, scratch)))
+        del os.environ["LSERVE_PREFILL_IMPL"]
 
     # the timed steps
     clocks = Clocks(local_rank)
@@ -398,16 +407,20 @@ def main():
                "sample": f"{rows} query rows x {wp.Hq} heads of the 128K prefill ({secs:.1f} s fp64 NumPy), "
                          f"rate scaled by each row's kept-tile FLOPs"}
 
+    n_dense = sum(1 for g in range(wp.Hkv) if setup.kind_p[g] == 0)
+    dense_density = (sum(setup.tiles[g] for g in range(wp.Hkv) if setup.kind_p[g] == 0)
+                     / max(1, n_dense * n * (n + 1) / 2))
     launches_per_step = 4 + 1 + 4   # tile count/scan/fill + attention; stats refresh; score/top-k/decode/merge
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{PREFILL_WL} prefill (B1 S131072 Hq32 Hkv8 d128, vertical-slash mask "
-                               f"{sum(setup.tiles[g] for g in range(wp.Hkv) if setup.kind_p[g] == 0) / (4 * n * (n + 1) / 2):.3f}"
-                               f" density) + {DECODE_WL} decode (B4 ctx262144 Hq32 Hkv32 d128, budget 8192)",
+        "config": {"workload": f"{wp.name} prefill (B{wp.B} S{wp.S} Hq{wp.Hq} Hkv{wp.Hkv} d{wp.d}, dense-head tile "
+                               f"density {dense_density:.3f}) + {wd.name} decode (B{wd.dec_B} ctx{wd.ctx} Hq{wd.Hq} "
+                               f"Hkv{wd.Hkv} d{wd.d}, budget {wd.token_budget})",
                    "l2": "flushed between steps (write of 252 MB)", "parallelism": f"replicas x{world}"},
         "prefill_ms": ms_prefill, "prefill_attention_ms": ms_attn, "tile_lists_ms": ms_tiles,
+        "prefill_mma_sync_ms": ms_legacy,
         "prefill_tflops": tflops_prefill, "kept_tile_tflop": setup.prefill_flops / 1e12,
         "decode_us_per_step": us_decode, "decode_GBps": gbps_decode, "decode_bytes": setup.dbytes,
         "roofline": {"bound": "tensor", "kernel": "prefill attention", "achieved": tflops_attn,
