@@ -137,6 +137,17 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   }
 }
 
+// 64-bit key masks over one tile (bit c <-> key offset c).
+__device__ __forceinline__ uint64_t bits_upto(int d) {   // offsets 0..d
+  return d < 0 ? 0ull : (d >= 63 ? ~0ull : (2ull << d) - 1ull);
+}
+__device__ __forceinline__ uint64_t bits_below(int h) {  // offsets 0..h-1
+  return h <= 0 ? 0ull : (h >= 64 ? ~0ull : (1ull << h) - 1ull);
+}
+__device__ __forceinline__ uint64_t bits_from(int l) {   // offsets l..63
+  return l <= 0 ? ~0ull : (l >= 64 ? 0ull : ~((1ull << l) - 1ull));
+}
+
 constexpr int kStages = 3;
 
 template <int D, int NM>
@@ -322,24 +333,37 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
       const uint32_t t_s = t_s0 + 64 * (2 * m + buf) + lane_off;
       wait_or_abort(&s_full[m][buf], (j >> 1) & 1, &s_abort, tmo);
       fence_after_sync();
-      uint32_t sr[64];
-      tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_wait_ld();
+      uint32_t x[64];
+      tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
       const int kt = cols[j];
-      const bool keep_tile = rb_valid && tile_keep(tp, streaming, mrow, qt, kt);
-      const bool full = keep_tile && tile_is_full(streaming, qt, kt, A.sink, A.local);
-      float s[64];
-      float mloc = kNegInf;
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const int key = kt * kTile + c;
-        bool keep = full;
-        if (!full)
-          keep = keep_tile && key <= i && (!streaming || key < A.sink || i - key < A.local);
-        s[c] = keep ? __uint_as_float(sr[c]) * sc : kNegInf;
-        mloc = fmaxf(mloc, s[c]);
+      // keep mask of this row over the tile's 64 keys (bit c <-> key 64 kt + c)
+      uint64_t keep = ~0ull;
+      const bool keep_tile = rb_valid && (T.QG == 1 || tile_keep(tp, streaming, mrow, qt, kt));
+      if (!keep_tile) {
+        keep = 0ull;
+      } else if (!tile_is_full(streaming, qt, kt, A.sink, A.local)) {
+        const int d0 = i - kt * kTile;   // offset of the query position inside the tile
+        keep = bits_upto(d0);
+        if (streaming) keep &= bits_below(A.sink - kt * kTile) | bits_from(d0 - A.local + 1);
       }
+      tmem_wait_ld();
+      float mx[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx[e] = kNegInf;
+      if (__all_sync(0xffffffffu, keep == ~0ull)) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(x[c]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float v = ((keep >> c) & 1ull) ? __uint_as_float(x[c]) : kNegInf;
+          x[c] = __float_as_uint(v);
+          mx[c & 7] = fmaxf(mx[c & 7], v);
+        }
+      }
+      const float mloc = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sc;
       // lazy rescale: move the reference max only when it grows by more than 8 (x256)
       const bool need = mloc > m_run + 8.f;
       const bool rescale = need && m_run != kNegInf;
@@ -347,14 +371,15 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
       if (need) m_run = mloc;
       const float m_use = m_run == kNegInf ? 0.f : m_run;
       uint32_t pk[32];
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float p0 = fast_exp2(s[2 * c] - m_use), p1 = fast_exp2(s[2 * c + 1] - m_use);
-        psum += p0 + p1;
+        const float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * c]), sc, -m_use));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * c + 1]), sc, -m_use));
+        ps[c & 3] += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
       }
-      l_run = l_run * f + psum;
+      l_run = l_run * f + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       tmem_st32(t_s, pk);   // P overwrites the first 32 columns of this S buffer
       // Observe the completion of PV of tile j-1 (every thread, every tile, in
       // order, so that the parity waits on o_done never fall two phases behind);
