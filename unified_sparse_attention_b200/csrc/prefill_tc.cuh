@@ -14,9 +14,10 @@
 // of their tile lists.
 //
 // Warp roles (64 + 128 NM threads):
-//   warp 0     TMA producer: Q once, then K and V of every listed tile into a
-//              3-stage shared-memory ring (128-byte swizzle), one mbarrier each.
-//   warp 1     allocates TMEM; lane 0 issues tcgen05.mma:
+//   warp 0     TMA producer (one elected lane issues): Q once, then K and V of every listed tile into a
+//              pair of 4-stage shared-memory rings (128-byte swizzle); K stages
+//              are released after the S MMAs, V stages after the PV MMAs.
+//   warp 1     allocates TMEM; runs the MMA loop converged, one elected lane issues tcgen05.mma:
 //                S[m] = Q[m] K^T      (M=128, N=64, K=d; A and B from smem)
 //                O[m] += P[m] V       (M=128, N=d, K=64; P from TMEM, V from smem)
 //              and signals completion with tcgen05.commit -> mbarrier.
@@ -53,16 +54,21 @@ __device__ __forceinline__ void fence_before_sync() {
 __device__ __forceinline__ void fence_after_sync() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
+__device__ __forceinline__ void commit(uint64_t* bar) {   // call from a converged warp
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(
+          smem_u32(bar))
+      : "memory");
 }
+// The issuing warp runs converged with warp-uniform operands; one lane chosen
+// by elect.sync issues the instruction.
 // D[tmem] (+)= A[smem] * B[smem]
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
   asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -70,10 +76,15 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
   asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.b32 %0, 1, 0, e;\n}\n" : "=r"(e));
+  return e != 0;
 }
 // 32 consecutive 32-bit TMEM columns of this thread's lane
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -148,14 +159,15 @@ __device__ __forceinline__ uint64_t bits_from(int l) {   // offsets l..63
   return l <= 0 ? ~0ull : (l >= 64 ? 0ull : ~((1ull << l) - 1ull));
 }
 
-constexpr int kStages = 3;
+constexpr int kKStages = 4;   // K ring: a stage is freed once the S MMAs that read it complete
+constexpr int kVStages = 4;   // V ring: a stage is freed once the PV MMAs that read it complete
 
 template <int D, int NM>
 struct Cfg {
   static constexpr int kBoxes = D / 64;
   static constexpr int kQTile = kBoxes * 16384;      // one M-tile of Q: [boxes][128 rows][128 B]
   static constexpr int kKVTile = kBoxes * 8192;      // one K (or V) tile: [boxes][64 rows][128 B]
-  static constexpr int kSmem = NM * kQTile + 2 * kStages * kKVTile + 1024;
+  static constexpr int kSmem = NM * kQTile + (kKStages + kVStages) * kKVTile + 1024;
   static constexpr int kThreads = 64 + 128 * NM;
   static constexpr int kTmemCols = (NM * D + NM * 128) <= 256 ? 256 : 512;
 };
@@ -177,14 +189,14 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
   const PrefillArgs& A = T.p;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full;
-  __shared__ __align__(8) uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+  __shared__ __align__(8) uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   __shared__ __align__(8) uint64_t s_full[NM][2], p_full[NM][2], o_done[NM];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_s = smem;
   uint8_t* k_s = q_s + NM * C::kQTile;
-  uint8_t* v_s = k_s + kStages * C::kKVTile;
+  uint8_t* v_s = k_s + kKStages * C::kKVTile;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // ---- work item
@@ -206,10 +218,13 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int m = 0; m < NM; ++m) {
       mbar_init(&s_full[m][0], 1);
@@ -235,34 +250,55 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
 
   if (warp == 0) {
     // ================================================================ producer
-    if (lane == 0 && n > 0) {
-      prefetch_tensormap(&tmQ);
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
+    // The whole warp walks the list (warp-uniform coordinates); one elected lane issues.
+    const bool leader = elect_one();
+    if (n > 0) {
+      if (leader) {
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+      }
       int valid_rb = 0;
       for (int rb = 0; rb < 2 * NM; ++rb) valid_rb += rb_qt(rb) < A.nQT;
-      mbar_arrive_expect_tx(&q_full, valid_rb * C::kBoxes * 8192);
-      for (int rb = 0; rb < 2 * NM; ++rb) {
-        if (rb_qt(rb) >= A.nQT) continue;
-        uint8_t* dst = q_s + (rb >> 1) * C::kQTile + (rb & 1) * 8192;
-        for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_3d(dst + x * 16384, &tmQ, &q_full, x * 64, rb_head(rb), tok0 + rb_qt(rb) * kTile);
+      if (leader) {
+        mbar_arrive_expect_tx(&q_full, valid_rb * C::kBoxes * 8192);
+        for (int rb = 0; rb < 2 * NM; ++rb) {
+          if (rb_qt(rb) >= A.nQT) continue;
+          uint8_t* dst = q_s + (rb >> 1) * C::kQTile + (rb & 1) * 8192;
+          for (int x = 0; x < C::kBoxes; ++x)
+            tma_load_3d(dst + x * 16384, &tmQ, &q_full, x * 64, rb_head(rb), tok0 + rb_qt(rb) * kTile);
+        }
       }
-      for (int j = 0; j < n; ++j) {
-        const int st = j % kStages;
-        if (j >= kStages && !wait_or_abort(&kv_empty[st], ((j / kStages) - 1) & 1, &s_abort, tmo)) break;
-        const int kt = cols[j];
-        mbar_arrive_expect_tx(&k_full[st], C::kKVTile);
-        for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_3d(k_s + st * C::kKVTile + x * 8192, &tmK, &k_full[st], x * 64, g, tok0 + kt * kTile);
-        mbar_arrive_expect_tx(&v_full[st], C::kKVTile);
-        for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_3d(v_s + st * C::kKVTile + x * 8192, &tmV, &v_full[st], x * 64, g, tok0 + kt * kTile);
+      // K of tile t+1 goes out before V of tile t: S MMAs run one tile ahead of PV MMAs
+      for (int t = 0; t <= n; ++t) {
+        if (t < n) {
+          const int st = t % kKStages;
+          if (t >= kKStages && !wait_or_abort(&k_empty[st], ((t / kKStages) - 1) & 1, &s_abort, tmo)) break;
+          const int kt = cols[t];
+          if (leader) {
+            mbar_arrive_expect_tx(&k_full[st], C::kKVTile);
+            for (int x = 0; x < C::kBoxes; ++x)
+              tma_load_3d(k_s + st * C::kKVTile + x * 8192, &tmK, &k_full[st], x * 64, g, tok0 + kt * kTile);
+          }
+        }
+        if (t >= 1) {
+          const int u = t - 1;
+          const int st = u % kVStages;
+          if (u >= kVStages && !wait_or_abort(&v_empty[st], ((u / kVStages) - 1) & 1, &s_abort, tmo)) break;
+          const int kt = cols[u];
+          if (leader) {
+            mbar_arrive_expect_tx(&v_full[st], C::kKVTile);
+            for (int x = 0; x < C::kBoxes; ++x)
+              tma_load_3d(v_s + st * C::kKVTile + x * 8192, &tmV, &v_full[st], x * 64, g, tok0 + kt * kTile);
+          }
+        }
       }
     }
   } else if (warp == 1) {
     // ================================================================== MMA
-    if (lane == 0 && n > 0) {
+    // The whole warp runs the loop (waits and descriptors warp-uniform); MMAs and
+    // commits are issued by one elected lane.
+    if (n > 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, 64, false);
       constexpr uint32_t kIdPV = idesc_bf16(128, D, true);
       int o_seen[NM];
@@ -275,8 +311,8 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
       };
       const uint32_t qa = smem_u32(q_s), ka = smem_u32(k_s), va = smem_u32(v_s);
       auto issue_s = [&](int j) {
-        const int st = j % kStages;
-        wait_or_abort(&k_full[st], (j / kStages) & 1, &s_abort, tmo);
+        const int st = j % kKStages;
+        wait_or_abort(&k_full[st], (j / kKStages) & 1, &s_abort, tmo);
         for (int m = 0; m < NM; ++m) {
           const int buf = j & 1;
           if (j >= 2) wait_pv(m, j - 2);   // S[m][buf] still holds P of tile j-2 until its PV is done
@@ -289,13 +325,14 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
           }
           commit(&s_full[m][buf]);
         }
+        if (j + kKStages < n) commit(&k_empty[st]);
       };
       wait_or_abort(&q_full, 0, &s_abort, tmo);
       issue_s(0);
       for (int j = 0; j < n; ++j) {
         if (j + 1 < n) issue_s(j + 1);
-        const int st = j % kStages;
-        wait_or_abort(&v_full[st], (j / kStages) & 1, &s_abort, tmo);
+        const int st = j % kVStages;
+        wait_or_abort(&v_full[st], (j / kVStages) & 1, &s_abort, tmo);
         for (int m = 0; m < NM; ++m) {
           const int buf = j & 1;
           wait_or_abort(&p_full[m][buf], (j >> 1) & 1, &s_abort, tmo);
@@ -307,7 +344,7 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
           }
           commit(&o_done[m]);
         }
-        if (j + kStages < n) commit(&kv_empty[st]);
+        if (j + kVStages < n) commit(&v_empty[st]);
       }
     }
   } else {
