@@ -129,9 +129,9 @@ struct PrefillWs {
   int* counts;
   int* offsets;
   int* order;
-  int* hist;     // [nQT + 1]
-  int* fill;     // [nQT + 1]  (contiguous with hist: one memset clears both)
-  int* bucket;   // [nQT + 1]
+  int* hist;     // [B*Hkv][nQT + 1]
+  int* fill;     // [B*Hkv][nQT + 1]  (contiguous with hist: one memset clears both)
+  int* bucket;   // [B*Hkv][nQT + 1]
   int* overflow;
   uint16_t* cols;
   long long max_nnz;
@@ -149,9 +149,10 @@ PrefillWs carve_prefill(const lserve_shape* s, void* ws, size_t* bytes) {
   w.counts = c.take<int>(R);
   w.offsets = c.take<int>(R + 1);
   w.order = c.take<int>(R);
-  w.hist = c.take<int>(2 * (nQT + 1));
-  w.fill = w.hist + (nQT + 1);
-  w.bucket = c.take<int>(nQT + 1);
+  const long long groups = static_cast<long long>(s->B) * s->Hkv;
+  w.hist = c.take<int>(2 * groups * (nQT + 1));
+  w.fill = w.hist + groups * (nQT + 1);
+  w.bucket = c.take<int>(groups * (nQT + 1));
   w.overflow = c.take<int>(1);
   w.max_nnz = R * (nQT + 1) / 2;
   w.cols = c.take<uint16_t>(w.max_nnz);
@@ -179,11 +180,13 @@ lserve_status launch_tile_lists(const lserve_shape* s, const uint8_t* head_kind,
   const int nRow = (nQT + qg - 1) / qg;
   const int R = s->B * s->Hkv * nRow;
   TileListParams P{s->B, s->Hkv, nQT, sink, local, head_kind, block_mask, qg, nRow};
-  if (cudaMemsetAsync(w.hist, 0, sizeof(int) * 2 * (nQT + 1), st) != cudaSuccess)
+  const size_t hist_ints = 2ull * s->B * s->Hkv * (nQT + 1);
+  if (cudaMemsetAsync(w.hist, 0, sizeof(int) * hist_ints, st) != cudaSuccess)
     return fail(LSERVE_ERR_CUDA, "prefill: memset failed");
   const int blocks = (R + 7) / 8;
   tile_count_kernel<<<blocks, 256, 0, st>>>(P, w.counts, w.hist);
-  tile_scan_kernel<<<1, 1024, 0, st>>>(w.counts, R, offsets, w.hist, nQT + 1, w.bucket, max_nnz, w.overflow);
+  tile_scan_kernel<<<1, 1024, 0, st>>>(w.counts, R, offsets, w.hist, nQT + 1, w.bucket, nRow, max_nnz,
+                                       w.overflow);
   tile_fill_kernel<<<blocks, 256, 0, st>>>(P, offsets, w.counts, cols, w.bucket, w.fill, order, w.overflow);
   return check_launch("tile lists");
 }
@@ -208,25 +211,24 @@ struct TcPlan {
 };
 
 bool tc_plan(int G, TcPlan* p) {
-  if (G % 4 == 0) *p = {1, 4, 2};
-  else if (G == 2) *p = {1, 2, 1};
+  if (G % 2 == 0) *p = {1, 2, 1};
   else if (G == 1) *p = {2, 1, 1};
   else return false;
   return true;
 }
 
-template <int D, int NM>
+template <int D>
 lserve_status launch_prefill_tc(const lserve_shape* s, const void* q, const void* k, const void* v,
                                 const tc::TcArgs& T, int n_rows, cudaStream_t st) {
-  using C = tc::Cfg<D, NM>;
+  using C = tc::Cfg<D>;
   CUtensorMap tq, tk, tv;
   const uint64_t Tn = static_cast<uint64_t>(s->B) * s->S;
   if (!make_map_3d(&tq, q, D, s->Hq, Tn) || !make_map_3d(&tk, k, D, s->Hkv, Tn) ||
       !make_map_3d(&tv, v, D, s->Hkv, Tn))
     return fail(LSERVE_ERR_CUDA, "prefill: cuTensorMapEncodeTiled failed");
-  ensure_smem(tc::prefill_tc_kernel<D, NM>, C::kSmem);
+  ensure_smem(tc::prefill_tc_kernel<D>, C::kSmem);
   const long long grid = static_cast<long long>(n_rows) * T.hsplit;
-  tc::prefill_tc_kernel<D, NM><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, st>>>(tq, tk, tv, T);
+  tc::prefill_tc_kernel<D><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, st>>>(tq, tk, tv, T);
   return check_launch("prefill attention (tcgen05)");
 }
 
@@ -427,12 +429,8 @@ lserve_status lserve_prefill(const lserve_shape* shape, const void* q, const voi
     const int nRow = (nQT + tp.QG - 1) / tp.QG;
     tc::TcArgs T{A, block_mask, tp.QG, tp.HG, nRow, G / tp.HG};
     const int n_rows = shape->B * shape->Hkv * nRow;
-    if (shape->d == 128)
-      s = tp.NM == 2 ? launch_prefill_tc<128, 2>(shape, q, k, v, T, n_rows, st)
-                     : launch_prefill_tc<128, 1>(shape, q, k, v, T, n_rows, st);
-    else
-      s = tp.NM == 2 ? launch_prefill_tc<64, 2>(shape, q, k, v, T, n_rows, st)
-                     : launch_prefill_tc<64, 1>(shape, q, k, v, T, n_rows, st);
+    s = shape->d == 128 ? launch_prefill_tc<128>(shape, q, k, v, T, n_rows, st)
+                        : launch_prefill_tc<64>(shape, q, k, v, T, n_rows, st);
     return s == LSERVE_OK ? ok() : s;
   }
   s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz, w.order, st);

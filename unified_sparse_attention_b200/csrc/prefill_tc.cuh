@@ -6,27 +6,34 @@
 // the Lambda support of sink + local window); elements of kept boundary tiles
 // are masked exactly.
 //
-// One CTA per work item: NM M-tiles of 128 query rows that share one KV tile
-// list.  Each M-tile holds two 64-row blocks: with grouped-query attention the
-// blocks are different query heads of the same KV head and query tile (G = 4:
-// four heads, two M-tiles, every K/V tile feeds both); with G = 2 one M-tile of
-// two heads; with G = 1 one M-tile of two adjacent query tiles walking the union
-// of their tile lists.
+// One CTA per work item: one M-tile of 128 query rows = two 64-row blocks that
+// share one KV tile list.  With grouped-query attention the blocks are two
+// query heads of the same KV head and query tile (G = 4: two CTAs per tile
+// row); with G = 1 they are two adjacent query tiles of one head walking the
+// union of their tile lists.
 //
-// Warp roles (64 + 128 NM threads):
-//   warp 0     TMA producer (one elected lane issues): Q once, then K and V of every listed tile into a
-//              pair of 4-stage shared-memory rings (128-byte swizzle); K stages
-//              are released after the S MMAs, V stages after the PV MMAs.
-//   warp 1     allocates TMEM; runs the MMA loop converged, one elected lane issues tcgen05.mma:
-//                S[m] = Q[m] K^T      (M=128, N=64, K=d; A and B from smem)
-//                O[m] += P[m] V       (M=128, N=d, K=64; P from TMEM, V from smem)
-//              and signals completion with tcgen05.commit -> mbarrier.
-//   warps 2..  one warpgroup per M-tile: thread = query row.  tcgen05.ld of
-//              its S row, exact element mask, base-2 online softmax with lazy
-//              rescaling (O in TMEM is rescaled only when the running max grows
-//              by more than 2^8), P packed to bf16 and written back over S with
-//              tcgen05.st, then the epilogue normalises O and stores bf16 rows.
-// TMEM columns: O[m] at m*d, S[m][buf] at NM*d + 64*(2m + buf) (double-buffered).
+// Warp roles (320 threads, one CTA per SM):
+//   warp 0     TMA producer (one elected lane issues): Q once, then K and V of
+//              every listed tile pair into shared-memory rings (128-byte
+//              swizzle); K stages are released after the S MMAs, V stages after
+//              the PV MMAs.
+//   warp 1     allocates TMEM; runs the MMA loop converged, one elected lane
+//              issues tcgen05.mma and tcgen05.commit:
+//                S[x]  = Q [K_a;K_b]^T      (M=128, N=128, K=d; A and B from smem)
+//                O[x] += P[x] [V_a;V_b]     (M=128, N=d, K=128; P from TMEM)
+//              for step p on stream x = p & 1, in the order S(0) S(1) PV(0) S(2)
+//              PV(1) S(3) ...
+//   warps 2-9  two softmax warpgroups, one per stream (thread = query row): the
+//              steps of a row are split between two independent online
+//              softmaxes (own running max, sum and accumulator), which run out of
+//              phase and keep both the exponential unit and the tensor core busy;
+//              tcgen05.ld of S, exact element mask, base-2 exponentials with lazy
+//              rescaling (O[x] is rescaled only when its running max grows by more
+//              than 2^8), P packed to bf16 over S with tcgen05.st.  The epilogue
+//              merges the two streams by log-sum-exp; each warpgroup normalises and
+//              stores half of the output columns.
+// TMEM (512 columns): O[0] at 0, O[1] at 128, S[0] at 256, S[1] at 384; P[x]
+// (bf16 pairs) is aliased over the first 64 columns of S[x].
 #pragma once
 
 #include "common.cuh"
@@ -98,6 +105,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+// 16 consecutive 32-bit TMEM columns of this thread's lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -159,17 +174,28 @@ __device__ __forceinline__ uint64_t bits_from(int l) {   // offsets l..63
   return l <= 0 ? ~0ull : (l >= 64 ? 0ull : ~((1ull << l) - 1ull));
 }
 
-constexpr int kKStages = 4;   // K ring: a stage is freed once the S MMAs that read it complete
-constexpr int kVStages = 4;   // V ring: a stage is freed once the PV MMAs that read it complete
+// A pipeline step covers two consecutive entries of the row's tile list (any two
+// kept 64-key tiles; an odd tail repeats the last tile and masks the copy), so
+// that S is a 128 x 128 tile and every barrier round trip and tcgen05.commit of
+// the single issuing thread is amortised over 128 keys.
+constexpr int kKStages = 3;   // K ring (tile pairs): freed once the S MMAs that read it complete
+constexpr int kVStages = 2;   // V ring (tile pairs): freed once the PV MMAs that read it complete
 
-template <int D, int NM>
+template <int D>
 struct Cfg {
   static constexpr int kBoxes = D / 64;
-  static constexpr int kQTile = kBoxes * 16384;      // one M-tile of Q: [boxes][128 rows][128 B]
-  static constexpr int kKVTile = kBoxes * 8192;      // one K (or V) tile: [boxes][64 rows][128 B]
-  static constexpr int kSmem = NM * kQTile + (kKStages + kVStages) * kKVTile + 1024;
-  static constexpr int kThreads = 64 + 128 * NM;
-  static constexpr int kTmemCols = (NM * D + NM * 128) <= 256 ? 256 : 512;
+  static constexpr int kQTile = kBoxes * 16384;     // Q: [boxes][128 rows][128 B]
+  static constexpr int kPair = kBoxes * 16384;      // one K (or V) tile pair: [boxes][128 keys][128 B]
+  // at least ~half of the SM's shared memory, so that only one CTA (and one 512-column
+  // TMEM allocation) is resident per SM
+  static constexpr int kSmemUsed = kQTile + (kKStages + kVStages) * kPair + 1024;
+  static constexpr int kSmem = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
+  static constexpr int kThreads = 64 + 256;   // producer, MMA, two softmax warpgroups
+  // TMEM: O[x] (fp32, D columns) at 128 x; S[x] (fp32, 128 columns) at 256 + 128 x,
+  // with P[x] (bf16 pairs, 64 columns) aliased over the first half of S[x]
+  static constexpr int kColO = 0;
+  static constexpr int kColS = 256;
+  static constexpr int kTmemCols = 512;
 };
 
 struct TcArgs {
@@ -181,25 +207,26 @@ struct TcArgs {
   int hsplit;                  // work items per row = G / HG
 };
 
-template <int D, int NM>
-__global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
+template <int D>
+__global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, TcArgs T) {
-  using C = Cfg<D, NM>;
+  using C = Cfg<D>;
   const PrefillArgs& A = T.p;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full;
   __shared__ __align__(8) uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
-  __shared__ __align__(8) uint64_t s_full[NM][2], p_full[NM][2], o_done[NM];
+  __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_done[2];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
+  __shared__ float s_ml[2][2][128];   // [warpgroup][m, l][row]: epilogue merge
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_s = smem;
-  uint8_t* k_s = q_s + NM * C::kQTile;
-  uint8_t* v_s = k_s + kKStages * C::kKVTile;
+  uint8_t* k_s = q_s + C::kQTile;
+  uint8_t* v_s = k_s + kKStages * C::kPair;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // ---- work item
+  // ---- work item: 128 query rows = two 64-row blocks
   const int w = blockIdx.x;
   const int r = A.order[w / T.hsplit];
   const int hs = w % T.hsplit;
@@ -210,11 +237,14 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
   const int h0 = g * A.G + hs * T.HG;
   const bool streaming = A.head_kind[g] != LSERVE_HEAD_DENSE;
   const int beg = A.row_offsets[r];
-  const int n = A.row_offsets[r + 1] - beg;
+  const int n = A.row_offsets[r + 1] - beg;   // kept tiles
+  const int np = (n + 1) >> 1;                 // pipeline steps (tile pairs)
   const uint16_t* cols = A.cols + beg;
   const int tok0 = b * A.S;
   auto rb_head = [&](int rb) { return h0 + rb % T.HG; };
   auto rb_qt = [&](int rb) { return qgi * T.QG + rb / T.HG; };
+  // list entry of half h of step p (the odd tail repeats the last entry)
+  auto pair_tile = [&](int p, int h) { return cols[min(2 * p + h, n - 1)]; };
 
   if (tid == 0) {
     mbar_init(&q_full, 1);
@@ -226,12 +256,10 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int m = 0; m < NM; ++m) {
-      mbar_init(&s_full[m][0], 1);
-      mbar_init(&s_full[m][1], 1);
-      mbar_init(&p_full[m][0], 128);
-      mbar_init(&p_full[m][1], 128);
-      mbar_init(&o_done[m], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 128);
+      mbar_init(&o_done[x], 1);
     }
     s_abort = 0;
     fence_barrier_init();
@@ -244,8 +272,6 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = s_tmem;
-  const uint32_t t_o0 = tmem;                  // O[m] at column m*D
-  const uint32_t t_s0 = tmem + NM * D;         // S[m][buf] at NM*D + 64*(2m+buf)
   const unsigned long long tmo = A.timeout_ns;
 
   if (warp == 0) {
@@ -259,217 +285,303 @@ __global__ void __launch_bounds__(Cfg<D, NM>::kThreads, 1)
         prefetch_tensormap(&tmV);
       }
       int valid_rb = 0;
-      for (int rb = 0; rb < 2 * NM; ++rb) valid_rb += rb_qt(rb) < A.nQT;
+      for (int rb = 0; rb < 2; ++rb) valid_rb += rb_qt(rb) < A.nQT;
       if (leader) {
         mbar_arrive_expect_tx(&q_full, valid_rb * C::kBoxes * 8192);
-        for (int rb = 0; rb < 2 * NM; ++rb) {
+        for (int rb = 0; rb < 2; ++rb) {
           if (rb_qt(rb) >= A.nQT) continue;
-          uint8_t* dst = q_s + (rb >> 1) * C::kQTile + (rb & 1) * 8192;
           for (int x = 0; x < C::kBoxes; ++x)
-            tma_load_3d(dst + x * 16384, &tmQ, &q_full, x * 64, rb_head(rb), tok0 + rb_qt(rb) * kTile);
+            tma_load_3d(q_s + x * 16384 + rb * 8192, &tmQ, &q_full, x * 64, rb_head(rb), tok0 + rb_qt(rb) * kTile);
         }
       }
-      // K of tile t+1 goes out before V of tile t: S MMAs run one tile ahead of PV MMAs
-      for (int t = 0; t <= n; ++t) {
-        if (t < n) {
+      // K of step t+1 goes out before V of step t: S MMAs run ahead of PV MMAs
+      for (int t = 0; t <= np; ++t) {
+        if (t < np) {
           const int st = t % kKStages;
           if (t >= kKStages && !wait_or_abort(&k_empty[st], ((t / kKStages) - 1) & 1, &s_abort, tmo)) break;
-          const int kt = cols[t];
+          const int ka = pair_tile(t, 0), kb = pair_tile(t, 1);
           if (leader) {
-            mbar_arrive_expect_tx(&k_full[st], C::kKVTile);
-            for (int x = 0; x < C::kBoxes; ++x)
-              tma_load_3d(k_s + st * C::kKVTile + x * 8192, &tmK, &k_full[st], x * 64, g, tok0 + kt * kTile);
+            mbar_arrive_expect_tx(&k_full[st], C::kPair);
+            for (int x = 0; x < C::kBoxes; ++x) {
+              uint8_t* dst = k_s + st * C::kPair + x * 16384;
+              tma_load_3d(dst, &tmK, &k_full[st], x * 64, g, tok0 + ka * kTile);
+              tma_load_3d(dst + 8192, &tmK, &k_full[st], x * 64, g, tok0 + kb * kTile);
+            }
           }
         }
         if (t >= 1) {
           const int u = t - 1;
           const int st = u % kVStages;
           if (u >= kVStages && !wait_or_abort(&v_empty[st], ((u / kVStages) - 1) & 1, &s_abort, tmo)) break;
-          const int kt = cols[u];
+          const int ka = pair_tile(u, 0), kb = pair_tile(u, 1);
           if (leader) {
-            mbar_arrive_expect_tx(&v_full[st], C::kKVTile);
-            for (int x = 0; x < C::kBoxes; ++x)
-              tma_load_3d(v_s + st * C::kKVTile + x * 8192, &tmV, &v_full[st], x * 64, g, tok0 + kt * kTile);
+            mbar_arrive_expect_tx(&v_full[st], C::kPair);
+            for (int x = 0; x < C::kBoxes; ++x) {
+              uint8_t* dst = v_s + st * C::kPair + x * 16384;
+              tma_load_3d(dst, &tmV, &v_full[st], x * 64, g, tok0 + ka * kTile);
+              tma_load_3d(dst + 8192, &tmV, &v_full[st], x * 64, g, tok0 + kb * kTile);
+            }
           }
         }
       }
     }
   } else if (warp == 1) {
     // ================================================================== MMA
-    // The whole warp runs the loop (waits and descriptors warp-uniform); MMAs and
-    // commits are issued by one elected lane.
+    // Step p belongs to stream x = p & 1 (S[x], P[x], O[x]).  The whole warp runs
+    // the loop (waits and descriptors warp-uniform); one elected lane issues.
+    // Tensor-core order: S(0) S(1) PV(0) S(2) PV(1) S(3) ...  S(p+2) overwrites the
+    // S/P buffer of PV(p), so it is issued once PV(p) has completed.
     if (n > 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 64, false);
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false);
       constexpr uint32_t kIdPV = idesc_bf16(128, D, true);
-      int o_seen[NM];
-      for (int m = 0; m < NM; ++m) o_seen[m] = 0;
-      auto wait_pv = [&](int m, int t) {   // PV of tile t (M-tile m) has completed
-        while (o_seen[m] <= t) {
-          if (!wait_or_abort(&o_done[m], o_seen[m] & 1, &s_abort, tmo)) return;
-          ++o_seen[m];
-        }
-      };
       const uint32_t qa = smem_u32(q_s), ka = smem_u32(k_s), va = smem_u32(v_s);
-      auto issue_s = [&](int j) {
-        const int st = j % kKStages;
-        wait_or_abort(&k_full[st], (j / kKStages) & 1, &s_abort, tmo);
-        for (int m = 0; m < NM; ++m) {
-          const int buf = j & 1;
-          if (j >= 2) wait_pv(m, j - 2);   // S[m][buf] still holds P of tile j-2 until its PV is done
-          fence_after_sync();
+      auto issue_s = [&](int p) {   // S[p&1] = Q [K_a; K_b]^T
+        const int st = p % kKStages, x = p & 1;
+        wait_or_abort(&k_full[st], (p / kKStages) & 1, &s_abort, tmo);
+        if (p >= 2) wait_or_abort(&o_done[x], ((p >> 1) - 1) & 1, &s_abort, tmo);   // PV(p-2) read P[x]
+        fence_after_sync();
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t ad = sdesc(qa + m * C::kQTile + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc(ka + st * C::kKVTile + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-            mma_ss(t_s0 + 64 * (2 * m + buf), ad, bd, kIdS, ks > 0);
-          }
-          commit(&s_full[m][buf]);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t ad = sdesc(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc(ka + st * C::kPair + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+          mma_ss(tmem + C::kColS + 128 * x, ad, bd, kIdS, ks > 0);
         }
-        if (j + kKStages < n) commit(&k_empty[st]);
+        commit(&s_full[x]);
+        if (p + kKStages < np) commit(&k_empty[st]);
       };
       wait_or_abort(&q_full, 0, &s_abort, tmo);
       issue_s(0);
-      for (int j = 0; j < n; ++j) {
-        if (j + 1 < n) issue_s(j + 1);
-        const int st = j % kVStages;
-        wait_or_abort(&v_full[st], (j / kVStages) & 1, &s_abort, tmo);
-        for (int m = 0; m < NM; ++m) {
-          const int buf = j & 1;
-          wait_or_abort(&p_full[m][buf], (j >> 1) & 1, &s_abort, tmo);
-          fence_after_sync();
+      if (np > 1) issue_s(1);
+      for (int p = 0; p < np; ++p) {
+        const int st = p % kVStages, x = p & 1;
+        wait_or_abort(&v_full[st], (p / kVStages) & 1, &s_abort, tmo);
+        wait_or_abort(&p_full[x], (p >> 1) & 1, &s_abort, tmo);
+        fence_after_sync();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bd = sdesc(va + st * C::kKVTile + kk * 2048, 8192, 1024);
-            mma_ts(t_o0 + m * D, t_s0 + 64 * (2 * m + buf) + 8 * kk, bd, kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          commit(&o_done[m]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = sdesc(va + st * C::kPair + kk * 2048, 16384, 1024);
+          mma_ts(tmem + C::kColO + 128 * x, tmem + C::kColS + 128 * x + 8 * kk, bd, kIdPV,
+                 (p >= 2 || kk > 0) ? 1u : 0u);
         }
-        if (j + kVStages < n) commit(&v_empty[st]);
+        commit(&o_done[x]);
+        if (p + kVStages < np) commit(&v_empty[st]);
+        if (p + 2 < np) issue_s(p + 2);
       }
     }
   } else {
     // ============================================================== softmax
-    const int m = (warp - 2) >> 2;          // M-tile of this warpgroup
+    // Warpgroup x runs an independent online softmax over the steps p = x, x+2, ...
+    // with its own (m, l) and accumulator O[x]; the two are merged at the end.
+    const int x = (warp - 2) >> 2;
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;    // row within the M-tile
-    const int rb = 2 * m + (row >> 6);
+    const int rb = row >> 6;
     const int h = rb_head(rb), qt = rb_qt(rb);
     const bool rb_valid = qt < A.nQT;
     const int i = qt * kTile + (row & 63);  // query position
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t t_o = t_o0 + m * D + lane_off;
+    const uint32_t t_o = tmem + C::kColO + 128 * x + lane_off;
+    const uint32_t t_s = tmem + C::kColS + 128 * x + lane_off;
     const uint8_t* mrow = (!streaming && T.block_mask && rb_valid)
                               ? T.block_mask + (static_cast<long>(bg) * A.nQT + qt) * A.nQT
                               : nullptr;
     float m_run = kNegInf, l_run = 0.f;
     const float sc = A.scale_log2;
     TileListParams tp{0, A.Hkv, A.nQT, A.sink, A.local, nullptr, nullptr};
-
-    for (int j = 0; j < n; ++j) {
-      const int buf = j & 1;
-      const uint32_t t_s = t_s0 + 64 * (2 * m + buf) + lane_off;
-      wait_or_abort(&s_full[m][buf], (j >> 1) & 1, &s_abort, tmo);
-      fence_after_sync();
-      uint32_t x[64];
-      tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-      const int kt = cols[j];
-      // keep mask of this row over the tile's 64 keys (bit c <-> key 64 kt + c)
-      uint64_t keep = ~0ull;
-      const bool keep_tile = rb_valid && (T.QG == 1 || tile_keep(tp, streaming, mrow, qt, kt));
-      if (!keep_tile) {
-        keep = 0ull;
-      } else if (!tile_is_full(streaming, qt, kt, A.sink, A.local)) {
-        const int d0 = i - kt * kTile;   // offset of the query position inside the tile
-        keep = bits_upto(d0);
-        if (streaming) keep &= bits_below(A.sink - kt * kTile) | bits_from(d0 - A.local + 1);
-      }
+    // keep mask of this row over one 64-key tile (bit c <-> key 64 kt + c)
+    auto tile_mask = [&](int kt) -> uint64_t {
+      if (!rb_valid || !(T.QG == 1 || tile_keep(tp, streaming, mrow, qt, kt))) return 0ull;
+      if (tile_is_full(streaming, qt, kt, A.sink, A.local)) return ~0ull;
+      const int d0 = i - kt * kTile;   // offset of the query position inside the tile
+      uint64_t k = bits_upto(d0);
+      if (streaming) k &= bits_below(A.sink - kt * kTile) | bits_from(d0 - A.local + 1);
+      return k;
+    };
+    // raw scores of one 64-key half, masked keys set to -inf
+    auto load_half = [&](int half, uint64_t keep, uint32_t (&v)[64]) {
+      tmem_ld32(t_s + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(t_s + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
       tmem_wait_ld();
-      float mx[8];
+      if (!__all_sync(0xffffffffu, keep == ~0ull)) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx[e] = kNegInf;
-      if (__all_sync(0xffffffffu, keep == ~0ull)) {
+        for (int c = 0; c < 64; ++c)
+          if (!((keep >> c) & 1ull)) v[c] = 0xff800000u;   // -inf: exp2 gives exactly 0
+      }
+    };
+    int seen = 0;   // completions of o_done[x] observed by this warpgroup
+
+    float rebase = 0.f;   // shift of the reference max decided at this stream's previous step
+    // tile indices of this stream's next step, loaded one step ahead (hides the load latency)
+    int nkt0 = 0, nkt1 = 0;
+    if (x < np) {
+      nkt0 = pair_tile(x, 0);
+      nkt1 = pair_tile(x, 1);
+    }
+    for (int p = x; p < np; p += 2) {
+      const int j = p >> 1;   // this stream's step index
+      const int kt0 = nkt0, kt1 = nkt1;
+      if (p + 2 < np) {
+        nkt0 = pair_tile(p + 2, 0);
+        nkt1 = pair_tile(p + 2, 1);
+      }
+      const uint64_t keep0 = tile_mask(kt0);
+      const uint64_t keep1 = (2 * p + 1 < n) ? tile_mask(kt1) : 0ull;
+      wait_or_abort(&s_full[x], j & 1, &s_abort, tmo);
+      fence_after_sync();
+      uint32_t v[64];
+      uint32_t pk0[32], pk1[32];
+      float ps[4];
+      // exponentials 2^(s*scale - m) of one 64-key half, packed to bf16 pairs;
+      // tracks the largest argument and the row sum
+      // one 32-column chunk of S (already in registers): exponentials, max, sum, bf16 pairs
+      auto exp_chunk = [&](uint32_t (&u)[32], uint64_t keep, int q, float m_use, uint32_t* pk, float (&am)[4]) {
+        if (!__all_sync(0xffffffffu, keep == ~0ull)) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(x[c]));
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float v = ((keep >> c) & 1ull) ? __uint_as_float(x[c]) : kNegInf;
-          x[c] = __float_as_uint(v);
-          mx[c & 7] = fmaxf(mx[c & 7], v);
+          for (int c = 0; c < 32; ++c)
+            if (!((keep >> (32 * q + c)) & 1ull)) u[c] = 0xff800000u;   // -inf: exp2 gives 0
         }
-      }
-      const float mloc = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sc;
-      // lazy rescale: move the reference max only when it grows by more than 8 (x256)
-      const bool need = mloc > m_run + 8.f;
-      const bool rescale = need && m_run != kNegInf;
-      const float f = rescale ? fast_exp2(m_run - mloc) : 1.f;
-      if (need) m_run = mloc;
-      const float m_use = m_run == kNegInf ? 0.f : m_run;
-      uint32_t pk[32];
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * c]), sc, -m_use));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * c + 1]), sc, -m_use));
-        ps[c & 3] += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < 16; ++c) {
+          const float a0 = fmaf(__uint_as_float(u[2 * c]), sc, -m_use);
+          const float a1 = fmaf(__uint_as_float(u[2 * c + 1]), sc, -m_use);
+          am[c & 3] = max3(am[c & 3], a0, a1);
+          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+          ps[c & 3] += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+      };
+      auto exp_pass = [&](float m) -> float {   // returns the largest argument
+        const float m_use = m == kNegInf ? 0.f : m;
+        float am[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ps[e] = 0.f;
+        // four 32-column chunks; the TMEM load of chunk c+1 is in flight while chunk c is processed
+        uint32_t ua[32], ub[32];
+        tmem_ld32(t_s, ua);
+        tmem_wait_ld();
+        tmem_ld32(t_s + 32, ub);
+        exp_chunk(ua, keep0, 0, m_use, pk0, am);
+        tmem_wait_ld();
+        tmem_ld32(t_s + 64, ua);
+        exp_chunk(ub, keep0, 1, m_use, pk0 + 16, am);
+        tmem_wait_ld();
+        tmem_ld32(t_s + 96, ub);
+        exp_chunk(ua, keep1, 0, m_use, pk1, am);
+        tmem_wait_ld();
+        exp_chunk(ub, keep1, 1, m_use, pk1 + 16, am);
+        return max3(am[0], am[1], fmaxf(am[2], am[3]));
+      };
+      // O[x] and l are multiplied by f before this step's P is added
+      float f = 1.f;
+      if (rebase != 0.f) {
+        f = fast_exp2(-rebase);
+        m_run += rebase;
+        rebase = 0.f;
       }
-      l_run = l_run * f + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-      tmem_st32(t_s, pk);   // P overwrites the first 32 columns of this S buffer
-      // Observe the completion of PV of tile j-1 (every thread, every tile, in
-      // order, so that the parity waits on o_done never fall two phases behind);
-      // then O holds exactly the tiles < j and may be rescaled.
-      if (j > 0) {
-        wait_or_abort(&o_done[m], (j - 1) & 1, &s_abort, tmo);
-        fence_after_sync();
+      float amax = kNegInf;
+      bool ok = false;
+      if (m_run != kNegInf) {   // steady state: one pass against the current reference
+        amax = exp_pass(m_run);
+        ok = !__any_sync(0xffffffffu, amax > 64.f);   // no exponential near the fp32/bf16 limit
       }
-      if (__any_sync(0xffffffffu, rescale)) {
+      if (!ok) {                // first step of the stream, or a jump: exact row max first
+        float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t ov[32];
-          tmem_ld32(t_o + c0, ov);
-          tmem_wait_ld();
+        for (int half = 0; half < 2; ++half) {
+          load_half(half, half ? keep1 : keep0, v);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * f);
-          tmem_st32(t_o + c0, ov);
+          for (int c = 0; c < 64; c += 8) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              mx[e] = max3(mx[e], __uint_as_float(v[c + 2 * e]), __uint_as_float(v[c + 2 * e + 1]));
+          }
+        }
+        const float mloc = max3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;
+        const float m_new = fmaxf(m_run, mloc);
+        if (m_run != kNegInf && m_new != m_run) f *= fast_exp2(m_run - m_new);
+        m_run = m_new;
+        amax = exp_pass(m_run);
+      }
+      // values above the reference by more than 2^8: move the reference at the next
+      // step of this stream (O must first absorb this step)
+      if (m_run != kNegInf && amax > 8.f) rebase = amax;
+      tmem_st32(t_s, pk0);        // P[x] over S[x] columns 0..63 (S is no longer needed)
+      tmem_st32(t_s + 32, pk1);
+      l_run = l_run * f + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+      // O[x] holds this stream's steps < p; PV(p-2) completed before S(p) was issued,
+      // observe it (in order) before touching O[x]
+      if (j > 0) {
+        wait_or_abort(&o_done[x], (j - 1) & 1, &s_abort, tmo);
+        ++seen;
+        fence_after_sync();
+        if (__any_sync(0xffffffffu, f != 1.f)) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld32(t_o + c0, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * f);
+            tmem_st32(t_o + c0, ov);
+          }
         }
       }
       tmem_wait_st();
       fence_before_sync();
-      mbar_arrive(&p_full[m][buf]);
+      mbar_arrive(&p_full[x]);
     }
-    // ---- epilogue
+    // a pending shift is never needed for the result: (m, l, O) stay consistent
+    // ---- epilogue: merge the two streams (log-sum-exp), each warpgroup stores half of O
+    const int nx = (np > x) ? (np - x + 1) >> 1 : 0;   // steps of this stream
+    if (nx > 0) {
+      wait_or_abort(&o_done[x], (nx - 1) & 1, &s_abort, tmo);   // PV of its last step
+      fence_after_sync();
+    }
+    s_ml[x][0][row] = m_run;
+    s_ml[x][1][row] = l_run;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    const float m_o = s_ml[x ^ 1][0][row], l_o = s_ml[x ^ 1][1][row];
+    const int nx_o = (np > (x ^ 1)) ? (np - (x ^ 1) + 1) >> 1 : 0;
+    const float m_all = fmaxf(m_run, m_o);
+    const float m_ref = m_all == kNegInf ? 0.f : m_all;
+    const float w_own = nx > 0 ? fast_exp2(m_run - m_ref) : 0.f;
+    const float w_oth = nx_o > 0 ? fast_exp2(m_o - m_ref) : 0.f;
+    const float l_tot = l_run * w_own + l_o * w_oth;
     if (rb_valid) {
-      bf16* orow = A.out + (static_cast<long>(tok0 + i) * Hq + h) * D;
-      const bool has = n > 0 && m_run != kNegInf && l_run > 0.f;
-      if (n > 0) {
-        wait_or_abort(&o_done[m], (n - 1) & 1, &s_abort, tmo);   // PV of the last tile
-        fence_after_sync();
-      }
-      const float inv = has ? 1.f / l_run : 0.f;
+      const int c_lo = x * (D / 2);   // this warpgroup's half of the output columns
+      bf16* orow = A.out + (static_cast<long>(tok0 + i) * Hq + h) * D + c_lo;
+      const bool has = n > 0 && m_all != kNegInf && l_tot > 0.f;
+      const float inv = has ? 1.f / l_tot : 0.f;
+      const uint32_t t_own = tmem + C::kColO + 128 * x + lane_off + c_lo;
+      const uint32_t t_oth = tmem + C::kColO + 128 * (x ^ 1) + lane_off + c_lo;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t ov[32];
-        if (n > 0) {
-          tmem_ld32(t_o + c0, ov);
-          tmem_wait_ld();
+      for (int c0 = 0; c0 < D / 2; c0 += 16) {
+        uint32_t oa[16], ob[16];
+        if (nx > 0) tmem_ld16(t_own + c0, oa);
+        if (nx_o > 0) tmem_ld16(t_oth + c0, ob);
+        tmem_wait_ld();
+        uint32_t pk[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float a0 = 0.f, a1 = 0.f;
+          if (nx > 0) {
+            a0 = __uint_as_float(oa[2 * c]) * w_own;
+            a1 = __uint_as_float(oa[2 * c + 1]) * w_own;
+          }
+          if (nx_o > 0) {
+            a0 = fmaf(__uint_as_float(ob[2 * c]), w_oth, a0);
+            a1 = fmaf(__uint_as_float(ob[2 * c + 1]), w_oth, a1);
+          }
+          pk[c] = pack_bf16x2(a0 * inv, a1 * inv);
         }
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          pk[c] = n > 0 ? pack_bf16x2(__uint_as_float(ov[2 * c]) * inv, __uint_as_float(ov[2 * c + 1]) * inv) : 0u;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(orow + c0 + 8 * c) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(orow + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(orow + c0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
-      if (A.lse)
+      if (A.lse && x == 0)
         A.lse[(static_cast<long>(b) * Hq + h) * A.S + i] =
-            has ? (m_run + __log2f(l_run)) * 0.6931471805599453f : kNegInf;
-    } else if (n > 0) {
-      wait_or_abort(&o_done[m], (n - 1) & 1, &s_abort, tmo);
+            has ? (m_all + __log2f(l_tot)) * 0.6931471805599453f : kNegInf;
     }
+    (void)seen;
   }
   fence_before_sync();
   __syncthreads();

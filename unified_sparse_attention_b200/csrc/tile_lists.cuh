@@ -10,11 +10,14 @@
 //   streaming  kt <= qt  and (64 kt < sink  or  max(64 qt - 64 kt - 63, 0) < local)
 // Built in three launches, all on device, no host round trip:
 //   tile_count_kernel  one warp per row: count kept tiles (4 mask bytes per lane
-//                      per step), histogram of row lengths
+//                      per step), histogram of row lengths per (b, kvh)
 //   tile_scan_kernel   one CTA: CSR offsets (exclusive scan of the counts) and the
-//                      start of every row-length bucket in longest-first order
+//                      start of every row-length bucket in the work order
 //   tile_fill_kernel   one warp per row: ballot-ordered compaction of kt into the
-//                      CSR, and the row's slot in the longest-first work order
+//                      CSR, and the row's slot in the work order
+// Work order: (b, kvh) groups one after another, longest rows first inside a
+// group.  Concurrent CTAs then share one KV head's K/V, which stays in L2 even
+// when the whole K/V of a long sequence does not.
 #pragma once
 
 #include "common.cuh"
@@ -78,15 +81,16 @@ __global__ void __launch_bounds__(256) tile_count_kernel(TileListParams P, int* 
   for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
   if ((threadIdx.x & 31) == 0) {
     counts[r] = cnt;
-    atomicAdd(&hist[cnt], 1);
+    atomicAdd(&hist[(r / P.nRow) * (P.nQT + 1) + cnt], 1);
   }
 }
 
-// One CTA of 1024 threads.  offsets[r] = sum_{r' < r} counts[r']; bucket[c] =
-// number of rows with more than c kept tiles (start of bucket c in the order).
+// One CTA of 1024 threads.  offsets[r] = sum_{r' < r} counts[r']; for group g
+// (rows g*nRow .. g*nRow + nRow - 1), bucket[g][c] = g*nRow + number of rows of
+// the group with more than c kept tiles (start of bucket c of that group).
 __global__ void __launch_bounds__(1024) tile_scan_kernel(const int* __restrict__ counts, int R,
                                                          int* __restrict__ offsets, const int* __restrict__ hist,
-                                                         int nbucket, int* __restrict__ bucket,
+                                                         int nbucket, int* __restrict__ bucket, int nRow,
                                                          long long max_nnz, int* __restrict__ overflow) {
   __shared__ int s_warp[32];
   __shared__ long long s_carry;
@@ -125,10 +129,12 @@ __global__ void __launch_bounds__(1024) tile_scan_kernel(const int* __restrict__
     offsets[R] = static_cast<int>(s_carry);
     *overflow = s_carry > max_nnz;
     if (s_carry > max_nnz) report(LSERVE_ERR_DEVICE_BOUNDS);
-    int above = 0;   // rows with more kept tiles than c
+  }
+  for (int grp = tid; grp < R / nRow; grp += blockDim.x) {
+    int above = grp * nRow;   // rows before this group + rows of it with more kept tiles than c
     for (int c = nbucket - 1; c >= 0; --c) {
-      bucket[c] = above;
-      above += hist[c];
+      bucket[grp * nbucket + c] = above;
+      above += hist[grp * nbucket + c];
     }
   }
 }
@@ -157,8 +163,8 @@ __global__ void __launch_bounds__(256) tile_fill_kernel(TileListParams P, const 
     pos += __shfl_sync(0xffffffffu, x, 31);
   });
   if (lane == 0 && order) {
-    const int cnt = counts[r];
-    order[bucket[cnt] + atomicAdd(&fill[cnt], 1)] = r;
+    const int k = (r / P.nRow) * (P.nQT + 1) + counts[r];
+    order[bucket[k] + atomicAdd(&fill[k], 1)] = r;
   }
 }
 

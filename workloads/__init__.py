@@ -100,6 +100,9 @@ WORKLOADS = {
         n_streaming=16, sink=64, local=256, anchors=64, dec_B=4, ctx=262144,
         token_budget=8192, pool_pages=16384, dec_anchors=64),
 }
+# Half-length version of the long prefill (same recipe), sized for profiler captures.
+WORKLOADS["llama3_8b_prefill_64k_vslash"] = dataclasses.replace(
+    WORKLOADS["llama3_8b_prefill_128k_vslash"], name="llama3_8b_prefill_64k_vslash", S=65536)
 # The literal reading of the long-prefill mask (5 % random fill, ~6.5 % density).
 WORKLOADS["llama3_8b_prefill_128k_vslash_literal"] = dataclasses.replace(
     WORKLOADS["llama3_8b_prefill_128k_vslash"],
