@@ -410,7 +410,7 @@ def main():
     n_dense = sum(1 for g in range(wp.Hkv) if setup.kind_p[g] == 0)
     dense_density = (sum(setup.tiles[g] for g in range(wp.Hkv) if setup.kind_p[g] == 0)
                      / max(1, n_dense * n * (n + 1) / 2))
-    launches_per_step = 4 + 1 + 4   # tile count/scan/fill + attention; stats refresh; score/top-k/decode/merge
+    launches_per_step = 4 + 1 + 3   # tile count/scan/fill + attention; stats refresh; score/top-k/decode (+merge)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",

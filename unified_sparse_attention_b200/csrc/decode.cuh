@@ -22,8 +22,9 @@
 // (not arithmetic) and their V rows are zeroed in the MMA operand, so even NaN
 // garbage there cannot reach the result.
 //
-// lse_merge_kernel: one CTA per (b, query head): out = sum_s w_s o_s with
-// w_s = 2^(lse_s - lse), lse = log2 sum_s 2^lse_s.
+// The last split CTA of each (b, KV head) to finish (a counter per unit, zeroed
+// by the top-k kernel and reset by that CTA) merges the partials by log-sum-exp:
+// out = sum_s w_s o_s with w_s = 2^(lse_s - lse), lse = log2 sum_s 2^lse_s.
 #pragma once
 
 #include "common.cuh"
@@ -49,7 +50,8 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(
     const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind,
     const int32_t* __restrict__ sel, const int32_t* __restrict__ sel_n, int kcap, int pages_per_split,
     int nsplit, int Hkv, int G, int num_pages, int sink, int local, float scale_log2,
-    unsigned long long timeout_ns, float* __restrict__ part_o, float* __restrict__ part_lse) {
+    unsigned long long timeout_ns, float* __restrict__ part_o, float* __restrict__ part_lse,
+    int32_t* __restrict__ done_count, bf16* __restrict__ out, float* __restrict__ lse_out) {
   using Cfg = DecodeCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kDecodeStages];
@@ -59,8 +61,17 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(
   const int split = blockIdx.x;
   const int b = unit / Hkv, g = unit % Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();   // the selection comes from the previous kernel
   const int n_sel = min(sel_n[unit], kcap);
   const int p_begin = split * pages_per_split;
+  if (n_sel == 0 && split == 0) {   // nothing to attend to: out = 0, lse = -inf
+    for (int idx = tid; idx < G * D; idx += kDecodeThreads) {
+      const long bh = static_cast<long>(b) * Hkv * G + static_cast<long>(g) * G + idx / D;
+      out[bh * D + idx % D] = __float2bfloat16_rn(0.f);
+      if (lse_out && idx % D == 0) lse_out[bh] = kNegInf;
+    }
+    return;
+  }
   if (p_begin >= n_sel) return;
   const int n_my = min(pages_per_split, n_sel - p_begin);
   const int L = seq_lens[b];
@@ -282,36 +293,55 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(
     part_o[(part * G + h) * D + c] = has ? o / l : 0.f;
     if (c == 0) part_lse[part * G + h] = has ? m + __log2f(l) : kNegInf;
   }
-}
-
-template <int D>
-__global__ void __launch_bounds__(D) lse_merge_kernel(const float* __restrict__ part_o,
-                                                      const float* __restrict__ part_lse,
-                                                      const int32_t* __restrict__ sel_n, int kcap,
-                                                      int pages_per_split, int nsplit, int Hkv, int G,
-                                                      bf16* __restrict__ out, float* __restrict__ lse_out) {
-  const int bh = blockIdx.x;              // b * Hq + h
-  const int Hq = Hkv * G;
-  const int b = bh / Hq, h = bh % Hq;
-  const int unit = b * Hkv + h / G, hh = h % G;
-  const int n_sel = min(sel_n[unit], kcap);
+  // ---- the last split of this (sequence, KV head) to finish merges all splits:
+  // out = sum_s w_s o_s with w_s = 2^(lse_s - lse), lse = log2 sum_s 2^lse_s
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
   const int ns = (n_sel + pages_per_split - 1) / pages_per_split;
-  const int c = threadIdx.x;
-  float m = kNegInf;
-  for (int s = 0; s < ns; ++s) m = fmaxf(m, part_lse[(static_cast<long>(unit) * nsplit + s) * G + hh]);
-  float o = 0.f, w = 0.f;
-  if (m != kNegInf) {
-    for (int s = 0; s < ns; ++s) {
-      const long part = static_cast<long>(unit) * nsplit + s;
-      const float ls = part_lse[part * G + hh];
-      const float sc = fast_exp2(ls - m);
-      o += sc * part_o[(part * G + hh) * D + c];
-      w += sc;
-    }
+  if (tid == 0) s_last = atomicAdd(&done_count[unit], 1) == ns - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // per query head: m = max_s lse_s, lse = m + log2 sum_s 2^(lse_s - m); warp w owns heads w, w + 4, ...
+  __shared__ float s_lse[16];
+  const long base = static_cast<long>(unit) * nsplit;
+  for (int hh = warp; hh < G; hh += 4) {
+    float m = kNegInf;
+    for (int sp = lane; sp < ns; sp += 32) m = fmaxf(m, __ldcg(&part_lse[(base + sp) * G + hh]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    if (m != kNegInf)
+      for (int sp = lane; sp < ns; sp += 32) l += fast_exp2(__ldcg(&part_lse[(base + sp) * G + hh]) - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) s_lse[hh] = (m != kNegInf && l > 0.f) ? m + __log2f(l) : kNegInf;
   }
-  const bool has = m != kNegInf && w > 0.f;
-  out[static_cast<long>(bh) * D + c] = __float2bfloat16_rn(has ? o / w : 0.f);
-  if (lse_out && c == 0) lse_out[bh] = has ? (m + __log2f(w)) * 0.6931471805599453f : kNegInf;
+  __syncthreads();
+  // out = sum_s 2^(lse_s - lse) o_s, four channels per thread; the split loads are independent
+  for (int idx = tid * 4; idx < G * D; idx += kDecodeThreads * 4) {
+    const int hh = idx / D, c = idx % D;
+    const float lse_h = s_lse[hh];
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lse_h != kNegInf) {
+#pragma unroll 4
+      for (int sp = 0; sp < ns; ++sp) {
+        const float w = fast_exp2(__ldcg(&part_lse[(base + sp) * G + hh]) - lse_h);
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(&part_o[((base + sp) * G + hh) * D + c]));
+        o.x += w * x.x;
+        o.y += w * x.y;
+        o.z += w * x.z;
+        o.w += w * x.w;
+      }
+    }
+    const long bh = static_cast<long>(b) * Hkv * G + static_cast<long>(g) * G + hh;
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + bh * D + c);
+    dst[0] = __floats2bfloat162_rn(o.x, o.y);
+    dst[1] = __floats2bfloat162_rn(o.z, o.w);
+    if (lse_out && c == 0) lse_out[bh] = lse_h == kNegInf ? kNegInf : lse_h * 0.6931471805599453f;
+  }
+  if (tid == 0) done_count[unit] = 0;   // ready for the next call
 }
 
 }  // namespace lserve

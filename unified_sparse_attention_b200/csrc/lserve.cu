@@ -245,8 +245,27 @@ struct DecodePlan {
   int32_t* sel_n;
   float* part_o;
   float* part_lse;
+  int32_t* done_count;   // per (b, kvh): finished splits (zeroed by the top-k kernel)
   size_t bytes;
 };
+
+// Launch with programmatic stream serialisation: the kernel may start while its
+// predecessor finishes and waits on griddepcontrol.wait before reading its output.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 int streaming_page_bound(int sink, int local) {
   return (sink + kPage - 1) / kPage + (local + kPage - 1) / kPage + 1;
@@ -278,7 +297,7 @@ DecodePlan plan_decode(const lserve_decode_args* a, void* ws) {
   p.budget_pages = a->token_budget / kPage;
   const int dense_cap = std::min(p.budget_pages, a->maxP);
   p.kcap = std::max(1, std::max(dense_cap, std::min(streaming_page_bound(a->sink, a->local), a->maxP)));
-  // split-KV: aim for ~8 CTAs per SM over the dense selections
+  // split-KV: aim for ~8 CTAs per SM over the selections
   const long long total = static_cast<long long>(a->B) * a->Hkv * p.kcap;
   long long pps = (total + 8 * 148 - 1) / (8 * 148);
   p.pps = static_cast<int>(std::max(2ll, std::min<long long>(pps, 64)));
@@ -294,6 +313,7 @@ DecodePlan plan_decode(const lserve_decode_args* a, void* ws) {
   p.sel_n = c.take<int32_t>(units);
   p.part_o = c.take<float>(units * p.nsplit * p.G * a->d);
   p.part_lse = c.take<float>(units * p.nsplit * p.G);
+  p.done_count = c.take<int32_t>(units);
   p.bytes = c.used();
   return p;
 }
@@ -317,22 +337,23 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
   }
   ensure_smem(topk_pages_kernel, kTopkSmemKeys * static_cast<int>(sizeof(uint32_t)));
   const int topk_smem = std::min(a->maxP, kTopkSmemKeys) * static_cast<int>(sizeof(uint32_t));
-  topk_pages_kernel<<<a->B * a->Hkv, kTopkThreads, topk_smem, st>>>(p.scores, a->maxP, a->seq_lens, a->head_kind,
-                                                                     a->Hkv, p.budget_pages, a->sink, a->local, sel,
-                                                                     sel_n, p.kcap);
+  if (launch_pdl(topk_pages_kernel, dim3(a->B * a->Hkv), dim3(kTopkThreads), topk_smem, st, p.scores, a->maxP,
+                 a->seq_lens, a->head_kind, a->Hkv, p.budget_pages, a->sink, a->local, sel, sel_n, p.kcap,
+                 p.done_count) != cudaSuccess)
+    return check_launch("decode top-k");
   CUtensorMap tk, tv;
   const uint64_t rows = static_cast<uint64_t>(a->num_pages) * a->Hkv * kPage;
   if (!make_map_2d(&tk, a->k_pages, D, rows) || !make_map_2d(&tv, a->v_pages, D, rows))
     return fail(LSERVE_ERR_CUDA, "decode: cuTensorMapEncodeTiled failed");
   ensure_smem(paged_decode_kernel<D>, DecodeCfg<D>::kSmemBytes);
   const float scale = a->scale > 0.f ? a->scale : 1.f / std::sqrt(static_cast<float>(D));
-  dim3 grid(p.nsplit, a->B * a->Hkv);
-  paged_decode_kernel<D><<<grid, kDecodeThreads, DecodeCfg<D>::kSmemBytes, st>>>(
-      tk, tv, static_cast<const bf16*>(a->q), a->page_table, a->maxP, a->seq_lens, a->head_kind, sel, sel_n, p.kcap,
-      p.pps, p.nsplit, a->Hkv, p.G, a->num_pages, a->sink, a->local, scale * 1.4426950408889634f, wait_timeout_ns(),
-      p.part_o, p.part_lse);
-  lse_merge_kernel<D><<<a->B * a->Hq, D, 0, st>>>(p.part_o, p.part_lse, sel_n, p.kcap, p.pps, p.nsplit, a->Hkv, p.G,
-                                                  static_cast<bf16*>(out), lse);
+  if (launch_pdl(paged_decode_kernel<D>, dim3(p.nsplit, a->B * a->Hkv), dim3(kDecodeThreads),
+                 DecodeCfg<D>::kSmemBytes, st, tk, tv, static_cast<const bf16*>(a->q), a->page_table, a->maxP,
+                 a->seq_lens, a->head_kind, static_cast<const int32_t*>(sel), static_cast<const int32_t*>(sel_n),
+                 p.kcap, p.pps, p.nsplit, a->Hkv, p.G, a->num_pages, a->sink, a->local,
+                 scale * 1.4426950408889634f, wait_timeout_ns(), p.part_o, p.part_lse, p.done_count,
+                 static_cast<bf16*>(out), lse) != cudaSuccess)
+    return check_launch("decode attention");
   return check_launch("decode");
 }
 

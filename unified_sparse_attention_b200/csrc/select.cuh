@@ -158,7 +158,7 @@ constexpr int kTopkSmemKeys = 16384;   // scores cached in shared memory up to t
 __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
     const float* __restrict__ scores, int maxP, const int32_t* __restrict__ seq_lens,
     const uint8_t* __restrict__ head_kind, int Hkv, int budget_pages, int sink, int local,
-    int32_t* __restrict__ sel, int32_t* __restrict__ sel_n, int kcap) {
+    int32_t* __restrict__ sel, int32_t* __restrict__ sel_n, int kcap, int32_t* __restrict__ done_count) {
   extern __shared__ uint32_t s_keys[];
   __shared__ int s_hist[256];
   __shared__ int s_scan[32];
@@ -166,6 +166,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
   __shared__ int s_remaining;
   const int unit = blockIdx.x;   // b * Hkv + g
   const int b = unit / Hkv, g = unit % Hkv;
+  pdl_wait();   // the scores come from the previous kernel
+  if (threadIdx.x == 0) done_count[unit] = 0;   // split-completion counter of the decode kernel
   const int L = max(0, seq_lens[b]);
   int n = (L + kPage - 1) / kPage;
   if (n > maxP) {   // sequence longer than its page-table row
