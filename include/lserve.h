@@ -183,7 +183,11 @@ typedef struct lserve_decode_args {
 /* Capacity (pages) of one selection row: max(min(budget/64, maxP), streaming pages). */
 int32_t lserve_decode_max_selected(const lserve_decode_args* args);
 
-/* Bytes of workspace lserve_decode needs (page scores, selection, split partials). */
+/* Bytes of workspace lserve_decode needs (page scores, selection, partition,
+ * per-warp partials).  It depends on the current device's SM count (the
+ * attention grid is one wave of SMs x 2 CTAs) or, when the environment
+ * variable LSERVE_DECODE_GRID holds a positive integer, on that grid size;
+ * ask again after changing either. */
 size_t lserve_decode_workspace_size(const lserve_decode_args* args);
 
 /*
@@ -196,7 +200,9 @@ size_t lserve_decode_workspace_size(const lserve_decode_args* args);
  *   selection      the k = min(token_budget/64, n) highest-scoring pages, ties to
  *                  the lower page index, listed in ascending page order
  *   attention      softmax(scale * q.k_t) over every valid token t of the
- *                  selected pages, computed split-KV and merged by log-sum-exp.
+ *                  selected pages.  All units' selected pages are dealt out
+ *                  evenly to one wave of CTAs; the partial results of a unit
+ *                  are merged by log-sum-exp.
  * Streaming KV head: the pages holding tokens [0, sink) and
  * [seq_len - local, seq_len), attending to exactly those tokens.
  * The query is at position seq_len - 1 (its own key/value are in the cache).

@@ -137,3 +137,30 @@ def test_out_of_range_page_id_is_reported_not_read():
                                torch.zeros(1, dtype=torch.uint8, device=dev))
     assert U.lserve_get_device_status() == 6
     assert U.lserve_get_device_status() == 0   # read clears it
+
+
+# The attention grid deals all selected pages out evenly to its CTAs.  Forcing a
+# small grid makes one CTA stream many pages (more than one 256-page chunk) and
+# many units (more than the 128 one chunk window spans), and lets the grid
+# exceed the page count elsewhere.
+def test_one_cta_crosses_page_chunks(monkeypatch):
+    monkeypatch.setenv("LSERVE_DECODE_GRID", "1")
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2, Hkv=1, d=64, dec_anchors=8)
+    r = run_decode(w, 1, 20000, 300 * 64, 64, 100, kind=[0])
+    assert len(r["sel"][(0, 0)]) == 300
+
+
+@pytest.mark.parametrize("grid", ["1", "3", "7", "1000"])
+def test_small_grid_spans_many_units(monkeypatch, grid):
+    monkeypatch.setenv("LSERVE_DECODE_GRID", grid)
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=8, Hkv=4, d=64, dec_anchors=4)
+    B = 40
+    lens = [(37 * b) % 300 for b in range(B)]     # ragged, some sequences empty
+    run_decode(w, B, 300, 128, 16, 70, lens=lens, kind=[0, 1, 0, 1])
+
+
+@pytest.mark.parametrize("grid", ["2", "5"])
+def test_small_grid_gqa_d128(monkeypatch, grid):
+    monkeypatch.setenv("LSERVE_DECODE_GRID", grid)
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=16, Hkv=2, d=128, dec_anchors=16)
+    run_decode(w, 3, 1000, 512, 64, 100, lens=[1000, 333, 65], kind=[0, 1])

@@ -1,347 +1,627 @@
-// decode.cuh -- split-KV sparse paged decode attention + log-sum-exp merge.
+// decode.cuh -- sparse paged decode attention over the selected pages, split
+// evenly across a persistent grid, with the log-sum-exp merge folded in.
 //
 // LServe + SampleAttention blog post, "LServe - Decode Phase" and Fig. 2:
 // token-level attention only inside the selected pages.  Streaming heads attend
 // to their sink + local tokens (mlsanity LServe page, Abstract: streaming heads
 // in both the prefilling and the decoding stages).
 //
-// paged_decode_kernel: one CTA per (sequence b, KV head g, split s); a split
-// covers `pages_per_split` consecutive entries of the (b, g) selection.  The CTA
-// streams each selected K and V page (64 x d bf16, contiguous in the pool)
-// into a 3-stage shared-memory ring with TMA (128-byte swizzle, completion on
-// an mbarrier; thread 0 is the producer).  Each of the 4 warps owns 16 tokens
-// of every page and keeps its own online-softmax state for the G query heads of
-// the group: q.k and p.v run on mma.sync m16n8k16 with the G heads as the M
-// rows (zero-padded to 16), so the kernel spends its issue slots on moving
-// bytes, not on dot-product reductions.  At the end the 4 warp states are
-// merged through shared memory into one (o, lse) partial per head and split.
+// Work split.  Unit u = (sequence b, KV head g) has n_u selected pages; the
+// pages of all units, laid end to end in unit order, form one flat list of
+// T = sum_u n_u pages with unit u at [off_u, off_u + n_u).
+// decode_partition_kernel builds `off` and, for each of the P CTAs of the
+// attention grid (P = SMs x resident CTAs per SM, one wave), the unit holding
+// the first page of CTA c's equal share [floor(c T / P), floor((c + 1) T / P)).
+// A share that crosses unit boundaries is cut into segments, one per unit.
+// Every CTA then streams about T / P pages whatever the mix of long dense
+// selections and short streaming ones, so the grid ends in one wave with no
+// tail, where one CTA per (unit, fixed-size split) left a partial last wave.
+//
+// paged_decode_kernel (per CTA):
+//   * resolves its pages (unit, logical page, physical page) into shared memory
+//     up front, in chunks of up to 256 pages, so the producer issues loads with
+//     no dependent global lookups on its path;
+//   * streams each page's K and V (64 x d bf16 each, contiguous in the pool)
+//     through a 3-stage ring with TMA (128-byte swizzle): a producer warp
+//     issues a stage's loads once the 4 consumer warps have released it (full
+//     and empty mbarriers per stage), so no consumer ever waits for an issue
+//     or for another consumer; the first page of a segment also brings the
+//     group's G query rows with a bulk copy;
+//   * each of the 4 warps owns 16 tokens of every page and keeps an online
+//     softmax for the G <= 8 query heads, on mma.sync m16n8k16 tiles laid out
+//     transposed: S^T = K Q^T (M = 16 tokens, N = 8 heads) and O^T += V^T P^T
+//     (M = channels, N = heads), with P^T made by movmatrix -- the heads fill N
+//     exactly, so no MMA work or accumulator register goes to padding, and
+//     issue slots go to moving bytes rather than to dot-product reductions;
+//   * at the end of a segment each warp writes its own normalised partial
+//     (o, lse) -- no cross-warp exchange, the ring keeps streaming -- and bumps
+//     the unit's counter; the warp that completes the count merges all of the
+//     unit's partials: out = sum_i 2^(lse_i - lse) o_i, lse = log2 sum_i 2^lse_i.
+//
+// Partial slots.  Segment (CTA c, unit u) uses slot c + u: along the flat list
+// both c and u never decrease and one of them grows at every segment boundary,
+// so slots are distinct, and unit u's slots are the contiguous run
+// c_first(u) + u .. c_last(u) + u.  Slots <= P + units - 1.
 //
 // Bytes per selected page: 2 * 64 * d * 2 (K and V); the kernel is HBM-bound.
 // Tokens outside the attended set (past seq_len; outside the Lambda set of a
 // streaming head) are masked exactly: their logits become -inf by selection
 // (not arithmetic) and their V rows are zeroed in the MMA operand, so even NaN
-// garbage there cannot reach the result.
-//
-// The last split CTA of each (b, KV head) to finish (a counter per unit, zeroed
-// by the top-k kernel and reset by that CTA) merges the partials by log-sum-exp:
-// out = sum_s w_s o_s with w_s = 2^(lse_s - lse), lse = log2 sum_s 2^lse_s.
+// garbage there cannot reach the result.  No CTA ever waits for another.
 #pragma once
 
+#include <climits>
+
 #include "common.cuh"
+#include "select.cuh"
 
 namespace lserve {
 
 constexpr int kDecodeStages = 3;
-constexpr int kDecodeThreads = 128;
+constexpr int kDecodeWarps = 4;                           // consumer warps
+constexpr int kIssuerWarp = kDecodeWarps;                  // issues the TMA loads
+constexpr int kResolverWarp = kDecodeWarps + 1;            // claims ranges, resolves their pages
+constexpr int kDecodeThreads = (kDecodeWarps + 2) * 32;
+constexpr int kDecodeCtasPerSm = 2;
+constexpr int kDecodeMaxG = 8;
+constexpr int kRangesPerCta = 4;   // ranges of the flat page list per attention CTA
+constexpr int kMetaRing = 64;      // resolved pages buffered ahead of the loads
+
+constexpr int kSegStart = 1, kSegEnd = 2, kSegStreaming = 4;
 
 template <int D>
 struct DecodeCfg {
   static constexpr int kBoxes = D / 64;                 // 64-channel TMA boxes per row
   static constexpr int kBoxBytes = 64 * 128;            // 64 rows x 128 bytes
   static constexpr int kKVBytes = kBoxes * kBoxBytes;   // one K (or V) page
-  static constexpr int kStageBytes = 2 * kKVBytes;
-  static constexpr int kSmemBytes = kDecodeStages * kStageBytes + 1024;   // + alignment slack
+  // stage = K page | V page | q rows of the group (rounded up to 1 KB)
+  __host__ __device__ static int stage_bytes(int G) { return 2 * kKVBytes + ((G * D * 2 + 1023) / 1024) * 1024; }
+  __host__ __device__ static int smem_bytes(int G) { return kDecodeStages * stage_bytes(G) + 1024; }   // + alignment slack
 };
 
+// CTA owning flat position f: the largest c with floor(c T / P) <= f.  With
+// P <= T no share is empty, so the owners of a range are every CTA between the
+// owners of its ends.
+__host__ __device__ __forceinline__ int flat_owner(long long f, long long T, long long P) {
+  return static_cast<int>(((f + 1) * P + T - 1) / T - 1);
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// By one block of 1024 threads, once every unit's selection is written.
+// off[u] = sum_{u' < u} min(sel_n[u'], kcap), off[units] = T; with Re = min(R, T)
+// ranges sharing the pages, range_unit[r] = unit holding flat position
+// floor(r T / Re) for r < Re; the range counter zeroed for the attention
+// kernel.  Units with nothing selected get their output here: out = 0, lse = -inf.
+__device__ __forceinline__ void decode_partition(const int32_t* sel_n, int units, int kcap, int R, int G, int D,
+                                                 int32_t* off, int32_t* range_unit, int32_t* range_counter,
+                                                 bf16* out, float* lse_out) {
+  __shared__ int s_warp[32];
+  __shared__ int s_carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
+  for (int base = 0; base < units; base += 1024) {
+    const int u = base + tid;
+    const int v = u < units ? min(max(__ldcg(sel_n + u), 0), kcap) : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = s_warp[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      s_warp[lane] = w;
+    }
+    __syncthreads();
+    const int carry = s_carry;
+    if (u < units) off[u] = carry + (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
+    __syncthreads();
+    if (tid == 1023) s_carry = carry + s_warp[31];
+    __syncthreads();
+  }
+  const long long T = s_carry;
+  if (tid == 0) {
+    off[units] = static_cast<int>(T);
+    *range_counter = 0;
+  }
+  __syncthreads();   // off[] of this block is visible to the block from here on
+  const long long Re = min(static_cast<long long>(R), T);   // every range below Re gets >= 1 page
+  for (int u = tid; u < units; u += 1024) {
+    const long long a = off[u], e = off[u + 1];
+    if (e == a) {   // nothing selected: out = 0, lse = -inf
+      for (int idx = 0; idx < G * D; idx += 8)
+        *reinterpret_cast<uint4*>(out + static_cast<long>(u) * G * D + idx) = make_uint4(0u, 0u, 0u, 0u);
+      if (lse_out)
+        for (int h = 0; h < G; ++h) lse_out[static_cast<long>(u) * G + h] = kNegInf;
+      continue;
+    }
+    // ranges whose share starts inside [a, e): ceil(a Re / T) .. ceil(e Re / T) - 1
+    const int r0 = static_cast<int>((a * Re + T - 1) / T);
+    const int r1 = static_cast<int>((e * Re + T - 1) / T) - 1;
+    for (int r = r0; r <= r1; ++r) range_unit[r] = u;
+  }
+}
+
+// One CTA of 1024 threads after the top-k grid (whose sel_n it reads after the
+// dependency wait, with L2 loads).
+__global__ void __launch_bounds__(1024) decode_partition_kernel(const int32_t* sel_n, int units, int kcap, int R,
+                                                                int G, int D, int32_t* off, int32_t* range_unit,
+                                                                int32_t* range_counter, bf16* out, float* lse_out) {
+  pdl_launch_dependents();   // the attention grid may get resident; it waits for this grid
+  pdl_wait();
+  decode_partition(sel_n, units, kcap, R, G, D, off, range_unit, range_counter, out, lse_out);
+}
+
+// Spin (with short sleeps) until cond() holds; false (and LSERVE_ERR_DEVICE_TIMEOUT
+// recorded) once timeout_ns has passed.
+template <typename F>
+__device__ __forceinline__ bool spin_until(F&& cond, uint64_t timeout_ns) {
+  if (cond()) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < 32; ++i) {
+      if (cond()) return true;
+      __nanosleep(32);
+    }
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      report(LSERVE_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 template <int D>
-__global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(
+__global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const bf16* __restrict__ q, const int32_t* __restrict__ page_table, int maxP,
     const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind,
-    const int32_t* __restrict__ sel, const int32_t* __restrict__ sel_n, int kcap, int pages_per_split,
-    int nsplit, int Hkv, int G, int num_pages, int sink, int local, float scale_log2,
-    unsigned long long timeout_ns, float* __restrict__ part_o, float* __restrict__ part_lse,
-    int32_t* __restrict__ done_count, bf16* __restrict__ out, float* __restrict__ lse_out) {
+    const int32_t* sel, const int32_t* off, const int32_t* range_unit, int32_t* range_counter, int R,
+    int kcap, int units, int Hkv, int G, int num_pages, int sink, int local, float scale_log2,
+    unsigned long long timeout_ns, float* __restrict__ part_o, float* __restrict__ part_lse) {
   using Cfg = DecodeCfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kDecodeStages];
+  __shared__ __align__(8) uint64_t full_bar[kDecodeStages];    // stage loaded (issuer's expect_tx + bytes)
+  __shared__ __align__(8) uint64_t empty_bar[kDecodeStages];   // stage consumed (one arrive per consumer warp)
+  __shared__ int4 s_meta[kMetaRing];   // {unit, logical page, physical page (-1: invalid), seq_len << 3 | flags}
+  __shared__ int4 s_seg[kMetaRing];    // {range, first range of the unit, last range of the unit, -}
+  __shared__ int s_resolved;           // pages whose metadata is in the ring
+  __shared__ int s_total;              // pages this CTA processes (INT_MAX until the ranges run out)
+  __shared__ int s_issued;             // pages whose loads were issued
+  __shared__ int s_abort;              // a bounded wait ran out or the plan was inconsistent
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-  const int unit = blockIdx.y;   // b * Hkv + g
-  const int split = blockIdx.x;
-  const int b = unit / Hkv, g = unit % Hkv;
+  const int stage_bytes = Cfg::stage_bytes(G);
+  const int q_bytes = G * D * 2;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  pdl_wait();   // the selection comes from the previous kernel
-  const int n_sel = min(sel_n[unit], kcap);
-  const int p_begin = split * pages_per_split;
-  if (n_sel == 0 && split == 0) {   // nothing to attend to: out = 0, lse = -inf
-    for (int idx = tid; idx < G * D; idx += kDecodeThreads) {
-      const long bh = static_cast<long>(b) * Hkv * G + static_cast<long>(g) * G + idx / D;
-      out[bh * D + idx % D] = __float2bfloat16_rn(0.f);
-      if (lse_out && idx % D == 0) lse_out[bh] = kNegInf;
-    }
-    return;
-  }
-  if (p_begin >= n_sel) return;
-  const int n_my = min(pages_per_split, n_sel - p_begin);
-  const int L = seq_lens[b];
-  const bool streaming = head_kind[g] != LSERVE_HEAD_DENSE;
-  const int32_t* my_sel = sel + static_cast<long>(unit) * kcap + p_begin;
-
   if (tid == 0) {
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
-    for (int s = 0; s < kDecodeStages; ++s) mbar_init(&full_bar[s], 1);
+    for (int s = 0; s < kDecodeStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kDecodeWarps);
+    }
     fence_barrier_init();
+    s_resolved = 0;
+    s_total = INT_MAX;
+    s_issued = 0;
+    s_abort = 0;
   }
   __syncthreads();
-
-  // physical page of selection entry `it`, or -1 when out of range
-  auto phys_page = [&](int it) -> int {
-    const int pidx = my_sel[it];
-    if (pidx < 0 || pidx >= maxP) return -1;
-    const int p = page_table[static_cast<long>(b) * maxP + pidx];
-    return (p >= 0 && p < num_pages) ? p : -1;
-  };
-  auto issue = [&](int it) {
-    const int st = it % kDecodeStages;
-    int p = phys_page(it);
-    if (p < 0) {
-      report(LSERVE_ERR_DEVICE_BOUNDS);
-      p = 0;   // load a harmless in-range page; every token of it is masked below
-    }
-    uint8_t* kdst = smem + st * Cfg::kStageBytes;
-    uint8_t* vdst = kdst + Cfg::kKVBytes;
-    mbar_arrive_expect_tx(&full_bar[st], Cfg::kStageBytes);
-    const int row = (p * Hkv + g) * kPage;
-#pragma unroll
-    for (int x = 0; x < Cfg::kBoxes; ++x) {
-      tma_load_2d(kdst + x * Cfg::kBoxBytes, &tmK, &full_bar[st], x * 64, row);
-      tma_load_2d(vdst + x * Cfg::kBoxBytes, &tmV, &full_bar[st], x * 64, row);
-    }
-  };
-  if (tid == 0)
-    for (int it = 0; it < min(kDecodeStages, n_my); ++it) issue(it);
-
-  // Q as the A operand: rows = the G query heads of the group (zero-padded to 16)
-  constexpr int KS = D / 16;
-  uint32_t qa[KS][4];
-  {
-    const int r = lane >> 2, c = 2 * (lane & 3);
-    const bf16* qb = q + (static_cast<long>(b) * Hkv * G + static_cast<long>(g) * G) * D;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      qa[ks][0] = r < G ? __ldg(reinterpret_cast<const uint32_t*>(qb + r * D + ks * 16 + c)) : 0u;
-      qa[ks][2] = r < G ? __ldg(reinterpret_cast<const uint32_t*>(qb + r * D + ks * 16 + 8 + c)) : 0u;
-      qa[ks][1] = r + 8 < G ? __ldg(reinterpret_cast<const uint32_t*>(qb + (r + 8) * D + ks * 16 + c)) : 0u;
-      qa[ks][3] = r + 8 < G ? __ldg(reinterpret_cast<const uint32_t*>(qb + (r + 8) * D + ks * 16 + 8 + c)) : 0u;
-    }
-  }
-
-  float acc[D / 8][4];
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-  float m_run[2] = {kNegInf, kNegInf}, l_run[2] = {0.f, 0.f};
-  const int mi = lane >> 3, rr = lane & 7;
-
-  bool timed_out = false;
-  for (int it = 0; it < n_my; ++it) {
-    const int st = it % kDecodeStages;
-    const uint32_t parity = (it / kDecodeStages) & 1;
-    if (!mbar_wait_bounded(&full_bar[st], parity, timeout_ns)) timed_out = true;
-    const uint8_t* ks_base = smem + st * Cfg::kStageBytes;
-    const uint8_t* vs_base = ks_base + Cfg::kKVBytes;
-    const int pidx = my_sel[it];
-    const bool page_ok = phys_page(it) >= 0;
-    const int t_warp = pidx * kPage + warp * 16;   // first token of this warp's slice
-
-    // ---- S = Q K^T for this warp's 16 tokens (two n-tiles of 8)
-    float s[2][4];
-#pragma unroll
-    for (int n = 0; n < 2; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const int box = ks >> 2, chunk = (ks & 3) * 2 + (mi & 1);
-      const int row = warp * 16 + (mi >> 1) * 8 + rr;
-      uint32_t b0, b1, b2, b3;
-      ldmatrix_x4(smem_u32(ks_base + box * Cfg::kBoxBytes + swz128(row, chunk)), b0, b1, b2, b3);
-      mma_bf16_16816(s[0], qa[ks], b0, b1);
-      mma_bf16_16816(s[1], qa[ks], b2, b3);
-    }
-    // ---- mask + online softmax (rows lane/4 and lane/4 + 8)
-    const int tc = 2 * (lane & 3);
-    auto valid = [&](int t) -> bool {
-      return page_ok && t < L && (!streaming || t < sink || t >= L - local);
-    };
-    bool all_valid = true;
-    float mloc[2] = {kNegInf, kNegInf};
-#pragma unroll
-    for (int n = 0; n < 2; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int t = t_warp + n * 8 + tc + (e & 1);
-        const bool ok = valid(t);
-        all_valid &= ok;
-        s[n][e] = ok ? s[n][e] * scale_log2 : kNegInf;
-        mloc[e >> 1] = fmaxf(mloc[e >> 1], s[n][e]);
-      }
-    float corr[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      mloc[h] = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], 1));
-      mloc[h] = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], 2));
-      const float m_new = fmaxf(m_run[h], mloc[h]);
-      const float m_use = m_new == kNegInf ? 0.f : m_new;
-      corr[h] = fast_exp2(m_run[h] - m_use);
-      m_run[h] = m_new;
-      mloc[h] = m_use;
-    }
-    float psum[2] = {0.f, 0.f};
-#pragma unroll
-    for (int n = 0; n < 2; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        s[n][e] = fast_exp2(s[n][e] - mloc[e >> 1]);
-        psum[e >> 1] += s[n][e];
-      }
-    l_run[0] = l_run[0] * corr[0] + psum[0];
-    l_run[1] = l_run[1] * corr[1] + psum[1];
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      acc[n][0] *= corr[0];
-      acc[n][1] *= corr[0];
-      acc[n][2] *= corr[1];
-      acc[n][3] *= corr[1];
-    }
-    // ---- O += P V
-    uint32_t pa[4];
-    pa[0] = pack_bf16x2(s[0][0], s[0][1]);
-    pa[1] = pack_bf16x2(s[0][2], s[0][3]);
-    pa[2] = pack_bf16x2(s[1][0], s[1][1]);
-    pa[3] = pack_bf16x2(s[1][2], s[1][3]);
-    const bool warp_all_valid = __all_sync(0xffffffffu, all_valid);
-    uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;   // zero V of masked tokens (may hold NaN)
-    if (!warp_all_valid) {
-      const int t0 = t_warp + tc;
-      vm0 = (valid(t0) ? 0x0000ffffu : 0u) | (valid(t0 + 1) ? 0xffff0000u : 0u);
-      vm1 = (valid(t0 + 8) ? 0x0000ffffu : 0u) | (valid(t0 + 9) ? 0xffff0000u : 0u);
-    }
-#pragma unroll
-    for (int np = 0; np < D / 16; ++np) {
-      const int ch = np * 16 + (mi >> 1) * 8;   // first channel of this lane's matrix
-      const int row = warp * 16 + (mi & 1) * 8 + rr;
-      uint32_t b0, b1, b2, b3;
-      ldmatrix_x4_trans(smem_u32(vs_base + (ch >> 6) * Cfg::kBoxBytes + swz128(row, (ch & 63) >> 3)), b0, b1,
-                        b2, b3);
-      b0 &= vm0;
-      b1 &= vm1;
-      b2 &= vm0;
-      b3 &= vm1;
-      mma_bf16_16816(acc[2 * np], pa, b0, b1);
-      mma_bf16_16816(acc[2 * np + 1], pa, b2, b3);
-    }
-    // ---- release the stage and refill it
-    if (__syncthreads_or(timed_out)) {
-      timed_out = true;
-      break;
-    }
-    if (tid == 0 && it + kDecodeStages < n_my) issue(it + kDecodeStages);
-  }
-  if (timed_out) {
-    // let every load this CTA issued land before the CTA (and its smem) goes away
-    if (tid == 0) {
-      for (int it = 0; it < n_my; ++it) {
-        const int st = it % kDecodeStages;
-        mbar_wait_bounded(&full_bar[st], (it / kDecodeStages) & 1, timeout_ns);
-      }
-    }
-    __syncthreads();
+  volatile int* v_resolved = &s_resolved;
+  volatile int* v_total = &s_total;
+  volatile int* v_issued = &s_issued;
+  volatile int* v_abort = &s_abort;
+  // off / range_unit / the selection come from the previous kernels, which may
+  // still be running: they are read only after this wait, with L2 loads through
+  // pointers that are not restrict-qualified (no load of them can move above it).
+  pdl_wait();
+  const long long T = __ldcg(off + units);
+  if (T <= 0 || T > static_cast<long long>(units) * kcap) {   // nothing selected anywhere, or a bad plan
+    if (T != 0 && tid == 0) report(LSERVE_ERR_DEVICE_BOUNDS);
     return;
   }
+  const long long Re = min(static_cast<long long>(R), T);   // ranges that hold pages
 
-  // ---- merge the 4 warps' states through shared memory (the ring is idle now)
-  float* o_w = reinterpret_cast<float*>(smem);           // [4][16][D]
-  float* m_w = o_w + 4 * 16 * D;                          // [4][16]
-  float* l_w = m_w + 4 * 16;                              // [4][16]
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
-    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
-  }
-  {
-    const int r = lane >> 2, c = 2 * (lane & 3);
-    if ((lane & 3) == 0) {
-      m_w[warp * 16 + r] = m_run[0];
-      m_w[warp * 16 + r + 8] = m_run[1];
-      l_w[warp * 16 + r] = l_run[0];
-      l_w[warp * 16 + r + 8] = l_run[1];
-    }
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      if (r < G) *reinterpret_cast<float2*>(&o_w[(warp * 16 + r) * D + n * 8 + c]) = make_float2(acc[n][0], acc[n][1]);
-      if (r + 8 < G)
-        *reinterpret_cast<float2*>(&o_w[(warp * 16 + r + 8) * D + n * 8 + c]) = make_float2(acc[n][2], acc[n][3]);
-    }
-  }
-  __syncthreads();
-  const long part = static_cast<long>(unit) * nsplit + split;
-  for (int idx = tid; idx < G * D; idx += kDecodeThreads) {
-    const int h = idx / D, c = idx % D;
-    float m = kNegInf;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) m = fmaxf(m, m_w[w * 16 + h]);
-    float o = 0.f, l = 0.f;
-    if (m != kNegInf) {
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float sc = fast_exp2(m_w[w * 16 + h] - m);
-        o += sc * o_w[(w * 16 + h) * D + c];
-        l += sc * l_w[w * 16 + h];
+  if (warp == kResolverWarp) {
+    // ---- claim ranges one after another and resolve their pages into the ring.
+    // Window: unit wu + l (lane l) ends at flat position wend (INT_MAX past the
+    // last unit); the window is shifted so that it always starts at the unit of
+    // the next page to resolve.
+    int gp = 0;   // pages resolved
+    bool ok = true;
+    while (ok) {
+      int r = 0;
+      if (lane == 0) r = atomicAdd(range_counter, 1);
+      r = __shfl_sync(0xffffffffu, r, 0);
+      if (r >= Re) break;
+      const int lo = static_cast<int>(r * T / Re), hi = static_cast<int>((r + 1) * T / Re);
+      int wu = __ldcg(range_unit + r);
+      if (wu < 0 || wu >= units) {
+        ok = false;
+        break;
+      }
+      int wstart = __ldcg(off + wu);
+      int wend = wu + lane < units ? __ldcg(off + wu + lane + 1) : INT_MAX;
+      int f0 = lo;
+      while (f0 < hi && ok) {
+        // shift the window to the unit of f0
+        int k0 = 0;
+#pragma unroll 8
+        for (int l = 0; l < 32; ++l) k0 += __shfl_sync(0xffffffffu, wend, l) <= f0;
+        if (k0 > 0) {
+          wu += k0;
+          if (wu >= units) {
+            ok = false;
+            break;
+          }
+          wstart = __ldcg(off + wu);
+          wend = wu + lane < units ? __ldcg(off + wu + lane + 1) : INT_MAX;
+          continue;
+        }
+        if (wstart > f0) {
+          ok = false;
+          break;
+        }
+        // page f of this lane lies in unit wu + k (k < 32 inside the window)
+        const int f = f0 + lane;
+        int k = 0;
+#pragma unroll 8
+        for (int l = 0; l < 32; ++l) k += __shfl_sync(0xffffffffu, wend, l) <= f;
+        const int kk = min(k, 31);
+        const int end_k = __shfl_sync(0xffffffffu, wend, kk);
+        const int prev_end = __shfl_sync(0xffffffffu, wend, max(kk - 1, 0));
+        const bool act = f < hi && k < 32;   // a prefix of the lanes
+        const int cnt = __popc(__ballot_sync(0xffffffffu, act));
+        // ring entries gp .. gp + cnt - 1 are free once page (entry - ring) is past the consumers
+        bool room = true;
+        if (lane == 0)
+          room = spin_until([&] { return *v_issued >= gp + cnt - kMetaRing + kDecodeStages || *v_abort; },
+                            timeout_ns) && !*v_abort;
+        if (!__shfl_sync(0xffffffffu, room, 0)) {
+          ok = false;
+          break;
+        }
+        bool bad = false;
+        if (act) {
+          const int u = wu + k;
+          const int start = k == 0 ? wstart : prev_end;
+          const int j = f - start, n_u = end_k - start;
+          bad = j < 0 || j >= n_u || n_u > kcap;
+          int pidx = -1, phys = -1, flags = 0, L = 0;
+          int c_first = 0, c_last = -1;
+          if (!bad) {
+            const int b = u / Hkv, g = u % Hkv;
+            pidx = __ldcg(sel + static_cast<long>(u) * kcap + j);
+            if (pidx >= 0 && pidx < maxP) {
+              const int p = page_table[static_cast<long>(b) * maxP + pidx];
+              if (p >= 0 && p < num_pages) phys = p;
+            }
+            if (phys < 0) report(LSERVE_ERR_DEVICE_BOUNDS);
+            L = seq_lens[b];
+            flags = ((j == 0 || f == lo) ? kSegStart : 0) | ((j == n_u - 1 || f == hi - 1) ? kSegEnd : 0) |
+                    (head_kind[g] != LSERVE_HEAD_DENSE ? kSegStreaming : 0);
+            c_first = flat_owner(start, T, Re);
+            c_last = flat_owner(start + n_u - 1, T, Re);
+          }
+          const int e = (gp + lane) % kMetaRing;
+          s_meta[e] = make_int4(u, pidx, phys, (max(L, 0) << 3) | flags);
+          s_seg[e] = make_int4(r, c_first, c_last, 0);
+        }
+        if (__any_sync(0xffffffffu, bad)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        __threadfence_block();
+        gp += cnt;
+        f0 += cnt;
+        if (lane == 0) *v_resolved = gp;
       }
     }
-    const bool has = m != kNegInf && l > 0.f;
-    part_o[(part * G + h) * D + c] = has ? o / l : 0.f;
-    if (c == 0) part_lse[part * G + h] = has ? m + __log2f(l) : kNegInf;
-  }
-  // ---- the last split of this (sequence, KV head) to finish merges all splits:
-  // out = sum_s w_s o_s with w_s = 2^(lse_s - lse), lse = log2 sum_s 2^lse_s
-  __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  const int ns = (n_sel + pages_per_split - 1) / pages_per_split;
-  if (tid == 0) s_last = atomicAdd(&done_count[unit], 1) == ns - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // per query head: m = max_s lse_s, lse = m + log2 sum_s 2^(lse_s - m); warp w owns heads w, w + 4, ...
-  __shared__ float s_lse[16];
-  const long base = static_cast<long>(unit) * nsplit;
-  for (int hh = warp; hh < G; hh += 4) {
-    float m = kNegInf;
-    for (int sp = lane; sp < ns; sp += 32) m = fmaxf(m, __ldcg(&part_lse[(base + sp) * G + hh]));
+    if (lane == 0) {
+      if (!ok) {
+        report(LSERVE_ERR_DEVICE_BOUNDS);
+        *v_abort = 1;
+      }
+      __threadfence_block();
+      *v_total = gp;
+    }
+  } else if (warp == kIssuerWarp) {
+    // ---- issue each resolved page's loads once its stage is free
+    if (lane == 0) {
+      for (int gp = 0;; ++gp) {
+        if (!spin_until([&] { return *v_resolved > gp || *v_total <= gp || *v_abort; }, timeout_ns)) {
+          *v_abort = 1;
+          break;
+        }
+        if (*v_resolved <= gp || *v_abort) break;   // no page gp: the ranges ran out
+        __threadfence_block();
+        const int st = gp % kDecodeStages;
+        if (gp >= kDecodeStages && !mbar_wait_bounded(&empty_bar[st], ((gp / kDecodeStages) - 1) & 1, timeout_ns)) {
+          *v_abort = 1;
+          break;
+        }
+        const int4 md = s_meta[gp % kMetaRing];
+        const int g = md.x % Hkv;
+        const int p = md.z >= 0 ? md.z : 0;   // an invalid page loads page 0; all its tokens are masked
+        uint8_t* kdst = smem + st * stage_bytes;
+        uint8_t* vdst = kdst + Cfg::kKVBytes;
+        const bool with_q = md.w & kSegStart;
+        mbar_arrive_expect_tx(&full_bar[st], 2 * Cfg::kKVBytes + (with_q ? q_bytes : 0));
+        const int row = (p * Hkv + g) * kPage;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float l = 0.f;
-    if (m != kNegInf)
-      for (int sp = lane; sp < ns; sp += 32) l += fast_exp2(__ldcg(&part_lse[(base + sp) * G + hh]) - m);
+        for (int x = 0; x < Cfg::kBoxes; ++x) {
+          tma_load_2d(kdst + x * Cfg::kBoxBytes, &tmK, &full_bar[st], x * 64, row);
+          tma_load_2d(vdst + x * Cfg::kBoxBytes, &tmV, &full_bar[st], x * 64, row);
+        }
+        if (with_q) bulk_load(vdst + Cfg::kKVBytes, q + static_cast<long>(md.x) * G * D, q_bytes, &full_bar[st]);
+        *v_issued = gp + 1;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---- consumers.  Transposed tiles: S^T = K Q^T (M = the warp's 16 tokens,
+    // N = 8 query heads, K = channels) and O^T += V^T P^T (M = channels, N =
+    // heads, K = tokens), so the G <= 8 heads fill N exactly.  A lane holds
+    // heads tc, tc + 1 of the tile.
+    constexpr int KS = D / 16;
+    uint32_t qb[KS][2];                   // Q^T as the B operand (heads >= G are zero)
+    float acc[D / 16][4];                 // O^T: m-tile mt = channels 16 mt .. 16 mt + 15
+    float m_run[2], l_run[2];             // online softmax of heads tc, tc + 1
+    const int mi = lane >> 3, rr = lane & 7;
+    const int qr = lane >> 2, tc = 2 * (lane & 3);
+    for (int gp = 0;; ++gp) {
+      bool have = false;
+      if (lane == 0)
+        have = spin_until([&] { return *v_resolved > gp || *v_total <= gp || *v_abort; }, timeout_ns) &&
+               *v_resolved > gp && !*v_abort;
+      if (!__shfl_sync(0xffffffffu, have, 0)) break;
+      const int st = gp % kDecodeStages;
+      const bool landed = mbar_wait_bounded(&full_bar[st], (gp / kDecodeStages) & 1, timeout_ns);
+      if (__any_sync(0xffffffffu, !landed || *v_abort != 0)) {
+        if (lane == 0) *v_abort = 1;
+        break;
+      }
+      const int4 md = s_meta[gp % kMetaRing];
+      const int4 sg = s_seg[gp % kMetaRing];
+      const int u = md.x, pidx = md.y;
+      const bool page_ok = md.z >= 0, streaming = md.w & kSegStreaming;
+      const int L = md.w >> 3;
+      const uint8_t* ks_base = smem + st * stage_bytes;
+      const uint8_t* vs_base = ks_base + Cfg::kKVBytes;
+      if (md.w & kSegStart) {
+        const uint8_t* qs = vs_base + Cfg::kKVBytes;   // [G][D] bf16, row-major
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) s_lse[hh] = (m != kNegInf && l > 0.f) ? m + __log2f(l) : kNegInf;
+        for (int ks = 0; ks < KS; ++ks) {   // lane: head qr, channels 16 ks + tc, +1 and + 8, + 9
+          const int c0 = ks * 16 + tc;
+          qb[ks][0] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c0) * 2) : 0u;
+          qb[ks][1] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c0 + 8) * 2) : 0u;
+        }
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+        m_run[0] = m_run[1] = kNegInf;
+        l_run[0] = l_run[1] = 0.f;
+      }
+      const int t_warp = pidx * kPage + warp * 16;   // first token of this warp's slice
+
+      // ---- this warp's K and V fragments into registers, then the stage goes back
+      // to the producer at once: the ring spends its time loading, not waiting for math
+      uint32_t kf[KS][4], vf[D / 16][4];
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {   // K as the A operand of S^T: rows = tokens, k = channels
+        const int box = ks >> 2, chunk = (ks & 3) * 2 + (lane >> 4);
+        const int row = warp * 16 + (mi & 1) * 8 + rr;
+        ldmatrix_x4(smem_u32(ks_base + box * Cfg::kBoxBytes + swz128(row, chunk)), kf[ks][0], kf[ks][1], kf[ks][2],
+                    kf[ks][3]);
+      }
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {   // V^T as the A operand of O^T: rows = channels, k = tokens
+        const int ch = mt * 16 + (mi & 1) * 8;   // channels of this lane's 8x8 source block
+        const int row = warp * 16 + (mi >> 1) * 8 + rr;
+        ldmatrix_x4_trans(smem_u32(vs_base + (ch >> 6) * Cfg::kBoxBytes + swz128(row, (ch & 63) >> 3)), vf[mt][0],
+                          vf[mt][1], vf[mt][2], vf[mt][3]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[st]);   // release orders the shared-memory reads above
+
+      // ---- S^T = K Q^T: 16 tokens x 8 heads; alternate k-steps feed two accumulators
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        if (ks & 1)
+          mma_bf16_16816(sb, kf[ks], qb[ks][0], qb[ks][1]);
+        else
+          mma_bf16_16816(sa, kf[ks], qb[ks][0], qb[ks][1]);
+      }
+      // ---- mask + online softmax.  Element e: token t_warp + qr + 8 (e >> 1), head tc + (e & 1)
+      auto valid = [&](int t) -> bool {
+        return page_ok && t < L && (!streaming || t < sink || t >= L - local);
+      };
+      const bool ok0 = valid(t_warp + qr), ok1 = valid(t_warp + qr + 8);
+      float p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) p[e] = ((e >> 1) ? ok1 : ok0) ? (sa[e] + sb[e]) * scale_log2 : kNegInf;
+      // per-head max over the 16 tokens: the lanes with one lane % 4 hold one head pair
+      float mh[2] = {fmaxf(p[0], p[2]), fmaxf(p[1], p[3])};
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mh[0] = fmaxf(mh[0], __shfl_xor_sync(0xffffffffu, mh[0], o));
+        mh[1] = fmaxf(mh[1], __shfl_xor_sync(0xffffffffu, mh[1], o));
+      }
+      float corr[2], m_use[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float m_new = fmaxf(m_run[h], mh[h]);
+        m_use[h] = m_new == kNegInf ? 0.f : m_new;
+        corr[h] = fast_exp2(m_run[h] - m_use[h]);
+        m_run[h] = m_new;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) p[e] = fast_exp2(p[e] - m_use[e & 1]);
+      l_run[0] = l_run[0] * corr[0] + p[0] + p[2];   // lane-partial sums; reduced at the segment's end
+      l_run[1] = l_run[1] * corr[1] + p[1] + p[3];
+      if (__any_sync(0xffffffffu, corr[0] != 1.f || corr[1] != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          acc[mt][0] *= corr[0];
+          acc[mt][1] *= corr[1];
+          acc[mt][2] *= corr[0];
+          acc[mt][3] *= corr[1];
+        }
+      }
+      // ---- P^T as the B operand (k = tokens, n = heads): transpose the two 8x8 blocks
+      const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p[0], p[1]));   // tokens 0..7
+      const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p[2], p[3]));   // tokens 8..15
+      // ---- O^T += V^T P^T.  V^T fragments hold tokens tc, tc + 1 (a0, a1) and tc + 8, + 9
+      // (a2, a3) of the slice; rows of masked tokens are zeroed (the pool may hold NaN there)
+      uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
+      if (!__all_sync(0xffffffffu, ok0 && ok1)) {
+        const int t0 = t_warp + tc;
+        vm0 = (valid(t0) ? 0x0000ffffu : 0u) | (valid(t0 + 1) ? 0xffff0000u : 0u);
+        vm1 = (valid(t0 + 8) ? 0x0000ffffu : 0u) | (valid(t0 + 9) ? 0xffff0000u : 0u);
+      }
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        vf[mt][0] &= vm0;
+        vf[mt][1] &= vm0;
+        vf[mt][2] &= vm1;
+        vf[mt][3] &= vm1;
+        mma_bf16_16816(acc[mt], vf[mt], pb0, pb1);
+      }
+
+      // ---- end of a segment: this warp's partial, and the merge if it completes the unit
+      if (md.w & kSegEnd) {
+        const int vr = sg.x, c_first = sg.y, c_last = sg.z;   // this range; the unit's first and last range
+        const bool slots_ok = c_first >= 0 && c_first <= vr && vr <= c_last && c_last < Re;
+        // (slot vr + u of every range of the unit is read by decode_merge_kernel)
+        // l of heads tc, tc + 1: sum over the 8 lanes that share lane % 4
+        float lh[2] = {l_run[0], l_run[1]};
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          lh[0] += __shfl_xor_sync(0xffffffffu, lh[0], o);
+          lh[1] += __shfl_xor_sync(0xffffffffu, lh[1], o);
+        }
+        const long pbase = (static_cast<long>(vr + u) * kDecodeWarps + warp) * G;   // this warp's partial
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int h = tc + h2;
+          if (h < G && slots_ok) {
+            const bool has = m_run[h2] != kNegInf && lh[h2] > 0.f;
+            const float inv = has ? 1.f / lh[h2] : 0.f;
+            float* po = part_o + (pbase + h) * D + qr;
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+              po[mt * 16] = acc[mt][h2] * inv;
+              po[mt * 16 + 8] = acc[mt][2 + h2] * inv;
+            }
+            if (qr == 0) part_lse[pbase + h] = has ? m_run[h2] + __log2f(lh[h2]) : kNegInf;
+          }
+        }
+        if (!slots_ok && lane == 0) report(LSERVE_ERR_DEVICE_BOUNDS);
+      }
+    }
   }
   __syncthreads();
-  // out = sum_s 2^(lse_s - lse) o_s, four channels per thread; the split loads are independent
-  for (int idx = tid * 4; idx < G * D; idx += kDecodeThreads * 4) {
-    const int hh = idx / D, c = idx % D;
-    const float lse_h = s_lse[hh];
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (lse_h != kNegInf) {
+  if (*v_abort && warp == kIssuerWarp && lane == 0) {
+    // let every load this CTA issued land before the CTA (and its smem) goes away;
+    // the last kDecodeStages issued pages sit in distinct stages, earlier ones have landed
+    const int issued = *v_issued;
+    for (int gp = max(0, issued - kDecodeStages); gp < issued; ++gp)
+      mbar_wait_bounded(&full_bar[gp % kDecodeStages], (gp / kDecodeStages) & 1, timeout_ns);
+  }
+}
+
+// One CTA per unit, after the attention grid: out = sum_i 2^(lse_i - lse) o_i,
+// lse = log2 sum_i 2^lse_i over the unit's per-warp partials (slots c_first(u)
+// + u .. c_last(u) + u, 4 warp partials each).  The threads split into groups
+// over the partials; a thread keeps a running (max, sum, vector) of one float4
+// of the output over its group's partials -- a single pass whose loads do not
+// depend on one another -- and the groups are combined through shared memory.
+constexpr int kMergeThreads = 1024;
+
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const int32_t* off, int units, int R, int G, int D,
+                                                                     const float* part_o, const float* part_lse,
+                                                                     bf16* __restrict__ out,
+                                                                     float* __restrict__ lse_out) {
+  __shared__ float4 s_o[kMergeThreads];
+  __shared__ float2 s_ml[kMergeThreads];
+  pdl_wait();   // the partials come from the attention grid: read after this, with L2 loads
+  const int u = blockIdx.x;
+  const long long T = __ldcg(off + units);
+  const long long a = __ldcg(off + u), e = __ldcg(off + u + 1);
+  if (T <= 0 || e <= a) return;   // nothing selected: written by the partition kernel
+  const long long Re = min(static_cast<long long>(R), T);
+  const int c_first = flat_owner(a, T, Re), c_last = flat_owner(e - 1, T, Re);
+  if (c_first < 0 || c_last < c_first || c_last >= Re) {
+    if (threadIdx.x == 0) report(LSERVE_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  const long first = static_cast<long>(c_first + u) * kDecodeWarps;   // first partial of the unit
+  const int nparts = (c_last - c_first + 1) * kDecodeWarps;
+  const int tid = threadIdx.x;
+  const int n4 = G * D / 4;   // float4s of the unit's output (<= 256)
+  const int groups = kMergeThreads / n4;
+  const int pg = tid / n4, q4 = tid % n4, h = q4 * 4 / D;
+  float m = kNegInf, l = 0.f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (pg < groups) {
+    const float4* po = reinterpret_cast<const float4*>(part_o) + first * n4 + q4;
 #pragma unroll 4
-      for (int sp = 0; sp < ns; ++sp) {
-        const float w = fast_exp2(__ldcg(&part_lse[(base + sp) * G + hh]) - lse_h);
-        const float4 x = __ldcg(reinterpret_cast<const float4*>(&part_o[((base + sp) * G + hh) * D + c]));
-        o.x += w * x.x;
-        o.y += w * x.y;
-        o.z += w * x.z;
-        o.w += w * x.w;
-      }
+    for (int x = pg; x < nparts; x += groups) {
+      const float lx = __ldcg(part_lse + (first + x) * G + h);
+      const float4 v = __ldcg(po + static_cast<long>(x) * n4);
+      if (lx == kNegInf) continue;   // an empty partial (its o is 0)
+      const float mn = fmaxf(m, lx);
+      const float sc = fast_exp2(m - mn), w = fast_exp2(lx - mn);
+      m = mn;
+      l = l * sc + w;
+      o.x = o.x * sc + w * v.x;
+      o.y = o.y * sc + w * v.y;
+      o.z = o.z * sc + w * v.z;
+      o.w = o.w * sc + w * v.w;
     }
-    const long bh = static_cast<long>(b) * Hkv * G + static_cast<long>(g) * G + hh;
-    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + bh * D + c);
-    dst[0] = __floats2bfloat162_rn(o.x, o.y);
-    dst[1] = __floats2bfloat162_rn(o.z, o.w);
-    if (lse_out && c == 0) lse_out[bh] = lse_h == kNegInf ? kNegInf : lse_h * 0.6931471805599453f;
   }
-  if (tid == 0) done_count[unit] = 0;   // ready for the next call
+  s_o[tid] = o;
+  s_ml[tid] = make_float2(m, l);
+  __syncthreads();
+  if (tid < n4) {
+    float mm = kNegInf;
+    for (int gg = 0; gg < groups; ++gg) mm = fmaxf(mm, s_ml[gg * n4 + tid].x);
+    float ll = 0.f;
+    float4 oo = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (mm != kNegInf)
+      for (int gg = 0; gg < groups; ++gg) {
+        const float2 ml = s_ml[gg * n4 + tid];
+        if (ml.x == kNegInf) continue;
+        const float sc = fast_exp2(ml.x - mm);
+        const float4 v = s_o[gg * n4 + tid];
+        ll += ml.y * sc;
+        oo.x += v.x * sc;
+        oo.y += v.y * sc;
+        oo.z += v.z * sc;
+        oo.w += v.w * sc;
+      }
+    const bool has = mm != kNegInf && ll > 0.f;
+    const float inv = has ? 1.f / ll : 0.f;
+    const int c = tid * 4 % D;
+    const long bh = static_cast<long>(u) * G + h;
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + bh * D + c);
+    dst[0] = __floats2bfloat162_rn(oo.x * inv, oo.y * inv);
+    dst[1] = __floats2bfloat162_rn(oo.z * inv, oo.w * inv);
+    if (lse_out && c == 0) lse_out[bh] = has ? (mm + __log2f(ll)) * 0.6931471805599453f : kNegInf;
+  }
 }
 
 }  // namespace lserve

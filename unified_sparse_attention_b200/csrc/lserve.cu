@@ -239,15 +239,43 @@ bool use_legacy_prefill() {
 
 // ----------------------------------------------------------------- decode
 struct DecodePlan {
-  int kcap, budget_pages, pps, nsplit, G, ppb;
+  int kcap, budget_pages, G, ppb;
+  int P;                 // CTAs of the attention grid (one wave)
+  int R;                 // ranges of the flat page list (kRangesPerCta per CTA)
   float* scores;
   int32_t* sel;
   int32_t* sel_n;
-  float* part_o;
-  float* part_lse;
-  int32_t* done_count;   // per (b, kvh): finished splits (zeroed by the top-k kernel)
+  int32_t* off;          // [units + 1] flat offsets of the units' selections
+  int32_t* range_unit;   // [R] unit holding the first page of each range
+  int32_t* range_counter;   // next range to claim (zeroed by the partition step)
+  float* part_o;         // [R + units][4 warps][G][d]
+  float* part_lse;       // [R + units][4 warps][G]
   size_t bytes;
 };
+
+// Attention CTAs for the current device: SMs x resident CTAs per SM, or the
+// value of LSERVE_DECODE_GRID (a positive integer) when that is set.
+int decode_grid() {
+  if (const char* e = getenv("LSERVE_DECODE_GRID")) {
+    const long v = strtol(e, nullptr, 10);
+    if (v > 0 && v <= (1 << 20)) return static_cast<int>(v);
+  }
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 148 * kDecodeCtasPerSm;
+  }
+  if (!cached[dev]) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+      cudaGetLastError();
+      sms = 148;
+    }
+    cached[dev] = sms * kDecodeCtasPerSm;
+  }
+  return cached[dev];
+}
 
 // Launch with programmatic stream serialisation: the kernel may start while its
 // predecessor finishes and waits on griddepcontrol.wait before reading its output.
@@ -284,6 +312,12 @@ lserve_status validate_decode(const lserve_decode_args* a) {
   if (a->sink < 0 || a->local < 0) return fail(LSERVE_ERR_INVALID_ARG, "decode: sink/local must be >= 0");
   if (static_cast<long long>(a->num_pages) * a->Hkv * kPage > (1ll << 31) - 1)
     return fail(LSERVE_ERR_UNSUPPORTED, "decode: page pool too large for 32-bit TMA coordinates");
+  if (static_cast<long long>(a->B) * a->Hkv * std::max(1, std::min(a->maxP, std::max(a->token_budget / kPage,
+                                                                    streaming_page_bound(a->sink, a->local)))) >
+      (1ll << 31) - 1)
+    return fail(LSERVE_ERR_UNSUPPORTED, "decode: B * Hkv * selected pages exceeds 32-bit offsets");
+  if (static_cast<long long>(a->maxP) * kPage >= (1ll << 28))
+    return fail(LSERVE_ERR_UNSUPPORTED, "decode: maxP * 64 tokens must stay below 2^28");
   if (!a->q || !a->k_pages || !a->v_pages || !a->page_table || !a->seq_lens || !a->stats || !a->head_kind)
     return fail(LSERVE_ERR_INVALID_ARG, "decode: null tensor pointer");
   if (!aligned16(a->q) || !aligned16(a->k_pages) || !aligned16(a->v_pages) || !aligned16(a->stats))
@@ -297,11 +331,8 @@ DecodePlan plan_decode(const lserve_decode_args* a, void* ws) {
   p.budget_pages = a->token_budget / kPage;
   const int dense_cap = std::min(p.budget_pages, a->maxP);
   p.kcap = std::max(1, std::max(dense_cap, std::min(streaming_page_bound(a->sink, a->local), a->maxP)));
-  // split-KV: aim for ~8 CTAs per SM over the selections
-  const long long total = static_cast<long long>(a->B) * a->Hkv * p.kcap;
-  long long pps = (total + 8 * 148 - 1) / (8 * 148);
-  p.pps = static_cast<int>(std::max(2ll, std::min<long long>(pps, 64)));
-  p.nsplit = (p.kcap + p.pps - 1) / p.pps;
+  p.P = decode_grid();
+  p.R = kRangesPerCta * p.P;
   // scoring: aim for >= ~4 CTAs per SM
   const long long pages = static_cast<long long>(a->B) * a->maxP;
   long long ppb = pages / (4 * 148);
@@ -311,9 +342,11 @@ DecodePlan plan_decode(const lserve_decode_args* a, void* ws) {
   p.scores = c.take<float>(units * a->maxP);
   p.sel = c.take<int32_t>(units * p.kcap);
   p.sel_n = c.take<int32_t>(units);
-  p.part_o = c.take<float>(units * p.nsplit * p.G * a->d);
-  p.part_lse = c.take<float>(units * p.nsplit * p.G);
-  p.done_count = c.take<int32_t>(units);
+  p.off = c.take<int32_t>(units + 1);
+  p.range_unit = c.take<int32_t>(p.R);
+  p.range_counter = c.take<int32_t>(1);
+  p.part_o = c.take<float>((p.R + units) * kDecodeWarps * p.G * a->d);
+  p.part_lse = c.take<float>((p.R + units) * kDecodeWarps * p.G);
   p.bytes = c.used();
   return p;
 }
@@ -337,23 +370,32 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
   }
   ensure_smem(topk_pages_kernel, kTopkSmemKeys * static_cast<int>(sizeof(uint32_t)));
   const int topk_smem = std::min(a->maxP, kTopkSmemKeys) * static_cast<int>(sizeof(uint32_t));
-  if (launch_pdl(topk_pages_kernel, dim3(a->B * a->Hkv), dim3(kTopkThreads), topk_smem, st, p.scores, a->maxP,
-                 a->seq_lens, a->head_kind, a->Hkv, p.budget_pages, a->sink, a->local, sel, sel_n, p.kcap,
-                 p.done_count) != cudaSuccess)
+  const int units = a->B * a->Hkv;
+  if (launch_pdl(topk_pages_kernel, dim3(units), dim3(kTopkThreads), topk_smem, st,
+                 static_cast<const float*>(p.scores), a->maxP, a->seq_lens, a->head_kind, a->Hkv, p.budget_pages,
+                 a->sink, a->local, sel, sel_n, p.kcap) != cudaSuccess)
     return check_launch("decode top-k");
+  if (launch_pdl(decode_partition_kernel, dim3(1), dim3(1024), 0, st, static_cast<const int32_t*>(sel_n), units,
+                 p.kcap, p.R, p.G, D, p.off, p.range_unit, p.range_counter, static_cast<bf16*>(out), lse) !=
+      cudaSuccess)
+    return check_launch("decode partition");
   CUtensorMap tk, tv;
   const uint64_t rows = static_cast<uint64_t>(a->num_pages) * a->Hkv * kPage;
   if (!make_map_2d(&tk, a->k_pages, D, rows) || !make_map_2d(&tv, a->v_pages, D, rows))
     return fail(LSERVE_ERR_CUDA, "decode: cuTensorMapEncodeTiled failed");
-  ensure_smem(paged_decode_kernel<D>, DecodeCfg<D>::kSmemBytes);
+  ensure_smem(paged_decode_kernel<D>, DecodeCfg<D>::smem_bytes(kDecodeMaxG));
   const float scale = a->scale > 0.f ? a->scale : 1.f / std::sqrt(static_cast<float>(D));
-  if (launch_pdl(paged_decode_kernel<D>, dim3(p.nsplit, a->B * a->Hkv), dim3(kDecodeThreads),
-                 DecodeCfg<D>::kSmemBytes, st, tk, tv, static_cast<const bf16*>(a->q), a->page_table, a->maxP,
-                 a->seq_lens, a->head_kind, static_cast<const int32_t*>(sel), static_cast<const int32_t*>(sel_n),
-                 p.kcap, p.pps, p.nsplit, a->Hkv, p.G, a->num_pages, a->sink, a->local,
-                 scale * 1.4426950408889634f, wait_timeout_ns(), p.part_o, p.part_lse, p.done_count,
-                 static_cast<bf16*>(out), lse) != cudaSuccess)
+  if (launch_pdl(paged_decode_kernel<D>, dim3(p.P), dim3(kDecodeThreads), DecodeCfg<D>::smem_bytes(p.G), st, tk,
+                 tv, static_cast<const bf16*>(a->q), a->page_table, a->maxP, a->seq_lens, a->head_kind,
+                 static_cast<const int32_t*>(sel), static_cast<const int32_t*>(p.off),
+                 static_cast<const int32_t*>(p.range_unit), p.range_counter, p.R, p.kcap, units, a->Hkv, p.G,
+                 a->num_pages, a->sink, a->local, scale * 1.4426950408889634f, wait_timeout_ns(), p.part_o,
+                 p.part_lse) != cudaSuccess)
     return check_launch("decode attention");
+  if (launch_pdl(decode_merge_kernel, dim3(units), dim3(kMergeThreads), 0, st, static_cast<const int32_t*>(p.off),
+                 units, p.R, p.G, D, static_cast<const float*>(p.part_o), static_cast<const float*>(p.part_lse),
+                 static_cast<bf16*>(out), lse) != cudaSuccess)
+    return check_launch("decode merge");
   return check_launch("decode");
 }
 

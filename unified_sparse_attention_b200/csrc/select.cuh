@@ -155,10 +155,15 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkSmemKeys = 16384;   // scores cached in shared memory up to this many pages
 
+// One block per unit (b, g) = blockIdx.x.  The scores come from the scoring
+// kernel, which may still be running: they are read only after the dependency
+// wait, with L2 loads through a pointer that is not restrict-qualified (no load
+// of them can move above the wait).
 __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
-    const float* __restrict__ scores, int maxP, const int32_t* __restrict__ seq_lens,
-    const uint8_t* __restrict__ head_kind, int Hkv, int budget_pages, int sink, int local,
-    int32_t* __restrict__ sel, int32_t* __restrict__ sel_n, int kcap, int32_t* __restrict__ done_count) {
+    const float* scores, int maxP, const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind,
+    int Hkv, int budget_pages, int sink, int local, int32_t* sel, int32_t* sel_n, int kcap) {
+  pdl_launch_dependents();   // the one-CTA partition grid may get resident; it waits for this grid
+  pdl_wait();
   extern __shared__ uint32_t s_keys[];
   __shared__ int s_hist[256];
   __shared__ int s_scan[32];
@@ -166,8 +171,6 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
   __shared__ int s_remaining;
   const int unit = blockIdx.x;   // b * Hkv + g
   const int b = unit / Hkv, g = unit % Hkv;
-  pdl_wait();   // the scores come from the previous kernel
-  if (threadIdx.x == 0) done_count[unit] = 0;   // split-completion counter of the decode kernel
   const int L = max(0, seq_lens[b]);
   int n = (L + kPage - 1) / kPage;
   if (n > maxP) {   // sequence longer than its page-table row
@@ -207,13 +210,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
   const float* srow = scores + static_cast<long>(unit) * maxP;
   const bool cached = n <= kTopkSmemKeys;
   if (cached)
-    for (int j = tid; j < n; j += blockDim.x) s_keys[j] = order_key(srow[j]);
+    for (int j = tid; j < n; j += blockDim.x) s_keys[j] = order_key(__ldcg(srow + j));
   if (tid == 0) {
     s_prefix = 0;
     s_remaining = k;
   }
   __syncthreads();
-  auto key_at = [&](int j) -> uint32_t { return cached ? s_keys[j] : order_key(srow[j]); };
+  auto key_at = [&](int j) -> uint32_t { return cached ? s_keys[j] : order_key(__ldcg(srow + j)); };
 
   uint32_t prefix = 0, mask = 0;
 #pragma unroll 1
