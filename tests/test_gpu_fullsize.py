@@ -1,0 +1,122 @@
+"""GPU parity at the full sizes of the workload configurations, in the launch
+configuration the benchmark times (default grid, tcgen05 prefill kernel).
+
+The oracle cannot take whole long-context layers, so it is given samples that
+it can compute exactly:
+
+* prefill: seeded query rows (the first and last tiles, tile edges, random
+  rows) of one dense and one streaming KV head with their query heads.  A row
+  of masked attention depends on that row's query and on K, V only, so each
+  sampled row is an exact row of the full layer.
+* decode: (sequence, KV head) units -- every unit of the 32K case, seeded
+  samples of the large batches -- each re-laid out as a one-sequence,
+  one-head cache (its pages gathered in logical order, identity page table).
+  The oracle recomputes that unit's page summaries (compared bit-exact with
+  the GPU's), bound scores and page selection (tie-aware), and attention over
+  the pages the GPU selected, compared with what the GPU produced for the unit
+  inside the full batch.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import attention as OA
+from oracle import decode as OD
+from oracle import selection as OS
+from parity import assert_attn_close, assert_lse_close, check_selection, f64
+
+pytestmark = pytest.mark.gpu
+
+U = pytest.importorskip("unified_sparse_attention_b200")
+
+PAGE = 64
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_32k", "llama3_8b_prefill_128k_vslash", "llama2_7b_mha"])
+def test_prefill_full_size_sampled_rows(name):
+    w = W.WORKLOADS[name]
+    dev = "cuda"
+    q, k, v = W.prefill_inputs(w, device=dev)
+    bm = W.block_mask(w, device=dev)
+    kind = W.head_kind(w).tolist()
+    out, lse = U.lserve_prefill(q, k, v, torch.tensor(kind, dtype=torch.uint8, device=dev), w.sink, w.local, bm,
+                                return_lse=True)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+    S, G = w.S, w.Hq // w.Hkv
+    rng = np.random.default_rng(w.seed + 101)
+    rows = np.unique(np.concatenate([[0, 1, 63, 64, 65, S // 2, S - 65, S - 64, S - 2, S - 1],
+                                     rng.integers(0, S, 10)])).astype(np.int64)
+    rows_t = torch.from_numpy(rows).to(dev)
+    for g in (kind.index(0), kind.index(1)):   # one dense and one streaming KV head
+        heads = torch.arange(g * G, (g + 1) * G, device=dev)
+        q_rows = q[:, rows_t][:, :, heads]
+        bm_g = None if bm is None else bm[:, g:g + 1].cpu().numpy()
+        ref, ref_lse = OA.masked_attention(f64(q_rows), f64(k[:, :, g:g + 1]), f64(v[:, :, g:g + 1]), [kind[g]],
+                                           w.sink, w.local, bm_g, rows=rows, q_at_rows=True)
+        got = out[:, rows_t][:, :, heads]
+        got_lse = lse[:, heads][:, :, rows_t]
+        what = f"{name} KV head {g} ({'streaming' if kind[g] else 'dense'})"
+        assert_attn_close(f64(got), ref, what)
+        assert_lse_close(f64(got_lse), ref_lse, what + " lse")
+
+
+def _units(w, kind, sample):
+    B = w.dec_B
+    if sample is None:
+        return [(b, g) for b in range(B) for g in range(w.Hkv)]
+    dense = [g for g in range(w.Hkv) if kind[g] == 0]
+    stream = [g for g in range(w.Hkv) if kind[g] == 1]
+    rng = np.random.default_rng(w.seed + 202)
+    picked = [(0, dense[0]), (B - 1, stream[0]), (B // 2, dense[-1])]
+    while len(picked) < sample:
+        u = (int(rng.integers(B)), int(rng.integers(w.Hkv)))
+        if u not in picked:
+            picked.append(u)
+    return picked[:max(sample, 3)]
+
+
+@pytest.mark.parametrize("name,sample", [("llama3_8b_32k", None), ("llama3_8b_decode_b16_64k", 4),
+                                         ("llama2_7b_mha", 3)])
+def test_decode_full_size_units(name, sample):
+    w = W.WORKLOADS[name]
+    dev = "cuda"
+    pc = W.decode_cache(w, device=dev)
+    q = W.decode_query(w, device=dev)
+    kind = W.head_kind(w).tolist()
+    hk = torch.tensor(kind, dtype=torch.uint8, device=dev)
+    pt, sl = pc.page_table.to(dev), pc.seq_lens.to(dev)
+    stats = U.lserve_update_page_stats(pc.k_pages, pt, sl, hk)
+    B, G = w.dec_B, w.Hq // w.Hkv
+    lse = torch.empty(B, w.Hq, dtype=torch.float32, device=dev)
+    out, _, sel, sel_n = U.lserve_decode(q, pc.k_pages, pc.v_pages, pt, sl, stats, hk, w.sink, w.local,
+                                         w.token_budget, lse=lse, return_selection=True)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+    sel_np, seln_np = sel.cpu().numpy(), sel_n.cpu().numpy()
+    ties = 0
+    for b, g in _units(w, kind, sample):
+        L = int(pc.seq_lens[b])
+        n = OS.n_pages(L)
+        phys = pc.page_table[b, :n].to(dev, torch.long)
+        kc, vc = pc.k_pages[phys, g:g + 1], pc.v_pages[phys, g:g + 1]   # [n, 1, 64, d], logical order
+        ptc = np.arange(n, dtype=np.int32)[None, :]
+        Lc = np.array([L])
+        st_ref = OS.page_stats(f64(kc), ptc, Lc, [kind[g]])
+        np.testing.assert_array_equal(f64(stats[phys, g:g + 1]), st_ref)   # bit-exact summaries
+        heads = slice(g * G, (g + 1) * G)
+        qc = f64(q[b:b + 1, heads])
+        sel_ref, _, scores = OS.select(qc, st_ref, ptc, Lc, [kind[g]], w.token_budget, w.sink, w.local)
+        row = sel_np[b, g, :seln_np[b, g]]
+        assert np.all(sel_np[b, g, seln_np[b, g]:] == -1)
+        if kind[g]:
+            assert list(row) == list(sel_ref[(0, 0)]), f"{name} unit {(b, g)}: streaming pages"
+        else:
+            ties += check_selection(row, OS.budget_pages(w.token_budget, L), scores[0, 0, :n])
+        ref_out, ref_lse = OD.decode_attention(qc, f64(kc), f64(vc), ptc, Lc, [kind[g]], {(0, 0): row},
+                                               w.sink, w.local)
+        what = f"{name} unit {(b, g)} ({'streaming' if kind[g] else 'dense'})"
+        assert_attn_close(f64(out[b:b + 1, heads]), ref_out, what)
+        assert_lse_close(f64(lse[b:b + 1, heads]), ref_lse, what + " lse")
+    print(f"{name}: tied selections {ties}")

@@ -68,6 +68,10 @@ constexpr int kRangesPerCta = 4;   // ranges of the flat page list per attention
 constexpr int kMetaRing = 64;      // resolved pages buffered ahead of the loads
 
 constexpr int kSegStart = 1, kSegEnd = 2, kSegStreaming = 4;
+// Wait for the loads still in flight when a CTA gives up: fixed, independent of
+// the (possibly very short) limit of the ordinary waits, so that no copy can
+// land in shared memory after the CTA has left.
+constexpr unsigned long long kDrainTimeoutNs = 1000000000ull;
 
 template <int D>
 struct DecodeCfg {
@@ -78,6 +82,17 @@ struct DecodeCfg {
   __host__ __device__ static int stage_bytes(int G) { return 2 * kKVBytes + ((G * D * 2 + 1023) / 1024) * 1024; }
   __host__ __device__ static int smem_bytes(int G) { return kDecodeStages * stage_bytes(G) + 1024; }   // + alignment slack
 };
+
+// Ranges the T selected pages are cut into: at most R (the workspace's
+// capacity), each of at least kMinRangePages pages so that the per-range costs
+// (resolving, a partial per warp, merging) stay small next to streaming the
+// pages; one range when T is smaller.  Every kernel of the step computes it
+// alike from T.
+constexpr int kMinRangePages = 8;
+__host__ __device__ __forceinline__ long long ranges_in_use(long long R, long long T) {
+  const long long r = T / kMinRangePages;
+  return r < 1 ? 1 : (r < R ? r : R);
+}
 
 // CTA owning flat position f: the largest c with floor(c T / P) <= f.  With
 // P <= T no share is empty, so the owners of a range are every CTA between the
@@ -138,7 +153,7 @@ __device__ __forceinline__ void decode_partition(const int32_t* sel_n, int units
     *range_counter = 0;
   }
   __syncthreads();   // off[] of this block is visible to the block from here on
-  const long long Re = min(static_cast<long long>(R), T);   // every range below Re gets >= 1 page
+  const long long Re = ranges_in_use(R, T);   // every range below Re gets >= 1 page
   for (int u = tid; u < units; u += 1024) {
     const long long a = off[u], e = off[u + 1];
     if (e == a) {   // nothing selected: out = 0, lse = -inf
@@ -190,7 +205,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
     const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind,
     const int32_t* sel, const int32_t* off, const int32_t* range_unit, int32_t* range_counter, int R,
     int kcap, int units, int Hkv, int G, int num_pages, int sink, int local, float scale_log2,
-    unsigned long long timeout_ns, float* __restrict__ part_o, float* __restrict__ part_lse) {
+    unsigned long long timeout_ns, int debug_stall, float* __restrict__ part_o, float* __restrict__ part_lse) {
   using Cfg = DecodeCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kDecodeStages];    // stage loaded (issuer's expect_tx + bytes)
@@ -232,16 +247,19 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
     if (T != 0 && tid == 0) report(LSERVE_ERR_DEVICE_BOUNDS);
     return;
   }
-  const long long Re = min(static_cast<long long>(R), T);   // ranges that hold pages
+  const long long Re = ranges_in_use(R, T);   // ranges that hold pages
 
-  if (warp == kResolverWarp) {
+  if (warp == kResolverWarp && debug_stall) {
+    // failure-detection test: publish nothing, so that every other wait of the
+    // CTA runs out (nothing is issued, so nothing is in flight when it leaves)
+  } else if (warp == kResolverWarp) {
     // ---- claim ranges one after another and resolve their pages into the ring.
     // Window: unit wu + l (lane l) ends at flat position wend (INT_MAX past the
     // last unit); the window is shifted so that it always starts at the unit of
     // the next page to resolve.
     int gp = 0;   // pages resolved
-    bool ok = true;
-    while (ok) {
+    bool ok = true, stopped = false;   // !ok: inconsistent plan; stopped: the CTA is giving up
+    while (ok && !stopped) {
       int r = 0;
       if (lane == 0) r = atomicAdd(range_counter, 1);
       r = __shfl_sync(0xffffffffu, r, 0);
@@ -255,7 +273,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
       int wstart = __ldcg(off + wu);
       int wend = wu + lane < units ? __ldcg(off + wu + lane + 1) : INT_MAX;
       int f0 = lo;
-      while (f0 < hi && ok) {
+      while (f0 < hi && ok && !stopped) {
         // shift the window to the unit of f0
         int k0 = 0;
 #pragma unroll 8
@@ -290,7 +308,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
           room = spin_until([&] { return *v_issued >= gp + cnt - kMetaRing + kDecodeStages || *v_abort; },
                             timeout_ns) && !*v_abort;
         if (!__shfl_sync(0xffffffffu, room, 0)) {
-          ok = false;
+          stopped = true;
           break;
         }
         bool bad = false;
@@ -331,10 +349,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
       }
     }
     if (lane == 0) {
-      if (!ok) {
-        report(LSERVE_ERR_DEVICE_BOUNDS);
-        *v_abort = 1;
-      }
+      if (!ok) report(LSERVE_ERR_DEVICE_BOUNDS);
+      if (!ok || stopped) *v_abort = 1;
       __threadfence_block();
       *v_total = gp;
     }
@@ -384,9 +400,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
     const int qr = lane >> 2, tc = 2 * (lane & 3);
     for (int gp = 0;; ++gp) {
       bool have = false;
-      if (lane == 0)
-        have = spin_until([&] { return *v_resolved > gp || *v_total <= gp || *v_abort; }, timeout_ns) &&
-               *v_resolved > gp && !*v_abort;
+      if (lane == 0) {
+        const bool known = spin_until([&] { return *v_resolved > gp || *v_total <= gp || *v_abort; }, timeout_ns);
+        if (!known) *v_abort = 1;
+        have = known && *v_resolved > gp && !*v_abort;
+      }
       if (!__shfl_sync(0xffffffffu, have, 0)) break;
       const int st = gp % kDecodeStages;
       const bool landed = mbar_wait_bounded(&full_bar[st], (gp / kDecodeStages) & 1, timeout_ns);
@@ -539,7 +557,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
     // the last kDecodeStages issued pages sit in distinct stages, earlier ones have landed
     const int issued = *v_issued;
     for (int gp = max(0, issued - kDecodeStages); gp < issued; ++gp)
-      mbar_wait_bounded(&full_bar[gp % kDecodeStages], (gp / kDecodeStages) & 1, timeout_ns);
+      mbar_wait_bounded(&full_bar[gp % kDecodeStages], (gp / kDecodeStages) & 1, kDrainTimeoutNs);
   }
 }
 
@@ -562,7 +580,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const int32
   const long long T = __ldcg(off + units);
   const long long a = __ldcg(off + u), e = __ldcg(off + u + 1);
   if (T <= 0 || e <= a) return;   // nothing selected: written by the partition kernel
-  const long long Re = min(static_cast<long long>(R), T);
+  const long long Re = ranges_in_use(R, T);
   const int c_first = flat_owner(a, T, Re), c_last = flat_owner(e - 1, T, Re);
   if (c_first < 0 || c_last < c_first || c_last >= Re) {
     if (threadIdx.x == 0) report(LSERVE_ERR_DEVICE_BOUNDS);

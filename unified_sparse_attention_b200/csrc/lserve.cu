@@ -47,13 +47,17 @@ lserve_status check_launch(const char* what) {
   return LSERVE_OK;
 }
 
+// Failure-detection test hook: with LSERVE_DEBUG_STALL_DECODE set, the decode
+// attention kernel's page resolver publishes nothing, so its other waits run
+// out and the call records LSERVE_ERR_DEVICE_TIMEOUT (no copy is in flight).
+int debug_stall_decode() { return getenv("LSERVE_DEBUG_STALL_DECODE") ? 1 : 0; }
+
+// Limit of every bounded wait inside the kernels: LSERVE_WAIT_TIMEOUT_NS when it
+// holds a positive integer (read at each launch), else 2 s.
 unsigned long long wait_timeout_ns() {
-  static unsigned long long v = [] {
-    const char* s = getenv("LSERVE_WAIT_TIMEOUT_NS");
-    unsigned long long t = s ? strtoull(s, nullptr, 10) : 0ull;
-    return t ? t : 2000000000ull;   // 2 s
-  }();
-  return v;
+  const char* s = getenv("LSERVE_WAIT_TIMEOUT_NS");
+  const unsigned long long t = s ? strtoull(s, nullptr, 10) : 0ull;
+  return t ? t : 2000000000ull;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -389,7 +393,8 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
                  tv, static_cast<const bf16*>(a->q), a->page_table, a->maxP, a->seq_lens, a->head_kind,
                  static_cast<const int32_t*>(sel), static_cast<const int32_t*>(p.off),
                  static_cast<const int32_t*>(p.range_unit), p.range_counter, p.R, p.kcap, units, a->Hkv, p.G,
-                 a->num_pages, a->sink, a->local, scale * 1.4426950408889634f, wait_timeout_ns(), p.part_o,
+                 a->num_pages, a->sink, a->local, scale * 1.4426950408889634f, wait_timeout_ns(),
+                 debug_stall_decode(), p.part_o,
                  p.part_lse) != cudaSuccess)
     return check_launch("decode attention");
   if (launch_pdl(decode_merge_kernel, dim3(units), dim3(kMergeThreads), 0, st, static_cast<const int32_t*>(p.off),

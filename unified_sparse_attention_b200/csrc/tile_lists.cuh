@@ -130,11 +130,21 @@ __global__ void __launch_bounds__(1024) tile_scan_kernel(const int* __restrict__
     *overflow = s_carry > max_nnz;
     if (s_carry > max_nnz) report(LSERVE_ERR_DEVICE_BOUNDS);
   }
-  for (int grp = tid; grp < R / nRow; grp += blockDim.x) {
-    int above = grp * nRow;   // rows before this group + rows of it with more kept tiles than c
-    for (int c = nbucket - 1; c >= 0; --c) {
-      bucket[grp * nbucket + c] = above;
-      above += hist[grp * nbucket + c];
+  // bucket[grp][c] = grp * nRow + (rows of the group with more than c kept
+  // tiles): a suffix sum over c per group, one warp per group, 32 buckets a step
+  for (int grp = warp; grp < R / nRow; grp += blockDim.x / 32) {
+    int carry = grp * nRow;
+    for (int c0 = nbucket - 1; c0 >= 0; c0 -= 32) {
+      const int c = c0 - lane;   // lane 0 takes the largest c of the step
+      const int hv = c >= 0 ? hist[grp * nbucket + c] : 0;
+      int x = hv;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (c >= 0) bucket[grp * nbucket + c] = carry + x - hv;
+      carry += __shfl_sync(0xffffffffu, x, 31);
     }
   }
 }
