@@ -243,7 +243,7 @@ bool use_legacy_prefill() {
 
 // ----------------------------------------------------------------- decode
 struct DecodePlan {
-  int kcap, budget_pages, G, ppb;
+  int kcap, budget_pages, G;
   int P;                 // CTAs of the attention grid (one wave)
   int R;                 // ranges of the flat page list (kRangesPerCta per CTA)
   float* scores;
@@ -257,18 +257,13 @@ struct DecodePlan {
   size_t bytes;
 };
 
-// Attention CTAs for the current device: SMs x resident CTAs per SM, or the
-// value of LSERVE_DECODE_GRID (a positive integer) when that is set.
-int decode_grid() {
-  if (const char* e = getenv("LSERVE_DECODE_GRID")) {
-    const long v = strtol(e, nullptr, 10);
-    if (v > 0 && v <= (1 << 20)) return static_cast<int>(v);
-  }
+// SMs of the current device (148 if it cannot be asked).
+int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
-    return 148 * kDecodeCtasPerSm;
+    return 148;
   }
   if (!cached[dev]) {
     int sms = 0;
@@ -276,9 +271,19 @@ int decode_grid() {
       cudaGetLastError();
       sms = 148;
     }
-    cached[dev] = sms * kDecodeCtasPerSm;
+    cached[dev] = sms;
   }
   return cached[dev];
+}
+
+// Attention CTAs for the current device: SMs x resident CTAs per SM, or the
+// value of LSERVE_DECODE_GRID (a positive integer) when that is set.
+int decode_grid() {
+  if (const char* e = getenv("LSERVE_DECODE_GRID")) {
+    const long v = strtol(e, nullptr, 10);
+    if (v > 0 && v <= (1 << 20)) return static_cast<int>(v);
+  }
+  return sm_count() * kDecodeCtasPerSm;
 }
 
 // Launch with programmatic stream serialisation: the kernel may start while its
@@ -337,10 +342,7 @@ DecodePlan plan_decode(const lserve_decode_args* a, void* ws) {
   p.kcap = std::max(1, std::max(dense_cap, std::min(streaming_page_bound(a->sink, a->local), a->maxP)));
   p.P = decode_grid();
   p.R = kRangesPerCta * p.P;
-  // scoring: aim for >= ~4 CTAs per SM
-  const long long pages = static_cast<long long>(a->B) * a->maxP;
-  long long ppb = pages / (4 * 148);
-  p.ppb = static_cast<int>(std::max(4ll, std::min<long long>(ppb, 64)));
+
   Carver c(ws);
   const long long units = static_cast<long long>(a->B) * a->Hkv;
   p.scores = c.take<float>(units * a->maxP);
@@ -355,23 +357,28 @@ DecodePlan plan_decode(const lserve_decode_args* a, void* ws) {
   return p;
 }
 
-template <int D, int G>
-void launch_score(const lserve_decode_args* a, const DecodePlan& p, cudaStream_t st) {
-  dim3 grid((a->maxP + p.ppb - 1) / p.ppb, a->B);
-  score_pages_kernel<D, G><<<grid, 256, 0, st>>>(static_cast<const bf16*>(a->q), static_cast<const bf16*>(a->stats),
-                                                 a->page_table, a->maxP, a->seq_lens, a->head_kind, a->Hkv,
-                                                 a->num_pages, p.ppb, p.scores);
-}
-
 template <int D>
 lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, int32_t* sel, int32_t* sel_n,
                               void* out, float* lse, cudaStream_t st) {
-  switch (p.G) {
-    case 1: launch_score<D, 1>(a, p, st); break;
-    case 2: launch_score<D, 2>(a, p, st); break;
-    case 4: launch_score<D, 4>(a, p, st); break;
-    default: launch_score<D, 8>(a, p, st); break;
+  if (p.G == 1) {
+    // one query head per KV head: per-lane fp32 products over 16-byte summary
+    // loads, one warp per (page, dense head), ~4 CTAs per SM
+    const long long pages = static_cast<long long>(a->B) * a->maxP;
+    const int ppb = static_cast<int>(std::max(4ll, std::min<long long>(pages / (4ll * sm_count()), 64)));
+    score_pages_kernel<D, 1><<<dim3((a->maxP + ppb - 1) / ppb, a->B), 256, 0, st>>>(
+        static_cast<const bf16*>(a->q), static_cast<const bf16*>(a->stats), a->page_table, a->maxP, a->seq_lens,
+        a->head_kind, a->Hkv, a->num_pages, ppb, p.scores);
+  } else {
+    // G query heads per KV head: the bound as a contraction on the tensor cores,
+    // one wave of SMs x resident CTAs (fewer when there is less work)
+    const long long items = static_cast<long long>(a->B) * a->Hkv * ((a->maxP + 3) / 4);
+    const long long want = (items + kScoreThreads / 32 - 1) / (kScoreThreads / 32);
+    const int grid = static_cast<int>(std::min<long long>(want, static_cast<long long>(sm_count()) * kScoreCtasPerSm));
+    score_pages_mma_kernel<D><<<grid, kScoreThreads, 0, st>>>(
+        static_cast<const bf16*>(a->q), static_cast<const bf16*>(a->stats), a->page_table, a->B, a->maxP,
+        a->seq_lens, a->head_kind, a->Hkv, p.G, a->num_pages, p.scores);
   }
+
   ensure_smem(topk_pages_kernel, kTopkSmemKeys * static_cast<int>(sizeof(uint32_t)));
   const int topk_smem = std::min(a->maxP, kTopkSmemKeys) * static_cast<int>(sizeof(uint32_t));
   const int units = a->B * a->Hkv;

@@ -5,13 +5,15 @@
 // only; mlsanity LServe page, Abstract: a hierarchical KV page selection policy
 // by query-centric similarity, with a constant number of pages kept.
 //
-// score_pages_kernel  (HBM-bound stream over the summaries)
+// Bound scoring (HBM-bound stream over the summaries)
 //   bound of query head h on logical page l:  sum_c max(q_hc * kmax_c, q_hc * kmin_c)
 //   group score: max over the G query heads of the KV head; page score: max over
-//   the page's logical pages that hold a valid token.  One warp per physical
-//   page: lane = (logical page l = lane/8, 16 (d=128) or 8 (d=64) channels),
-//   four 16-byte loads per lane, fp32 products (exact for bf16 operands) and a
-//   3-step shuffle sum per head, then shuffle max over heads and logical pages.
+//   the page's logical pages that hold a valid token.
+//   score_pages_kernel (G = 1): one warp per physical page: lane = (logical
+//     page l = lane/8, 16 (d=128) or 8 (d=64) channels), four 16-byte loads per
+//     lane, fp32 products (exact for bf16 operands) and a 3-step shuffle sum.
+//   score_pages_mma_kernel (G >= 2): the same bound as a contraction on the
+//     tensor cores (see there); per-lane products would cost G x as much issue.
 //
 // topk_pages_kernel  (latency-bound, one CTA per (sequence, KV head))
 //   k = min(budget/64, n_pages) pages by 4-pass 8-bit radix select on the
@@ -115,6 +117,158 @@ __global__ void __launch_bounds__(256) score_pages_kernel(
     s = fmaxf(s, __shfl_xor_sync(0xffffffffu, s, 8));
     s = fmaxf(s, __shfl_xor_sync(0xffffffffu, s, 16));
     if (lane == 0) scores[(static_cast<long>(b) * Hkv + g) * maxP + i] = s;
+  }
+}
+
+// Bound scoring on the tensor cores.  max(q_c kmax_c, q_c kmin_c) is q_c kmax_c
+// when q_c >= 0 and q_c kmin_c otherwise, so the bound of query head h on a
+// logical page is  q-_h . kmin + q+_h . kmax  (q- = min(q, 0), q+ = max(q, 0)):
+// one contraction of the summary row [kmin | kmax] (2d bf16, as stored) with
+// [q- | q+].  One warp takes 4 physical pages = 16 logical pages of one dense
+// KV head as the M = 16 rows of m16n8k16 tiles, K = 2d, and the group's G <= 8
+// query heads as N = 8 (q- and q+ are exact bf16 values; products are exact
+// and sums are fp32).  The K order inside the tiles is permuted so that every
+// lane reads 16 contiguous bytes of a row per 32 channels (channels 32 j + 8 t
+// .. + 7 of lane t of a quad feed k-steps 2 j and 2 j + 1); the q fragments use
+// the same order.  The group max is over the valid heads of each row, the page
+// max over the rows of a page that hold a valid token (quad shuffles).
+constexpr int kScoreThreads = 256;
+constexpr int kScoreCtasPerSm = 2;
+
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads, kScoreCtasPerSm) score_pages_mma_kernel(
+    const bf16* __restrict__ q, const bf16* __restrict__ stats, const int32_t* __restrict__ page_table, int B,
+    int maxP, const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind, int Hkv, int G,
+    int num_pages, float* __restrict__ scores) {
+  constexpr int NJ = 2 * D / 32;   // 32-channel groups of [kmin | kmax]
+  __shared__ int s_dense[256];
+  __shared__ int s_ndense;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int g = 0; g < Hkv; ++g)
+      if (head_kind[g] == LSERVE_HEAD_DENSE) s_dense[n++] = g;
+    s_ndense = n;
+  }
+  __syncthreads();
+  // items (b, dense head, group of 4 pages) in that order; each warp takes an
+  // equal contiguous run of them (the grid is one wave)
+  const int ngrp = (maxP + 3) / 4;
+  const long long items = static_cast<long long>(B) * s_ndense * ngrp;
+  const long long total_warps = static_cast<long long>(gridDim.x) * nwarps;
+  const long long per = (items + total_warps - 1) / total_warps;
+  const long long it0 = (static_cast<long long>(blockIdx.x) * nwarps + warp) * per;
+  const long long it1 = min(items, it0 + per);
+  const int r = lane >> 2, t = lane & 3;   // fragment row (and row + 8), lane of the quad
+  const float ninf = kNegInf;
+
+  struct Item {
+    int b, g, ib, n_pages, L;
+    int p[2];   // physical pages of rows r and r + 8 (-1: none)
+  };
+  auto locate = [&](long long it) -> Item {
+    Item m;
+    m.b = static_cast<int>(it / (static_cast<long long>(s_ndense) * ngrp));
+    const int rem = static_cast<int>(it % (static_cast<long long>(s_ndense) * ngrp));
+    m.g = s_dense[rem / ngrp];
+    m.ib = (rem % ngrp) * 4;
+    m.L = seq_lens[m.b];
+    m.n_pages = min(maxP, (max(m.L, 0) + kPage - 1) / kPage);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = m.ib + (r + 8 * h) / 4;
+      int pg = -1;
+      if (i < m.n_pages) {
+        pg = page_table[static_cast<long>(m.b) * maxP + i];
+        if (pg < 0 || pg >= num_pages) {
+          if (((r + 8 * h) & 3) == 0 && t == 0) report(LSERVE_ERR_DEVICE_BOUNDS);
+          pg = -1;
+        }
+      }
+      m.p[h] = pg;
+    }
+    return m;
+  };
+
+  int cur_b = -1, cur_g = -1;
+  uint32_t qb[NJ][4];   // per 32-channel group: b0, b1 of k-step 2j, then of 2j + 1 (query head r)
+  Item nx = it0 < it1 ? locate(it0) : Item{};
+  for (long long it = it0; it < it1; ++it) {
+    const Item m = nx;
+    if (m.ib >= m.n_pages) {   // past the end of this sequence
+      if (it + 1 < it1) nx = locate(it + 1);
+      continue;
+    }
+    // the summaries of rows r and r + 8 (logical page (row % 4) of page ib + row / 4)
+    uint4 a[NJ][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = r + 8 * h;
+      const bf16* srow =
+          m.p[h] >= 0 ? stats + ((static_cast<long>(m.p[h]) * Hkv + m.g) * kNL + (row & 3)) * 2 * D + 8 * t
+                      : nullptr;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j)
+        a[j][h] = srow ? __ldg(reinterpret_cast<const uint4*>(srow + 32 * j)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (it + 1 < it1) nx = locate(it + 1);   // the next item's pages load meanwhile
+    if (m.b != cur_b || m.g != cur_g) {
+      cur_b = m.b;
+      cur_g = m.g;
+      const bf16* qh = q + (static_cast<long>(m.b) * Hkv * G + static_cast<long>(m.g) * G + r) * D;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const bool plus = 32 * j >= D;   // kmax half: q+, kmin half: q-
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (r < G) w = __ldg(reinterpret_cast<const uint4*>(qh + (32 * j) % D + 8 * t));
+        auto half = [&](uint32_t x) -> uint32_t {
+          uint32_t o = 0u;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const uint32_t hb = (x >> (16 * e)) & 0xffffu;
+            if (((hb & 0x8000u) != 0) != plus) o |= hb << (16 * e);
+          }
+          return o;
+        };
+        qb[j][0] = half(w.x);
+        qb[j][1] = half(w.y);
+        qb[j][2] = half(w.z);
+        qb[j][3] = half(w.w);
+      }
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const uint32_t fa[4] = {a[j][0].x, a[j][1].x, a[j][0].y, a[j][1].y};   // k-step 2j
+      const uint32_t fb[4] = {a[j][0].z, a[j][1].z, a[j][0].w, a[j][1].w};   // k-step 2j + 1
+      mma_bf16_16816(acc, fa, qb[j][0], qb[j][1]);
+      mma_bf16_16816(acc, fb, qb[j][2], qb[j][3]);
+    }
+    // element e: row r + 8 (e >> 1), head 2 t + (e & 1)
+    float sc[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float mx = ninf;
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (2 * t + e < G) mx = fmaxf(mx, acc[2 * h + e]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const int row = r + 8 * h;
+      const int i = m.ib + row / 4;
+      // logical pages without a valid token (and missing pages) do not count
+      sc[h] = (m.p[h] >= 0 && i * kPage + (row & 3) * kLogical < m.L) ? mx : ninf;
+      sc[h] = fmaxf(sc[h], __shfl_xor_sync(0xffffffffu, sc[h], 4));
+      sc[h] = fmaxf(sc[h], __shfl_xor_sync(0xffffffffu, sc[h], 8));
+    }
+    // lanes 0 and 16 hold pages r / 4 and r / 4 + 2 of the group
+    if ((lane & 15) == 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int i = m.ib + (r + 8 * h) / 4;
+        if (i < m.n_pages) scores[(static_cast<long>(m.b) * Hkv + m.g) * maxP + i] = sc[h];
+      }
+    }
   }
 }
 
