@@ -431,10 +431,11 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       uint32_t v[64];
       uint32_t pk0[32], pk1[32];
       float ps[4];
-      // exponentials 2^(s*scale - m) of one 64-key half, packed to bf16 pairs;
-      // tracks the largest argument and the row sum
-      // one 32-column chunk of S (already in registers): exponentials, max, sum, bf16 pairs
-      auto exp_chunk = [&](uint32_t (&u)[32], uint64_t keep, int q, float m_use, uint32_t* pk, float (&am)[4]) {
+      // One 32-column chunk of S (already in registers): exponentials 2^(s*scale - m),
+      // packed fp32 pairs for the scale/subtract and the running sums (half the
+      // instructions: the softmax is issue-bound), bf16 pairs of P.
+      auto exp_chunk = [&](uint32_t (&u)[32], uint64_t keep, int q, uint64_t sc2, uint64_t nm2, uint32_t* pk,
+                           uint64_t (&ps2)[2]) {
         if (!__all_sync(0xffffffffu, keep == ~0ull)) {
 #pragma unroll
           for (int c = 0; c < 32; ++c)
@@ -442,34 +443,34 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         }
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float a0 = fmaf(__uint_as_float(u[2 * c]), sc, -m_use);
-          const float a1 = fmaf(__uint_as_float(u[2 * c + 1]), sc, -m_use);
-          am[c & 3] = max3(am[c & 3], a0, a1);
+          float a0, a1;
+          split_f32x2(fma_f32x2(f32x2(__uint_as_float(u[2 * c]), __uint_as_float(u[2 * c + 1])), sc2, nm2), a0, a1);
           const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
-          ps[c & 3] += p0 + p1;
+          ps2[c & 1] = add_f32x2(ps2[c & 1], f32x2(p0, p1));
           pk[c] = pack_bf16x2(p0, p1);
         }
       };
-      auto exp_pass = [&](float m) -> float {   // returns the largest argument
+      auto exp_pass = [&](float m) -> float {   // returns the row sum of the exponentials
         const float m_use = m == kNegInf ? 0.f : m;
-        float am[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) ps[e] = 0.f;
+        const uint64_t sc2 = f32x2(sc, sc), nm2 = f32x2(-m_use, -m_use);
+        uint64_t ps2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
         // four 32-column chunks; the TMEM load of chunk c+1 is in flight while chunk c is processed
         uint32_t ua[32], ub[32];
         tmem_ld32(t_s, ua);
         tmem_wait_ld();
         tmem_ld32(t_s + 32, ub);
-        exp_chunk(ua, keep0, 0, m_use, pk0, am);
+        exp_chunk(ua, keep0, 0, sc2, nm2, pk0, ps2);
         tmem_wait_ld();
         tmem_ld32(t_s + 64, ua);
-        exp_chunk(ub, keep0, 1, m_use, pk0 + 16, am);
+        exp_chunk(ub, keep0, 1, sc2, nm2, pk0 + 16, ps2);
         tmem_wait_ld();
         tmem_ld32(t_s + 96, ub);
-        exp_chunk(ua, keep1, 0, m_use, pk1, am);
+        exp_chunk(ua, keep1, 0, sc2, nm2, pk1, ps2);
         tmem_wait_ld();
-        exp_chunk(ub, keep1, 1, m_use, pk1 + 16, am);
-        return max3(am[0], am[1], fmaxf(am[2], am[3]));
+        exp_chunk(ub, keep1, 1, sc2, nm2, pk1 + 16, ps2);
+        split_f32x2(ps2[0], ps[0], ps[1]);
+        split_f32x2(ps2[1], ps[2], ps[3]);
+        return (ps[0] + ps[1]) + (ps[2] + ps[3]);
       };
       // O[x] and l are multiplied by f before this step's P is added
       float f = 1.f;
@@ -478,11 +479,12 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         m_run += rebase;
         rebase = 0.f;
       }
-      float amax = kNegInf;
+      float rsum = 0.f;
       bool ok = false;
       if (m_run != kNegInf) {   // steady state: one pass against the current reference
-        amax = exp_pass(m_run);
-        ok = !__any_sync(0xffffffffu, amax > 64.f);   // no exponential near the fp32/bf16 limit
+        rsum = exp_pass(m_run);
+        // every weight is at most the row sum: none near the fp32/bf16 limit (catches inf/NaN too)
+        ok = !__any_sync(0xffffffffu, !(rsum <= 1099511627776.f));   // 2^40
       }
       if (!ok) {                // first step of the stream, or a jump: exact row max first
         float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
@@ -500,11 +502,18 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         const float m_new = fmaxf(m_run, mloc);
         if (m_run != kNegInf && m_new != m_run) f *= fast_exp2(m_run - m_new);
         m_run = m_new;
-        amax = exp_pass(m_run);
+        rsum = exp_pass(m_run);
       }
-      // values above the reference by more than 2^8: move the reference at the next
-      // step of this stream (O must first absorb this step)
-      if (m_run != kNegInf && amax > 8.f) rebase = amax;
+      // weights well above the reference (row sum beyond 2^12): move the reference to the
+      // largest argument at this stream's next step (O must first absorb this step); the
+      // largest weight is read back from the bf16 pairs of P
+      if (m_run != kNegInf && rsum > 4096.f) {
+        uint32_t mp = 0u;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) mp = max_bf16x2(mp, max_bf16x2(pk0[c], pk1[c]));
+        const float wmax = fmaxf(bf16_lo(mp), bf16_hi(mp));
+        if (wmax > 1.f) rebase = __log2f(wmax);
+      }
       tmem_st32(t_s, pk0);        // P[x] over S[x] columns 0..63 (S is no longer needed)
       tmem_st32(t_s + 32, pk1);
       l_run = l_run * f + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
