@@ -69,23 +69,31 @@ __device__ __forceinline__ void commit(uint64_t* bar) {   // call from a converg
       : "memory");
 }
 // The issuing warp runs converged with warp-uniform operands; one lane chosen
-// by elect.sync issues the instruction.
-// D[tmem] (+)= A[smem] * B[smem]
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
+// by elect.sync issues the instructions.
+// Four MMAs from one elected lane: the first takes `accumulate`, the others
+// accumulate.  D[tmem] (+)= A[smem] * B[smem]  /  D[tmem] (+)= A[tmem] * B[smem]
+__device__ __forceinline__ void mma_ss4(uint32_t d_tmem, uint64_t a0, uint64_t a1, uint64_t a2, uint64_t a3,
+                                        uint64_t b0, uint64_t b1, uint64_t b2, uint64_t b3, uint32_t idesc,
+                                        uint32_t accumulate) {
   asm volatile(
-      "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
-      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n .reg .pred p, e, t;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %9, 0;\n setp.eq.b32 t, %9, %9;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %10, p;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %10, t;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %10, t;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %10, t;\n}\n" ::"r"(d_tmem),
+      "l"(a0), "l"(a1), "l"(a2), "l"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(accumulate), "r"(idesc)
       : "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem]
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
+__device__ __forceinline__ void mma_ts4(uint32_t d_tmem, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint64_t b0, uint64_t b1, uint64_t b2, uint64_t b3, uint32_t idesc,
+                                        uint32_t accumulate) {
   asm volatile(
-      "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
-      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n .reg .pred p, e, t;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %9, 0;\n setp.eq.b32 t, %9, %9;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %10, p;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %10, t;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %10, t;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %10, t;\n}\n" ::"r"(d_tmem),
+      "r"(a0), "r"(a1), "r"(a2), "r"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(accumulate), "r"(idesc)
       : "memory");
 }
 __device__ __forceinline__ bool elect_one() {
@@ -330,7 +338,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     // Step p belongs to stream x = p & 1 (S[x], P[x], O[x]).  The whole warp runs
     // the loop (waits and descriptors warp-uniform); one elected lane issues.
     // Tensor-core order: S(0) S(1) PV(0) S(2) PV(1) S(3) ...  S(p+2) overwrites the
-    // S/P buffer of PV(p), so it is issued once PV(p) has completed.
+    // S/P buffer that PV(p) reads; tcgen05.mma instructions of one kind issued by
+    // one thread are pipelined in issue order, so S(p+2) is issued right after
+    // PV(p) without waiting for its completion (checked: parity, and bit-identical
+    // results over repeated runs).
     if (n > 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, false);
       constexpr uint32_t kIdPV = idesc_bf16(128, D, true);
@@ -338,13 +349,17 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       auto issue_s = [&](int p) {   // S[p&1] = Q [K_a; K_b]^T
         const int st = p % kKStages, x = p & 1;
         wait_or_abort(&k_full[st], (p / kKStages) & 1, &s_abort, tmo);
-        if (p >= 2) wait_or_abort(&o_done[x], ((p >> 1) - 1) & 1, &s_abort, tmo);   // PV(p-2) read P[x]
         fence_after_sync();
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t ad = sdesc(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc(ka + st * C::kPair + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-          mma_ss(tmem + C::kColS + 128 * x, ad, bd, kIdS, ks > 0);
+        for (int k4 = 0; k4 < D / 16; k4 += 4) {
+          uint64_t ad[4], bd[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int ks = k4 + e;
+            ad[e] = sdesc(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+            bd[e] = sdesc(ka + st * C::kPair + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+          }
+          mma_ss4(tmem + C::kColS + 128 * x, ad[0], ad[1], ad[2], ad[3], bd[0], bd[1], bd[2], bd[3], kIdS, k4 > 0);
         }
         commit(&s_full[x]);
         if (p + kKStages < np) commit(&k_empty[st]);
@@ -358,10 +373,16 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         wait_or_abort(&p_full[x], (p >> 1) & 1, &s_abort, tmo);
         fence_after_sync();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = sdesc(va + st * C::kPair + kk * 2048, 16384, 1024);
-          mma_ts(tmem + C::kColO + 128 * x, tmem + C::kColS + 128 * x + 8 * kk, bd, kIdPV,
-                 (p >= 2 || kk > 0) ? 1u : 0u);
+        for (int k4 = 0; k4 < 8; k4 += 4) {
+          uint64_t bd[4];
+          uint32_t at[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            bd[e] = sdesc(va + st * C::kPair + (k4 + e) * 2048, 16384, 1024);
+            at[e] = tmem + C::kColS + 128 * x + 8 * (k4 + e);
+          }
+          mma_ts4(tmem + C::kColO + 128 * x, at[0], at[1], at[2], at[3], bd[0], bd[1], bd[2], bd[3], kIdPV,
+                  (p >= 2 || k4 > 0) ? 1u : 0u);
         }
         commit(&o_done[x]);
         if (p + kVStages < np) commit(&v_empty[st]);
