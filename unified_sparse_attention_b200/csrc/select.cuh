@@ -322,7 +322,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
   __shared__ int s_hist[256];
   __shared__ int s_scan[32];
   __shared__ uint32_t s_prefix;
-  __shared__ int s_remaining;
+  __shared__ int s_remaining, s_count;
+  __shared__ uint32_t s_mm[2][32];
   const int unit = blockIdx.x;   // b * Hkv + g
   const int b = unit / Hkv, g = unit % Hkv;
   const int L = max(0, seq_lens[b]);
@@ -365,21 +366,52 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
   const bool cached = n <= kTopkSmemKeys;
   if (cached)
     for (int j = tid; j < n; j += blockDim.x) s_keys[j] = order_key(__ldcg(srow + j));
-  if (tid == 0) {
-    s_prefix = 0;
-    s_remaining = k;
-  }
   __syncthreads();
   auto key_at = [&](int j) -> uint32_t { return cached ? s_keys[j] : order_key(__ldcg(srow + j)); };
 
-  uint32_t prefix = 0, mask = 0;
+  // The bits above the highest one in which the keys differ are common to all
+  // of them (scores of similar magnitude share sign and exponent): the radix
+  // digits start below them, so that no pass piles every key into one bin.
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int j = tid; j < n; j += blockDim.x) {
+    const uint32_t kk = key_at(j);
+    kmin = min(kmin, kk);
+    kmax = max(kmax, kk);
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if ((tid & 31) == 0) {
+    s_mm[0][tid >> 5] = kmin;
+    s_mm[1][tid >> 5] = kmax;
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const int nw = blockDim.x >> 5;
+    kmin = __reduce_min_sync(0xffffffffu, tid < nw ? s_mm[0][tid] : 0xffffffffu);
+    kmax = __reduce_max_sync(0xffffffffu, tid < nw ? s_mm[1][tid] : 0u);
+    if (tid == 0) {
+      s_mm[0][0] = kmin;
+      s_mm[1][0] = kmax;
+    }
+  }
+  __syncthreads();
+  kmin = s_mm[0][0];
+  kmax = s_mm[1][0];
+  int shift = (kmin ^ kmax) ? 32 - __clz(kmin ^ kmax) : 0;   // low bits still to resolve
+  uint32_t mask = shift >= 32 ? 0u : ~((1u << shift) - 1u);    // bits fixed so far
+  uint32_t prefix = kmax & mask;                                // their value for the k-th key
+  int remaining = k;                                            // keys still to take at prefix
+  // 8-bit digits (the first may be narrower); a pass ends the search when the
+  // k-th key's bin is taken whole -- the lower bits need not be resolved
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  while (shift > 0) {
+    const int w = min(8, shift);
+    shift -= w;
     for (int j = tid; j < 256; j += blockDim.x) s_hist[j] = 0;
     __syncthreads();
     for (int j = tid; j < n; j += blockDim.x) {
       const uint32_t kk = key_at(j);
-      if ((kk & mask) == prefix) atomicAdd(&s_hist[(kk >> shift) & 255], 1);
+      if ((kk & mask) == prefix) atomicAdd(&s_hist[(kk >> shift) & ((1u << w) - 1u)], 1);
     }
     __syncthreads();
     if (tid < 32) {
@@ -398,39 +430,44 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
         if (tid + o < 32) suf += y;
       }
       const int above = suf - sum;   // keys with a higher digit
-      const int rem = s_remaining;
-      if (above < rem && rem <= suf) {   // exactly one lane
-        int acc = above, digit = tid * 8;
+      if (above < remaining && remaining <= suf) {   // exactly one lane
+        int acc = above, digit = tid * 8, cnt = 0;
+#pragma unroll
         for (int e = 7; e >= 0; --e) {
-          if (acc + c[e] >= rem) {
+          if (cnt == 0 && acc + c[e] >= remaining) {
             digit = tid * 8 + e;
-            break;
+            cnt = c[e];
+          } else if (cnt == 0) {
+            acc += c[e];
           }
-          acc += c[e];
         }
         s_prefix = prefix | (static_cast<uint32_t>(digit) << shift);
-        s_remaining = rem - acc;
+        s_remaining = remaining - acc;
+        s_count = cnt;
       }
     }
     __syncthreads();
     prefix = s_prefix;
-    mask |= 255u << shift;
+    mask |= ((1u << w) - 1u) << shift;
+    remaining = s_remaining;
+    if (s_count == remaining) break;   // the whole bin is taken
   }
-  const uint32_t T = prefix;        // key of the k-th largest score
-  const int take_eq = s_remaining;  // how many keys equal to T are taken (lowest indices)
+  // keys compare on the fixed bits: above T is taken, at T the lowest indices
+  const uint32_t T = prefix;
+  const int take_eq = remaining;
 
   // ascending emission: each thread owns a contiguous run of indices
   const int per = (n + blockDim.x - 1) / blockDim.x;
   const int j0 = min(n, tid * per), j1 = min(n, j0 + per);
   int n_eq = 0;
-  for (int j = j0; j < j1; ++j) n_eq += key_at(j) == T;
+  for (int j = j0; j < j1; ++j) n_eq += (key_at(j) & mask) == T;
   int tot;
   int eq_before = block_exclusive_scan(n_eq, s_scan, &tot);
   int n_sel = 0;
   {
     int e = eq_before;
     for (int j = j0; j < j1; ++j) {
-      const uint32_t kk = key_at(j);
+      const uint32_t kk = key_at(j) & mask;
       if (kk > T) ++n_sel;
       else if (kk == T) n_sel += (e++ < take_eq);
     }
@@ -439,7 +476,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
   {
     int e = eq_before, pos = sel_before;
     for (int j = j0; j < j1; ++j) {
-      const uint32_t kk = key_at(j);
+      const uint32_t kk = key_at(j) & mask;
       bool take = kk > T;
       if (kk == T) take = (e++ < take_eq);
       if (take && pos < kcap) row[pos++] = j;
