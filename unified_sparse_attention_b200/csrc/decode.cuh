@@ -1,5 +1,5 @@
-// decode.cuh -- sparse paged decode attention over the selected pages, split
-// evenly across a persistent grid, with the log-sum-exp merge folded in.
+// decode.cuh -- sparse paged decode attention over the selected pages: the
+// selection step's kernel, the attention grid and the log-sum-exp merge.
 //
 // LServe + SampleAttention blog post, "LServe - Decode Phase" and Fig. 2:
 // token-level attention only inside the selected pages.  Streaming heads attend
@@ -8,40 +8,35 @@
 //
 // Work split.  Unit u = (sequence b, KV head g) has n_u selected pages; the
 // pages of all units, laid end to end in unit order, form one flat list of
-// T = sum_u n_u pages with unit u at [off_u, off_u + n_u).
-// decode_partition_kernel builds `off` and, for each of the P CTAs of the
-// attention grid (P = SMs x resident CTAs per SM, one wave), the unit holding
-// the first page of CTA c's equal share [floor(c T / P), floor((c + 1) T / P)).
-// A share that crosses unit boundaries is cut into segments, one per unit.
-// Every CTA then streams about T / P pages whatever the mix of long dense
-// selections and short streaming ones, so the grid ends in one wave with no
-// tail, where one CTA per (unit, fixed-size split) left a partial last wave.
+// T = sum_u n_u pages with unit u at [off_u, off_u + n_u).  The list is cut
+// into Re = ranges_in_use(R, T) equal ranges of at least kMinRangePages pages.
+// n_u follows from the sequence lengths alone, so one extra block of the top-k
+// grid builds this plan (decode_partition) while the other blocks select.
 //
-// paged_decode_kernel (per CTA):
-//   * resolves its pages (unit, logical page, physical page) into shared memory
-//     up front, in chunks of up to 256 pages, so the producer issues loads with
-//     no dependent global lookups on its path;
-//   * streams each page's K and V (64 x d bf16 each, contiguous in the pool)
-//     through a 3-stage ring with TMA (128-byte swizzle): a producer warp
-//     issues a stage's loads once the 4 consumer warps have released it (full
-//     and empty mbarriers per stage), so no consumer ever waits for an issue
-//     or for another consumer; the first page of a segment also brings the
-//     group's G query rows with a bulk copy;
-//   * each of the 4 warps owns 16 tokens of every page and keeps an online
-//     softmax for the G <= 8 query heads, on mma.sync m16n8k16 tiles laid out
+// paged_decode_kernel: one wave of CTAs (SMs x 2) that claim ranges from a
+// counter, so that SMs that run ahead take more.  Per CTA:
+//   * a resolver warp claims ranges and resolves their pages (unit, logical
+//     page, physical page, segment flags) into a shared-memory ring ahead of
+//     the loads; a range that crosses unit boundaries is cut into segments,
+//     one per unit;
+//   * an issuer warp streams each page's K and V (64 x d bf16 each, contiguous
+//     in the pool) through a 3-stage ring with TMA (128-byte swizzle), and the
+//     group's G query rows with a bulk copy at a segment start (full and empty
+//     mbarriers per stage);
+//   * four consumer warps each own 16 tokens of every page, copy their K/V
+//     fragments to registers and release the stage at once, then keep an online
+//     softmax for the G <= 8 query heads on mma.sync m16n8k16 tiles laid out
 //     transposed: S^T = K Q^T (M = 16 tokens, N = 8 heads) and O^T += V^T P^T
-//     (M = channels, N = heads), with P^T made by movmatrix -- the heads fill N
-//     exactly, so no MMA work or accumulator register goes to padding, and
-//     issue slots go to moving bytes rather than to dot-product reductions;
-//   * at the end of a segment each warp writes its own normalised partial
-//     (o, lse) -- no cross-warp exchange, the ring keeps streaming -- and bumps
-//     the unit's counter; the warp that completes the count merges all of the
-//     unit's partials: out = sum_i 2^(lse_i - lse) o_i, lse = log2 sum_i 2^lse_i.
+//     with P^T from movmatrix, so the heads fill N exactly;
+//   * at the end of a segment each consumer warp writes its own normalised
+//     partial (o, lse) -- no cross-warp exchange, the ring keeps streaming.
+// decode_merge_kernel (one CTA per unit) then combines a unit's partials:
+// out = sum_i 2^(lse_i - lse) o_i, lse = log2 sum_i 2^lse_i.
 //
-// Partial slots.  Segment (CTA c, unit u) uses slot c + u: along the flat list
-// both c and u never decrease and one of them grows at every segment boundary,
-// so slots are distinct, and unit u's slots are the contiguous run
-// c_first(u) + u .. c_last(u) + u.  Slots <= P + units - 1.
+// Partial slots.  Segment (range r, unit u) uses slot r + u: along the flat
+// list both r and u never decrease and one of them grows at every segment
+// boundary, so slots are distinct, and unit u's slots are the contiguous run
+// r_first(u) + u .. r_last(u) + u.  Slots <= Re + units - 1.
 //
 // Bytes per selected page: 2 * 64 * d * 2 (K and V); the kernel is HBM-bound.
 // Tokens outside the attended set (past seq_len; outside the Lambda set of a
@@ -107,22 +102,29 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
-// By one block of 1024 threads, once every unit's selection is written.
-// off[u] = sum_{u' < u} min(sel_n[u'], kcap), off[units] = T; with Re = min(R, T)
-// ranges sharing the pages, range_unit[r] = unit holding flat position
-// floor(r T / Re) for r < Re; the range counter zeroed for the attention
-// kernel.  Units with nothing selected get their output here: out = 0, lse = -inf.
-__device__ __forceinline__ void decode_partition(const int32_t* sel_n, int units, int kcap, int R, int G, int D,
-                                                 int32_t* off, int32_t* range_unit, int32_t* range_counter,
-                                                 bf16* out, float* lse_out) {
+// The plan of the attention grid, by one block (any multiple of 32 threads).
+// The selection sizes are known from the sequence lengths alone
+// (unit_selected(), the counts the top-k blocks write), so this runs beside
+// the top-k blocks instead of after them.  off[u] = pages selected before unit
+// u, off[units] = T; with Re = ranges_in_use(R, T) ranges sharing the pages,
+// range_unit[r] = unit holding flat position floor(r T / Re) for r < Re; the
+// range counter zeroed for the attention kernel.  Units with nothing selected
+// get their output here: out = 0, lse = -inf.
+__device__ __forceinline__ void decode_partition(const int32_t* __restrict__ seq_lens,
+                                                 const uint8_t* __restrict__ head_kind, int Hkv, int maxP,
+                                                 int budget_pages, int sink, int local, int units, int kcap, int R,
+                                                 int G, int D, int32_t* off, int32_t* range_unit,
+                                                 int32_t* range_counter, bf16* out, float* lse_out) {
   __shared__ int s_warp[32];
   __shared__ int s_carry;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x, nw = nt >> 5;
   if (tid == 0) s_carry = 0;
   __syncthreads();
-  for (int base = 0; base < units; base += 1024) {
+  for (int base = 0; base < units; base += nt) {
     const int u = base + tid;
-    const int v = u < units ? min(max(__ldcg(sel_n + u), 0), kcap) : 0;
+    const int v = u < units ? unit_selected(seq_lens[u / Hkv], maxP, head_kind[u % Hkv] == LSERVE_HEAD_DENSE,
+                                            budget_pages, sink, local, kcap)
+                            : 0;
     int x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -132,19 +134,19 @@ __device__ __forceinline__ void decode_partition(const int32_t* sel_n, int units
     if (lane == 31) s_warp[warp] = x;
     __syncthreads();
     if (warp == 0) {
-      int w = s_warp[lane];
+      int w = lane < nw ? s_warp[lane] : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, w, o);
         if (lane >= o) w += y;
       }
-      s_warp[lane] = w;
+      if (lane < nw) s_warp[lane] = w;
     }
     __syncthreads();
     const int carry = s_carry;
     if (u < units) off[u] = carry + (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
     __syncthreads();
-    if (tid == 1023) s_carry = carry + s_warp[31];
+    if (tid == nt - 1) s_carry = carry + s_warp[nw - 1];
     __syncthreads();
   }
   const long long T = s_carry;
@@ -154,7 +156,7 @@ __device__ __forceinline__ void decode_partition(const int32_t* sel_n, int units
   }
   __syncthreads();   // off[] of this block is visible to the block from here on
   const long long Re = ranges_in_use(R, T);   // every range below Re gets >= 1 page
-  for (int u = tid; u < units; u += 1024) {
+  for (int u = tid; u < units; u += nt) {
     const long long a = off[u], e = off[u + 1];
     if (e == a) {   // nothing selected: out = 0, lse = -inf
       for (int idx = 0; idx < G * D; idx += 8)
@@ -170,14 +172,24 @@ __device__ __forceinline__ void decode_partition(const int32_t* sel_n, int units
   }
 }
 
-// One CTA of 1024 threads after the top-k grid (whose sel_n it reads after the
-// dependency wait, with L2 loads).
-__global__ void __launch_bounds__(1024) decode_partition_kernel(const int32_t* sel_n, int units, int kcap, int R,
-                                                                int G, int D, int32_t* off, int32_t* range_unit,
-                                                                int32_t* range_counter, bf16* out, float* lse_out) {
-  pdl_launch_dependents();   // the attention grid may get resident; it waits for this grid
+// Selection step: blocks 0 .. units-1 select the pages of one unit each
+// (topk_unit); block `units` lays out the attention grid's work
+// (decode_partition), which does not depend on the selected pages.
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_pages_kernel(
+    const float* scores, int maxP, const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind,
+    int Hkv, int budget_pages, int sink, int local, int32_t* sel, int32_t* sel_n, int kcap, int units, int R, int G,
+    int D, int32_t* off, int32_t* range_unit, int32_t* range_counter, bf16* out, float* lse_out) {
+  const int unit = blockIdx.x;
+  // sequence length and head kind are inputs of the step, not results of the scoring grid
+  const int L = unit < units ? seq_lens[unit / Hkv] : 0;
+  const bool dense = unit < units && head_kind[unit % Hkv] == LSERVE_HEAD_DENSE;
   pdl_wait();
-  decode_partition(sel_n, units, kcap, R, G, D, off, range_unit, range_counter, out, lse_out);
+  pdl_launch_dependents();   // the attention grid may get resident; it waits for this grid
+  if (unit < units)
+    topk_unit(scores, unit, maxP, L, dense, budget_pages, sink, local, sel, sel_n, kcap);
+  else
+    decode_partition(seq_lens, head_kind, Hkv, maxP, budget_pages, sink, local, units, kcap, R, G, D, off,
+                     range_unit, range_counter, out, lse_out);
 }
 
 // Spin (with short sleeps) until cond() holds; false (and LSERVE_ERR_DEVICE_TIMEOUT
@@ -357,6 +369,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
   } else if (warp == kIssuerWarp) {
     // ---- issue each resolved page's loads once its stage is free
     if (lane == 0) {
+      const uint64_t pol = l2_evict_first();   // every page is read once per step
       for (int gp = 0;; ++gp) {
         if (!spin_until([&] { return *v_resolved > gp || *v_total <= gp || *v_abort; }, timeout_ns)) {
           *v_abort = 1;
@@ -379,8 +392,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
         const int row = (p * Hkv + g) * kPage;
 #pragma unroll
         for (int x = 0; x < Cfg::kBoxes; ++x) {
-          tma_load_2d(kdst + x * Cfg::kBoxBytes, &tmK, &full_bar[st], x * 64, row);
-          tma_load_2d(vdst + x * Cfg::kBoxBytes, &tmV, &full_bar[st], x * 64, row);
+          tma_load_2d_hint(kdst + x * Cfg::kBoxBytes, &tmK, &full_bar[st], x * 64, row, pol);
+          tma_load_2d_hint(vdst + x * Cfg::kBoxBytes, &tmV, &full_bar[st], x * 64, row, pol);
         }
         if (with_q) bulk_load(vdst + Cfg::kKVBytes, q + static_cast<long>(md.x) * G * D, q_bytes, &full_bar[st]);
         *v_issued = gp + 1;
@@ -575,11 +588,13 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const int32
                                                                      float* __restrict__ lse_out) {
   __shared__ float4 s_o[kMergeThreads];
   __shared__ float2 s_ml[kMergeThreads];
-  pdl_wait();   // the partials come from the attention grid: read after this, with L2 loads
+  // the plan and the partials come from the previous grids: read after the
+  // wait, with L2 loads
+  pdl_wait();
   const int u = blockIdx.x;
   const long long T = __ldcg(off + units);
   const long long a = __ldcg(off + u), e = __ldcg(off + u + 1);
-  if (T <= 0 || e <= a) return;   // nothing selected: written by the partition kernel
+  if (T <= 0 || e <= a) return;   // nothing selected: written by the partition block
   const long long Re = ranges_in_use(R, T);
   const int c_first = flat_owner(a, T, Re), c_last = flat_owner(e - 1, T, Re);
   if (c_first < 0 || c_last < c_first || c_last >= Re) {

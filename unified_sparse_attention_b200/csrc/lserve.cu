@@ -362,12 +362,19 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
                               void* out, float* lse, cudaStream_t st) {
   if (p.G == 1) {
     // one query head per KV head: per-lane fp32 products over 16-byte summary
-    // loads, one warp per (page, dense head), ~4 CTAs per SM
-    const long long pages = static_cast<long long>(a->B) * a->maxP;
-    const int ppb = static_cast<int>(std::max(4ll, std::min<long long>(pages / (4ll * sm_count()), 64)));
-    score_pages_kernel<D, 1><<<dim3((a->maxP + ppb - 1) / ppb, a->B), 256, 0, st>>>(
-        static_cast<const bf16*>(a->q), static_cast<const bf16*>(a->stats), a->page_table, a->maxP, a->seq_lens,
-        a->head_kind, a->Hkv, a->num_pages, ppb, p.scores);
+    // loads, one warp per (page, dense head); exactly one wave of CTAs, each
+    // with an equal share of the (sequence, dense head, page) list
+    static const int occ = [] {
+      int o = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, score_pages_kernel<D, 1>, 256, 0) != cudaSuccess) o = 0;
+      return std::max(1, o);
+    }();
+    const long long work = static_cast<long long>(a->B) * a->Hkv * a->maxP;
+    const int grid = static_cast<int>(std::max(1ll, std::min<long long>(static_cast<long long>(sm_count()) * occ,
+                                                                        (work + 63) / 64)));
+    score_pages_kernel<D, 1><<<grid, 256, 0, st>>>(
+        static_cast<const bf16*>(a->q), static_cast<const bf16*>(a->stats), a->page_table, a->B, a->maxP,
+        a->seq_lens, a->head_kind, a->Hkv, a->num_pages, p.scores);
   } else {
     // G query heads per KV head: the bound as a contraction on the tensor cores,
     // one wave of SMs x resident CTAs (fewer when there is less work)
@@ -382,14 +389,12 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
   ensure_smem(topk_pages_kernel, kTopkSmemKeys * static_cast<int>(sizeof(uint32_t)));
   const int topk_smem = std::min(a->maxP, kTopkSmemKeys) * static_cast<int>(sizeof(uint32_t));
   const int units = a->B * a->Hkv;
-  if (launch_pdl(topk_pages_kernel, dim3(units), dim3(kTopkThreads), topk_smem, st,
+  // one block per unit selects its pages; one more lays out the attention grid's work
+  if (launch_pdl(topk_pages_kernel, dim3(units + 1), dim3(kTopkThreads), topk_smem, st,
                  static_cast<const float*>(p.scores), a->maxP, a->seq_lens, a->head_kind, a->Hkv, p.budget_pages,
-                 a->sink, a->local, sel, sel_n, p.kcap) != cudaSuccess)
+                 a->sink, a->local, sel, sel_n, p.kcap, units, p.R, p.G, D, p.off, p.range_unit, p.range_counter,
+                 static_cast<bf16*>(out), lse) != cudaSuccess)
     return check_launch("decode top-k");
-  if (launch_pdl(decode_partition_kernel, dim3(1), dim3(1024), 0, st, static_cast<const int32_t*>(sel_n), units,
-                 p.kcap, p.R, p.G, D, p.off, p.range_unit, p.range_counter, static_cast<bf16*>(out), lse) !=
-      cudaSuccess)
-    return check_launch("decode partition");
   CUtensorMap tk, tv;
   const uint64_t rows = static_cast<uint64_t>(a->num_pages) * a->Hkv * kPage;
   if (!make_map_2d(&tk, a->k_pages, D, rows) || !make_map_2d(&tv, a->v_pages, D, rows))

@@ -15,11 +15,12 @@
 //   score_pages_mma_kernel (G >= 2): the same bound as a contraction on the
 //     tensor cores (see there); per-lane products would cost G x as much issue.
 //
-// topk_pages_kernel  (latency-bound, one CTA per (sequence, KV head))
-//   k = min(budget/64, n_pages) pages by 4-pass 8-bit radix select on the
-//   order-preserving uint32 image of the fp32 scores, ties to the lower page
-//   index, emitted in ascending page order by a block-wide scan.  Streaming
-//   heads get their fixed sink + local page list from the same kernel.
+// topk_unit  (latency-bound, one CTA per (sequence, KV head); the kernel that
+//   runs it is in decode.cuh)
+//   k = min(budget/64, n_pages) pages by radix select (8-bit digits below the
+//   bits all keys share) on the order-preserving uint32 image of the fp32
+//   scores, ties to the lower page index, emitted in ascending page order by a
+//   block-wide scan.  Streaming heads get their fixed sink + local page list.
 #pragma once
 
 #include "common.cuh"
@@ -27,18 +28,23 @@
 namespace lserve {
 
 // ------------------------------------------------------------------ scoring
+// Per-lane fp32 products (one query head per KV head).  The work -- every
+// (sequence, dense KV head, page) -- is one flat list, v = (b * ndense + i_g) *
+// maxP + page, cut into gridDim.x equal contiguous shares (one wave of CTAs,
+// so that no SM is left with an extra CTA's worth of pages at the end); a warp
+// takes every nwarps-th (page, head) of its CTA's share and scores its four
+// logical pages with 16-byte loads.
 template <int D, int G>
-__global__ void __launch_bounds__(256) score_pages_kernel(
-    const bf16* __restrict__ q, const bf16* __restrict__ stats, const int32_t* __restrict__ page_table, int maxP,
-    const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind, int Hkv, int num_pages,
-    int pages_per_block, float* __restrict__ scores) {
+__global__ void __launch_bounds__(256, 5) score_pages_kernel(
+    const bf16* __restrict__ q, const bf16* __restrict__ stats, const int32_t* __restrict__ page_table, int B,
+    int maxP, const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind, int Hkv, int num_pages,
+    float* __restrict__ scores) {
   constexpr int CPL = D / 8;   // channels per lane
   __shared__ int s_dense[256];
   __shared__ int s_ndense;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
-  const int b = blockIdx.y;
   if (threadIdx.x == 0) {
     int n = 0;
     for (int g = 0; g < Hkv; ++g)
@@ -46,31 +52,36 @@ __global__ void __launch_bounds__(256) score_pages_kernel(
     s_ndense = n;
   }
   __syncthreads();
-  const int L = seq_lens[b];
-  const int n_pages = min(maxP, (L + kPage - 1) / kPage);
-  const int i0 = blockIdx.x * pages_per_block;
-  const int i1 = min(i0 + pages_per_block, n_pages);
-  if (i0 >= i1) return;
-  const int npg = i1 - i0;
-  const int units = s_ndense * npg;
+  const long long V = static_cast<long long>(B) * s_ndense * maxP;
+  const long long v0 = V * blockIdx.x / gridDim.x, v1 = V * (blockIdx.x + 1) / gridDim.x;
   const int l = lane >> 3;           // logical page of this lane
   const int c0 = (lane & 7) * CPL;   // first channel of this lane
   const float ninf = kNegInf;
 
-  int cur_g = -1;
+  int cur_bg = -1, L = 0, n_pages = 0;
   float qf[G][CPL];
-  for (int u = warp; u < units; u += nwarps) {
-    const int g = s_dense[u / npg];
-    const int i = i0 + u % npg;
-    if (g != cur_g) {
-      cur_g = g;
+  int bgi = static_cast<int>((v0 + warp) / maxP);                   // b * ndense + i_g
+  int i = static_cast<int>(v0 + warp - static_cast<long long>(bgi) * maxP);   // page
+  auto advance = [&] {
+    i += nwarps;
+    while (i >= maxP) {
+      i -= maxP;
+      ++bgi;
+    }
+  };
+  for (long long v = v0 + warp; v < v1; v += nwarps, advance()) {
+    const int b = bgi / s_ndense, g = s_dense[bgi % s_ndense];
+    if (bgi != cur_bg) {
+      cur_bg = bgi;
+      L = seq_lens[b];
+      n_pages = L > 0 ? min(maxP, (L - 1) / kPage + 1) : 0;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const bf16* qp = q + (static_cast<long>(b) * Hkv * G + g * G + h) * D + c0;
 #pragma unroll
         for (int c = 0; c < CPL; c += 8) {
-          uint4 v = __ldg(reinterpret_cast<const uint4*>(qp + c));
-          const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
+          uint4 u = __ldg(reinterpret_cast<const uint4*>(qp + c));
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             qf[h][c + 2 * e] = bf16_lo(w[e]);
@@ -79,6 +90,7 @@ __global__ void __launch_bounds__(256) score_pages_kernel(
         }
       }
     }
+    if (i >= n_pages) continue;   // past the sequence: no score
     const int p = page_table[static_cast<long>(b) * maxP + i];
     float s = ninf;
     if (p >= 0 && p < num_pages) {
@@ -161,6 +173,7 @@ __global__ void __launch_bounds__(kScoreThreads, kScoreCtasPerSm) score_pages_mm
   const long long it1 = min(items, it0 + per);
   const int r = lane >> 2, t = lane & 3;   // fragment row (and row + 8), lane of the quad
   const float ninf = kNegInf;
+  const uint64_t pol = l2_evict_first();
 
   struct Item {
     int b, g, ib, n_pages, L;
@@ -209,7 +222,7 @@ __global__ void __launch_bounds__(kScoreThreads, kScoreCtasPerSm) score_pages_mm
                       : nullptr;
 #pragma unroll
       for (int j = 0; j < NJ; ++j)
-        a[j][h] = srow ? __ldg(reinterpret_cast<const uint4*>(srow + 32 * j)) : make_uint4(0u, 0u, 0u, 0u);
+        a[j][h] = srow ? ld_once_u4(srow + 32 * j, pol) : make_uint4(0u, 0u, 0u, 0u);
     }
     if (it + 1 < it1) nx = locate(it + 1);   // the next item's pages load meanwhile
     if (m.b != cur_b || m.g != cur_g) {
@@ -309,44 +322,85 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkSmemKeys = 16384;   // scores cached in shared memory up to this many pages
 
-// One block per unit (b, g) = blockIdx.x.  The scores come from the scoring
-// kernel, which may still be running: they are read only after the dependency
-// wait, with L2 loads through a pointer that is not restrict-qualified (no load
-// of them can move above the wait).
-__global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
-    const float* scores, int maxP, const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind,
-    int Hkv, int budget_pages, int sink, int local, int32_t* sel, int32_t* sel_n, int kcap) {
-  pdl_launch_dependents();   // the one-CTA partition grid may get resident; it waits for this grid
-  pdl_wait();
+// Pages of a sequence of L tokens.
+__device__ __forceinline__ int seq_pages(int L) { return L > 0 ? (L - 1) / kPage + 1 : 0; }
+
+// Streaming head over the n pages of a sequence of L tokens: the pages holding
+// a token of [0, sink) or [L - local, L) are [0, a) and [bb, bb + cnt - a);
+// returns cnt.
+__device__ __forceinline__ int streaming_pages(int L, int n, int sink, int local, int& a, int& bb) {
+  const int w0 = local > 0 ? max(0, L - local) / kPage : n;   // first window page
+  const int w1 = local > 0 ? seq_pages(L) : n;                 // one past the last
+  a = min(seq_pages(min(sink, L)), n);
+  bb = max(w0, a);
+  return L > 0 ? a + max(0, min(w1, n) - bb) : 0;
+}
+
+// Pages the selection keeps for one unit (sequence of L tokens, one KV head):
+// a dense head min(budget, pages), a streaming head its sink and window pages,
+// at most kcap.  topk_unit() writes exactly this many.
+__device__ __forceinline__ int unit_selected(int L, int maxP, bool dense, int budget_pages, int sink, int local,
+                                             int kcap) {
+  L = max(0, L);
+  const int n = min(seq_pages(L), maxP);
+  if (dense) return min(budget_pages, n);
+  int a, bb;
+  return min(streaming_pages(L, n, sink, local, a, bb), kcap);
+}
+
+// Block-wide exclusive scan of one 64-bit value per thread (two packed 32-bit
+// counts); returns the prefix.  Needs blockDim.x/32 values of scratch.
+__device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned long long v,
+                                                                     unsigned long long* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  unsigned long long before = x - v;
+  for (int w = 0; w < warp; ++w) before += scratch[w];   // broadcast reads, no second barrier
+  return before;
+}
+
+// Top-k pages of one unit (b, g) = `unit`, by one block.  The scores come from
+// the scoring kernel, which may still be running when the block starts: they
+// are read only after the caller's dependency wait, with L2 loads through a
+// pointer that is not restrict-qualified (no load of them can move above it).
+// Dense head: k = min(budget, pages) pages with the largest scores, ties to
+// the lower index, written in ascending order.  Radix select over the order-
+// preserving integer keys: the digits start below the bits that all keys
+// share, a pass costs two barriers (the histogram of the next pass is cleared
+// while this one fills), and the search ends once the k-th key's bin is
+// taken whole; one scan of (above, equal) counts places the output.
+__device__ __forceinline__ void topk_unit(const float* scores, int unit, int maxP, int L, bool dense,
+                                          int budget_pages, int sink, int local, int32_t* sel, int32_t* sel_n,
+                                          int kcap) {
   extern __shared__ uint32_t s_keys[];
-  __shared__ int s_hist[256];
-  __shared__ int s_scan[32];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_remaining, s_count;
+  __shared__ __align__(16) int s_hist[2][256];
+  __shared__ unsigned long long s_scan[32];
   __shared__ uint32_t s_mm[2][32];
-  const int unit = blockIdx.x;   // b * Hkv + g
-  const int b = unit / Hkv, g = unit % Hkv;
-  const int L = max(0, seq_lens[b]);
-  int n = (L + kPage - 1) / kPage;
+  __shared__ int s_step[3];   // prefix, remaining, count of the k-th key's bin
+  L = max(0, L);
+  int n = seq_pages(L);
   if (n > maxP) {   // sequence longer than its page-table row
     if (threadIdx.x == 0) report(LSERVE_ERR_DEVICE_BOUNDS);
     n = maxP;
   }
   int32_t* row = sel + static_cast<long>(unit) * kcap;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, nt = blockDim.x;
 
-  if (head_kind[g] != LSERVE_HEAD_DENSE) {
-    // pages holding a token of [0, sink) or [L - local, L)
-    const int n_sink = (min(sink, L) + kPage - 1) / kPage;
-    const int w0 = local > 0 ? max(0, L - local) / kPage : n;   // first window page
-    const int w1 = local > 0 ? (L - 1) / kPage + 1 : n;         // one past the last
-    const int a = min(n_sink, n), bb = max(w0, a);
-    int cnt = L > 0 ? a + max(0, min(w1, n) - bb) : 0;
+  if (!dense) {
+    int a, bb;
+    int cnt = streaming_pages(L, n, sink, local, a, bb);
     if (cnt > kcap) {
       if (tid == 0) report(LSERVE_ERR_DEVICE_BOUNDS);
       cnt = kcap;
     }
-    for (int j = tid; j < kcap; j += blockDim.x) {
+    for (int j = tid; j < kcap; j += nt) {
       int v = -1;
       if (j < a) v = j;
       else if (j < cnt) v = bb + (j - a);
@@ -358,26 +412,35 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
 
   const int k = min(budget_pages, n);
   if (k >= n) {
-    for (int j = tid; j < kcap; j += blockDim.x) row[j] = j < n ? j : -1;
+    for (int j = tid; j < kcap; j += nt) row[j] = j < n ? j : -1;
     if (tid == 0 && sel_n) sel_n[unit] = n;
     return;
   }
   const float* srow = scores + static_cast<long>(unit) * maxP;
   const bool cached = n <= kTopkSmemKeys;
-  if (cached)
-    for (int j = tid; j < n; j += blockDim.x) s_keys[j] = order_key(__ldcg(srow + j));
-  __syncthreads();
   auto key_at = [&](int j) -> uint32_t { return cached ? s_keys[j] : order_key(__ldcg(srow + j)); };
 
-  // The bits above the highest one in which the keys differ are common to all
-  // of them (scores of similar magnitude share sign and exponent): the radix
-  // digits start below them, so that no pass piles every key into one bin.
+  // keys (cached), their min and max, both histograms cleared
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int j = tid; j < n; j += blockDim.x) {
-    const uint32_t kk = key_at(j);
-    kmin = min(kmin, kk);
-    kmax = max(kmax, kk);
+  for (int j0 = 0; j0 < n; j0 += 4 * nt) {   // four independent loads in flight per thread
+    float f[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = j0 + r * nt + tid;
+      f[r] = j < n ? __ldcg(srow + j) : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = j0 + r * nt + tid;
+      if (j < n) {
+        const uint32_t kk = order_key(f[r]);
+        if (cached) s_keys[j] = kk;
+        kmin = min(kmin, kk);
+        kmax = max(kmax, kk);
+      }
+    }
   }
+  for (int j = tid; j < 2 * 256; j += nt) (&s_hist[0][0])[j] = 0;
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   if ((tid & 31) == 0) {
@@ -385,48 +448,42 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
     s_mm[1][tid >> 5] = kmax;
   }
   __syncthreads();
-  if (tid < 32) {
-    const int nw = blockDim.x >> 5;
-    kmin = __reduce_min_sync(0xffffffffu, tid < nw ? s_mm[0][tid] : 0xffffffffu);
-    kmax = __reduce_max_sync(0xffffffffu, tid < nw ? s_mm[1][tid] : 0u);
-    if (tid == 0) {
-      s_mm[0][0] = kmin;
-      s_mm[1][0] = kmax;
-    }
+  for (int w = 0; w < (nt >> 5); ++w) {   // every thread reduces the per-warp values itself
+    kmin = min(kmin, s_mm[0][w]);
+    kmax = max(kmax, s_mm[1][w]);
   }
-  __syncthreads();
-  kmin = s_mm[0][0];
-  kmax = s_mm[1][0];
+  // The bits above the highest one in which the keys differ are common to all
+  // of them (scores of similar magnitude share sign and exponent): the radix
+  // digits start below them, so that no pass piles every key into one bin.
   int shift = (kmin ^ kmax) ? 32 - __clz(kmin ^ kmax) : 0;   // low bits still to resolve
   uint32_t mask = shift >= 32 ? 0u : ~((1u << shift) - 1u);    // bits fixed so far
   uint32_t prefix = kmax & mask;                                // their value for the k-th key
   int remaining = k;                                            // keys still to take at prefix
+  int pass = 0;
   // 8-bit digits (the first may be narrower); a pass ends the search when the
   // k-th key's bin is taken whole -- the lower bits need not be resolved
 #pragma unroll 1
   while (shift > 0) {
     const int w = min(8, shift);
     shift -= w;
-    for (int j = tid; j < 256; j += blockDim.x) s_hist[j] = 0;
-    __syncthreads();
-    for (int j = tid; j < n; j += blockDim.x) {
+    int* hist = s_hist[pass & 1];
+    for (int j = tid; j < n; j += nt) {
       const uint32_t kk = key_at(j);
-      if ((kk & mask) == prefix) atomicAdd(&s_hist[(kk >> shift) & ((1u << w) - 1u)], 1);
+      if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & ((1u << w) - 1u)], 1);
     }
+    // the other histogram was last read before the previous pass's final barrier
+    for (int j = tid; j < 256; j += nt) s_hist[(pass + 1) & 1][j] = 0;
     __syncthreads();
     if (tid < 32) {
       // lane t owns digits 8t..8t+7; find the digit holding the remaining-th largest
-      int c[8], sum = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        c[e] = s_hist[tid * 8 + e];
-        sum += c[e];
-      }
-      // inclusive suffix sum over lanes (sum of lanes >= tid)
-      int suf = sum;
+      const int4 h0 = *reinterpret_cast<const int4*>(hist + tid * 8);
+      const int4 h1 = *reinterpret_cast<const int4*>(hist + tid * 8 + 4);
+      const int c[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+      const int sum = ((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7]));
+      int suf = sum;   // inclusive suffix sum over lanes (sum of lanes >= tid)
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_down_sync(0xffffffffu, suf, o);
+        const int y = __shfl_down_sync(0xffffffffu, suf, o);
         if (tid + o < 32) suf += y;
       }
       const int above = suf - sum;   // keys with a higher digit
@@ -441,48 +498,43 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pages_kernel(
             acc += c[e];
           }
         }
-        s_prefix = prefix | (static_cast<uint32_t>(digit) << shift);
-        s_remaining = remaining - acc;
-        s_count = cnt;
+        s_step[0] = static_cast<int>(prefix | (static_cast<uint32_t>(digit) << shift));
+        s_step[1] = remaining - acc;
+        s_step[2] = cnt;
       }
     }
     __syncthreads();
-    prefix = s_prefix;
+    prefix = static_cast<uint32_t>(s_step[0]);
     mask |= ((1u << w) - 1u) << shift;
-    remaining = s_remaining;
-    if (s_count == remaining) break;   // the whole bin is taken
+    remaining = s_step[1];
+    ++pass;
+    if (s_step[2] == remaining) break;   // the whole bin is taken
   }
   // keys compare on the fixed bits: above T is taken, at T the lowest indices
   const uint32_t T = prefix;
   const int take_eq = remaining;
 
-  // ascending emission: each thread owns a contiguous run of indices
-  const int per = (n + blockDim.x - 1) / blockDim.x;
+  // ascending emission: each thread owns a contiguous run of indices; one scan
+  // of the packed counts (equal << 32 | above) gives every thread its place
+  const int per = (n + nt - 1) / nt;
   const int j0 = min(n, tid * per), j1 = min(n, j0 + per);
-  int n_eq = 0;
-  for (int j = j0; j < j1; ++j) n_eq += (key_at(j) & mask) == T;
-  int tot;
-  int eq_before = block_exclusive_scan(n_eq, s_scan, &tot);
-  int n_sel = 0;
-  {
-    int e = eq_before;
-    for (int j = j0; j < j1; ++j) {
-      const uint32_t kk = key_at(j) & mask;
-      if (kk > T) ++n_sel;
-      else if (kk == T) n_sel += (e++ < take_eq);
-    }
+  unsigned int n_eq = 0, n_gt = 0;
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t kk = key_at(j) & mask;
+    n_eq += kk == T;
+    n_gt += kk > T;
   }
-  int sel_before = block_exclusive_scan(n_sel, s_scan, &tot);
-  {
-    int e = eq_before, pos = sel_before;
-    for (int j = j0; j < j1; ++j) {
-      const uint32_t kk = key_at(j) & mask;
-      bool take = kk > T;
-      if (kk == T) take = (e++ < take_eq);
-      if (take && pos < kcap) row[pos++] = j;
-    }
+  const unsigned long long before =
+      block_exclusive_scan64((static_cast<unsigned long long>(n_eq) << 32) | n_gt, s_scan);
+  int e = static_cast<int>(before >> 32);
+  int pos = static_cast<int>(before & 0xffffffffu) + min(e, take_eq);
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t kk = key_at(j) & mask;
+    bool take = kk > T;
+    if (kk == T) take = (e++ < take_eq);
+    if (take && pos < kcap) row[pos++] = j;
   }
-  for (int j = k + tid; j < kcap; j += blockDim.x) row[j] = -1;
+  for (int j = k + tid; j < kcap; j += nt) row[j] = -1;
   if (tid == 0 && sel_n) sel_n[unit] = k;
 }
 
