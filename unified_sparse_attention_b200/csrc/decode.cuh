@@ -611,19 +611,32 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const int32
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
   if (pg < groups) {
     const float4* po = reinterpret_cast<const float4*>(part_o) + first * n4 + q4;
-#pragma unroll 4
-    for (int x = pg; x < nparts; x += groups) {
-      const float lx = __ldcg(part_lse + (first + x) * G + h);
-      const float4 v = __ldcg(po + static_cast<long>(x) * n4);
-      if (lx == kNegInf) continue;   // an empty partial (its o is 0)
-      const float mn = fmaxf(m, lx);
-      const float sc = fast_exp2(m - mn), w = fast_exp2(lx - mn);
-      m = mn;
-      l = l * sc + w;
-      o.x = o.x * sc + w * v.x;
-      o.y = o.y * sc + w * v.y;
-      o.z = o.z * sc + w * v.z;
-      o.w = o.w * sc + w * v.w;
+    // eight partials per thread in flight at once: one L2 round trip for a unit
+    // of up to 8 * groups partials
+    for (int x0 = pg; x0 < nparts; x0 += 8 * groups) {
+      float lx[8];
+      float4 v[8];
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const int x = x0 + s * groups;
+        lx[s] = kNegInf;
+        if (x < nparts) {
+          lx[s] = __ldcg(part_lse + (first + x) * G + h);
+          v[s] = __ldcg(po + static_cast<long>(x) * n4);
+        }
+      }
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        if (lx[s] == kNegInf) continue;   // no partial, or an empty one (its o is 0)
+        const float mn = fmaxf(m, lx[s]);
+        const float sc = fast_exp2(m - mn), w = fast_exp2(lx[s] - mn);
+        m = mn;
+        l = l * sc + w;
+        o.x = o.x * sc + w * v[s].x;
+        o.y = o.y * sc + w * v[s].y;
+        o.z = o.z * sc + w * v[s].z;
+        o.w = o.w * sc + w * v[s].w;
+      }
     }
   }
   s_o[tid] = o;

@@ -319,7 +319,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
   return before;
 }
 
-constexpr int kTopkThreads = 1024;
+constexpr int kTopkThreads = 512;
 constexpr int kTopkSmemKeys = 16384;   // scores cached in shared memory up to this many pages
 
 // Pages of a sequence of L tokens.
