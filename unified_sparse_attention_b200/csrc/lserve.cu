@@ -231,6 +231,15 @@ lserve_status launch_prefill_tc(const lserve_shape* s, const void* q, const void
       !make_map_3d(&tv, v, D, s->Hkv, Tn))
     return fail(LSERVE_ERR_CUDA, "prefill: cuTensorMapEncodeTiled failed");
   ensure_smem(tc::prefill_tc_kernel<D>, C::kSmem);
+  // the kernel's register split (setmaxnreg) needs the launch to hand out at
+  // least kRegsNeeded registers per thread, or its warpgroups would wait forever
+  static const int regs = [] {
+    cudaFuncAttributes fa{};
+    return cudaFuncGetAttributes(&fa, tc::prefill_tc_kernel<D>) == cudaSuccess ? fa.numRegs : 0;
+  }();
+  if (regs < C::kRegsNeeded)
+    return fail(LSERVE_ERR_UNSUPPORTED, "prefill: kernel built with %d registers per thread, its split needs %d",
+                regs, C::kRegsNeeded);
   const long long grid = static_cast<long long>(n_rows) * T.hsplit;
   tc::prefill_tc_kernel<D><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, st>>>(tq, tk, tv, T);
   return check_launch("prefill attention (tcgen05)");

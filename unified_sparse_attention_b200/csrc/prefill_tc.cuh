@@ -12,26 +12,31 @@
 // row); with G = 1 they are two adjacent query tiles of one head walking the
 // union of their tile lists.
 //
-// Warp roles (320 threads, one CTA per SM):
-//   warp 0     TMA producer (one elected lane issues): Q once, then K and V of
+// Warp roles (384 threads, one CTA per SM; the third warpgroup hands registers
+// to the two softmax warpgroups with setmaxnreg):
+//   warp 8     TMA producer (one elected lane issues): Q once, then K and V of
 //              every listed tile pair into shared-memory rings (128-byte
 //              swizzle); K stages are released after the S MMAs, V stages after
 //              the PV MMAs.
-//   warp 1     allocates TMEM; runs the MMA loop converged, one elected lane
+//   warp 9     allocates TMEM; runs the MMA loop converged, one elected lane
 //              issues tcgen05.mma and tcgen05.commit:
 //                S[x]  = Q [K_a;K_b]^T      (M=128, N=128, K=d; A and B from smem)
 //                O[x] += P[x] [V_a;V_b]     (M=128, N=d, K=128; P from TMEM)
 //              for step p on stream x = p & 1, in the order S(0) S(1) PV(0) S(2)
 //              PV(1) S(3) ...
-//   warps 2-9  two softmax warpgroups, one per stream (thread = query row): the
+//   warps 0-7  two softmax warpgroups, one per stream (thread = query row): the
 //              steps of a row are split between two independent online
-//              softmaxes (own running max, sum and accumulator), which run out of
+//              softmaxes (own reference, sum and accumulator), which run out of
 //              phase and keep both the exponential unit and the tensor core busy;
-//              tcgen05.ld of S, exact element mask, base-2 exponentials with lazy
-//              rescaling (O[x] is rescaled only when its running max grows by more
-//              than 2^8), P packed to bf16 over S with tcgen05.st.  The epilogue
-//              merges the two streams by log-sum-exp; each warpgroup normalises and
-//              stores half of the output columns.
+//              tcgen05.ld of S, exact element mask, base-2 exponentials in one
+//              pass against a reference that moves only when the row sum shows
+//              that it must: the first step of a stream takes the exact row max
+//              (its largest weight is then exactly 1 in bf16); a row sum above
+//              2^40 redoes a step against the exact row max; one above 2^12
+//              moves the reference to the largest weight at the stream's next
+//              step.  P is packed to bf16 over S with tcgen05.st.  The epilogue
+//              merges the two streams by log-sum-exp; each warpgroup normalises
+//              and stores half of the output columns.
 // TMEM (512 columns): O[0] at 0, O[1] at 128, S[0] at 256, S[1] at 384; P[x]
 // (bf16 pairs) is aliased over the first 64 columns of S[x].
 #pragma once
@@ -198,7 +203,16 @@ struct Cfg {
   // TMEM allocation) is resident per SM
   static constexpr int kSmemUsed = kQTile + (kKStages + kVStages) * kPair + 1024;
   static constexpr int kSmem = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
-  static constexpr int kThreads = 64 + 256;   // producer, MMA, two softmax warpgroups
+  // warps 0-7: two softmax warpgroups; warp 8: TMA producer; warp 9: MMA issue;
+  // warps 10-11 complete the third warpgroup so that it can hand registers to
+  // the softmax warpgroups (setmaxnreg acts on whole warpgroups)
+  static constexpr int kThreads = 384;
+  static constexpr int kWarpProducer = 8, kWarpMma = 9;
+  // registers per thread after the split: the launch gives every thread the
+  // kernel's count (168 at 384 threads, one CTA per SM); 128 x kRegsAux +
+  // 256 x kRegsSoftmax must not exceed 384 x that count
+  static constexpr int kRegsAux = 56, kRegsSoftmax = 216;
+  static constexpr int kRegsNeeded = (128 * kRegsAux + 256 * kRegsSoftmax + kThreads - 1) / kThreads;
   // TMEM: O[x] (fp32, D columns) at 128 x; S[x] (fp32, 128 columns) at 256 + 128 x,
   // with P[x] (bf16 pairs, 64 columns) aliased over the first half of S[x]
   static constexpr int kColO = 0;
@@ -272,7 +286,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     s_abort = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == C::kWarpMma) {
     tmem_alloc(&s_tmem, C::kTmemCols);
     tmem_relinquish();
   }
@@ -282,7 +296,11 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   const uint32_t tmem = s_tmem;
   const unsigned long long tmo = A.timeout_ns;
 
-  if (warp == 0) {
+  // Each warpgroup changes its register count at the top of its own branch
+  // (code after a merge of the two would be held to the smaller count).
+  if (warp >= C::kWarpProducer) {   // the third warpgroup gives registers to the softmax
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegsAux));
+   if (warp == C::kWarpProducer) {
     // ================================================================ producer
     // The whole warp walks the list (warp-uniform coordinates); one elected lane issues.
     const bool leader = elect_one();
@@ -333,7 +351,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == C::kWarpMma) {
     // ================================================================== MMA
     // Step p belongs to stream x = p & 1 (S[x], P[x], O[x]).  The whole warp runs
     // the loop (waits and descriptors warp-uniform); one elected lane issues.
@@ -389,11 +407,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         if (p + 2 < np) issue_s(p + 2);
       }
     }
+   }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kRegsSoftmax));
     // ============================================================== softmax
     // Warpgroup x runs an independent online softmax over the steps p = x, x+2, ...
     // with its own (m, l) and accumulator O[x]; the two are merged at the end.
-    const int x = (warp - 2) >> 2;
+    const int x = warp >> 2;
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;    // row within the M-tile
     const int rb = row >> 6;
@@ -615,7 +635,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   }
   fence_before_sync();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == C::kWarpMma) {
     fence_after_sync();
     tmem_dealloc(tmem, C::kTmemCols);
   }
