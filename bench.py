@@ -17,6 +17,7 @@ Prints ONE JSON line on rank 0.  Multi-GPU runs are independent replicas
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -38,6 +39,34 @@ METRIC = "prefill attn ms & kept-tile TFLOPS at 128K; decode attn µs/step & HBM
 PREFILL_WL = "llama3_8b_prefill_128k_vslash"
 DECODE_WL = "llama2_7b_mha"
 L2_BYTES = 126 * 1024 * 1024
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) from a one-pass ncu
+# capture of this script's default workloads (launch list under profiles/):
+# per launch of the prefill attention kernel, and per decode step (stats
+# refresh, scoring, top-k + plan, paged attention, merge).  Reported only while
+# the kernel sources hash as they did when the counters were taken.
+TRAFFIC = {
+    "prefill": {"bytes": 3655072256,
+                "sources": ["prefill_tc.cuh", "prefill_mma.cuh", "tile_lists.cuh", "common.cuh", "lserve.cu"],
+                "sha256": "b50ce53bdada557e5659e799c0a420d1df533369215699f06c93008829cf1f53"},
+    "decode": {"bytes": 821951232,
+               "sources": ["select.cuh", "decode.cuh", "page_stats.cuh", "common.cuh", "lserve.cu"],
+               "sha256": "396ae7de7ed4bbe2020efbe42443793efc02d5f5ba80aadc8e9237ca6ad5d3dd"},
+}
+
+
+def traffic(key, workload_is_default):
+    """Counter-measured DRAM bytes for `key`, or None when the workload is not the
+    captured one or the kernel sources changed since the capture."""
+    t = TRAFFIC[key]
+    if not workload_is_default:
+        return None
+    h = hashlib.sha256()
+    for f in t["sources"]:
+        with open(os.path.join(ROOT, "unified_sparse_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return t["bytes"] if h.hexdigest() == t["sha256"] else None
 
 
 def peaks():
@@ -423,7 +452,7 @@ def main():
     n_dense = sum(1 for g in range(wp.Hkv) if setup.kind_p[g] == 0)
     dense_density = (sum(setup.tiles[g] for g in range(wp.Hkv) if setup.kind_p[g] == 0)
                      / max(1, n_dense * n * (n + 1) / 2))
-    launches_per_step = 4 + 1 + 5   # tile count/scan/fill + attention; stats refresh; score/top-k/partition/attention/merge
+    launches_per_step = 4 + 1 + 4   # tile count/scan/fill + attention; stats refresh; score/top-k+plan/attention/merge
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -442,11 +471,15 @@ def main():
         "decode_us_per_step_l2_flushed": float(np.median(t_decode_flushed)) * 1e3,
         "roofline": {"bound": "tensor", "kernel": "prefill attention", "achieved": tflops_attn,
                      "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tflops_attn / pk["bf16"],
-                     "traffic": None, "peak_source": pk["source"] + " bf16 burst",
+                     "traffic": traffic("prefill", wp.name == PREFILL_WL), "traffic_unit": "bytes per launch",
+                     "algorithmic_bytes_note": "compulsory: q, k, v, mask read once, out and lse written once",
+                     "peak_source": pk["source"] + " bf16 burst",
                      "achieved_note": "kept-tile FLOPs / (lserve_prefill - tile-list build) time"},
-        "roofline_decode": {"bound": "hbm", "kernel": "decode step (score, top-k, partition, paged attention, merge)",
+        "roofline_decode": {"bound": "hbm", "kernel": "decode step (score, top-k + plan, paged attention, merge)",
                             "achieved": gbps_decode, "peak": pk["hbm"], "unit": "GB/s",
-                            "frac": gbps_decode / pk["hbm"], "traffic": None, "peak_source": pk["source"]},
+                            "frac": gbps_decode / pk["hbm"],
+                            "traffic": traffic("decode", wd.name == DECODE_WL), "traffic_unit": "bytes per step",
+                            "algorithmic_bytes": setup.dbytes["total"], "peak_source": pk["source"]},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "e2e": e2e,
