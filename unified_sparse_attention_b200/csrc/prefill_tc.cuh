@@ -317,7 +317,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         for (int rb = 0; rb < 2; ++rb) {
           if (rb_qt(rb) >= A.nQT) continue;
           for (int x = 0; x < C::kBoxes; ++x)
-            tma_load_3d(q_s + x * 16384 + rb * 8192, &tmQ, &q_full, x * 64, rb_head(rb), tok0 + rb_qt(rb) * kTile);
+            tma_load_3d_hint(q_s + x * 16384 + rb * 8192, &tmQ, &q_full, x * 64, rb_head(rb),
+                             tok0 + rb_qt(rb) * kTile, l2_evict_first());
         }
       }
       // K of step t+1 goes out before V of step t: S MMAs run ahead of PV MMAs
@@ -624,8 +625,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           }
           pk[c] = pack_bf16x2(a0 * inv, a1 * inv);
         }
-        *reinterpret_cast<uint4*>(orow + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(orow + c0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        // Q and O are touched once per item: streaming stores (and evict-first Q
+        // loads) leave L2 to the K/V tiles that other query tiles read again
+        __stcs(reinterpret_cast<uint4*>(orow + c0), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+        __stcs(reinterpret_cast<uint4*>(orow + c0 + 8), make_uint4(pk[4], pk[5], pk[6], pk[7]));
       }
       if (A.lse && x == 0)
         A.lse[(static_cast<long>(b) * Hq + h) * A.S + i] =
