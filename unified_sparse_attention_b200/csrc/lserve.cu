@@ -128,6 +128,25 @@ struct Carver {
   size_t used() const { return cur - base + 256; }
 };
 
+// SMs of the current device (148 if it cannot be asked).
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (!cached[dev]) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+      cudaGetLastError();
+      sms = 148;
+    }
+    cached[dev] = sms;
+  }
+  return cached[dev];
+}
+
 // ---------------------------------------------------------------- prefill
 struct PrefillWs {
   int* counts;
@@ -135,6 +154,7 @@ struct PrefillWs {
   int* order;
   int* hist;     // [B*Hkv][nQT + 1]
   int* fill;     // [B*Hkv][nQT + 1]  (contiguous with hist: one memset clears both)
+  int* work_counter;   // next unclaimed work item of the persistent prefill (cleared with hist)
   int* bucket;   // [B*Hkv][nQT + 1]
   int* overflow;
   uint16_t* cols;
@@ -154,8 +174,9 @@ PrefillWs carve_prefill(const lserve_shape* s, void* ws, size_t* bytes) {
   w.offsets = c.take<int>(R + 1);
   w.order = c.take<int>(R);
   const long long groups = static_cast<long long>(s->B) * s->Hkv;
-  w.hist = c.take<int>(2 * groups * (nQT + 1));
+  w.hist = c.take<int>(2 * groups * (nQT + 1) + 1);
   w.fill = w.hist + groups * (nQT + 1);
+  w.work_counter = w.hist + 2 * groups * (nQT + 1);
   w.bucket = c.take<int>(groups * (nQT + 1));
   w.overflow = c.take<int>(1);
   w.max_nnz = R * (nQT + 1) / 2;
@@ -184,7 +205,7 @@ lserve_status launch_tile_lists(const lserve_shape* s, const uint8_t* head_kind,
   const int nRow = (nQT + qg - 1) / qg;
   const int R = s->B * s->Hkv * nRow;
   TileListParams P{s->B, s->Hkv, nQT, sink, local, head_kind, block_mask, qg, nRow};
-  const size_t hist_ints = 2ull * s->B * s->Hkv * (nQT + 1);
+  const size_t hist_ints = 2ull * s->B * s->Hkv * (nQT + 1) + 1;   // + the work counter
   if (cudaMemsetAsync(w.hist, 0, sizeof(int) * hist_ints, st) != cudaSuccess)
     return fail(LSERVE_ERR_CUDA, "prefill: memset failed");
   const int blocks = (R + 7) / 8;
@@ -240,7 +261,10 @@ lserve_status launch_prefill_tc(const lserve_shape* s, const void* q, const void
   if (regs < C::kRegsNeeded)
     return fail(LSERVE_ERR_UNSUPPORTED, "prefill: kernel built with %d registers per thread, its split needs %d",
                 regs, C::kRegsNeeded);
-  const long long grid = static_cast<long long>(n_rows) * T.hsplit;
+  // persistent: one CTA per SM (its shared memory and TMEM admit no second), each
+  // claiming work items from the counter until they run out
+  const long long grid = std::min<long long>(T.n_items, sm_count());
+  if (grid <= 0) return LSERVE_OK;
   tc::prefill_tc_kernel<D><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, st>>>(tq, tk, tv, T);
   return check_launch("prefill attention (tcgen05)");
 }
@@ -266,24 +290,6 @@ struct DecodePlan {
   size_t bytes;
 };
 
-// SMs of the current device (148 if it cannot be asked).
-int sm_count() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-    cudaGetLastError();
-    return 148;
-  }
-  if (!cached[dev]) {
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
-      cudaGetLastError();
-      sms = 148;
-    }
-    cached[dev] = sms;
-  }
-  return cached[dev];
-}
 
 // Attention CTAs for the current device: SMs x resident CTAs per SM, or the
 // value of LSERVE_DECODE_GRID (a positive integer) when that is set.
@@ -516,8 +522,8 @@ lserve_status lserve_prefill(const lserve_shape* shape, const void* q, const voi
                           tp.QG);
     if (s != LSERVE_OK) return s;
     const int nRow = (nQT + tp.QG - 1) / tp.QG;
-    tc::TcArgs T{A, block_mask, tp.QG, tp.HG, nRow, G / tp.HG};
     const int n_rows = shape->B * shape->Hkv * nRow;
+    tc::TcArgs T{A, block_mask, tp.QG, tp.HG, nRow, G / tp.HG, n_rows * (G / tp.HG), w.work_counter};
     s = shape->d == 128 ? launch_prefill_tc<128>(shape, q, k, v, T, n_rows, st)
                         : launch_prefill_tc<64>(shape, q, k, v, T, n_rows, st);
     return s == LSERVE_OK ? ok() : s;

@@ -6,11 +6,20 @@
 // the Lambda support of sink + local window); elements of kept boundary tiles
 // are masked exactly.
 //
-// One CTA per work item: one M-tile of 128 query rows = two 64-row blocks that
-// share one KV tile list.  With grouped-query attention the blocks are two
-// query heads of the same KV head and query tile (G = 4: two CTAs per tile
-// row); with G = 1 they are two adjacent query tiles of one head walking the
-// union of their tile lists.
+// Work item: one M-tile of 128 query rows = two 64-row blocks that share one KV
+// tile list.  With grouped-query attention the blocks are two query heads of
+// the same KV head and query tile (G = 4: two items per tile row); with G = 1
+// they are two adjacent query tiles of one head walking the union of their
+// tile lists.
+//
+// Persistent CTAs, one per SM: the producer warp claims items from a global
+// counter (in the device-built order: grouped by KV head, longest rows first)
+// and hands each to the other roles through a two-slot ring in shared memory.
+// Barrier phases (K/V rings, S/P/O handshakes) run on across items, so the next
+// item's Q and K/V loads and its first S MMAs overlap this item's last steps and
+// epilogue; q_empty frees the Q buffer once an item's last S MMA completed, and
+// o_free lets the next item's first P.V overwrite the O accumulators once both
+// softmax warpgroups have read them.
 //
 // Warp roles (384 threads, one CTA per SM; the third warpgroup hands registers
 // to the two softmax warpgroups with setmaxnreg):
@@ -193,6 +202,7 @@ __device__ __forceinline__ uint64_t bits_from(int l) {   // offsets l..63
 // the single issuing thread is amortised over 128 keys.
 constexpr int kKStages = 3;   // K ring (tile pairs): freed once the S MMAs that read it complete
 constexpr int kVStages = 2;   // V ring (tile pairs): freed once the PV MMAs that read it complete
+constexpr int kItemReaders = 9;   // warps that read a claimed item index: the MMA warp and 8 softmax warps
 
 template <int D>
 struct Cfg {
@@ -211,7 +221,7 @@ struct Cfg {
   // registers per thread after the split: the launch gives every thread the
   // kernel's count (168 at 384 threads, one CTA per SM); 128 x kRegsAux +
   // 256 x kRegsSoftmax must not exceed 384 x that count
-  static constexpr int kRegsAux = 56, kRegsSoftmax = 216;
+  static constexpr int kRegsAux = 88, kRegsSoftmax = 200;
   static constexpr int kRegsNeeded = (128 * kRegsAux + 256 * kRegsSoftmax + kThreads - 1) / kThreads;
   // TMEM: O[x] (fp32, D columns) at 128 x; S[x] (fp32, 128 columns) at 256 + 128 x,
   // with P[x] (bf16 pairs, 64 columns) aliased over the first half of S[x]
@@ -227,7 +237,43 @@ struct TcArgs {
   int HG;                      // query heads per work item
   int nRow;                    // work rows per (b, kvh) = ceil(nQT / QG)
   int hsplit;                  // work items per row = G / HG
+  int n_items;                 // work items in all = rows x hsplit
+  int* work_counter;           // next unclaimed work item; zero at launch
 };
+
+// One work item (128 query rows sharing a KV tile list), decoded from its index.
+struct Item {
+  int n, np;      // kept tiles; pipeline steps (tile pairs)
+  int g, b, bg;   // KV head, sequence, b * Hkv + g
+  int qgi, h0, tok0, QG, HG;
+  bool streaming;
+  const uint16_t* cols;
+  __device__ int rb_head(int rb) const { return h0 + rb % HG; }
+  __device__ int rb_qt(int rb) const { return qgi * QG + rb / HG; }
+  // list entry of half h of step p (the odd tail repeats the last entry)
+  __device__ int pair_tile(int p, int h) const { return cols[min(2 * p + h, n - 1)]; }
+};
+
+__device__ __forceinline__ Item item_at(const TcArgs& T, int w) {
+  const PrefillArgs& A = T.p;
+  Item it;
+  const int r = A.order[w / T.hsplit];
+  const int hs = w % T.hsplit;
+  it.qgi = r % T.nRow;
+  it.bg = r / T.nRow;
+  it.g = it.bg % A.Hkv;
+  it.b = it.bg / A.Hkv;
+  it.h0 = it.g * A.G + hs * T.HG;
+  it.QG = T.QG;
+  it.HG = T.HG;
+  it.streaming = A.head_kind[it.g] != LSERVE_HEAD_DENSE;
+  const int beg = A.row_offsets[r];
+  it.n = A.row_offsets[r + 1] - beg;
+  it.np = (it.n + 1) >> 1;
+  it.cols = A.cols + beg;
+  it.tok0 = it.b * A.S;
+  return it;
+}
 
 template <int D>
 __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
@@ -239,34 +285,23 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   __shared__ __align__(8) uint64_t q_full;
   __shared__ __align__(8) uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_done[2];
+  // persistent CTA: the producer claims work items and passes them on through a
+  // two-slot ring; q_empty frees the Q buffer (all S MMAs of an item done), o_free
+  // frees the O accumulators (both warpgroups have read them in the epilogue)
+  __shared__ __align__(8) uint64_t item_full[2], item_empty[2], q_empty, o_free;
+  __shared__ int s_item[2];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
-  __shared__ float s_ml[2][2][128];   // [warpgroup][m, l][row]: epilogue merge
+  __shared__ float s_ml[2][2][2][128];   // [item parity][warpgroup][m, l][row]: epilogue merge
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_s = smem;
   uint8_t* k_s = q_s + C::kQTile;
   uint8_t* v_s = k_s + kKStages * C::kPair;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // ---- work item: 128 query rows = two 64-row blocks
-  const int w = blockIdx.x;
-  const int r = A.order[w / T.hsplit];
-  const int hs = w % T.hsplit;
-  const int qgi = r % T.nRow;
-  const int bg = r / T.nRow;
-  const int g = bg % A.Hkv, b = bg / A.Hkv;
   const int Hq = A.Hkv * A.G;
-  const int h0 = g * A.G + hs * T.HG;
-  const bool streaming = A.head_kind[g] != LSERVE_HEAD_DENSE;
-  const int beg = A.row_offsets[r];
-  const int n = A.row_offsets[r + 1] - beg;   // kept tiles
-  const int np = (n + 1) >> 1;                 // pipeline steps (tile pairs)
-  const uint16_t* cols = A.cols + beg;
-  const int tok0 = b * A.S;
-  auto rb_head = [&](int rb) { return h0 + rb % T.HG; };
-  auto rb_qt = [&](int rb) { return qgi * T.QG + rb / T.HG; };
-  // list entry of half h of step p (the odd tail repeats the last entry)
-  auto pair_tile = [&](int p, int h) { return cols[min(2 * p + h, n - 1)]; };
+  // item index of ring slot `slot` (written before item_full completes)
+  auto claimed = [&](int slot) { return *reinterpret_cast<volatile int*>(&s_item[slot]); };
 
   if (tid == 0) {
     mbar_init(&q_full, 1);
@@ -282,7 +317,11 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       mbar_init(&s_full[x], 1);
       mbar_init(&p_full[x], 128);
       mbar_init(&o_done[x], 1);
+      mbar_init(&item_full[x], 1);
+      mbar_init(&item_empty[x], kItemReaders);
     }
+    mbar_init(&q_empty, 1);
+    mbar_init(&o_free, 256);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -302,31 +341,55 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegsAux));
    if (warp == C::kWarpProducer) {
     // ================================================================ producer
-    // The whole warp walks the list (warp-uniform coordinates); one elected lane issues.
+    // The whole warp walks the lists (warp-uniform coordinates); one elected lane
+    // issues.  Work items are claimed from the global counter one at a time and
+    // handed to the other roles through the item ring.  K and V stage indices and
+    // phases run on across items (gk, gv: tile pairs issued so far).
     const bool leader = elect_one();
-    if (n > 0) {
+    if (leader) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+    }
+    int gk = 0, gv = 0, nq = 0;   // K and V steps issued; items with tiles (Q loads)
+    bool live = true;
+    for (int ii = 0; live; ++ii) {
+      const int slot = ii & 1;
+      if (ii >= 2 && !wait_or_abort(&item_empty[slot], ((ii >> 1) - 1) & 1, &s_abort, tmo)) break;
+      int w = 0;
       if (leader) {
-        prefetch_tensormap(&tmQ);
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
+        w = atomicAdd(T.work_counter, 1);
+        s_item[slot] = w;
+        mbar_arrive(&item_full[slot]);   // release: the index is visible to the waiters
       }
+      w = __shfl_sync(0xffffffffu, w, __ffs(__ballot_sync(0xffffffffu, leader)) - 1);
+      if (w >= T.n_items || s_abort) break;
+      const Item it = item_at(T, w);
+      const int n = it.n, np = it.np, g = it.g, tok0 = it.tok0;
+      if (n == 0) continue;
+      // the Q buffer is free once every S MMA of the previous item with tiles completed
+      if (nq > 0 && !wait_or_abort(&q_empty, (nq - 1) & 1, &s_abort, tmo)) break;
+      ++nq;
       int valid_rb = 0;
-      for (int rb = 0; rb < 2; ++rb) valid_rb += rb_qt(rb) < A.nQT;
+      for (int rb = 0; rb < 2; ++rb) valid_rb += it.rb_qt(rb) < A.nQT;
       if (leader) {
         mbar_arrive_expect_tx(&q_full, valid_rb * C::kBoxes * 8192);
         for (int rb = 0; rb < 2; ++rb) {
-          if (rb_qt(rb) >= A.nQT) continue;
+          if (it.rb_qt(rb) >= A.nQT) continue;
           for (int x = 0; x < C::kBoxes; ++x)
-            tma_load_3d_hint(q_s + x * 16384 + rb * 8192, &tmQ, &q_full, x * 64, rb_head(rb),
-                             tok0 + rb_qt(rb) * kTile, l2_evict_first());
+            tma_load_3d_hint(q_s + x * 16384 + rb * 8192, &tmQ, &q_full, x * 64, it.rb_head(rb),
+                             tok0 + it.rb_qt(rb) * kTile, l2_evict_first());
         }
       }
       // K of step t+1 goes out before V of step t: S MMAs run ahead of PV MMAs
-      for (int t = 0; t <= np; ++t) {
+      for (int t = 0; t <= np && live; ++t) {
         if (t < np) {
-          const int st = t % kKStages;
-          if (t >= kKStages && !wait_or_abort(&k_empty[st], ((t / kKStages) - 1) & 1, &s_abort, tmo)) break;
-          const int ka = pair_tile(t, 0), kb = pair_tile(t, 1);
+          const int gt = gk + t, st = gt % kKStages;
+          if (gt >= kKStages && !wait_or_abort(&k_empty[st], ((gt / kKStages) - 1) & 1, &s_abort, tmo)) {
+            live = false;
+            break;
+          }
+          const int ka = it.pair_tile(t, 0), kb = it.pair_tile(t, 1);
           if (leader) {
             mbar_arrive_expect_tx(&k_full[st], C::kPair);
             for (int x = 0; x < C::kBoxes; ++x) {
@@ -337,10 +400,12 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           }
         }
         if (t >= 1) {
-          const int u = t - 1;
-          const int st = u % kVStages;
-          if (u >= kVStages && !wait_or_abort(&v_empty[st], ((u / kVStages) - 1) & 1, &s_abort, tmo)) break;
-          const int ka = pair_tile(u, 0), kb = pair_tile(u, 1);
+          const int gu = gv + t - 1, st = gu % kVStages;
+          if (gu >= kVStages && !wait_or_abort(&v_empty[st], ((gu / kVStages) - 1) & 1, &s_abort, tmo)) {
+            live = false;
+            break;
+          }
+          const int ka = it.pair_tile(t - 1, 0), kb = it.pair_tile(t - 1, 1);
           if (leader) {
             mbar_arrive_expect_tx(&v_full[st], C::kPair);
             for (int x = 0; x < C::kBoxes; ++x) {
@@ -351,23 +416,38 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           }
         }
       }
+      gk += np;
+      gv += np;
     }
   } else if (warp == C::kWarpMma) {
     // ================================================================== MMA
-    // Step p belongs to stream x = p & 1 (S[x], P[x], O[x]).  The whole warp runs
-    // the loop (waits and descriptors warp-uniform); one elected lane issues.
-    // Tensor-core order: S(0) S(1) PV(0) S(2) PV(1) S(3) ...  S(p+2) overwrites the
-    // S/P buffer that PV(p) reads; tcgen05.mma instructions of one kind issued by
-    // one thread are pipelined in issue order, so S(p+2) is issued right after
-    // PV(p) without waiting for its completion (checked: parity, and bit-identical
-    // results over repeated runs).
-    if (n > 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false);
-      constexpr uint32_t kIdPV = idesc_bf16(128, D, true);
-      const uint32_t qa = smem_u32(q_s), ka = smem_u32(k_s), va = smem_u32(v_s);
+    // Step p of an item belongs to stream x = p & 1 (S[x], P[x], O[x]).  The whole
+    // warp runs the loop (waits and descriptors warp-uniform); one elected lane
+    // issues.  Tensor-core order within an item: S(0) S(1) PV(0) S(2) PV(1) S(3) ...
+    // S(p+2) overwrites the S/P buffer that PV(p) reads; tcgen05.mma instructions
+    // issued by one thread are pipelined in issue order, so S(p+2) is issued right
+    // after PV(p) without waiting for its completion (checked: parity, and
+    // bit-identical results over repeated runs).  The same order makes S(0), S(1)
+    // of the next item safe right after the last PV of this one, so they run while
+    // the softmax warpgroups finish this item's epilogue.
+    constexpr uint32_t kIdS = idesc_bf16(128, 128, false);
+    constexpr uint32_t kIdPV = idesc_bf16(128, D, true);
+    const uint32_t qa = smem_u32(q_s), ka = smem_u32(k_s), va = smem_u32(v_s);
+    int gk = 0, gv = 0, nq = 0;   // K and V steps consumed; items with tiles
+    int cs[2] = {0, 0};           // steps of each stream over the previous items
+    for (int ii = 0;; ++ii) {
+      const int slot = ii & 1;
+      if (!wait_or_abort(&item_full[slot], (ii >> 1) & 1, &s_abort, tmo)) break;
+      const int w = claimed(slot);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&item_empty[slot]);
+      if (w >= T.n_items) break;
+      const Item it = item_at(T, w);
+      const int np = it.np;
+      if (it.n == 0) continue;
       auto issue_s = [&](int p) {   // S[p&1] = Q [K_a; K_b]^T
-        const int st = p % kKStages, x = p & 1;
-        wait_or_abort(&k_full[st], (p / kKStages) & 1, &s_abort, tmo);
+        const int gt = gk + p, st = gt % kKStages, x = p & 1;
+        wait_or_abort(&k_full[st], (gt / kKStages) & 1, &s_abort, tmo);
         fence_after_sync();
 #pragma unroll
         for (int k4 = 0; k4 < D / 16; k4 += 4) {
@@ -381,15 +461,20 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           mma_ss4(tmem + C::kColS + 128 * x, ad[0], ad[1], ad[2], ad[3], bd[0], bd[1], bd[2], bd[3], kIdS, k4 > 0);
         }
         commit(&s_full[x]);
-        if (p + kKStages < np) commit(&k_empty[st]);
+        commit(&k_empty[st]);
+        if (p == np - 1) commit(&q_empty);   // the item's last read of Q
       };
-      wait_or_abort(&q_full, 0, &s_abort, tmo);
+      wait_or_abort(&q_full, nq & 1, &s_abort, tmo);
+      ++nq;
       issue_s(0);
       if (np > 1) issue_s(1);
       for (int p = 0; p < np; ++p) {
-        const int st = p % kVStages, x = p & 1;
-        wait_or_abort(&v_full[st], (p / kVStages) & 1, &s_abort, tmo);
-        wait_or_abort(&p_full[x], (p >> 1) & 1, &s_abort, tmo);
+        const int gu = gv + p, st = gu % kVStages, x = p & 1;
+        wait_or_abort(&v_full[st], (gu / kVStages) & 1, &s_abort, tmo);
+        wait_or_abort(&p_full[x], (cs[x] + (p >> 1)) & 1, &s_abort, tmo);
+        // PV(0) overwrites O[0] (and PV(1) O[1]): the previous item's epilogue must
+        // have read both accumulators
+        if (p == 0 && ii > 0) wait_or_abort(&o_free, (ii - 1) & 1, &s_abort, tmo);
         fence_after_sync();
 #pragma unroll
         for (int k4 = 0; k4 < 8; k4 += 4) {
@@ -404,9 +489,14 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
                   (p >= 2 || k4 > 0) ? 1u : 0u);
         }
         commit(&o_done[x]);
-        if (p + kVStages < np) commit(&v_empty[st]);
+        commit(&v_empty[st]);
         if (p + 2 < np) issue_s(p + 2);
       }
+      gk += np;
+      gv += np;
+      cs[0] += (np + 1) >> 1;
+      cs[1] += np >> 1;
+      if (s_abort) break;
     }
    }
   } else {
@@ -418,223 +508,246 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;    // row within the M-tile
     const int rb = row >> 6;
-    const int h = rb_head(rb), qt = rb_qt(rb);
-    const bool rb_valid = qt < A.nQT;
-    const int i = qt * kTile + (row & 63);  // query position
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t t_o = tmem + C::kColO + 128 * x + lane_off;
     const uint32_t t_s = tmem + C::kColS + 128 * x + lane_off;
-    const uint8_t* mrow = (!streaming && T.block_mask && rb_valid)
-                              ? T.block_mask + (static_cast<long>(bg) * A.nQT + qt) * A.nQT
-                              : nullptr;
-    float m_run = kNegInf, l_run = 0.f;
     const float sc = A.scale_log2;
     TileListParams tp{0, A.Hkv, A.nQT, A.sink, A.local, nullptr, nullptr};
-    // keep mask of this row over one 64-key tile (bit c <-> key 64 kt + c)
-    auto tile_mask = [&](int kt) -> uint64_t {
-      if (!rb_valid || !(T.QG == 1 || tile_keep(tp, streaming, mrow, qt, kt))) return 0ull;
-      if (tile_is_full(streaming, qt, kt, A.sink, A.local)) return ~0ull;
-      const int d0 = i - kt * kTile;   // offset of the query position inside the tile
-      uint64_t k = bits_upto(d0);
-      if (streaming) k &= bits_below(A.sink - kt * kTile) | bits_from(d0 - A.local + 1);
-      return k;
-    };
-    // raw scores of one 64-key half, masked keys set to -inf
-    auto load_half = [&](int half, uint64_t keep, uint32_t (&v)[64]) {
-      tmem_ld32(t_s + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld32(t_s + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-      tmem_wait_ld();
-      if (!__all_sync(0xffffffffu, keep == ~0ull)) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (!((keep >> c) & 1ull)) v[c] = 0xff800000u;   // -inf: exp2 gives exactly 0
-      }
-    };
-    int seen = 0;   // completions of o_done[x] observed by this warpgroup
-
-    float rebase = 0.f;   // shift of the reference max decided at this stream's previous step
-    // tile indices of this stream's next step, loaded one step ahead (hides the load latency)
-    int nkt0 = 0, nkt1 = 0;
-    if (x < np) {
-      nkt0 = pair_tile(x, 0);
-      nkt1 = pair_tile(x, 1);
-    }
-    for (int p = x; p < np; p += 2) {
-      const int j = p >> 1;   // this stream's step index
-      const int kt0 = nkt0, kt1 = nkt1;
-      if (p + 2 < np) {
-        nkt0 = pair_tile(p + 2, 0);
-        nkt1 = pair_tile(p + 2, 1);
-      }
-      const uint64_t keep0 = tile_mask(kt0);
-      const uint64_t keep1 = (2 * p + 1 < n) ? tile_mask(kt1) : 0ull;
-      wait_or_abort(&s_full[x], j & 1, &s_abort, tmo);
-      fence_after_sync();
-      uint32_t v[64];
-      uint32_t pk0[32], pk1[32];
-      float ps[4];
-      // One 32-column chunk of S (already in registers): exponentials 2^(s*scale - m),
-      // packed fp32 pairs for the scale/subtract and the running sums (half the
-      // instructions: the softmax is issue-bound), bf16 pairs of P.
-      auto exp_chunk = [&](uint32_t (&u)[32], uint64_t keep, int q, uint64_t sc2, uint64_t nm2, uint32_t* pk,
-                           uint64_t (&ps2)[2]) {
+    int cs_own = 0;   // steps of this stream over the previous items (barrier phases)
+    for (int ii = 0;; ++ii) {
+      const int slot = ii & 1;
+      if (!wait_or_abort(&item_full[slot], (ii >> 1) & 1, &s_abort, tmo)) break;
+      const int w = claimed(slot);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&item_empty[slot]);
+      if (w >= T.n_items) break;
+      const Item it = item_at(T, w);
+      const int n = it.n, np = it.np, b = it.b, bg = it.bg;
+      const bool streaming = it.streaming;
+      const int h = it.rb_head(rb), qt = it.rb_qt(rb);
+      const bool rb_valid = qt < A.nQT;
+      const int i = qt * kTile + (row & 63);  // query position
+      const int tok0 = it.tok0;
+      const uint8_t* mrow = (!streaming && T.block_mask && rb_valid)
+                                ? T.block_mask + (static_cast<long>(bg) * A.nQT + qt) * A.nQT
+                                : nullptr;
+      float m_run = kNegInf, l_run = 0.f;
+      // keep mask of this row over one 64-key tile (bit c <-> key 64 kt + c)
+      auto tile_mask = [&](int kt) -> uint64_t {
+        if (!rb_valid || !(T.QG == 1 || tile_keep(tp, streaming, mrow, qt, kt))) return 0ull;
+        if (tile_is_full(streaming, qt, kt, A.sink, A.local)) return ~0ull;
+        const int d0 = i - kt * kTile;   // offset of the query position inside the tile
+        uint64_t k = bits_upto(d0);
+        if (streaming) k &= bits_below(A.sink - kt * kTile) | bits_from(d0 - A.local + 1);
+        return k;
+      };
+      // raw scores of one 64-key half, masked keys set to -inf
+      auto load_half = [&](int half, uint64_t keep, uint32_t (&v)[64]) {
+        tmem_ld32(t_s + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(t_s + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_wait_ld();
         if (!__all_sync(0xffffffffu, keep == ~0ull)) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (!((keep >> (32 * q + c)) & 1ull)) u[c] = 0xff800000u;   // -inf: exp2 gives 0
-        }
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          float a0, a1;
-          split_f32x2(fma_f32x2(f32x2(__uint_as_float(u[2 * c]), __uint_as_float(u[2 * c + 1])), sc2, nm2), a0, a1);
-          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
-          ps2[c & 1] = add_f32x2(ps2[c & 1], f32x2(p0, p1));
-          pk[c] = pack_bf16x2(p0, p1);
+  #pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (!((keep >> c) & 1ull)) v[c] = 0xff800000u;   // -inf: exp2 gives exactly 0
         }
       };
-      auto exp_pass = [&](float m) -> float {   // returns the row sum of the exponentials
-        const float m_use = m == kNegInf ? 0.f : m;
-        const uint64_t sc2 = f32x2(sc, sc), nm2 = f32x2(-m_use, -m_use);
-        uint64_t ps2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
-        // four 32-column chunks; the TMEM load of chunk c+1 is in flight while chunk c is processed
-        uint32_t ua[32], ub[32];
-        tmem_ld32(t_s, ua);
-        tmem_wait_ld();
-        tmem_ld32(t_s + 32, ub);
-        exp_chunk(ua, keep0, 0, sc2, nm2, pk0, ps2);
-        tmem_wait_ld();
-        tmem_ld32(t_s + 64, ua);
-        exp_chunk(ub, keep0, 1, sc2, nm2, pk0 + 16, ps2);
-        tmem_wait_ld();
-        tmem_ld32(t_s + 96, ub);
-        exp_chunk(ua, keep1, 0, sc2, nm2, pk1, ps2);
-        tmem_wait_ld();
-        exp_chunk(ub, keep1, 1, sc2, nm2, pk1 + 16, ps2);
-        split_f32x2(ps2[0], ps[0], ps[1]);
-        split_f32x2(ps2[1], ps[2], ps[3]);
-        return (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      };
-      // O[x] and l are multiplied by f before this step's P is added
-      float f = 1.f;
-      if (rebase != 0.f) {
-        f = fast_exp2(-rebase);
-        m_run += rebase;
-        rebase = 0.f;
+      int seen = 0;   // completions of o_done[x] observed by this warpgroup
+
+      float rebase = 0.f;   // shift of the reference max decided at this stream's previous step
+      // tile indices of this stream's next step, loaded one step ahead (hides the load latency)
+      int nkt0 = 0, nkt1 = 0;
+      if (x < np) {
+        nkt0 = it.pair_tile(x, 0);
+        nkt1 = it.pair_tile(x, 1);
       }
-      float rsum = 0.f;
-      bool ok = false;
-      if (m_run != kNegInf) {   // steady state: one pass against the current reference
-        rsum = exp_pass(m_run);
-        // every weight is at most the row sum: none near the fp32/bf16 limit (catches inf/NaN too)
-        ok = !__any_sync(0xffffffffu, !(rsum <= 1099511627776.f));   // 2^40
-      }
-      if (!ok) {                // first step of the stream, or a jump: exact row max first
-        float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          load_half(half, half ? keep1 : keep0, v);
-#pragma unroll
-          for (int c = 0; c < 64; c += 8) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              mx[e] = max3(mx[e], __uint_as_float(v[c + 2 * e]), __uint_as_float(v[c + 2 * e + 1]));
-          }
+      for (int p = x; p < np; p += 2) {
+        const int j = p >> 1;   // this stream's step index
+        const int kt0 = nkt0, kt1 = nkt1;
+        if (p + 2 < np) {
+          nkt0 = it.pair_tile(p + 2, 0);
+          nkt1 = it.pair_tile(p + 2, 1);
         }
-        const float mloc = max3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;
-        const float m_new = fmaxf(m_run, mloc);
-        if (m_run != kNegInf && m_new != m_run) f *= fast_exp2(m_run - m_new);
-        m_run = m_new;
-        rsum = exp_pass(m_run);
-      }
-      // weights well above the reference (row sum beyond 2^12): move the reference to the
-      // largest argument at this stream's next step (O must first absorb this step); the
-      // largest weight is read back from the bf16 pairs of P
-      if (m_run != kNegInf && rsum > 4096.f) {
-        uint32_t mp = 0u;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) mp = max_bf16x2(mp, max_bf16x2(pk0[c], pk1[c]));
-        const float wmax = fmaxf(bf16_lo(mp), bf16_hi(mp));
-        if (wmax > 1.f) rebase = __log2f(wmax);
-      }
-      tmem_st32(t_s, pk0);        // P[x] over S[x] columns 0..63 (S is no longer needed)
-      tmem_st32(t_s + 32, pk1);
-      l_run = l_run * f + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-      // O[x] holds this stream's steps < p; PV(p-2) completed before S(p) was issued,
-      // observe it (in order) before touching O[x]
-      if (j > 0) {
-        wait_or_abort(&o_done[x], (j - 1) & 1, &s_abort, tmo);
-        ++seen;
+        const uint64_t keep0 = tile_mask(kt0);
+        const uint64_t keep1 = (2 * p + 1 < n) ? tile_mask(kt1) : 0ull;
+        wait_or_abort(&s_full[x], (cs_own + j) & 1, &s_abort, tmo);
         fence_after_sync();
-        if (__any_sync(0xffffffffu, f != 1.f)) {
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t ov[32];
-            tmem_ld32(t_o + c0, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * f);
-            tmem_st32(t_o + c0, ov);
+        uint32_t v[64];
+        uint32_t pk0[32], pk1[32];
+        float ps[4];
+        // One 32-column chunk of S (already in registers): exponentials 2^(s*scale - m),
+        // packed fp32 pairs for the scale/subtract and the running sums (half the
+        // instructions: the softmax is issue-bound), bf16 pairs of P.
+        auto exp_chunk = [&](uint32_t (&u)[32], uint64_t keep, int q, uint64_t sc2, uint64_t nm2, uint32_t* pk,
+                             uint64_t (&ps2)[2]) {
+          if (!__all_sync(0xffffffffu, keep == ~0ull)) {
+  #pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (!((keep >> (32 * q + c)) & 1ull)) u[c] = 0xff800000u;   // -inf: exp2 gives 0
+          }
+  #pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            float a0, a1;
+            split_f32x2(fma_f32x2(f32x2(__uint_as_float(u[2 * c]), __uint_as_float(u[2 * c + 1])), sc2, nm2), a0, a1);
+            const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+            ps2[c & 1] = add_f32x2(ps2[c & 1], f32x2(p0, p1));
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+        };
+        auto exp_pass = [&](float m) -> float {   // returns the row sum of the exponentials
+          const float m_use = m == kNegInf ? 0.f : m;
+          const uint64_t sc2 = f32x2(sc, sc), nm2 = f32x2(-m_use, -m_use);
+          uint64_t ps2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
+          // four 32-column chunks; the TMEM load of chunk c+1 is in flight while chunk c is processed
+          uint32_t ua[32], ub[32];
+          tmem_ld32(t_s, ua);
+          tmem_wait_ld();
+          tmem_ld32(t_s + 32, ub);
+          exp_chunk(ua, keep0, 0, sc2, nm2, pk0, ps2);
+          tmem_wait_ld();
+          tmem_ld32(t_s + 64, ua);
+          exp_chunk(ub, keep0, 1, sc2, nm2, pk0 + 16, ps2);
+          tmem_wait_ld();
+          tmem_ld32(t_s + 96, ub);
+          exp_chunk(ua, keep1, 0, sc2, nm2, pk1, ps2);
+          tmem_wait_ld();
+          exp_chunk(ub, keep1, 1, sc2, nm2, pk1 + 16, ps2);
+          split_f32x2(ps2[0], ps[0], ps[1]);
+          split_f32x2(ps2[1], ps[2], ps[3]);
+          return (ps[0] + ps[1]) + (ps[2] + ps[3]);
+        };
+        // O[x] and l are multiplied by f before this step's P is added
+        float f = 1.f;
+        if (rebase != 0.f) {
+          f = fast_exp2(-rebase);
+          m_run += rebase;
+          rebase = 0.f;
+        }
+        float rsum = 0.f;
+        bool ok = false;
+        if (m_run != kNegInf) {   // steady state: one pass against the current reference
+          rsum = exp_pass(m_run);
+          // every weight is at most the row sum: none near the fp32/bf16 limit (catches inf/NaN too)
+          ok = !__any_sync(0xffffffffu, !(rsum <= 1099511627776.f));   // 2^40
+        }
+        if (!ok) {                // first step of the stream, or a jump: exact row max first
+          float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+  #pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            load_half(half, half ? keep1 : keep0, v);
+  #pragma unroll
+            for (int c = 0; c < 64; c += 8) {
+  #pragma unroll
+              for (int e = 0; e < 4; ++e)
+                mx[e] = max3(mx[e], __uint_as_float(v[c + 2 * e]), __uint_as_float(v[c + 2 * e + 1]));
+            }
+          }
+          const float mloc = max3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;
+          const float m_new = fmaxf(m_run, mloc);
+          if (m_run != kNegInf && m_new != m_run) f *= fast_exp2(m_run - m_new);
+          m_run = m_new;
+          rsum = exp_pass(m_run);
+        }
+        // weights well above the reference (row sum beyond 2^12): move the reference to the
+        // largest argument at this stream's next step (O must first absorb this step); the
+        // largest weight is read back from the bf16 pairs of P
+        if (m_run != kNegInf && rsum > 4096.f) {
+          uint32_t mp = 0u;
+  #pragma unroll
+          for (int c = 0; c < 32; ++c) mp = max_bf16x2(mp, max_bf16x2(pk0[c], pk1[c]));
+          const float wmax = fmaxf(bf16_lo(mp), bf16_hi(mp));
+          if (wmax > 1.f) rebase = __log2f(wmax);
+        }
+        tmem_st32(t_s, pk0);        // P[x] over S[x] columns 0..63 (S is no longer needed)
+        tmem_st32(t_s + 32, pk1);
+        l_run = l_run * f + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+        // O[x] holds this stream's steps < p; PV(p-2) completed before S(p) was issued,
+        // observe it (in order) before touching O[x]
+        if (j > 0) {
+          wait_or_abort(&o_done[x], (cs_own + j - 1) & 1, &s_abort, tmo);
+          ++seen;
+          fence_after_sync();
+          if (__any_sync(0xffffffffu, f != 1.f)) {
+  #pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t ov[32];
+              tmem_ld32(t_o + c0, ov);
+              tmem_wait_ld();
+  #pragma unroll
+              for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * f);
+              tmem_st32(t_o + c0, ov);
+            }
           }
         }
+        tmem_wait_st();
+        fence_before_sync();
+        mbar_arrive(&p_full[x]);
       }
-      tmem_wait_st();
+      // a pending shift is never needed for the result: (m, l, O) stay consistent
+      // ---- epilogue: merge the two streams (log-sum-exp), each warpgroup stores half of O
+      const int nx = (np > x) ? (np - x + 1) >> 1 : 0;   // steps of this stream
+      if (nx > 0) {
+        wait_or_abort(&o_done[x], (cs_own + nx - 1) & 1, &s_abort, tmo);   // PV of its last step
+        fence_after_sync();
+      }
+      s_ml[ii & 1][x][0][row] = m_run;
+      s_ml[ii & 1][x][1][row] = l_run;
+      // the other warpgroup observed its stream's last P.V before this barrier; the
+      // fences order that observation before this warpgroup's reads of O[x^1]
       fence_before_sync();
-      mbar_arrive(&p_full[x]);
-    }
-    // a pending shift is never needed for the result: (m, l, O) stay consistent
-    // ---- epilogue: merge the two streams (log-sum-exp), each warpgroup stores half of O
-    const int nx = (np > x) ? (np - x + 1) >> 1 : 0;   // steps of this stream
-    if (nx > 0) {
-      wait_or_abort(&o_done[x], (nx - 1) & 1, &s_abort, tmo);   // PV of its last step
+      asm volatile("bar.sync 1, 256;" ::: "memory");
       fence_after_sync();
-    }
-    s_ml[x][0][row] = m_run;
-    s_ml[x][1][row] = l_run;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    const float m_o = s_ml[x ^ 1][0][row], l_o = s_ml[x ^ 1][1][row];
-    const int nx_o = (np > (x ^ 1)) ? (np - (x ^ 1) + 1) >> 1 : 0;
-    const float m_all = fmaxf(m_run, m_o);
-    const float m_ref = m_all == kNegInf ? 0.f : m_all;
-    const float w_own = nx > 0 ? fast_exp2(m_run - m_ref) : 0.f;
-    const float w_oth = nx_o > 0 ? fast_exp2(m_o - m_ref) : 0.f;
-    const float l_tot = l_run * w_own + l_o * w_oth;
-    if (rb_valid) {
-      const int c_lo = x * (D / 2);   // this warpgroup's half of the output columns
-      bf16* orow = A.out + (static_cast<long>(tok0 + i) * Hq + h) * D + c_lo;
-      const bool has = n > 0 && m_all != kNegInf && l_tot > 0.f;
-      const float inv = has ? 1.f / l_tot : 0.f;
-      const uint32_t t_own = tmem + C::kColO + 128 * x + lane_off + c_lo;
-      const uint32_t t_oth = tmem + C::kColO + 128 * (x ^ 1) + lane_off + c_lo;
-#pragma unroll 1
-      for (int c0 = 0; c0 < D / 2; c0 += 16) {
-        uint32_t oa[16], ob[16];
-        if (nx > 0) tmem_ld16(t_own + c0, oa);
-        if (nx_o > 0) tmem_ld16(t_oth + c0, ob);
-        tmem_wait_ld();
-        uint32_t pk[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float a0 = 0.f, a1 = 0.f;
-          if (nx > 0) {
-            a0 = __uint_as_float(oa[2 * c]) * w_own;
-            a1 = __uint_as_float(oa[2 * c + 1]) * w_own;
+      const float m_o = s_ml[ii & 1][x ^ 1][0][row], l_o = s_ml[ii & 1][x ^ 1][1][row];
+      const int nx_o = (np > (x ^ 1)) ? (np - (x ^ 1) + 1) >> 1 : 0;
+      const float m_all = fmaxf(m_run, m_o);
+      const float m_ref = m_all == kNegInf ? 0.f : m_all;
+      const float w_own = nx > 0 ? fast_exp2(m_run - m_ref) : 0.f;
+      const float w_oth = nx_o > 0 ? fast_exp2(m_o - m_ref) : 0.f;
+      const float l_tot = l_run * w_own + l_o * w_oth;
+      if (rb_valid) {
+        const int c_lo = x * (D / 2);   // this warpgroup's half of the output columns
+        bf16* orow = A.out + (static_cast<long>(tok0 + i) * Hq + h) * D + c_lo;
+        const bool has = n > 0 && m_all != kNegInf && l_tot > 0.f;
+        const float inv = has ? 1.f / l_tot : 0.f;
+        const uint32_t t_own = tmem + C::kColO + 128 * x + lane_off + c_lo;
+        const uint32_t t_oth = tmem + C::kColO + 128 * (x ^ 1) + lane_off + c_lo;
+  #pragma unroll 1
+        for (int c0 = 0; c0 < D / 2; c0 += 16) {
+          uint32_t oa[16], ob[16];
+          if (nx > 0) tmem_ld16(t_own + c0, oa);
+          if (nx_o > 0) tmem_ld16(t_oth + c0, ob);
+          tmem_wait_ld();
+          uint32_t pk[8];
+  #pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            float a0 = 0.f, a1 = 0.f;
+            if (nx > 0) {
+              a0 = __uint_as_float(oa[2 * c]) * w_own;
+              a1 = __uint_as_float(oa[2 * c + 1]) * w_own;
+            }
+            if (nx_o > 0) {
+              a0 = fmaf(__uint_as_float(ob[2 * c]), w_oth, a0);
+              a1 = fmaf(__uint_as_float(ob[2 * c + 1]), w_oth, a1);
+            }
+            pk[c] = pack_bf16x2(a0 * inv, a1 * inv);
           }
-          if (nx_o > 0) {
-            a0 = fmaf(__uint_as_float(ob[2 * c]), w_oth, a0);
-            a1 = fmaf(__uint_as_float(ob[2 * c + 1]), w_oth, a1);
-          }
-          pk[c] = pack_bf16x2(a0 * inv, a1 * inv);
+          // Q and O are touched once per item: streaming stores (and evict-first Q
+          // loads) leave L2 to the K/V tiles that other query tiles read again
+          __stcs(reinterpret_cast<uint4*>(orow + c0), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+          __stcs(reinterpret_cast<uint4*>(orow + c0 + 8), make_uint4(pk[4], pk[5], pk[6], pk[7]));
         }
-        // Q and O are touched once per item: streaming stores (and evict-first Q
-        // loads) leave L2 to the K/V tiles that other query tiles read again
-        __stcs(reinterpret_cast<uint4*>(orow + c0), make_uint4(pk[0], pk[1], pk[2], pk[3]));
-        __stcs(reinterpret_cast<uint4*>(orow + c0 + 8), make_uint4(pk[4], pk[5], pk[6], pk[7]));
+        if (A.lse && x == 0)
+          A.lse[(static_cast<long>(b) * Hq + h) * A.S + i] =
+              has ? (m_all + __log2f(l_tot)) * 0.6931471805599453f : kNegInf;
       }
-      if (A.lse && x == 0)
-        A.lse[(static_cast<long>(b) * Hq + h) * A.S + i] =
-            has ? (m_all + __log2f(l_tot)) * 0.6931471805599453f : kNegInf;
+      (void)seen;
+      // both accumulators have been read: the MMA warp may let the next item's PV(0)
+      // overwrite them
+      fence_before_sync();
+      mbar_arrive(&o_free);
+      cs_own += nx;
+      if (s_abort) break;
     }
-    (void)seen;
   }
   fence_before_sync();
   __syncthreads();
