@@ -1,12 +1,18 @@
-"""Failure detection on the GPU without a fault: the decode kernel's bounded waits.
+"""Failure detection on the GPU without a fault: the kernels' bounded waits.
 
-Every wait inside the decode attention kernel (on a stage's loads, on a free
-stage, on the page resolver) gives up after LSERVE_WAIT_TIMEOUT_NS, records
-LSERVE_ERR_DEVICE_TIMEOUT and lets the CTA leave after its copies in flight
-have landed.  With LSERVE_DEBUG_STALL_DECODE set, the kernel's page resolver
-publishes nothing -- a flag nobody sets -- so the issuer's and the consumers'
-waits run out (with a 20 ms limit).  The status must say so, and the next call
-without the hook must give the same result as before on the same context.
+Every wait inside the decode attention kernel and the tcgen05 prefill kernel
+gives up after LSERVE_WAIT_TIMEOUT_NS, records LSERVE_ERR_DEVICE_TIMEOUT and
+lets the CTA leave once its copies (and MMAs) in flight have landed.
+
+* decode: with LSERVE_DEBUG_STALL_DECODE set, the page resolver publishes
+  nothing -- a flag nobody sets -- so the issuer's and the consumers' waits run
+  out;
+* prefill: with LSERVE_DEBUG_STALL_PREFILL set, the producer hands out no work
+  item, so the MMA and softmax warps' waits on the item ring run out.
+
+Both with a 20 ms limit and nothing in flight.  The status must say so, and the
+next call without the hook must give the same result as before on the same
+context.
 """
 import dataclasses
 
@@ -45,6 +51,31 @@ def test_decode_wait_limit_reports_timeout_and_context_survives(monkeypatch):
     monkeypatch.delenv("LSERVE_DEBUG_STALL_DECODE")
     monkeypatch.delenv("LSERVE_WAIT_TIMEOUT_NS")
     again = U.lserve_decode(*args)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+    assert torch.equal(again, ref)
+
+
+def test_prefill_wait_limit_reports_timeout_and_context_survives(monkeypatch):
+    monkeypatch.delenv("LSERVE_PREFILL_IMPL", raising=False)   # the tcgen05 kernel
+    w = W.WORKLOADS["tiny"]
+    dev = "cuda"
+    q, k, v = (t.to(dev) for t in W.prefill_inputs(w))
+    hk = W.head_kind(w).to(dev)
+    ref = U.lserve_prefill(q, k, v, hk, w.sink, w.local, None)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+
+    monkeypatch.setenv("LSERVE_WAIT_TIMEOUT_NS", "20000000")
+    monkeypatch.setenv("LSERVE_DEBUG_STALL_PREFILL", "1")
+    U.lserve_prefill(q, k, v, hk, w.sink, w.local, None)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == LSERVE_ERR_DEVICE_TIMEOUT
+    assert "bounded wait" in U.lserve_last_error_string()
+
+    monkeypatch.delenv("LSERVE_DEBUG_STALL_PREFILL")
+    monkeypatch.delenv("LSERVE_WAIT_TIMEOUT_NS")
+    again = U.lserve_prefill(q, k, v, hk, w.sink, w.local, None)
     torch.cuda.synchronize()
     assert U.lserve_get_device_status() == 0
     assert torch.equal(again, ref)

@@ -51,6 +51,9 @@ lserve_status check_launch(const char* what) {
 // attention kernel's page resolver publishes nothing, so its other waits run
 // out and the call records LSERVE_ERR_DEVICE_TIMEOUT (no copy is in flight).
 int debug_stall_decode() { return getenv("LSERVE_DEBUG_STALL_DECODE") ? 1 : 0; }
+// The same for the tcgen05 prefill (LSERVE_DEBUG_STALL_PREFILL): its producer
+// hands out no work item, so the MMA and softmax warps' waits run out.
+int debug_stall_prefill() { return getenv("LSERVE_DEBUG_STALL_PREFILL") ? 1 : 0; }
 
 // Limit of every bounded wait inside the kernels: LSERVE_WAIT_TIMEOUT_NS when it
 // holds a positive integer (read at each launch), else 2 s.
@@ -523,7 +526,8 @@ lserve_status lserve_prefill(const lserve_shape* shape, const void* q, const voi
     if (s != LSERVE_OK) return s;
     const int nRow = (nQT + tp.QG - 1) / tp.QG;
     const int n_rows = shape->B * shape->Hkv * nRow;
-    tc::TcArgs T{A, block_mask, tp.QG, tp.HG, nRow, G / tp.HG, n_rows * (G / tp.HG), w.work_counter};
+    tc::TcArgs T{A, block_mask, tp.QG, tp.HG, nRow, G / tp.HG, n_rows * (G / tp.HG), w.work_counter,
+                 debug_stall_prefill()};
     s = shape->d == 128 ? launch_prefill_tc<128>(shape, q, k, v, T, n_rows, st)
                         : launch_prefill_tc<64>(shape, q, k, v, T, n_rows, st);
     return s == LSERVE_OK ? ok() : s;

@@ -239,7 +239,13 @@ struct TcArgs {
   int hsplit;                  // work items per row = G / HG
   int n_items;                 // work items in all = rows x hsplit
   int* work_counter;           // next unclaimed work item; zero at launch
+  int debug_stall;             // failure-detection test hook: the producer hands out no item
 };
+
+// Wait for the loads and MMAs still in flight when a CTA gives up: fixed,
+// independent of the (possibly very short) limit of the ordinary waits, so that
+// nothing lands in shared memory or TMEM after the CTA has released them.
+constexpr unsigned long long kPrefillDrainNs = 1000000000ull;
 
 // One work item (128 query rows sharing a KV tile list), decoded from its index.
 struct Item {
@@ -288,7 +294,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   // persistent CTA: the producer claims work items and passes them on through a
   // two-slot ring; q_empty frees the Q buffer (all S MMAs of an item done), o_free
   // frees the O accumulators (both warpgroups have read them in the epilogue)
-  __shared__ __align__(8) uint64_t item_full[2], item_empty[2], q_empty, o_free;
+  __shared__ __align__(8) uint64_t item_full[2], item_empty[2], q_empty, o_free, mma_drain;
   __shared__ int s_item[2];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
@@ -322,6 +328,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     }
     mbar_init(&q_empty, 1);
     mbar_init(&o_free, 256);
+    mbar_init(&mma_drain, 1);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -352,7 +359,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       prefetch_tensormap(&tmV);
     }
     int gk = 0, gv = 0, nq = 0;   // K and V steps issued; items with tiles (Q loads)
-    bool live = true;
+    int kiss = 0, viss = 0;       // K and V stage loads actually issued (for the drain)
+    bool live = !T.debug_stall;   // the test hook publishes nothing: every other wait runs out
     for (int ii = 0; live; ++ii) {
       const int slot = ii & 1;
       if (ii >= 2 && !wait_or_abort(&item_empty[slot], ((ii >> 1) - 1) & 1, &s_abort, tmo)) break;
@@ -390,6 +398,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
             break;
           }
           const int ka = it.pair_tile(t, 0), kb = it.pair_tile(t, 1);
+          kiss = gt + 1;
           if (leader) {
             mbar_arrive_expect_tx(&k_full[st], C::kPair);
             for (int x = 0; x < C::kBoxes; ++x) {
@@ -406,6 +415,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
             break;
           }
           const int ka = it.pair_tile(t - 1, 0), kb = it.pair_tile(t - 1, 1);
+          viss = gu + 1;
           if (leader) {
             mbar_arrive_expect_tx(&v_full[st], C::kPair);
             for (int x = 0; x < C::kBoxes; ++x) {
@@ -418,6 +428,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       }
       gk += np;
       gv += np;
+    }
+    if (s_abort) {   // let the copies still in flight land: the latest load of each stage, and Q
+      for (int g0 = max(0, kiss - kKStages); g0 < kiss; ++g0)
+        mbar_wait_bounded(&k_full[g0 % kKStages], (g0 / kKStages) & 1, kPrefillDrainNs);
+      for (int g0 = max(0, viss - kVStages); g0 < viss; ++g0)
+        mbar_wait_bounded(&v_full[g0 % kVStages], (g0 / kVStages) & 1, kPrefillDrainNs);
+      if (nq > 0) mbar_wait_bounded(&q_full, (nq - 1) & 1, kPrefillDrainNs);
     }
   } else if (warp == C::kWarpMma) {
     // ================================================================== MMA
@@ -497,6 +514,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       cs[0] += (np + 1) >> 1;
       cs[1] += np >> 1;
       if (s_abort) break;
+    }
+    if (s_abort) {   // every MMA issued so far completes before TMEM is released
+      commit(&mma_drain);
+      mbar_wait_bounded(&mma_drain, 0, kPrefillDrainNs);
     }
    }
   } else {
