@@ -363,6 +363,14 @@ def main():
     def decode_only():
         U.lserve_decode(*dargs, out=out_d, workspace=ws_d)
 
+    # selection reuse across decode steps: a step that keeps the dense heads'
+    # pages of a selection step (no scoring, no summaries read)
+    _, _, sel_d, seln_d = U.lserve_decode(*dargs, out=out_d, workspace=ws_d, return_selection=True)
+
+    def decode_reuse():
+        U.lserve_decode_reuse(setup.qd, setup.kp, setup.vp, setup.pt, setup.sl, setup.hk_d, wd.sink, wd.local,
+                              wd.token_budget, sel_d, seln_d, out=out_d, workspace=ws_d)
+
     def step():
         prefill()
         decode()
@@ -379,6 +387,7 @@ def main():
     t_prefill = time_loop(prefill, args.steps, args.warmup, stream, fl)
     t_decode = time_loop(decode_only, args.steps, args.warmup, stream, fl)
     t_decode_flushed = time_loop(decode_only, args.steps, 2, stream, scratch)
+    t_reuse = time_loop(decode_reuse, args.steps, args.warmup, stream, fl)
     ms_legacy = None
     if not args.no_legacy:   # the mma.sync kernel on the same call, for comparison only
         os.environ["LSERVE_PREFILL_IMPL"] = "mma"
@@ -406,7 +415,9 @@ def main():
     ms_tiles = float(np.median(t_tiles))
     ms_attn = max(1e-6, ms_prefill - ms_tiles)
     us_decode = float(np.median(t_decode)) * 1e3
-    ms_step, ms_prefill, us_decode = max_over_ranks([ms_step, ms_prefill, us_decode], dist, dev)
+    us_reuse = float(np.median(t_reuse)) * 1e3
+    ms_step, ms_prefill, us_decode, us_reuse = max_over_ranks([ms_step, ms_prefill, us_decode, us_reuse], dist, dev)
+    reuse_bytes = setup.dbytes["total"] - setup.dbytes["stats"]
 
     tflops_prefill = setup.prefill_flops / (ms_prefill * 1e-3) / 1e12
     tflops_attn = setup.prefill_flops / (ms_attn * 1e-3) / 1e12
@@ -473,6 +484,13 @@ def main():
         "prefill_tflops": tflops_prefill, "kept_tile_tflop": setup.prefill_flops / 1e12,
         "decode_us_per_step": us_decode, "decode_GBps": gbps_decode, "decode_bytes": setup.dbytes,
         "decode_us_per_step_l2_flushed": float(np.median(t_decode_flushed)) * 1e3,
+        "decode_reuse": {"us_per_step": us_reuse, "bytes": reuse_bytes,
+                         "GBps": reuse_bytes / (us_reuse * 1e-6) / 1e9,
+                         "frac_hbm": reuse_bytes / (us_reuse * 1e-6) / 1e9 / pk["hbm"],
+                         "cadence4_us_per_step": (us_decode + 3 * us_reuse) / 4,
+                         "note": "selection reused across decode steps: the dense heads keep the pages of a "
+                                 "selection step (no scoring, no summaries read); cadence4 = one selection step "
+                                 "and three reuse steps"},
         "roofline": {"bound": "tensor", "kernel": "prefill attention", "achieved": tflops_attn,
                      "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tflops_attn / pk["bf16"],
                      "traffic": traffic("prefill", wp.name == PREFILL_WL), "traffic_unit": "bytes per launch",

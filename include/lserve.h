@@ -184,7 +184,8 @@ typedef struct lserve_decode_args {
 int32_t lserve_decode_max_selected(const lserve_decode_args* args);
 
 /* Bytes of workspace lserve_decode needs (page scores, selection, partition,
- * per-warp partials).  It depends on the current device's SM count (the
+ * per-warp partials); lserve_decode_reuse needs the same, and may ask with
+ * stats = NULL.  It depends on the current device's SM count (the
  * attention grid is one wave of SMs x 2 CTAs) or, when the environment
  * variable LSERVE_DECODE_GRID holds a positive integer, on that grid size;
  * ask again after changing either. */
@@ -248,6 +249,36 @@ lserve_status lserve_decode(const lserve_decode_args* args, void* out, float* ls
 #define LSERVE_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB per device */
 lserve_status lserve_decode_noalloc(const lserve_decode_args* args, void* out, float* lse,
                                     int32_t* sel_out, int32_t* sel_n, void* stream);
+
+/*
+ * lserve_decode_reuse -- a decode step that keeps an earlier page selection.
+ *
+ * LServe + SampleAttention blog post, "LServe - Decode Phase": selection
+ * results are reused across a small window of decode steps, so that the page
+ * scoring is not paid on every token.  This call computes lserve_decode's
+ * attention with each dense head's page set taken from sel_in / sel_n_in
+ * instead of being scored and selected; the page summaries are not read
+ * (args->stats may be NULL) and no scoring kernel runs.
+ *
+ *   sel_in    int32 [B, Hkv, lserve_decode_max_selected(args)]: page indices
+ *             within each sequence (ascending), as lserve_decode wrote them to
+ *             sel_out at an earlier step of the same batch (same B, Hkv, maxP,
+ *             token_budget, sink, local).  Only the rows of dense heads are read.
+ *   sel_n_in  int32 [B, Hkv]: valid entries of each row (clamped to the row
+ *             capacity).
+ *
+ * A dense head of sequence b attends to every token t < seq_lens[b] of those
+ * pages: tokens appended since the selection count where they fall in a
+ * selected page, not elsewhere.  A streaming head takes its sink and local
+ * window from the current seq_lens, as in lserve_decode.  A page index outside
+ * [0, maxP) is recorded as LSERVE_ERR_DEVICE_BOUNDS and its tokens are skipped.
+ * out, lse, sel_out, sel_n and the workspace are as for lserve_decode (the same
+ * workspace size suffices); sel_out / sel_n may be sel_in / sel_n_in (the dense
+ * rows are copied onto themselves, the streaming rows refreshed).
+ */
+lserve_status lserve_decode_reuse(const lserve_decode_args* args, const int32_t* sel_in,
+                                  const int32_t* sel_n_in, void* out, float* lse, int32_t* sel_out,
+                                  int32_t* sel_n, void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ status */
 

@@ -83,3 +83,16 @@ def sparse_decode(q, k_pages, v_pages, page_table, seq_lens, stats, head_kind,
     out, lse = decode_attention(q, k_pages, v_pages, page_table, seq_lens, head_kind, sel,
                                 sink, local, scale)
     return out, lse, sel, margin, scores
+
+
+def reuse_decode(q, k_pages, v_pages, page_table, seq_lens, head_kind, kept_sel, sink, local, scale=None):
+    """A decode step that keeps the page selection of an earlier step.
+
+    LServe + SampleAttention blog post, "LServe - Decode Phase": selection
+    results are reused across a small window of decode steps.  Reading where
+    the page is silent: a dense KV head attends to every token t < seq_len of
+    the kept pages (tokens appended since the selection count where they fall
+    in a kept page, not elsewhere); a streaming KV head takes its sink and local
+    window from the current seq_len.  This is decode_attention with the kept
+    selection.  Returns (out, lse)."""
+    return decode_attention(q, k_pages, v_pages, page_table, seq_lens, head_kind, kept_sel, sink, local, scale)

@@ -164,3 +164,71 @@ def test_small_grid_gqa_d128(monkeypatch, grid):
     monkeypatch.setenv("LSERVE_DECODE_GRID", grid)
     w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=16, Hkv=2, d=128, dec_anchors=16)
     run_decode(w, 3, 1000, 512, 64, 100, lens=[1000, 333, 65], kind=[0, 1])
+
+
+def _reuse_setup(w, B, ctx, L0, budget, sink, local):
+    """Cache holding ctx valid tokens per sequence; a selection step at lengths L0."""
+    dev = "cuda"
+    pc, q = make(w, B, ctx)
+    kind = [g % 2 for g in range(w.Hkv)]   # dense and streaming heads alternate
+    hk = torch.tensor(kind, dtype=torch.uint8, device=dev)
+    kp, vp, pt = pc.k_pages.to(dev), pc.v_pages.to(dev), pc.page_table.to(dev)
+    l0 = torch.tensor(L0, dtype=torch.int32, device=dev)
+    stats = U.lserve_update_page_stats(kp, pt, l0, hk)
+    out, _, sel, sel_n = U.lserve_decode(q.to(dev), kp, vp, pt, l0, stats, hk, sink, local, budget,
+                                         return_selection=True)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+    return pc, q, kind, hk, kp, vp, pt, l0, out, sel, sel_n
+
+
+@pytest.mark.parametrize("G,d", [(4, 128), (1, 64)])
+def test_reuse_at_the_same_lengths_is_bit_identical(G, d):
+    w = dataclasses.replace(W.WORKLOADS["llama3_8b_32k"], Hq=4 * G, Hkv=4, d=d)
+    B, ctx = 3, 5000
+    pc, q, kind, hk, kp, vp, pt, l0, out, sel, sel_n = _reuse_setup(w, B, ctx, [ctx, 3000, 777], 1024, 64, 256)
+    lse = torch.empty(B, w.Hq, dtype=torch.float32, device="cuda")
+    again = U.lserve_decode_reuse(q.to("cuda"), kp, vp, pt, l0, hk, 64, 256, 1024, sel, sel_n, lse=lse)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+    assert torch.equal(again, out)
+
+
+def test_reuse_after_appending_tokens_matches_oracle():
+    w = dataclasses.replace(W.WORKLOADS["llama3_8b_32k"], Hq=16, Hkv=4, d=128)
+    B, ctx, sink, local, budget = 3, 6000, 64, 256, 1024
+    L0, L1 = [5000, 2100, 700], [6000, 2170, 701]
+    pc, q, kind, hk, kp, vp, pt, l0, _, sel, sel_n = _reuse_setup(w, B, ctx, L0, budget, sink, local)
+    l1 = torch.tensor(L1, dtype=torch.int32, device="cuda")
+    q1 = W.decode_query(w, B=B, step=1)   # the query of a later step
+    lse = torch.empty(B, w.Hq, dtype=torch.float32, device="cuda")
+    # the selection buffers double as outputs: dense rows stay, streaming rows follow the new lengths
+    out = U.lserve_decode_reuse(q1.to("cuda"), kp, vp, pt, l1, hk, sink, local, budget, sel, sel_n, lse=lse,
+                                sel_out=sel, sel_n_out=sel_n)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+    sel_np, seln_np = sel.cpu().numpy(), sel_n.cpu().numpy()
+    kept = {(b, g): sel_np[b, g, : seln_np[b, g]] for b in range(B) for g in range(w.Hkv)}
+    ref_out, ref_lse = OD.reuse_decode(f64(q1), f64(pc.k_pages), f64(pc.v_pages), pc.page_table.numpy(),
+                                       np.array(L1), kind, kept, sink, local)
+    assert_attn_close(f64(out), ref_out, "reuse out")
+    assert_lse_close(f64(lse), ref_lse, "reuse lse")
+    for b in range(B):   # streaming rows were refreshed for the new lengths
+        t = np.arange(L1[b])
+        window = sorted(set((t[(t < sink) | (t >= L1[b] - local)] // 64).tolist()))
+        for g in range(w.Hkv):
+            if kind[g]:
+                assert list(kept[(b, g)]) == window
+
+
+def test_reuse_reports_a_page_index_outside_the_table():
+    w = dataclasses.replace(W.WORKLOADS["llama3_8b_32k"], Hq=8, Hkv=2, d=128)
+    B, ctx = 2, 3000
+    pc, q, kind, hk, kp, vp, pt, l0, _, sel, sel_n = _reuse_setup(w, B, ctx, [ctx, ctx], 1024, 64, 256)
+    dense = kind.index(0)
+    bad = sel.clone()
+    bad[0, dense, 0] = pt.shape[1] + 5            # not a page of the sequence's table
+    U.lserve_decode_reuse(q.to("cuda"), kp, vp, pt, l0, hk, 64, 256, 1024, bad, sel_n)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 6   # LSERVE_ERR_DEVICE_BOUNDS
+    assert U.lserve_get_device_status() == 0

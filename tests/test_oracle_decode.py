@@ -120,3 +120,37 @@ def test_cra_is_one_without_dropping_and_matches_weight_sums():
     keep = A.kept_mask(np.arange(S), S, True, 5, 30, None)
     np.testing.assert_allclose(r[0, 1], (full * keep).sum(axis=1), atol=1e-12)
     np.testing.assert_allclose(r[0, 0], 1.0, atol=1e-12)
+
+
+def test_reuse_at_the_same_lengths_is_the_selection_step():
+    """Keeping a selection at the step that made it reproduces that step."""
+    q, k, v, kp, vp, pt, L = make(5, lens=[333, 200])
+    kind = np.array([0, 1], np.uint8)
+    st = Sel.page_stats(kp, pt, L, kind)
+    out, lse, sel, _, _ = D.sparse_decode(q, kp, vp, pt, L, st, kind, 128, 64, 100)
+    out2, lse2 = D.reuse_decode(q, kp, vp, pt, L, kind, sel, 64, 100)
+    np.testing.assert_array_equal(out2, out)
+    np.testing.assert_array_equal(lse2, lse)
+
+
+def test_reuse_after_appending_tokens_matches_sdpa_with_the_kept_pages():
+    """Tokens appended since the selection count where they fall in a kept page;
+    a streaming head's window follows the current length (SDPA with the token
+    mask written out from the reading)."""
+    ctx = 333
+    q, k, v, kp, vp, pt, _ = make(6, ctx=ctx)
+    kind = np.array([0, 1], np.uint8)
+    L0 = np.array([250, 130], np.int32)          # lengths at the selection step
+    L1 = np.array([333, 200], np.int32)          # lengths now
+    st = Sel.page_stats(kp, pt, L0, kind)
+    _, _, sel, _, _ = D.sparse_decode(q, kp, vp, pt, L0, st, kind, 128, 64, 100)
+    out, _ = D.reuse_decode(q, kp, vp, pt, L1, kind, sel, 64, 100)
+    t = np.arange(ctx)
+    for b in range(2):
+        dense_mask = np.isin(t // 64, np.asarray(sel[(b, 0)])) & (t < L1[b])
+        stream_mask = ((t < 64) | (t >= L1[b] - 100)) & (t < L1[b])
+        for h in range(4):
+            kvh = h // 2
+            m = dense_mask if kvh == 0 else stream_mask
+            ref = sdpa_one(q[b, h], k[b, m, kvh], v[b, m, kvh])
+            np.testing.assert_allclose(out[b, h], ref, atol=1e-12)

@@ -38,6 +38,7 @@ EXPORTED_SYMBOLS = (
     "lserve_decode_workspace_size",
     "lserve_decode",
     "lserve_decode_noalloc",
+    "lserve_decode_reuse",
     "lserve_get_device_status",
     "lserve_last_error_string",
     "lserve_version",
@@ -92,6 +93,7 @@ def load_library():
         "lserve_decode_workspace_size": (sz, [ctypes.POINTER(DecodeArgs)]),
         "lserve_decode": (i32, [ctypes.POINTER(DecodeArgs), vp, vp, vp, vp, vp, sz, vp]),
         "lserve_decode_noalloc": (i32, [ctypes.POINTER(DecodeArgs), vp, vp, vp, vp, vp]),
+        "lserve_decode_reuse": (i32, [ctypes.POINTER(DecodeArgs), vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "lserve_get_device_status": (i32, [vp]),
         "lserve_last_error_string": (ctypes.c_char_p, []),
         "lserve_version": (ctypes.c_char_p, []),
@@ -239,10 +241,12 @@ def _decode_args(q, k_pages, v_pages, page_table, seq_lens, stats, head_kind, si
     if page_table.shape[0] != B:
         raise ValueError("page_table must be [B, maxP]")
     _dev(seq_lens, "seq_lens", torch.int32, (B,))
-    _dev(stats, "stats", torch.bfloat16, (NP, Hkv, 4, 2, d))
+    if stats is not None:
+        _dev(stats, "stats", torch.bfloat16, (NP, Hkv, 4, 2, d))
     _dev(head_kind, "head_kind", torch.uint8, (Hkv,))
     return DecodeArgs(B, Hq, Hkv, d, NP, page_table.shape[1], q.data_ptr(), k_pages.data_ptr(),
-                      v_pages.data_ptr(), page_table.data_ptr(), seq_lens.data_ptr(), stats.data_ptr(),
+                      v_pages.data_ptr(), page_table.data_ptr(), seq_lens.data_ptr(),
+                      None if stats is None else stats.data_ptr(),
                       head_kind.data_ptr(), int(sink), int(local), int(token_budget), float(scale))
 
 
@@ -285,6 +289,32 @@ def lserve_decode(q, k_pages, v_pages, page_table, seq_lens, stats, head_kind, s
                              ws.numel(), _stream(stream)))
     if return_selection:
         return out, lse, sel_out, sel_n
+    return out
+
+
+def lserve_decode_reuse(q, k_pages, v_pages, page_table, seq_lens, head_kind, sink: int, local: int,
+                        token_budget: int, sel, sel_n, scale: float = 0.0, out=None, lse=None, sel_out=None,
+                        sel_n_out=None, workspace=None, stream=None):
+    """A decode step that keeps an earlier page selection (`sel`, `sel_n`, as
+    lserve_decode returned them); see include/lserve.h.  Returns out."""
+    lib = load_library()
+    a = _decode_args(q, k_pages, v_pages, page_table, seq_lens, None, head_kind, sink, local, token_budget, scale)
+    B, Hq, d = q.shape
+    Hkv = a.Hkv
+    out = torch.empty_like(q) if out is None else _dev(out, "out", torch.bfloat16, q.shape)
+    if lse is not None:
+        _dev(lse, "lse", torch.float32, (B, Hq))
+    kcap = int(lib.lserve_decode_max_selected(ctypes.byref(a)))
+    _dev(sel, "sel", torch.int32, (B, Hkv, kcap))
+    _dev(sel_n, "sel_n", torch.int32, (B, Hkv))
+    if sel_out is not None:
+        _dev(sel_out, "sel_out", torch.int32, (B, Hkv, kcap))
+    if sel_n_out is not None:
+        _dev(sel_n_out, "sel_n_out", torch.int32, (B, Hkv))
+    need = int(lib.lserve_decode_workspace_size(ctypes.byref(a)))
+    ws = _workspace(need, q.device, workspace)
+    _check(lib.lserve_decode_reuse(ctypes.byref(a), _ptr(sel), _ptr(sel_n), _ptr(out), _ptr(lse), _ptr(sel_out),
+                                   _ptr(sel_n_out), _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 

@@ -114,7 +114,8 @@ __device__ __forceinline__ void decode_partition(const int32_t* __restrict__ seq
                                                  const uint8_t* __restrict__ head_kind, int Hkv, int maxP,
                                                  int budget_pages, int sink, int local, int units, int kcap, int R,
                                                  int G, int D, int32_t* off, int32_t* range_unit,
-                                                 int32_t* range_counter, bf16* out, float* lse_out) {
+                                                 int32_t* range_counter, bf16* out, float* lse_out,
+                                                 const int32_t* sel_n_in) {
   __shared__ int s_warp[32];
   __shared__ int s_carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x, nw = nt >> 5;
@@ -122,9 +123,12 @@ __device__ __forceinline__ void decode_partition(const int32_t* __restrict__ seq
   __syncthreads();
   for (int base = 0; base < units; base += nt) {
     const int u = base + tid;
-    const int v = u < units ? unit_selected(seq_lens[u / Hkv], maxP, head_kind[u % Hkv] == LSERVE_HEAD_DENSE,
-                                            budget_pages, sink, local, kcap)
-                            : 0;
+    int v = 0;
+    if (u < units) {
+      const bool dense = head_kind[u % Hkv] == LSERVE_HEAD_DENSE;
+      v = (dense && sel_n_in) ? min(max(sel_n_in[u], 0), kcap)   // a kept selection's size
+                              : unit_selected(seq_lens[u / Hkv], maxP, dense, budget_pages, sink, local, kcap);
+    }
     int x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -173,12 +177,14 @@ __device__ __forceinline__ void decode_partition(const int32_t* __restrict__ seq
 }
 
 // Selection step: blocks 0 .. units-1 select the pages of one unit each
-// (topk_unit); block `units` lays out the attention grid's work
+// (topk_unit; with a kept selection sel_in / sel_n_in the dense units copy
+// their rows instead); block `units` lays out the attention grid's work
 // (decode_partition), which does not depend on the selected pages.
 __global__ void __launch_bounds__(kTopkThreads, 2) topk_pages_kernel(
     const float* scores, int maxP, const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind,
     int Hkv, int budget_pages, int sink, int local, int32_t* sel, int32_t* sel_n, int kcap, int units, int R, int G,
-    int D, int32_t* off, int32_t* range_unit, int32_t* range_counter, bf16* out, float* lse_out) {
+    int D, int32_t* off, int32_t* range_unit, int32_t* range_counter, bf16* out, float* lse_out,
+    const int32_t* sel_in, const int32_t* sel_n_in) {
   const int unit = blockIdx.x;
   // sequence length and head kind are inputs of the step, not results of the scoring grid
   const int L = unit < units ? seq_lens[unit / Hkv] : 0;
@@ -186,10 +192,10 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_pages_kernel(
   pdl_wait();
   pdl_launch_dependents();   // the attention grid may get resident; it waits for this grid
   if (unit < units)
-    topk_unit(scores, unit, maxP, L, dense, budget_pages, sink, local, sel, sel_n, kcap);
+    topk_unit(scores, unit, maxP, L, dense, budget_pages, sink, local, sel, sel_n, kcap, sel_in, sel_n_in);
   else
     decode_partition(seq_lens, head_kind, Hkv, maxP, budget_pages, sink, local, units, kcap, R, G, D, off,
-                     range_unit, range_counter, out, lse_out);
+                     range_unit, range_counter, out, lse_out, sel_n_in);
 }
 
 // Spin (with short sleeps) until cond() holds; false (and LSERVE_ERR_DEVICE_TIMEOUT

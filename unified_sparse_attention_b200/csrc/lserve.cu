@@ -306,8 +306,9 @@ int decode_grid() {
 
 // Launch with programmatic stream serialisation: the kernel may start while its
 // predecessor finishes and waits on griddepcontrol.wait before reading its output.
+// With pdl = false (the first kernel of a step) it is an ordinary launch.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+cudaError_t launch_pdl(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                        Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -318,7 +319,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -326,7 +327,7 @@ int streaming_page_bound(int sink, int local) {
   return (sink + kPage - 1) / kPage + (local + kPage - 1) / kPage + 1;
 }
 
-lserve_status validate_decode(const lserve_decode_args* a) {
+lserve_status validate_decode(const lserve_decode_args* a, bool need_stats = true) {
   if (!a) return fail(LSERVE_ERR_INVALID_ARG, "decode: null args");
   if (a->B <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->d <= 0 || a->Hq % a->Hkv || a->num_pages <= 0 || a->maxP <= 0)
     return fail(LSERVE_ERR_INVALID_ARG, "decode: invalid shape");
@@ -345,9 +346,10 @@ lserve_status validate_decode(const lserve_decode_args* a) {
     return fail(LSERVE_ERR_UNSUPPORTED, "decode: B * Hkv * selected pages exceeds 32-bit offsets");
   if (static_cast<long long>(a->maxP) * kPage >= (1ll << 28))
     return fail(LSERVE_ERR_UNSUPPORTED, "decode: maxP * 64 tokens must stay below 2^28");
-  if (!a->q || !a->k_pages || !a->v_pages || !a->page_table || !a->seq_lens || !a->stats || !a->head_kind)
+  if (!a->q || !a->k_pages || !a->v_pages || !a->page_table || !a->seq_lens || (need_stats && !a->stats) ||
+      !a->head_kind)
     return fail(LSERVE_ERR_INVALID_ARG, "decode: null tensor pointer");
-  if (!aligned16(a->q) || !aligned16(a->k_pages) || !aligned16(a->v_pages) || !aligned16(a->stats))
+  if (!aligned16(a->q) || !aligned16(a->k_pages) || !aligned16(a->v_pages) || (a->stats && !aligned16(a->stats)))
     return fail(LSERVE_ERR_INVALID_ARG, "decode: tensors must be 16-byte aligned");
   return LSERVE_OK;
 }
@@ -377,8 +379,11 @@ DecodePlan plan_decode(const lserve_decode_args* a, void* ws) {
 
 template <int D>
 lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, int32_t* sel, int32_t* sel_n,
-                              void* out, float* lse, cudaStream_t st) {
-  if (p.G == 1) {
+                              void* out, float* lse, cudaStream_t st, const int32_t* sel_in = nullptr,
+                              const int32_t* sel_n_in = nullptr) {
+  if (sel_in) {
+    // a kept selection: no scoring (the top-k step copies the dense rows)
+  } else if (p.G == 1) {
     // one query head per KV head: per-lane fp32 products over 16-byte summary
     // loads, one warp per (page, dense head); exactly one wave of CTAs, each
     // with an equal share of the (sequence, dense head, page) list
@@ -408,10 +413,10 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
   const int topk_smem = std::min(a->maxP, kTopkSmemKeys) * static_cast<int>(sizeof(uint32_t));
   const int units = a->B * a->Hkv;
   // one block per unit selects its pages; one more lays out the attention grid's work
-  if (launch_pdl(topk_pages_kernel, dim3(units + 1), dim3(kTopkThreads), topk_smem, st,
+  if (launch_pdl(sel_in == nullptr, topk_pages_kernel, dim3(units + 1), dim3(kTopkThreads), topk_smem, st,
                  static_cast<const float*>(p.scores), a->maxP, a->seq_lens, a->head_kind, a->Hkv, p.budget_pages,
                  a->sink, a->local, sel, sel_n, p.kcap, units, p.R, p.G, D, p.off, p.range_unit, p.range_counter,
-                 static_cast<bf16*>(out), lse) != cudaSuccess)
+                 static_cast<bf16*>(out), lse, sel_in, sel_n_in) != cudaSuccess)
     return check_launch("decode top-k");
   CUtensorMap tk, tv;
   const uint64_t rows = static_cast<uint64_t>(a->num_pages) * a->Hkv * kPage;
@@ -419,7 +424,7 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
     return fail(LSERVE_ERR_CUDA, "decode: cuTensorMapEncodeTiled failed");
   ensure_smem(paged_decode_kernel<D>, DecodeCfg<D>::smem_bytes(kDecodeMaxG));
   const float scale = a->scale > 0.f ? a->scale : 1.f / std::sqrt(static_cast<float>(D));
-  if (launch_pdl(paged_decode_kernel<D>, dim3(p.P), dim3(kDecodeThreads), DecodeCfg<D>::smem_bytes(p.G), st, tk,
+  if (launch_pdl(true, paged_decode_kernel<D>, dim3(p.P), dim3(kDecodeThreads), DecodeCfg<D>::smem_bytes(p.G), st, tk,
                  tv, static_cast<const bf16*>(a->q), a->page_table, a->maxP, a->seq_lens, a->head_kind,
                  static_cast<const int32_t*>(sel), static_cast<const int32_t*>(p.off),
                  static_cast<const int32_t*>(p.range_unit), p.range_counter, p.R, p.kcap, units, a->Hkv, p.G,
@@ -427,7 +432,7 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
                  debug_stall_decode(), p.part_o,
                  p.part_lse) != cudaSuccess)
     return check_launch("decode attention");
-  if (launch_pdl(decode_merge_kernel, dim3(units), dim3(kMergeThreads), 0, st, static_cast<const int32_t*>(p.off),
+  if (launch_pdl(true, decode_merge_kernel, dim3(units), dim3(kMergeThreads), 0, st, static_cast<const int32_t*>(p.off),
                  units, p.R, p.G, D, static_cast<const float*>(p.part_o), static_cast<const float*>(p.part_lse),
                  static_cast<bf16*>(out), lse) != cudaSuccess)
     return check_launch("decode merge");
@@ -573,7 +578,8 @@ int32_t lserve_decode_max_selected(const lserve_decode_args* args) {
 }
 
 size_t lserve_decode_workspace_size(const lserve_decode_args* args) {
-  if (validate_decode(args) != LSERVE_OK) return 0;
+  // the size depends on the shapes only: a call with stats = NULL (lserve_decode_reuse) asks too
+  if (validate_decode(args, /*need_stats=*/false) != LSERVE_OK) return 0;
   return plan_decode(args, nullptr).bytes;
 }
 
@@ -616,6 +622,25 @@ lserve_status lserve_decode_noalloc(const lserve_decode_args* args, void* out, f
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   s = args->d == 128 ? launch_decode_d<128>(args, p, sel, seln, out, lse, st)
                      : launch_decode_d<64>(args, p, sel, seln, out, lse, st);
+  return s == LSERVE_OK ? ok() : s;
+}
+
+lserve_status lserve_decode_reuse(const lserve_decode_args* args, const int32_t* sel_in, const int32_t* sel_n_in,
+                                  void* out, float* lse, int32_t* sel_out, int32_t* sel_n, void* workspace,
+                                  size_t ws_bytes, void* stream) {
+  lserve_status s = validate_decode(args, /*need_stats=*/false);
+  if (s != LSERVE_OK) return s;
+  if (!sel_in || !sel_n_in) return fail(LSERVE_ERR_INVALID_ARG, "decode reuse: sel_in and sel_n_in are required");
+  if (!out || !aligned16(out)) return fail(LSERVE_ERR_INVALID_ARG, "decode: out must be non-null and 16-byte aligned");
+  const size_t need = plan_decode(args, nullptr).bytes;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < need)
+    return fail(LSERVE_ERR_WORKSPACE, "decode: workspace missing, misaligned or smaller than %zu bytes", need);
+  DecodePlan p = plan_decode(args, workspace);
+  int32_t* sel = sel_out ? sel_out : p.sel;
+  int32_t* seln = sel_n ? sel_n : p.sel_n;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = args->d == 128 ? launch_decode_d<128>(args, p, sel, seln, out, lse, st, sel_in, sel_n_in)
+                     : launch_decode_d<64>(args, p, sel, seln, out, lse, st, sel_in, sel_n_in);
   return s == LSERVE_OK ? ok() : s;
 }
 

@@ -378,7 +378,8 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned lo
 // taken whole; one scan of (above, equal) counts places the output.
 __device__ __forceinline__ void topk_unit(const float* scores, int unit, int maxP, int L, bool dense,
                                           int budget_pages, int sink, int local, int32_t* sel, int32_t* sel_n,
-                                          int kcap) {
+                                          int kcap, const int32_t* sel_in = nullptr,
+                                          const int32_t* sel_n_in = nullptr) {
   extern __shared__ uint32_t s_keys[];
   __shared__ __align__(16) int s_hist[2][256];
   __shared__ unsigned long long s_scan[32];
@@ -410,6 +411,13 @@ __device__ __forceinline__ void topk_unit(const float* scores, int unit, int max
     return;
   }
 
+  if (sel_in) {   // a selection kept from an earlier step: its row as it stands
+    const int m = min(max(sel_n_in[unit], 0), kcap);
+    const int32_t* src = sel_in + static_cast<long>(unit) * kcap;
+    for (int j = tid; j < kcap; j += nt) row[j] = j < m ? src[j] : -1;
+    if (tid == 0 && sel_n) sel_n[unit] = m;
+    return;
+  }
   const int k = min(budget_pages, n);
   if (k >= n) {
     for (int j = tid; j < kcap; j += nt) row[j] = j < n ? j : -1;
