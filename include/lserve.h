@@ -162,6 +162,28 @@ lserve_status lserve_update_page_stats(int32_t B, int32_t Hkv, int32_t d, int32_
                                        int32_t first_logical_page, const uint8_t* head_kind,
                                        void* stats, void* stream);
 
+/*
+ * lserve_cra -- cumulative residual attention of a sparse prefill mask.
+ *
+ * LServe + SampleAttention blog post, "CRA - The Accuracy Proxy", Fig. 4: for
+ * every query row i, the share r_i of its causal softmax probability mass that
+ * the sparse mask keeps, and CRA = the minimum of r_i over the rows -- the
+ * worst-kept query, which a mask is judged by.  The mask is given exactly as to
+ * lserve_prefill (head_kind, sink, local, block_mask).  Computed from two LSE-only
+ * passes of the prefill kernel (causal, and the sparse mask; no output written):
+ * r_i = exp(lse_sparse(i) - lse_causal(i)); a row that keeps nothing retains 0.
+ *
+ *   retained  fp32 [B, Hq, S] or NULL: r_i of every row
+ *   cra       fp32 [B, Hq]: min_i r_i
+ *   workspace >= lserve_cra_workspace_size(shape) bytes, 256-byte aligned
+ * Errors and stream behaviour as for lserve_prefill.
+ */
+size_t lserve_cra_workspace_size(const lserve_shape* shape);
+lserve_status lserve_cra(const lserve_shape* shape, const void* q, const void* k, const void* v,
+                         const uint8_t* head_kind, int32_t sink, int32_t local,
+                         const uint8_t* block_mask, float* retained, float* cra, void* workspace,
+                         size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------- decode */
 
 typedef struct lserve_decode_args {

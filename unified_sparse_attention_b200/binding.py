@@ -33,6 +33,8 @@ EXPORTED_SYMBOLS = (
     "lserve_prefill_workspace_size",
     "lserve_prefill",
     "lserve_prefill_tile_lists",
+    "lserve_cra_workspace_size",
+    "lserve_cra",
     "lserve_update_page_stats",
     "lserve_decode_max_selected",
     "lserve_decode_workspace_size",
@@ -86,6 +88,8 @@ def load_library():
     sig = {
         "lserve_prefill_workspace_size": (sz, [ctypes.POINTER(Shape)]),
         "lserve_prefill": (i32, [ctypes.POINTER(Shape), vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
+        "lserve_cra_workspace_size": (sz, [ctypes.POINTER(Shape)]),
+        "lserve_cra": (i32, [ctypes.POINTER(Shape), vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
         "lserve_prefill_tile_lists": (i32, [ctypes.POINTER(Shape), vp, i32, i32, vp, vp, vp, ctypes.c_int64,
                                             vp, sz, vp]),
         "lserve_update_page_stats": (i32, [i32, i32, i32, i32, vp, vp, i32, vp, i32, vp, vp, vp]),
@@ -183,6 +187,33 @@ def lserve_prefill(q, k, v, head_kind, sink: int, local: int, block_mask=None, o
                               int(local), _ptr(block_mask), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                               _stream(stream)))
     return (out, lse) if (return_lse or lse is not None) else out
+
+
+def lserve_cra_workspace_size(B: int, S: int, Hq: int, Hkv: int, d: int) -> int:
+    return int(load_library().lserve_cra_workspace_size(ctypes.byref(Shape(B, S, Hq, Hkv, d, 0.0))))
+
+
+def lserve_cra(q, k, v, head_kind, sink: int, local: int, block_mask=None, scale: float = 0.0,
+               return_retained: bool = False, workspace=None, stream=None):
+    """Cumulative residual attention of a sparse prefill mask; see include/lserve.h.
+    Returns cra fp32[B, Hq] (and the per-row retained mass fp32[B, Hq, S])."""
+    lib = load_library()
+    _dev(q, "q", torch.bfloat16)
+    B, S, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _dev(k, "k", torch.bfloat16, (B, S, Hkv, d))
+    _dev(v, "v", torch.bfloat16, (B, S, Hkv, d))
+    _dev(head_kind, "head_kind", torch.uint8, (Hkv,))
+    if block_mask is not None:
+        _dev(block_mask, "block_mask", torch.uint8, (B, Hkv, S // PAGE, S // PAGE))
+    cra = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    retained = torch.empty(B, Hq, S, dtype=torch.float32, device=q.device) if return_retained else None
+    shape = _shape(q, k, scale)
+    need = int(lib.lserve_cra_workspace_size(ctypes.byref(shape)))
+    ws = _workspace(need, q.device, workspace)
+    _check(lib.lserve_cra(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(head_kind), int(sink), int(local),
+                          _ptr(block_mask), _ptr(retained), _ptr(cra), _ptr(ws), ws.numel(), _stream(stream)))
+    return (cra, retained) if return_retained else cra
 
 
 def lserve_prefill_tile_lists(B, S, Hq, Hkv, d, head_kind, sink, local, block_mask=None, stream=None):

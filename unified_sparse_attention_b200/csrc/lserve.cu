@@ -15,6 +15,7 @@
 #include <utility>
 
 #include "common.cuh"
+#include "cra.cuh"
 #include "decode.cuh"
 #include "page_stats.cuh"
 #include "prefill_mma.cuh"
@@ -272,9 +273,46 @@ lserve_status launch_prefill_tc(const lserve_shape* s, const void* q, const void
   return check_launch("prefill attention (tcgen05)");
 }
 
+// One prefill pass: tile lists, then the attention kernel.  out may be null
+// (only the LSE is written: the CRA passes).
+lserve_status run_prefill(const lserve_shape* shape, const void* q, const void* k, const void* v,
+                          const uint8_t* head_kind, int sink, int local, const uint8_t* block_mask, void* out,
+                          float* lse, void* workspace, cudaStream_t st);
+
+size_t round_up256(size_t b) { return (b + 255) / 256 * 256; }
+
 bool use_legacy_prefill() {
   const char* e = getenv("LSERVE_PREFILL_IMPL");
   return e && strcmp(e, "mma") == 0;
+}
+
+lserve_status run_prefill(const lserve_shape* shape, const void* q, const void* k, const void* v,
+                          const uint8_t* head_kind, int sink, int local, const uint8_t* block_mask, void* out,
+                          float* lse, void* workspace, cudaStream_t st) {
+  PrefillWs w = carve_prefill(shape, workspace, nullptr);
+  const int G = shape->Hq / shape->Hkv;
+  const int nQT = shape->S / kTile;
+  const float scale = shape->scale > 0.f ? shape->scale : 1.f / std::sqrt(static_cast<float>(shape->d));
+  PrefillArgs A{w.offsets, w.cols, w.order, head_kind, static_cast<bf16*>(out), lse, G,
+                shape->Hkv, nQT, shape->S, sink, local, scale * 1.4426950408889634f, wait_timeout_ns()};
+  TcPlan tp;
+  lserve_status s;
+  if (!use_legacy_prefill() && tc_plan(G, &tp)) {
+    s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz, w.order, st,
+                          tp.QG);
+    if (s != LSERVE_OK) return s;
+    const int nRow = (nQT + tp.QG - 1) / tp.QG;
+    const int n_rows = shape->B * shape->Hkv * nRow;
+    tc::TcArgs T{A, block_mask, tp.QG, tp.HG, nRow, G / tp.HG, n_rows * (G / tp.HG), w.work_counter,
+                 debug_stall_prefill()};
+    return shape->d == 128 ? launch_prefill_tc<128>(shape, q, k, v, T, n_rows, st)
+                           : launch_prefill_tc<64>(shape, q, k, v, T, n_rows, st);
+  }
+  s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz, w.order, st);
+  if (s != LSERVE_OK) return s;
+  const int n_rows = shape->B * shape->Hkv * nQT;
+  return shape->d == 128 ? launch_prefill_mma<128>(shape, q, k, v, A, n_rows, st)
+                         : launch_prefill_mma<64>(shape, q, k, v, A, n_rows, st);
 }
 
 // ----------------------------------------------------------------- decode
@@ -517,31 +555,45 @@ lserve_status lserve_prefill(const lserve_shape* shape, const void* q, const voi
       ws_bytes < lserve_prefill_workspace_size(shape))
     return fail(LSERVE_ERR_WORKSPACE, "prefill: workspace missing, misaligned or smaller than %zu bytes",
                 lserve_prefill_workspace_size(shape));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  PrefillWs w = carve_prefill(shape, workspace, nullptr);
-  const int G = shape->Hq / shape->Hkv;
-  const int nQT = shape->S / kTile;
-  const float scale = shape->scale > 0.f ? shape->scale : 1.f / std::sqrt(static_cast<float>(shape->d));
-  PrefillArgs A{w.offsets, w.cols, w.order, head_kind, static_cast<bf16*>(out), lse, G,
-                shape->Hkv, nQT, shape->S, sink, local, scale * 1.4426950408889634f, wait_timeout_ns()};
-  TcPlan tp;
-  if (!use_legacy_prefill() && tc_plan(G, &tp)) {
-    s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz, w.order, st,
-                          tp.QG);
-    if (s != LSERVE_OK) return s;
-    const int nRow = (nQT + tp.QG - 1) / tp.QG;
-    const int n_rows = shape->B * shape->Hkv * nRow;
-    tc::TcArgs T{A, block_mask, tp.QG, tp.HG, nRow, G / tp.HG, n_rows * (G / tp.HG), w.work_counter,
-                 debug_stall_prefill()};
-    s = shape->d == 128 ? launch_prefill_tc<128>(shape, q, k, v, T, n_rows, st)
-                        : launch_prefill_tc<64>(shape, q, k, v, T, n_rows, st);
-    return s == LSERVE_OK ? ok() : s;
-  }
-  s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz, w.order, st);
+  s = run_prefill(shape, q, k, v, head_kind, sink, local, block_mask, out, lse, workspace,
+                  static_cast<cudaStream_t>(stream));
+  return s == LSERVE_OK ? ok() : s;
+}
+
+size_t lserve_cra_workspace_size(const lserve_shape* shape) {
+  const size_t pw = lserve_prefill_workspace_size(shape);
+  if (!pw) return 0;
+  const size_t lse_bytes = static_cast<size_t>(shape->B) * shape->Hq * shape->S * sizeof(float);
+  return round_up256(pw) + 2 * round_up256(lse_bytes) + round_up256(static_cast<size_t>(shape->Hkv));
+}
+
+lserve_status lserve_cra(const lserve_shape* shape, const void* q, const void* k, const void* v,
+                         const uint8_t* head_kind, int32_t sink, int32_t local, const uint8_t* block_mask,
+                         float* retained, float* cra, void* workspace, size_t ws_bytes, void* stream) {
+  lserve_status s = validate_prefill(shape, sink, local);
   if (s != LSERVE_OK) return s;
-  const int n_rows = shape->B * shape->Hkv * nQT;
-  s = shape->d == 128 ? launch_prefill_mma<128>(shape, q, k, v, A, n_rows, st)
-                      : launch_prefill_mma<64>(shape, q, k, v, A, n_rows, st);
+  if (!q || !k || !v || !head_kind || !cra) return fail(LSERVE_ERR_INVALID_ARG, "cra: null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v))
+    return fail(LSERVE_ERR_INVALID_ARG, "cra: q/k/v must be 16-byte aligned");
+  const size_t need = lserve_cra_workspace_size(shape);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < need)
+    return fail(LSERVE_ERR_WORKSPACE, "cra: workspace missing, misaligned or smaller than %zu bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  const size_t pw = round_up256(lserve_prefill_workspace_size(shape));
+  const size_t lse_bytes = round_up256(static_cast<size_t>(shape->B) * shape->Hq * shape->S * sizeof(float));
+  float* lse_full = reinterpret_cast<float*>(base + pw);
+  float* lse_sparse = reinterpret_cast<float*>(base + pw + lse_bytes);
+  uint8_t* all_dense = base + pw + 2 * lse_bytes;
+  if (cudaMemsetAsync(all_dense, LSERVE_HEAD_DENSE, static_cast<size_t>(shape->Hkv), st) != cudaSuccess)
+    return fail(LSERVE_ERR_CUDA, "cra: memset failed");
+  // the causal reference and the sparse mask, LSE only (no output written)
+  s = run_prefill(shape, q, k, v, all_dense, 0, 0, nullptr, nullptr, lse_full, workspace, st);
+  if (s != LSERVE_OK) return s;
+  s = run_prefill(shape, q, k, v, head_kind, sink, local, block_mask, nullptr, lse_sparse, workspace, st);
+  if (s != LSERVE_OK) return s;
+  cra_reduce_kernel<<<shape->B * shape->Hq, kCraThreads, 0, st>>>(lse_sparse, lse_full, shape->S, retained, cra);
+  s = check_launch("cra reduction");
   return s == LSERVE_OK ? ok() : s;
 }
 

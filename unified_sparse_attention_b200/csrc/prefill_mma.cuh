@@ -243,10 +243,12 @@ __global__ void __launch_bounds__(kPrefillThreads) prefill_mma_kernel(const __gr
     const int i = i_row0 + hr * 8;
     const bool has = m_run[hr] != kNegInf && l_run[hr] > 0.f;
     const float inv = has ? 1.f / l_run[hr] : 0.f;
-    bf16* orow = A.out + (static_cast<long>(tok0 + i) * Hq + h) * D;
+    if (A.out) {   // no output: only the LSE (CRA passes)
+      bf16* orow = A.out + (static_cast<long>(tok0 + i) * Hq + h) * D;
 #pragma unroll
-    for (int j = 0; j < D / 8; ++j)
-      *reinterpret_cast<uint32_t*>(orow + j * 8 + tc) = pack_bf16x2(acc[j][2 * hr] * inv, acc[j][2 * hr + 1] * inv);
+      for (int j = 0; j < D / 8; ++j)
+        *reinterpret_cast<uint32_t*>(orow + j * 8 + tc) = pack_bf16x2(acc[j][2 * hr] * inv, acc[j][2 * hr + 1] * inv);
+    }
     if (A.lse && (lane & 3) == 0)
       A.lse[(static_cast<long>(b) * Hq + h) * A.S + i] =
           has ? (m_run[hr] + __log2f(l_run[hr])) * 0.6931471805599453f : kNegInf;

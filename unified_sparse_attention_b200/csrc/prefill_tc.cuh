@@ -727,13 +727,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       const float l_tot = l_run * w_own + l_o * w_oth;
       if (rb_valid) {
         const int c_lo = x * (D / 2);   // this warpgroup's half of the output columns
-        bf16* orow = A.out + (static_cast<long>(tok0 + i) * Hq + h) * D + c_lo;
         const bool has = n > 0 && m_all != kNegInf && l_tot > 0.f;
         const float inv = has ? 1.f / l_tot : 0.f;
         const uint32_t t_own = tmem + C::kColO + 128 * x + lane_off + c_lo;
         const uint32_t t_oth = tmem + C::kColO + 128 * (x ^ 1) + lane_off + c_lo;
+        bf16* orow = A.out ? A.out + (static_cast<long>(tok0 + i) * Hq + h) * D + c_lo : nullptr;
   #pragma unroll 1
-        for (int c0 = 0; c0 < D / 2; c0 += 16) {
+        for (int c0 = 0; orow && c0 < D / 2; c0 += 16) {   // no output: only the LSE (CRA passes)
           uint32_t oa[16], ob[16];
           if (nx > 0) tmem_ld16(t_own + c0, oa);
           if (nx_o > 0) tmem_ld16(t_oth + c0, ob);
