@@ -115,6 +115,20 @@ def decode_bytes(w, kind, k_pages_per_seq, d):
                 total=stats + sel + stream + q_out + table)
 
 
+def decode_bytes_int4(w, kind, k_pages_per_seq, d):
+    """The same step over INT4 pages: a K or V row is d/2 bytes of codes; a page
+    adds its key steps/offsets (2 d fp32) and value steps/offsets (2 x 64 fp32)."""
+    b = decode_bytes(w, kind, k_pages_per_seq, d)
+    n_dense = sum(1 for x in kind if x == 0)
+    n_stream = len(kind) - n_dense
+    page = 64 * d + 2 * d * 4 + 2 * 64 * 4
+    sel = w.dec_B * n_dense * k_pages_per_seq * page
+    stream_tok = min(w.ctx, w.sink + w.local)
+    stream = w.dec_B * n_stream * (stream_tok * (d + 8) + -(-stream_tok // 64) * 2 * d * 4)
+    total = b["stats"] + sel + stream + b["q_out"] + b["table"]
+    return dict(stats=b["stats"], selected=sel, streaming=stream, q_out=b["q_out"], table=b["table"], total=total)
+
+
 class Setup:
     def __init__(self, device, prefill_wl=PREFILL_WL, decode_wl=DECODE_WL):
         self.dev = device
@@ -371,6 +385,14 @@ def main():
         U.lserve_decode_reuse(setup.qd, setup.kp, setup.vp, setup.pt, setup.sl, setup.hk_d, wd.sink, wd.local,
                               wd.token_budget, sel_d, seln_d, out=out_d, workspace=ws_d)
 
+    # INT4 pages: the decode pool quantised once (lserve_quantize_pages_int4), then
+    # the same decode step over codes dequantised on chip
+    kq, kpar, vq, vpar, stats4 = U.lserve_quantize_pages_int4(setup.kp, setup.vp, setup.pt, setup.sl, setup.hk_d)
+
+    def decode_int4():
+        U.lserve_decode_int4(setup.qd, kq, vq, kpar, vpar, setup.pt, setup.sl, stats4, setup.hk_d, wd.sink,
+                             wd.local, wd.token_budget, out=out_d, workspace=ws_d)
+
     def step():
         prefill()
         decode()
@@ -388,6 +410,7 @@ def main():
     t_decode = time_loop(decode_only, args.steps, args.warmup, stream, fl)
     t_decode_flushed = time_loop(decode_only, args.steps, 2, stream, scratch)
     t_reuse = time_loop(decode_reuse, args.steps, args.warmup, stream, fl)
+    t_int4 = time_loop(decode_int4, args.steps, args.warmup, stream, fl)
     ms_legacy = None
     if not args.no_legacy:   # the mma.sync kernel on the same call, for comparison only
         os.environ["LSERVE_PREFILL_IMPL"] = "mma"
@@ -416,7 +439,10 @@ def main():
     ms_attn = max(1e-6, ms_prefill - ms_tiles)
     us_decode = float(np.median(t_decode)) * 1e3
     us_reuse = float(np.median(t_reuse)) * 1e3
-    ms_step, ms_prefill, us_decode, us_reuse = max_over_ranks([ms_step, ms_prefill, us_decode, us_reuse], dist, dev)
+    us_int4 = float(np.median(t_int4)) * 1e3
+    ms_step, ms_prefill, us_decode, us_reuse, us_int4 = max_over_ranks(
+        [ms_step, ms_prefill, us_decode, us_reuse, us_int4], dist, dev)
+    int4_bytes = decode_bytes_int4(wd, setup.kind_d.tolist(), setup.k_sel, wd.d)
     reuse_bytes = setup.dbytes["total"] - setup.dbytes["stats"]
 
     tflops_prefill = setup.prefill_flops / (ms_prefill * 1e-3) / 1e12
@@ -491,6 +517,12 @@ def main():
                          "note": "selection reused across decode steps: the dense heads keep the pages of a "
                                  "selection step (no scoring, no summaries read); cadence4 = one selection step "
                                  "and three reuse steps"},
+        "decode_int4": {"us_per_step": us_int4, "bytes": int4_bytes["total"],
+                        "GBps": int4_bytes["total"] / (us_int4 * 1e-6) / 1e9,
+                        "frac_hbm": int4_bytes["total"] / (us_int4 * 1e-6) / 1e9 / pk["hbm"],
+                        "speedup_vs_bf16": us_decode / us_int4,
+                        "note": "decode step over INT4 pages (codes + fp32 steps/offsets, dequantised on chip); "
+                                "pool quantised once before timing"},
         "roofline": {"bound": "tensor", "kernel": "prefill attention", "achieved": tflops_attn,
                      "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tflops_attn / pk["bf16"],
                      "traffic": traffic("prefill", wp.name == PREFILL_WL), "traffic_unit": "bytes per launch",

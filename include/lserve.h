@@ -273,6 +273,64 @@ lserve_status lserve_decode_noalloc(const lserve_decode_args* args, void* out, f
                                     int32_t* sel_out, int32_t* sel_n, void* stream);
 
 /*
+ * lserve_quantize_pages_int4 -- INT4 KV pages for lserve_decode_int4.
+ *
+ * LServe + SampleAttention blog post, "LServe - Decode Phase" and Fig. 2: INT4
+ * KV quantization cuts the bytes of every page read.  The pages name no scheme;
+ * this one is asymmetric INT4 with one step s and offset lo per (page, KV
+ * head, channel) for keys (over the page's valid tokens) and per (page, KV
+ * head, token) for values (over the d channels), in float32:
+ *   s = (hi - lo) / 15,  code = clamp(rint((x - lo) / s), 0, 15) (0 when s == 0),
+ *   dequantised value = bf16(fma(code, s, lo)), rounded to nearest even.
+ * The pages sequence b holds from page index first_page onward (0: all) are
+ * quantised from the bf16 pools, and the page summaries of dense heads are
+ * written from the dequantised keys (so they bound what lserve_decode_int4
+ * attends to).  Rows past seq_len get code 0 (values: s = lo = 0).
+ *
+ *   k_pages, v_pages  bf16 [num_pages, Hkv, 64, d] (read)
+ *   kq, vq            uint8 [num_pages, Hkv, 64, d/2] (written; channel 2j in
+ *                     the low nibble of byte j of a row)
+ *   kpar              fp32 [num_pages, Hkv, 2, d] (s per channel; lo per channel)
+ *   vpar              fp32 [num_pages, Hkv, 2, 64] (s per token; lo per token)
+ *   stats             bf16 [num_pages, Hkv, 4, 2, d] (dense heads written)
+ * All device memory, owned by the caller; k_pages, v_pages, kq, vq and stats
+ * 16-byte aligned.  The call is asynchronous on the stream.
+ * Errors: LSERVE_ERR_INVALID_ARG (sizes, null or misaligned pointers),
+ * LSERVE_ERR_UNSUPPORTED (d not 64 or 128); a page_table entry outside
+ * [0, num_pages) is skipped and reported as LSERVE_ERR_DEVICE_BOUNDS by
+ * lserve_get_device_status.
+ */
+lserve_status lserve_quantize_pages_int4(int32_t B, int32_t Hkv, int32_t d, int32_t num_pages,
+                                        const void* k_pages, const void* v_pages,
+                                        const int32_t* page_table, int32_t maxP,
+                                        const int32_t* seq_lens, int32_t first_page,
+                                        const uint8_t* head_kind, void* kq, float* kpar, void* vq,
+                                        float* vpar, void* stats, void* stream);
+
+/*
+ * lserve_decode_int4 -- lserve_decode over INT4 pages.
+ *
+ * LServe + SampleAttention blog post, "LServe - Decode Phase" and Fig. 2: the
+ * same selection and attention as lserve_decode, with every K and V row read
+ * as INT4 codes and dequantised on chip to bf16(fma(code, s, lo)) -- the
+ * values lserve_quantize_pages_int4 defines.  args->k_pages / args->v_pages
+ * point at the code pools kq / vq (uint8 [num_pages, Hkv, 64, d/2]) and
+ * args->stats at the summaries that lserve_quantize_pages_int4 wrote (so the
+ * bound holds for the dequantised keys).  The result equals lserve_decode run
+ * on bf16 pools holding the dequantised values.
+ *
+ *   kpar   fp32 [num_pages, Hkv, 2, d], 16-byte aligned (read)
+ *   vpar   fp32 [num_pages, Hkv, 2, 64], 16-byte aligned (read)
+ *   out, lse, sel_out, sel_n, workspace: as lserve_decode (the same
+ *   lserve_decode_workspace_size).
+ * Errors: LSERVE_ERR_INVALID_ARG for a null or misaligned kpar / vpar, and
+ * every error lserve_decode returns.
+ */
+lserve_status lserve_decode_int4(const lserve_decode_args* args, const float* kpar,
+                                 const float* vpar, void* out, float* lse, int32_t* sel_out,
+                                 int32_t* sel_n, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * lserve_decode_reuse -- a decode step that keeps an earlier page selection.
  *
  * LServe + SampleAttention blog post, "LServe - Decode Phase": selection

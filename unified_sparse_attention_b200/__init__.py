@@ -17,6 +17,8 @@ from .binding import (  # noqa: F401
     lserve_decode_max_selected,
     lserve_decode_noalloc,
     lserve_decode_reuse,
+    lserve_decode_int4,
+    lserve_quantize_pages_int4,
     lserve_cra,
     lserve_cra_workspace_size,
     lserve_decode_workspace_size,

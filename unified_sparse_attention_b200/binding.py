@@ -41,6 +41,8 @@ EXPORTED_SYMBOLS = (
     "lserve_decode",
     "lserve_decode_noalloc",
     "lserve_decode_reuse",
+    "lserve_quantize_pages_int4",
+    "lserve_decode_int4",
     "lserve_get_device_status",
     "lserve_last_error_string",
     "lserve_version",
@@ -98,6 +100,9 @@ def load_library():
         "lserve_decode": (i32, [ctypes.POINTER(DecodeArgs), vp, vp, vp, vp, vp, sz, vp]),
         "lserve_decode_noalloc": (i32, [ctypes.POINTER(DecodeArgs), vp, vp, vp, vp, vp]),
         "lserve_decode_reuse": (i32, [ctypes.POINTER(DecodeArgs), vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "lserve_quantize_pages_int4": (i32, [i32, i32, i32, i32, vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, vp, vp,
+                                             vp]),
+        "lserve_decode_int4": (i32, [ctypes.POINTER(DecodeArgs), vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "lserve_get_device_status": (i32, [vp]),
         "lserve_last_error_string": (ctypes.c_char_p, []),
         "lserve_version": (ctypes.c_char_p, []),
@@ -346,6 +351,82 @@ def lserve_decode_reuse(q, k_pages, v_pages, page_table, seq_lens, head_kind, si
     ws = _workspace(need, q.device, workspace)
     _check(lib.lserve_decode_reuse(ctypes.byref(a), _ptr(sel), _ptr(sel_n), _ptr(out), _ptr(lse), _ptr(sel_out),
                                    _ptr(sel_n_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def lserve_quantize_pages_int4(k_pages, v_pages, page_table, seq_lens, head_kind, first_page: int = 0, kq=None,
+                               kpar=None, vq=None, vpar=None, stats=None, stream=None):
+    """INT4 codes, steps and offsets of the pages each sequence holds, and the
+    page summaries of the dequantised keys; see include/lserve.h.
+    Returns (kq, kpar, vq, vpar, stats); buffers passed in are updated in place."""
+    lib = load_library()
+    _dev(k_pages, "k_pages", torch.bfloat16)
+    NP, Hkv, P, d = k_pages.shape
+    if P != PAGE:
+        raise ValueError("k_pages must be [NP, Hkv, 64, d]")
+    _dev(v_pages, "v_pages", torch.bfloat16, k_pages.shape)
+    _dev(page_table, "page_table", torch.int32)
+    B, maxP = page_table.shape
+    _dev(seq_lens, "seq_lens", torch.int32, (B,))
+    _dev(head_kind, "head_kind", torch.uint8, (Hkv,))
+    dev = k_pages.device
+    mk = lambda t, name, dt, shape: (torch.zeros(shape, dtype=dt, device=dev) if t is None
+                                     else _dev(t, name, dt, shape))
+    kq = mk(kq, "kq", torch.uint8, (NP, Hkv, P, d // 2))
+    vq = mk(vq, "vq", torch.uint8, (NP, Hkv, P, d // 2))
+    kpar = mk(kpar, "kpar", torch.float32, (NP, Hkv, 2, d))
+    vpar = mk(vpar, "vpar", torch.float32, (NP, Hkv, 2, P))
+    stats = mk(stats, "stats", torch.bfloat16, (NP, Hkv, 4, 2, d))
+    _check(lib.lserve_quantize_pages_int4(B, Hkv, d, NP, _ptr(k_pages), _ptr(v_pages), _ptr(page_table), maxP,
+                                          _ptr(seq_lens), int(first_page), _ptr(head_kind), _ptr(kq), _ptr(kpar),
+                                          _ptr(vq), _ptr(vpar), _ptr(stats), _stream(stream)))
+    return kq, kpar, vq, vpar, stats
+
+
+def lserve_decode_int4(q, kq, vq, kpar, vpar, page_table, seq_lens, stats, head_kind, sink: int, local: int,
+                       token_budget: int, scale: float = 0.0, out=None, lse=None, sel_out=None, sel_n=None,
+                       workspace=None, stream=None, return_selection: bool = False):
+    """lserve_decode over INT4 pages (as lserve_quantize_pages_int4 wrote them);
+    see include/lserve.h.  Returns out (and lse, sel, sel_n)."""
+    lib = load_library()
+    _dev(q, "q", torch.bfloat16)
+    B, Hq, d = q.shape
+    _dev(kq, "kq", torch.uint8)
+    NP, Hkv, P, d2 = kq.shape
+    if P != PAGE or 2 * d2 != d:
+        raise ValueError("kq must be [NP, Hkv, 64, d/2]")
+    _dev(vq, "vq", torch.uint8, kq.shape)
+    _dev(kpar, "kpar", torch.float32, (NP, Hkv, 2, d))
+    _dev(vpar, "vpar", torch.float32, (NP, Hkv, 2, P))
+    _dev(page_table, "page_table", torch.int32)
+    if page_table.shape[0] != B:
+        raise ValueError("page_table must be [B, maxP]")
+    _dev(seq_lens, "seq_lens", torch.int32, (B,))
+    _dev(stats, "stats", torch.bfloat16, (NP, Hkv, 4, 2, d))
+    _dev(head_kind, "head_kind", torch.uint8, (Hkv,))
+    a = DecodeArgs(B, Hq, Hkv, d, NP, page_table.shape[1], q.data_ptr(), kq.data_ptr(), vq.data_ptr(),
+                   page_table.data_ptr(), seq_lens.data_ptr(), stats.data_ptr(), head_kind.data_ptr(), int(sink),
+                   int(local), int(token_budget), float(scale))
+    out = torch.empty_like(q) if out is None else _dev(out, "out", torch.bfloat16, q.shape)
+    if lse is not None:
+        _dev(lse, "lse", torch.float32, (B, Hq))
+    kcap = int(lib.lserve_decode_max_selected(ctypes.byref(a)))
+    if return_selection and sel_out is None:
+        sel_out = torch.empty(B, Hkv, kcap, dtype=torch.int32, device=q.device)
+        sel_n = torch.empty(B, Hkv, dtype=torch.int32, device=q.device) if sel_n is None else sel_n
+    if sel_out is not None:
+        _dev(sel_out, "sel_out", torch.int32, (B, Hkv, kcap))
+    if sel_n is not None:
+        _dev(sel_n, "sel_n", torch.int32, (B, Hkv))
+    need = int(lib.lserve_decode_workspace_size(ctypes.byref(a)))
+    if need == 0:   # invalid arguments: let the library report which
+        _check(lib.lserve_decode_int4(ctypes.byref(a), _ptr(kpar), _ptr(vpar), _ptr(out), None, None, None, None, 0,
+                                      _stream(stream)))
+    ws = _workspace(need, q.device, workspace)
+    _check(lib.lserve_decode_int4(ctypes.byref(a), _ptr(kpar), _ptr(vpar), _ptr(out), _ptr(lse), _ptr(sel_out),
+                                  _ptr(sel_n), _ptr(ws), ws.numel(), _stream(stream)))
+    if return_selection:
+        return out, lse, sel_out, sel_n
     return out
 
 

@@ -76,6 +76,15 @@ struct DecodeCfg {
   // stage = K page | V page | q rows of the group (rounded up to 1 KB)
   __host__ __device__ static int stage_bytes(int G) { return 2 * kKVBytes + ((G * D * 2 + 1023) / 1024) * 1024; }
   __host__ __device__ static int smem_bytes(int G) { return kDecodeStages * stage_bytes(G) + 1024; }   // + alignment slack
+  // INT4 pages (lserve_decode_int4): stage = K codes | V codes | K steps, offsets |
+  // V steps, offsets | q rows; the consumers dequantise their rows into a bf16
+  // staging area laid out like a bf16 stage (2 x kKVBytes after the ring)
+  static constexpr int kQ4Bytes = 64 * (D / 2);   // one page of codes
+  static constexpr int kParKBytes = 2 * D * 4;    // fp32 step and offset per channel
+  static constexpr int kParVBytes = 2 * 64 * 4;   // fp32 step and offset per token
+  static constexpr int kQ4ParK = 2 * kQ4Bytes, kQ4ParV = kQ4ParK + kParKBytes, kQ4Q = kQ4ParV + kParVBytes;
+  __host__ __device__ static int stage_bytes_q4(int G) { return ((kQ4Q + G * D * 2 + 1023) / 1024) * 1024; }
+  __host__ __device__ static int smem_bytes_q4(int G) { return kDecodeStages * stage_bytes_q4(G) + 2 * kKVBytes + 1024; }
 };
 
 // Ranges the T selected pages are cut into: at most R (the workspace's
@@ -216,14 +225,30 @@ __device__ __forceinline__ bool spin_until(F&& cond, uint64_t timeout_ns) {
   }
 }
 
-template <int D>
+// Eight INT4 codes (one 32-bit word, channel e in bits 4e..4e+3) to eight bf16
+// values bf16(fma(code, s_e, lo_e)), as one 16-byte row chunk.  The code becomes
+// a float exactly through the bit pattern of 2^23 + code.
+__device__ __forceinline__ uint4 dequant8(uint32_t w, const float (&s)[8], const float (&lo)[8]) {
+  float v[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    v[e] = fmaf(__uint_as_float(0x4B000000u | ((w >> (4 * e)) & 15u)) - 8388608.f, s[e], lo[e]);
+  return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                    pack_bf16x2(v[6], v[7]));
+}
+
+// Q4 = false: bf16 pages (tmK, tmV over [NP * Hkv * 64, d] bf16).  Q4 = true:
+// INT4 pages (tmK, tmV over [NP * Hkv * 64, d/2] bytes) with their steps and
+// offsets kpar, vpar (see quant.cuh); the math after dequantisation is the same.
+template <int D, bool Q4 = false>
 __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const bf16* __restrict__ q, const int32_t* __restrict__ page_table, int maxP,
     const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind,
     const int32_t* sel, const int32_t* off, const int32_t* range_unit, int32_t* range_counter, int R,
     int kcap, int units, int Hkv, int G, int num_pages, int sink, int local, float scale_log2,
-    unsigned long long timeout_ns, int debug_stall, float* __restrict__ part_o, float* __restrict__ part_lse) {
+    unsigned long long timeout_ns, int debug_stall, float* __restrict__ part_o, float* __restrict__ part_lse,
+    const float* __restrict__ kpar = nullptr, const float* __restrict__ vpar = nullptr) {
   using Cfg = DecodeCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kDecodeStages];    // stage loaded (issuer's expect_tx + bytes)
@@ -235,7 +260,9 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
   __shared__ int s_issued;             // pages whose loads were issued
   __shared__ int s_abort;              // a bounded wait ran out or the plan was inconsistent
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int stage_bytes = Cfg::stage_bytes(G);
+  const int stage_bytes = Q4 ? Cfg::stage_bytes_q4(G) : Cfg::stage_bytes(G);
+  uint8_t* stage_k = smem + kDecodeStages * stage_bytes;   // Q4: dequantised rows, bf16-stage layout
+  uint8_t* stage_v = stage_k + Cfg::kKVBytes;
   const int q_bytes = G * D * 2;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
@@ -392,16 +419,26 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
         const int g = md.x % Hkv;
         const int p = md.z >= 0 ? md.z : 0;   // an invalid page loads page 0; all its tokens are masked
         uint8_t* kdst = smem + st * stage_bytes;
-        uint8_t* vdst = kdst + Cfg::kKVBytes;
         const bool with_q = md.w & kSegStart;
-        mbar_arrive_expect_tx(&full_bar[st], 2 * Cfg::kKVBytes + (with_q ? q_bytes : 0));
         const int row = (p * Hkv + g) * kPage;
+        if constexpr (Q4) {
+          mbar_arrive_expect_tx(&full_bar[st], Cfg::kQ4Q + (with_q ? q_bytes : 0));
+          tma_load_2d_hint(kdst, &tmK, &full_bar[st], 0, row, pol);
+          tma_load_2d_hint(kdst + Cfg::kQ4Bytes, &tmV, &full_bar[st], 0, row, pol);
+          const long ph = static_cast<long>(p) * Hkv + g;
+          bulk_load(kdst + Cfg::kQ4ParK, kpar + ph * 2 * D, Cfg::kParKBytes, &full_bar[st]);
+          bulk_load(kdst + Cfg::kQ4ParV, vpar + ph * 2 * kPage, Cfg::kParVBytes, &full_bar[st]);
+          if (with_q) bulk_load(kdst + Cfg::kQ4Q, q + static_cast<long>(md.x) * G * D, q_bytes, &full_bar[st]);
+        } else {
+          uint8_t* vdst = kdst + Cfg::kKVBytes;
+          mbar_arrive_expect_tx(&full_bar[st], 2 * Cfg::kKVBytes + (with_q ? q_bytes : 0));
 #pragma unroll
-        for (int x = 0; x < Cfg::kBoxes; ++x) {
-          tma_load_2d_hint(kdst + x * Cfg::kBoxBytes, &tmK, &full_bar[st], x * 64, row, pol);
-          tma_load_2d_hint(vdst + x * Cfg::kBoxBytes, &tmV, &full_bar[st], x * 64, row, pol);
+          for (int x = 0; x < Cfg::kBoxes; ++x) {
+            tma_load_2d_hint(kdst + x * Cfg::kBoxBytes, &tmK, &full_bar[st], x * 64, row, pol);
+            tma_load_2d_hint(vdst + x * Cfg::kBoxBytes, &tmV, &full_bar[st], x * 64, row, pol);
+          }
+          if (with_q) bulk_load(vdst + Cfg::kKVBytes, q + static_cast<long>(md.x) * G * D, q_bytes, &full_bar[st]);
         }
-        if (with_q) bulk_load(vdst + Cfg::kKVBytes, q + static_cast<long>(md.x) * G * D, q_bytes, &full_bar[st]);
         *v_issued = gp + 1;
       }
     }
@@ -436,10 +473,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
       const int u = md.x, pidx = md.y;
       const bool page_ok = md.z >= 0, streaming = md.w & kSegStreaming;
       const int L = md.w >> 3;
-      const uint8_t* ks_base = smem + st * stage_bytes;
-      const uint8_t* vs_base = ks_base + Cfg::kKVBytes;
+      const uint8_t* stg = smem + st * stage_bytes;
+      const uint8_t* ks_base = Q4 ? stage_k : stg;
+      const uint8_t* vs_base = Q4 ? stage_v : stg + Cfg::kKVBytes;
       if (md.w & kSegStart) {
-        const uint8_t* qs = vs_base + Cfg::kKVBytes;   // [G][D] bf16, row-major
+        const uint8_t* qs = stg + (Q4 ? Cfg::kQ4Q : 2 * Cfg::kKVBytes);   // [G][D] bf16, row-major
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {   // lane: head qr, channels 16 ks + tc, +1 and + 8, + 9
           const int c0 = ks * 16 + tc;
@@ -452,6 +490,37 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
         l_run[0] = l_run[1] = 0.f;
       }
       const int t_warp = pidx * kPage + warp * 16;   // first token of this warp's slice
+      if constexpr (Q4) {
+        // ---- this warp's 16 rows of K and V, dequantised into the staging area
+        // (bf16-stage layout, 128-byte swizzle); then the stage goes back at once
+        constexpr int W8 = D / 8;   // 8-channel chunks (one code word) per row
+        const uint32_t* kw = reinterpret_cast<const uint32_t*>(stg);
+        const uint32_t* vw = reinterpret_cast<const uint32_t*>(stg + Cfg::kQ4Bytes);
+        const float* kp4 = reinterpret_cast<const float*>(stg + Cfg::kQ4ParK);   // s[D], lo[D]
+        const float* vp4 = reinterpret_cast<const float*>(stg + Cfg::kQ4ParV);   // s[64], lo[64]
+        __syncwarp();   // the previous page's fragment loads from these rows are done
+#pragma unroll 2
+        for (int idx = lane; idx < 16 * W8; idx += 32) {
+          const int r = warp * 16 + idx / W8, c8 = idx % W8;
+          float s8[8], l8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            s8[e] = kp4[c8 * 8 + e];
+            l8[e] = kp4[D + c8 * 8 + e];
+          }
+          const uint32_t off_b = (c8 >> 3) * Cfg::kBoxBytes + swz128(r, c8 & 7);
+          *reinterpret_cast<uint4*>(stage_k + off_b) = dequant8(kw[r * W8 + c8], s8, l8);
+          const float sv = vp4[r], lv = vp4[kPage + r];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            s8[e] = sv;
+            l8[e] = lv;
+          }
+          *reinterpret_cast<uint4*>(stage_v + off_b) = dequant8(vw[r * W8 + c8], s8, l8);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[st]);   // codes, steps and q rows are no longer needed
+      }
 
       // ---- this warp's K and V fragments into registers, then the stage goes back
       // to the producer at once: the ring spends its time loading, not waiting for math
@@ -471,7 +540,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
                           vf[mt][1], vf[mt][2], vf[mt][3]);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[st]);   // release orders the shared-memory reads above
+      if (!Q4 && lane == 0) mbar_arrive(&empty_bar[st]);   // release orders the shared-memory reads above
 
       // ---- S^T = K Q^T: 16 tokens x 8 heads; alternate k-steps feed two accumulators
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};

@@ -20,6 +20,7 @@
 #include "page_stats.cuh"
 #include "prefill_mma.cuh"
 #include "prefill_tc.cuh"
+#include "quant.cuh"
 #include "select.cuh"
 #include "tile_lists.cuh"
 
@@ -102,6 +103,20 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D byte view [rows, inner] (row stride = inner bytes), box inner x 64, no swizzle:
+// one page of INT4 codes per load.
+bool make_map_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(inner), 64};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -418,7 +433,8 @@ DecodePlan plan_decode(const lserve_decode_args* a, void* ws) {
 template <int D>
 lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, int32_t* sel, int32_t* sel_n,
                               void* out, float* lse, cudaStream_t st, const int32_t* sel_in = nullptr,
-                              const int32_t* sel_n_in = nullptr) {
+                              const int32_t* sel_n_in = nullptr, const float* kpar = nullptr,
+                              const float* vpar = nullptr) {
   if (sel_in) {
     // a kept selection: no scoring (the top-k step copies the dense rows)
   } else if (p.G == 1) {
@@ -456,19 +472,23 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
                  a->sink, a->local, sel, sel_n, p.kcap, units, p.R, p.G, D, p.off, p.range_unit, p.range_counter,
                  static_cast<bf16*>(out), lse, sel_in, sel_n_in) != cudaSuccess)
     return check_launch("decode top-k");
+  // kpar set: INT4 pages (codes of d/2 bytes a row, steps and offsets in kpar, vpar)
+  const bool q4 = kpar != nullptr;
   CUtensorMap tk, tv;
   const uint64_t rows = static_cast<uint64_t>(a->num_pages) * a->Hkv * kPage;
-  if (!make_map_2d(&tk, a->k_pages, D, rows) || !make_map_2d(&tv, a->v_pages, D, rows))
-    return fail(LSERVE_ERR_CUDA, "decode: cuTensorMapEncodeTiled failed");
-  ensure_smem(paged_decode_kernel<D>, DecodeCfg<D>::smem_bytes(kDecodeMaxG));
+  const bool mapped = q4 ? make_map_2d_u8(&tk, a->k_pages, D / 2, rows) && make_map_2d_u8(&tv, a->v_pages, D / 2, rows)
+                         : make_map_2d(&tk, a->k_pages, D, rows) && make_map_2d(&tv, a->v_pages, D, rows);
+  if (!mapped) return fail(LSERVE_ERR_CUDA, "decode: cuTensorMapEncodeTiled failed");
+  auto* kern = q4 ? paged_decode_kernel<D, true> : paged_decode_kernel<D, false>;
+  ensure_smem(kern, q4 ? DecodeCfg<D>::smem_bytes_q4(kDecodeMaxG) : DecodeCfg<D>::smem_bytes(kDecodeMaxG));
+  const int smem = q4 ? DecodeCfg<D>::smem_bytes_q4(p.G) : DecodeCfg<D>::smem_bytes(p.G);
   const float scale = a->scale > 0.f ? a->scale : 1.f / std::sqrt(static_cast<float>(D));
-  if (launch_pdl(true, paged_decode_kernel<D>, dim3(p.P), dim3(kDecodeThreads), DecodeCfg<D>::smem_bytes(p.G), st, tk,
+  if (launch_pdl(true, kern, dim3(p.P), dim3(kDecodeThreads), smem, st, tk,
                  tv, static_cast<const bf16*>(a->q), a->page_table, a->maxP, a->seq_lens, a->head_kind,
                  static_cast<const int32_t*>(sel), static_cast<const int32_t*>(p.off),
                  static_cast<const int32_t*>(p.range_unit), p.range_counter, p.R, p.kcap, units, a->Hkv, p.G,
                  a->num_pages, a->sink, a->local, scale * 1.4426950408889634f, wait_timeout_ns(),
-                 debug_stall_decode(), p.part_o,
-                 p.part_lse) != cudaSuccess)
+                 debug_stall_decode(), p.part_o, p.part_lse, kpar, vpar) != cudaSuccess)
     return check_launch("decode attention");
   if (launch_pdl(true, decode_merge_kernel, dim3(units), dim3(kMergeThreads), 0, st, static_cast<const int32_t*>(p.off),
                  units, p.R, p.G, D, static_cast<const float*>(p.part_o), static_cast<const float*>(p.part_lse),
@@ -674,6 +694,53 @@ lserve_status lserve_decode_noalloc(const lserve_decode_args* args, void* out, f
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   s = args->d == 128 ? launch_decode_d<128>(args, p, sel, seln, out, lse, st)
                      : launch_decode_d<64>(args, p, sel, seln, out, lse, st);
+  return s == LSERVE_OK ? ok() : s;
+}
+
+lserve_status lserve_quantize_pages_int4(int32_t B, int32_t Hkv, int32_t d, int32_t num_pages, const void* k_pages,
+                                        const void* v_pages, const int32_t* page_table, int32_t maxP,
+                                        const int32_t* seq_lens, int32_t first_page, const uint8_t* head_kind,
+                                        void* kq, float* kpar, void* vq, float* vpar, void* stats, void* stream) {
+  if (B <= 0 || Hkv <= 0 || num_pages <= 0 || maxP <= 0 || first_page < 0 || B > 65535 || Hkv > 65535)
+    return fail(LSERVE_ERR_INVALID_ARG, "quantize: invalid sizes");
+  if (d != 64 && d != 128) return fail(LSERVE_ERR_UNSUPPORTED, "quantize: head dim %d not in {64,128}", d);
+  if (!k_pages || !v_pages || !page_table || !seq_lens || !head_kind || !kq || !kpar || !vq || !vpar || !stats)
+    return fail(LSERVE_ERR_INVALID_ARG, "quantize: null pointer");
+  if (!aligned16(k_pages) || !aligned16(v_pages) || !aligned16(kq) || !aligned16(vq) || !aligned16(stats))
+    return fail(LSERVE_ERR_INVALID_ARG, "quantize: pools and stats must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid(maxP, B, Hkv);
+  if (d == 128)
+    quant_int4_kernel<128><<<grid, 128, 0, st>>>(static_cast<const bf16*>(k_pages), static_cast<const bf16*>(v_pages),
+                                                 page_table, maxP, seq_lens, first_page, head_kind, Hkv, num_pages,
+                                                 static_cast<uint8_t*>(kq), kpar, static_cast<uint8_t*>(vq), vpar,
+                                                 static_cast<bf16*>(stats));
+  else
+    quant_int4_kernel<64><<<grid, 128, 0, st>>>(static_cast<const bf16*>(k_pages), static_cast<const bf16*>(v_pages),
+                                                page_table, maxP, seq_lens, first_page, head_kind, Hkv, num_pages,
+                                                static_cast<uint8_t*>(kq), kpar, static_cast<uint8_t*>(vq), vpar,
+                                                static_cast<bf16*>(stats));
+  const lserve_status s = check_launch("quantize");
+  return s == LSERVE_OK ? ok() : s;
+}
+
+lserve_status lserve_decode_int4(const lserve_decode_args* args, const float* kpar, const float* vpar, void* out,
+                                 float* lse, int32_t* sel_out, int32_t* sel_n, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  lserve_status s = validate_decode(args);
+  if (s != LSERVE_OK) return s;
+  if (!kpar || !vpar || !aligned16(kpar) || !aligned16(vpar))
+    return fail(LSERVE_ERR_INVALID_ARG, "decode int4: kpar and vpar must be non-null and 16-byte aligned");
+  if (!out || !aligned16(out)) return fail(LSERVE_ERR_INVALID_ARG, "decode: out must be non-null and 16-byte aligned");
+  const size_t need = plan_decode(args, nullptr).bytes;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < need)
+    return fail(LSERVE_ERR_WORKSPACE, "decode: workspace missing, misaligned or smaller than %zu bytes", need);
+  DecodePlan p = plan_decode(args, workspace);
+  int32_t* sel = sel_out ? sel_out : p.sel;
+  int32_t* seln = sel_n ? sel_n : p.sel_n;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = args->d == 128 ? launch_decode_d<128>(args, p, sel, seln, out, lse, st, nullptr, nullptr, kpar, vpar)
+                     : launch_decode_d<64>(args, p, sel, seln, out, lse, st, nullptr, nullptr, kpar, vpar);
   return s == LSERVE_OK ? ok() : s;
 }
 
