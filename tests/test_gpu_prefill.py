@@ -141,3 +141,15 @@ def test_gqa_ratios_and_odd_tile_count(G, S):
 def test_d64_mha_pairs_with_mask():
     w = dataclasses.replace(W.WORKLOADS["tiny"], B=2, Hq=2, Hkv=2, d=64)
     run_case(w, 832, [0, 1], 32, 97, mask_fill=0.3, B=2)
+
+
+@pytest.mark.parametrize("G", [1, 2])
+@pytest.mark.parametrize("sink,local", [(0, 64), (0, 65), (0, 66), (130, 127), (0, 4096), (5000, 0), (63, 1),
+                                        (65, 129)])
+def test_streaming_tile_runs_edges(G, sink, local):
+    """Where the window's tile count steps (local 64 / 65 / 66), a window or sink
+    covering the whole sequence, and an odd tile count (G = 1 pairs query tiles,
+    so the last pair is ragged): the kernel's own tile runs for streaming and
+    unmasked dense heads against the oracle's token-level kept sets."""
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2 * G, Hkv=2, d=64)
+    run_case(w, 576, [1, 0], sink, local)

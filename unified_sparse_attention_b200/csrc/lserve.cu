@@ -219,11 +219,12 @@ lserve_status validate_prefill(const lserve_shape* s, int sink, int local) {
 
 lserve_status launch_tile_lists(const lserve_shape* s, const uint8_t* head_kind, int sink, int local,
                                 const uint8_t* block_mask, const PrefillWs& w, int* offsets, uint16_t* cols,
-                                long long max_nnz, int* order, cudaStream_t st, int qg = 1) {
+                                long long max_nnz, int* order, cudaStream_t st, int qg = 1,
+                                bool closed_form = false) {
   const int nQT = s->S / kTile;
   const int nRow = (nQT + qg - 1) / qg;
   const int R = s->B * s->Hkv * nRow;
-  TileListParams P{s->B, s->Hkv, nQT, sink, local, head_kind, block_mask, qg, nRow};
+  TileListParams P{s->B, s->Hkv, nQT, sink, local, head_kind, block_mask, qg, nRow, closed_form ? 1 : 0};
   const size_t hist_ints = 2ull * s->B * s->Hkv * (nQT + 1) + 1;   // + the work counter
   if (cudaMemsetAsync(w.hist, 0, sizeof(int) * hist_ints, st) != cudaSuccess)
     return fail(LSERVE_ERR_CUDA, "prefill: memset failed");
@@ -313,8 +314,10 @@ lserve_status run_prefill(const lserve_shape* shape, const void* q, const void* 
   TcPlan tp;
   lserve_status s;
   if (!use_legacy_prefill() && tc_plan(G, &tp)) {
+    // rows with a closed-form list (streaming heads; dense heads without a mask)
+    // get no CSR entries: the kernel computes their tiles
     s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz, w.order, st,
-                          tp.QG);
+                          tp.QG, /*closed_form=*/true);
     if (s != LSERVE_OK) return s;
     const int nRow = (nQT + tp.QG - 1) / tp.QG;
     const int n_rows = shape->B * shape->Hkv * nRow;

@@ -253,11 +253,15 @@ struct Item {
   int g, b, bg;   // KV head, sequence, b * Hkv + g
   int qgi, h0, tok0, QG, HG;
   bool streaming;
-  const uint16_t* cols;
+  const uint16_t* cols;   // CSR list, or null: the closed-form runs [0, ra), [rw, rw + n - ra)
+  int ra, rw;
   __device__ int rb_head(int rb) const { return h0 + rb % HG; }
   __device__ int rb_qt(int rb) const { return qgi * QG + rb / HG; }
   // list entry of half h of step p (the odd tail repeats the last entry)
-  __device__ int pair_tile(int p, int h) const { return cols[min(2 * p + h, n - 1)]; }
+  __device__ int pair_tile(int p, int h) const {
+    const int j = min(2 * p + h, n - 1);
+    return cols ? cols[j] : (j < ra ? j : rw + (j - ra));
+  }
 };
 
 __device__ __forceinline__ Item item_at(const TcArgs& T, int w) {
@@ -273,10 +277,21 @@ __device__ __forceinline__ Item item_at(const TcArgs& T, int w) {
   it.QG = T.QG;
   it.HG = T.HG;
   it.streaming = A.head_kind[it.g] != LSERVE_HEAD_DENSE;
-  const int beg = A.row_offsets[r];
-  it.n = A.row_offsets[r + 1] - beg;
+  // the same rows as the list builder's closed-form ones (no CSR entries)
+  TileListParams P{0, A.Hkv, A.nQT, A.sink, A.local, A.head_kind, T.block_mask, T.QG, T.nRow, 1};
+  RowRuns rr;
+  if (row_runs(P, r, &rr)) {
+    it.n = rr.n;
+    it.cols = nullptr;
+    it.ra = rr.a;
+    it.rw = rr.w;
+  } else {
+    const int beg = A.row_offsets[r];
+    it.n = A.row_offsets[r + 1] - beg;
+    it.cols = A.cols + beg;
+    it.ra = it.rw = 0;
+  }
   it.np = (it.n + 1) >> 1;
-  it.cols = A.cols + beg;
   it.tok0 = it.b * A.S;
   return it;
 }

@@ -18,6 +18,13 @@
 // Work order: (b, kvh) groups one after another, longest rows first inside a
 // group.  Concurrent CTAs then share one KV head's K/V, which stays in L2 even
 // when the whole K/V of a long sequence does not.
+//
+// Closed-form rows (TileListParams::closed_form, the tcgen05 prefill): the list
+// of a streaming head's row (Lambda at tile level: the sink tiles, then the
+// window of the row's query tiles) and of a dense head's row without a block
+// mask (every causal tile) is two runs of consecutive tiles, which the attention
+// kernel computes itself (row_runs).  Such rows get no CSR entries; their length
+// still orders the work.
 #pragma once
 
 #include "common.cuh"
@@ -30,7 +37,44 @@ struct TileListParams {
   const uint8_t* block_mask;   // [B, Hkv, nQT, nQT] or null
   int qg = 1;                  // query tiles per row (a row keeps the union of their lists)
   int nRow = 0;                // rows per (b, kvh) = ceil(nQT / qg)
+  int closed_form = 0;         // rows with a closed-form list get no CSR entries
 };
+
+// counts[r] of a closed-form row: its length with this flag set (the CSR holds
+// nothing for it; the work order uses the length)
+constexpr int kClosedRow = 1 << 30;
+__device__ __forceinline__ int csr_count(int v) { return (v & kClosedRow) ? 0 : v; }
+__device__ __forceinline__ int row_length(int v) { return v & ~kClosedRow; }
+
+// The kept list of row r as two runs, tiles [0, a) then [w, w + n - a), when it
+// has that form: a streaming head's row (tiles holding a sink token, 64 kt <
+// sink, then the union of the windows of its query tiles qt_lo..qt_hi: tile kt
+// meets the window of qt when max(64 (qt - kt) - 63, 0) < local, i.e. qt - kt <
+// nw with nw = (local + 62) / 64 + 1 for local > 0 and nw = 0 for local = 0),
+// or a dense head's row without a block mask (all tiles kt <= qt_hi).  Returns
+// false for a block-masked dense row.  Entry j of the list is j < a ? j : w + j - a.
+struct RowRuns {
+  int a, w, n;
+};
+__device__ __forceinline__ bool row_runs(const TileListParams& P, int r, RowRuns* rr) {
+  const int qgi = r % P.nRow;
+  const int g = (r / P.nRow) % P.Hkv;
+  const int qt_lo = qgi * P.qg;
+  const int qt_hi = min(P.nQT - 1, qt_lo + P.qg - 1);
+  if (P.head_kind[g] == LSERVE_HEAD_DENSE) {
+    if (P.block_mask) return false;
+    rr->a = rr->w = rr->n = qt_hi + 1;
+    return true;
+  }
+  const int a = min((P.sink + kTile - 1) / kTile, qt_hi + 1);
+  int w0 = qt_hi + 1;   // no window
+  if (P.local > 0) w0 = max(0, qt_lo - ((P.local + kTile - 2) / kTile + 1) + 1);
+  const int w = max(w0, a);
+  rr->a = a;
+  rr->w = w;
+  rr->n = a + (qt_hi + 1 - w);
+  return true;
+}
 
 __device__ __forceinline__ bool tile_keep(const TileListParams& P, bool streaming, const uint8_t* mrow, int qt,
                                           int kt) {
@@ -75,6 +119,14 @@ __global__ void __launch_bounds__(256) tile_count_kernel(TileListParams P, int* 
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int R = P.B * P.Hkv * P.nRow;
   if (r >= R) return;
+  RowRuns rr;
+  if (P.closed_form && row_runs(P, r, &rr)) {
+    if ((threadIdx.x & 31) == 0) {
+      counts[r] = rr.n | kClosedRow;
+      atomicAdd(&hist[(r / P.nRow) * (P.nQT + 1) + rr.n], 1);
+    }
+    return;
+  }
   int cnt = 0;
   tile_row_walk(P, r, [&](int, int, const bool (&k4)[4]) { cnt += k4[0] + k4[1] + k4[2] + k4[3]; });
 #pragma unroll
@@ -99,7 +151,7 @@ __global__ void __launch_bounds__(1024) tile_scan_kernel(const int* __restrict__
   __syncthreads();
   for (int base = 0; base < R; base += 1024) {
     const int r = base + tid;
-    const int v = r < R ? counts[r] : 0;
+    const int v = r < R ? csr_count(counts[r]) : 0;
     int x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -158,7 +210,8 @@ __global__ void __launch_bounds__(256) tile_fill_kernel(TileListParams P, const 
   if (r >= R || *overflow) return;
   const int lane = threadIdx.x & 31;
   int pos = offsets[r];
-  tile_row_walk(P, r, [&](int, int kt0, const bool (&k4)[4]) {
+  const int cr = counts[r];
+  if (!(cr & kClosedRow)) tile_row_walk(P, r, [&](int, int kt0, const bool (&k4)[4]) {
     const int c = k4[0] + k4[1] + k4[2] + k4[3];
     int x = c;
 #pragma unroll
@@ -173,7 +226,7 @@ __global__ void __launch_bounds__(256) tile_fill_kernel(TileListParams P, const 
     pos += __shfl_sync(0xffffffffu, x, 31);
   });
   if (lane == 0 && order) {
-    const int k = (r / P.nRow) * (P.nQT + 1) + counts[r];
+    const int k = (r / P.nRow) * (P.nQT + 1) + row_length(cr);
     order[bucket[k] + atomicAdd(&fill[k], 1)] = r;
   }
 }
