@@ -281,17 +281,26 @@ lserve_status lserve_decode_noalloc(const lserve_decode_args* args, void* out, f
  * head, channel) for keys (over the page's valid tokens) and per (page, KV
  * head, token) for values (over the d channels), in float32:
  *   s = (hi - lo) / 15,  code = clamp(rint((x - lo) / s), 0, 15) (0 when s == 0),
- *   dequantised value = bf16(fma(code, s, lo)), rounded to nearest even.
+ *   dequantised value = fma(code, s, lo) in float32.
  * The pages sequence b holds from page index first_page onward (0: all) are
  * quantised from the bf16 pools, and the page summaries of dense heads are
- * written from the dequantised keys (so they bound what lserve_decode_int4
- * attends to).  Rows past seq_len get code 0 (values: s = lo = 0).
+ * written from the dequantised keys, minimum rounded down and maximum rounded
+ * up to bf16 (so they bound what lserve_decode_int4 attends to).  Rows past seq_len get code 0 (values: s = lo = 0).
  *
  *   k_pages, v_pages  bf16 [num_pages, Hkv, 64, d] (read)
- *   kq, vq            uint8 [num_pages, Hkv, 64, d/2] (written; channel 2j in
- *                     the low nibble of byte j of a row)
- *   kpar              fp32 [num_pages, Hkv, 2, d] (s per channel; lo per channel)
- *   vpar              fp32 [num_pages, Hkv, 2, 64] (s per token; lo per token)
+ *   kq                uint8 [num_pages, Hkv, 64, d/2] (written): one key row per
+ *                     token, its codes in the order of the decode step's operand
+ *                     fragments: four chunks of d/8 bytes; word w of chunk t holds
+ *                     nibbles n = j + 4e (nibble n in bits 4n..4n+3) of channels
+ *                     16 (r/2) + 8 (r%2) + 2t + e, r = 4w + j
+ *   vq                uint8 [num_pages, Hkv, 64 * d/2] (written): four slices of
+ *                     16 tokens, each 32 chunks of d/4 bytes; word m of chunk
+ *                     4g + t holds nibbles n = j + 4e of channel 16m + g + 8 (j%2),
+ *                     token 16 slice + 2t + 8 (j/2) + e
+ *   kpar              fp32 [num_pages, Hkv, 2, d] (written): s, then lo, each in
+ *                     four chunks of d/4 channels, entry i of chunk t being
+ *                     channel 16 (i/4) + 8 ((i/2)%2) + 2t + i%2
+ *   vpar              fp32 [num_pages, Hkv, 64, 2] (written): (s, lo) per token
  *   stats             bf16 [num_pages, Hkv, 4, 2, d] (dense heads written)
  * All device memory, owned by the caller; k_pages, v_pages, kq, vq and stats
  * 16-byte aligned.  The call is asynchronous on the stream.
@@ -312,15 +321,17 @@ lserve_status lserve_quantize_pages_int4(int32_t B, int32_t Hkv, int32_t d, int3
  *
  * LServe + SampleAttention blog post, "LServe - Decode Phase" and Fig. 2: the
  * same selection and attention as lserve_decode, with every K and V row read
- * as INT4 codes and dequantised on chip to bf16(fma(code, s, lo)) -- the
- * values lserve_quantize_pages_int4 defines.  args->k_pages / args->v_pages
- * point at the code pools kq / vq (uint8 [num_pages, Hkv, 64, d/2]) and
- * args->stats at the summaries that lserve_quantize_pages_int4 wrote (so the
- * bound holds for the dequantised keys).  The result equals lserve_decode run
- * on bf16 pools holding the dequantised values.
+ * as INT4 codes: keys s_c code + lo_c, values s_t code + lo_t (the values
+ * lserve_quantize_pages_int4 defines).  The steps are folded into the other
+ * operand (the tensor cores multiply the integer codes by s q and s p, each
+ * carried as the sum of two bf16 parts, so about 2^-18 of each product is
+ * lost) and the offsets into one fp32 term per head; no dequantised value is
+ * ever rounded to bf16.  args->k_pages / args->v_pages point at
+ * the code pools kq / vq and args->stats at the summaries that
+ * lserve_quantize_pages_int4 wrote (so the bound holds for the dequantised keys).
  *
  *   kpar   fp32 [num_pages, Hkv, 2, d], 16-byte aligned (read)
- *   vpar   fp32 [num_pages, Hkv, 2, 64], 16-byte aligned (read)
+ *   vpar   fp32 [num_pages, Hkv, 64, 2], 16-byte aligned (read)
  *   out, lse, sel_out, sel_n, workspace: as lserve_decode (the same
  *   lserve_decode_workspace_size).
  * Errors: LSERVE_ERR_INVALID_ARG for a null or misaligned kpar / vpar, and

@@ -45,7 +45,7 @@ def test_quantiser_bit_exact(d, lens):
     kq, kpar, vq, vpar, kdeq, _ = OQ.quantize_pages(f64(pc.k_pages), f64(pc.v_pages), pc.page_table.numpy(),
                                                     pc.seq_lens.numpy())
     np.testing.assert_array_equal(g["kq"].cpu().numpy(), kq)
-    np.testing.assert_array_equal(g["vq"].cpu().numpy(), vq)
+    np.testing.assert_array_equal(g["vq"].cpu().numpy(), vq.reshape(g["vq"].shape))
     np.testing.assert_array_equal(g["kpar"].cpu().numpy(), kpar)
     np.testing.assert_array_equal(g["vpar"].cpu().numpy(), vpar)
     st = OQ.quantized_stats(kdeq, pc.page_table.numpy(), pc.seq_lens.numpy(), kind)
@@ -104,7 +104,7 @@ def run_int4(w, B, ctx, budget, sink, local, lens=None, kind=None):
                                            gpu_sel, sink, local)
     assert_attn_close(f64(out), ref_out, "int4 decode out")
     assert_lse_close(f64(lse), ref_lse, "int4 decode lse")
-    return dict(pc=pc, q=q, out=out, lse=lse, kdeq=kdeq, vdeq=vdeq, stats=g["stats"], kind=kind)
+    return dict(pc=pc, q=q, out=out, lse=lse, kdeq=kdeq, vdeq=vdeq, stats=g["stats"], kind=kind, sel=gpu_sel)
 
 
 @pytest.mark.parametrize("G,d", [(1, 128), (2, 64), (4, 128), (8, 128)])
@@ -123,9 +123,10 @@ def test_int4_decode_single_token_and_empty_sequence():
     run_int4(w, 3, 130, 128, 0, 1, lens=[1, 130, 0], kind=[0, 1])
 
 
-def test_int4_decode_equals_bf16_decode_on_dequantised_pools():
-    """Dequantisation on chip lands the same bf16 values in the same layout, so
-    the bf16 path over the dequantised pools gives the identical result."""
+def test_int4_decode_matches_bf16_decode_on_dequantised_pools():
+    """The bf16 path over pools holding the dequantised values, and the INT4
+    path (steps folded into bf16(s q) and bf16(s p)), agree within the
+    attention tolerance, and select the same pages (same summaries)."""
     w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=8, Hkv=2, d=128, dec_anchors=8)
     r = run_int4(w, 2, 1500, 256, 64, 100, lens=[1500, 1210], kind=[0, 1])
     dev = "cuda"
@@ -134,11 +135,13 @@ def test_int4_decode_equals_bf16_decode_on_dequantised_pools():
     vd = torch.from_numpy(r["vdeq"]).to(torch.bfloat16).to(dev)
     hk = torch.tensor(r["kind"], dtype=torch.uint8, device=dev)
     lse = torch.empty_like(r["lse"])
-    out = U.lserve_decode(r["q"].to(dev), kd, vd, pc.page_table.to(dev), pc.seq_lens.to(dev), r["stats"], hk, 64,
-                          100, 256, lse=lse)
+    out, _, sel, sel_n = U.lserve_decode(r["q"].to(dev), kd, vd, pc.page_table.to(dev), pc.seq_lens.to(dev),
+                                         r["stats"], hk, 64, 100, 256, lse=lse, return_selection=True)
     torch.cuda.synchronize()
-    assert torch.equal(out, r["out"])
-    assert torch.equal(lse, r["lse"])
+    for (b, h), row in r["sel"].items():
+        assert list(sel[b, h, : sel_n[b, h]].cpu().numpy()) == list(row)
+    assert_attn_close(f64(r["out"]), f64(out), "int4 vs bf16 on dequantised pools")
+    assert_lse_close(f64(r["lse"]), f64(lse), "int4 vs bf16 lse")
 
 
 def test_int4_decode_rejects_missing_params():
@@ -159,3 +162,31 @@ def test_int4_decode_rejects_missing_params():
     st = lib.lserve_decode_int4(ctypes.byref(a), None, g["vpar"].data_ptr(), out.data_ptr(), None, None, None,
                                 ws.data_ptr(), ws.numel(), None)
     assert st != 0 and "kpar" in U.lserve_last_error_string()
+
+
+def test_int4_unattended_parameters_are_never_used():
+    """NaN in the value steps/offsets of every row outside the attended token
+    sets, and in the key steps/offsets of every page holding no attended token:
+    the output is unchanged, bit for bit."""
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=8, Hkv=2, d=128, dec_anchors=8)
+    r = run_int4(w, 2, 1500, 256, 64, 100, lens=[1500, 1210], kind=[0, 1])
+    pc, kind = r["pc"], r["kind"]
+    g = quantize(pc, kind)
+    kpar, vpar = g["kpar"].cpu().clone(), g["vpar"].cpu().clone()
+    L = pc.seq_lens.tolist()
+    nan = float("nan")
+    for b in range(2):
+        for h in range(2):
+            toks = set(OD.token_set(L[b], bool(kind[h]), 64, 100, None if kind[h] else r["sel"][(b, h)]).tolist())
+            for i in range(OS.n_pages(L[b])):
+                p = int(pc.page_table[b, i])
+                rows = [row for row in range(64) if i * 64 + row not in toks]
+                vpar[p, h, rows] = nan
+                if len(rows) == 64:
+                    kpar[p, h] = nan
+    dev = "cuda"
+    out2 = U.lserve_decode_int4(r["q"].to(dev), g["kq"], g["vq"], kpar.to(dev), vpar.to(dev), pc.page_table.to(dev),
+                                pc.seq_lens.to(dev), g["stats"], torch.tensor(kind, dtype=torch.uint8, device=dev),
+                                64, 100, 256)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, r["out"])

@@ -2,13 +2,15 @@
 
 * codes lie in [0, 15], the extremes of every group map to codes 0 and 15,
   and codes are monotone in the value within a group;
-* dequantisation is within one step (plus bf16 rounding) of the input;
+* dequantisation is within half a step (plus the float32 rounding of the fma)
+  of the input;
 * a group whose values are all equal dequantises exactly;
-* the bf16 rounding of the dequantised values is round-to-nearest-even
-  (checked by hand on ties);
+* the directed bf16 roundings of the summaries are checked by hand and
+  against torch's bf16 conversion (bracketing, one step apart at most);
 * the summaries of the dequantised keys bound every dequantised key.
 """
 import numpy as np
+import pytest
 import torch
 
 import workloads as W
@@ -16,7 +18,7 @@ from oracle import quant as Q
 from oracle import selection as Sel
 
 
-def pool(seed=3, B=2, ctx=150, Hkv=2, d=16, lens=None):
+def pool(seed=3, B=2, ctx=150, Hkv=2, d=64, lens=None):
     rng = np.random.default_rng(seed)
     k = torch.from_numpy(rng.standard_normal((B, ctx, Hkv, d)).astype(np.float32) * 3).to(torch.bfloat16)
     v = torch.from_numpy(rng.standard_normal((B, ctx, Hkv, d)).astype(np.float32)).to(torch.bfloat16)
@@ -28,14 +30,72 @@ def pool(seed=3, B=2, ctx=150, Hkv=2, d=16, lens=None):
     return pc.k_pages.float().numpy(), pc.v_pages.float().numpy(), pt.numpy(), lens
 
 
-def unpack(q):
-    return np.stack([q & 15, q >> 4], axis=-1).reshape(*q.shape[:-1], -1)
+def unpack_k(row_bytes, d):
+    return Q.unpack_nibbles(row_bytes, Q.k_code_position(d))
 
 
-def test_bf16_rounding_is_nearest_even():
-    x = np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 1.0 + 5 * 2 ** -9], np.float32)
-    # ties go to the even 7-bit mantissa; 1 + 5/512 lies nearer 1 + 1/128 than 1 + 2/128
-    np.testing.assert_array_equal(Q.bf16_round(x), np.array([1.0, 1.0 + 2 ** -6, -2.5, 1.0 + 2 ** -7], np.float32))
+def unpack_v(page_bytes, d):
+    return Q.unpack_nibbles(page_bytes, Q.v_code_position(d))
+
+
+def test_code_layouts_are_bijections():
+    """Every code of a key row / value page has its own nibble, and every
+    nibble holds one code; the parameter order lists each channel once."""
+    for d in (32, 64, 128):
+        kp = Q.k_code_position(d)
+        assert sorted(kp.tolist()) == list(range(d))
+        vp = Q.v_code_position(d)
+        assert sorted(vp.ravel().tolist()) == list(range(64 * d))
+        order = Q.k_param_order(d)
+        assert len(order) == d and sorted(order.tolist()) == list(range(d))
+        # round trip through the packed bytes
+        rng = np.random.default_rng(d)
+        codes = rng.integers(0, 16, size=(64, d)).astype(np.uint8)
+        packed = Q.pack_nibbles(codes, vp, 32 * d)
+        np.testing.assert_array_equal(Q.unpack_nibbles(packed, vp), codes)
+        row = codes[0]
+        np.testing.assert_array_equal(Q.unpack_nibbles(Q.pack_nibbles(row, kp, d // 2), kp), row)
+    with pytest.raises(ValueError):
+        Q.k_code_position(16)
+
+
+def test_key_chunk_holds_the_lane_channels():
+    """Chunk t of a key row (d/8 bytes) holds exactly the channels 2t, 2t+1 of
+    every group of eight (the channels one lane of the decode step multiplies)."""
+    d = 128
+    kp = Q.k_code_position(d)
+    for t in range(4):
+        lo, hi = 2 * t * (d // 8), 2 * (t + 1) * (d // 8)
+        chans = sorted(int(c) for c in np.nonzero((kp >= lo) & (kp < hi))[0])
+        assert chans == sorted(c for c in range(d) if (c % 8) // 2 == t)
+
+
+def test_bf16_directed_rounding_by_hand():
+    # bf16 keeps 8 significant bits: next to 1 the representable values are 1 +- k 2^-7
+    x = np.array([1.0 + 2 ** -10, -1.0 - 2 ** -10, 1.5, -2.5, 2 ** -8 * 3.3, np.inf, -np.inf], np.float32)
+    np.testing.assert_array_equal(Q.bf16_round_down(x),
+                                  np.array([1.0, -1.0 - 2 ** -7, 1.5, -2.5, 2 ** -8 * 3.296875, np.inf, -np.inf],
+                                           np.float32))
+    np.testing.assert_array_equal(Q.bf16_round_up(x),
+                                  np.array([1.0 + 2 ** -7, -1.0, 1.5, -2.5, 2 ** -8 * 3.3125, np.inf, -np.inf],
+                                           np.float32))
+
+
+def test_bf16_directed_rounding_brackets_and_is_tight():
+    """Down <= x <= up, both bf16 (torch's own bf16 conversion leaves them
+    unchanged), and they are equal or one bf16 step apart."""
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal(20000) * np.exp(rng.uniform(-20, 20, 20000))).astype(np.float32)
+    dn, up = Q.bf16_round_down(x), Q.bf16_round_up(x)
+    assert np.all(dn <= x) and np.all(x <= up)
+    as_bf16 = lambda a: torch.from_numpy(a).to(torch.bfloat16).float().numpy()
+    np.testing.assert_array_equal(as_bf16(dn), dn)
+    np.testing.assert_array_equal(as_bf16(up), up)
+    exact = dn == up
+    np.testing.assert_array_equal(exact, as_bf16(x) == x)
+    # no bf16 lies strictly between: same sign, so their top halves differ by one
+    gap = np.abs(up.view(np.uint32).astype(np.int64) - dn.view(np.uint32).astype(np.int64))
+    assert np.all(gap[~exact] == 0x10000)
 
 
 def test_codes_range_extremes_monotone_and_error_bound():
@@ -45,7 +105,7 @@ def test_codes_range_extremes_monotone_and_error_bound():
         for i in range(Sel.n_pages(L[b])):
             p, nv = pt[b, i], min(64, L[b] - 64 * i)
             for g in range(2):
-                kc = unpack(kq[p, g])[:nv]
+                kc = np.stack([unpack_k(kq[p, g, r], 2 * kq.shape[-1]) for r in range(64)])[:nv]
                 x = kp[p, g, :nv]
                 assert kc.max() <= 15
                 for c in range(x.shape[1]):           # keys: per channel
@@ -54,16 +114,20 @@ def test_codes_range_extremes_monotone_and_error_bound():
                         assert kc[col.argmin(), c] == 0 and kc[col.argmax(), c] == 15
                     order = np.argsort(col, kind="stable")
                     assert np.all(np.diff(kc[order, c].astype(int)) >= 0)
-                step = kpar[p, g, 0]
+                step = np.empty_like(kpar[p, g, 0])
+                step[Q.k_param_order(step.size)] = kpar[p, g, 0]
                 err = np.abs(kdeq[p, g, :nv] - x)
-                assert np.all(err <= step[None, :] * 0.5 * (1 + 1e-5) + np.abs(x) * 2 ** -8 + 1e-6)
-                vc = unpack(vq[p, g])[:nv]
+                # half a step, plus the float32 rounding of the fma
+                rnd = np.maximum(np.abs(x), np.abs(kdeq[p, g, :nv])) * 2 ** -22
+                assert np.all(err <= step[None, :] * 0.5 * (1 + 1e-5) + rnd + 1e-7)
+                vc = unpack_v(vq[p, g], kp.shape[-1])[:nv]
                 y = vp[p, g, :nv]
                 for t in range(nv):                    # values: per token
                     if y[t].max() > y[t].min():
                         assert vc[t, y[t].argmin()] == 0 and vc[t, y[t].argmax()] == 15
                 err = np.abs(vdeq[p, g, :nv] - y)
-                assert np.all(err <= vpar[p, g, 0, :nv, None] * 0.5 * (1 + 1e-5) + np.abs(y) * 2 ** -8 + 1e-6)
+                rnd = np.maximum(np.abs(y), np.abs(vdeq[p, g, :nv])) * 2 ** -22
+                assert np.all(err <= vpar[p, g, :nv, 0, None] * 0.5 * (1 + 1e-5) + rnd + 1e-7)
 
 
 def test_constant_group_dequantises_exactly():

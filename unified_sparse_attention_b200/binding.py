@@ -373,9 +373,9 @@ def lserve_quantize_pages_int4(k_pages, v_pages, page_table, seq_lens, head_kind
     mk = lambda t, name, dt, shape: (torch.zeros(shape, dtype=dt, device=dev) if t is None
                                      else _dev(t, name, dt, shape))
     kq = mk(kq, "kq", torch.uint8, (NP, Hkv, P, d // 2))
-    vq = mk(vq, "vq", torch.uint8, (NP, Hkv, P, d // 2))
+    vq = mk(vq, "vq", torch.uint8, (NP, Hkv, P * d // 2))
     kpar = mk(kpar, "kpar", torch.float32, (NP, Hkv, 2, d))
-    vpar = mk(vpar, "vpar", torch.float32, (NP, Hkv, 2, P))
+    vpar = mk(vpar, "vpar", torch.float32, (NP, Hkv, P, 2))
     stats = mk(stats, "stats", torch.bfloat16, (NP, Hkv, 4, 2, d))
     _check(lib.lserve_quantize_pages_int4(B, Hkv, d, NP, _ptr(k_pages), _ptr(v_pages), _ptr(page_table), maxP,
                                           _ptr(seq_lens), int(first_page), _ptr(head_kind), _ptr(kq), _ptr(kpar),
@@ -395,9 +395,9 @@ def lserve_decode_int4(q, kq, vq, kpar, vpar, page_table, seq_lens, stats, head_
     NP, Hkv, P, d2 = kq.shape
     if P != PAGE or 2 * d2 != d:
         raise ValueError("kq must be [NP, Hkv, 64, d/2]")
-    _dev(vq, "vq", torch.uint8, kq.shape)
+    _dev(vq, "vq", torch.uint8, (NP, Hkv, P * d2))
     _dev(kpar, "kpar", torch.float32, (NP, Hkv, 2, d))
-    _dev(vpar, "vpar", torch.float32, (NP, Hkv, 2, P))
+    _dev(vpar, "vpar", torch.float32, (NP, Hkv, P, 2))
     _dev(page_table, "page_table", torch.int32)
     if page_table.shape[0] != B:
         raise ValueError("page_table must be [B, maxP]")

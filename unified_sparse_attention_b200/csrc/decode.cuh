@@ -77,14 +77,14 @@ struct DecodeCfg {
   __host__ __device__ static int stage_bytes(int G) { return 2 * kKVBytes + ((G * D * 2 + 1023) / 1024) * 1024; }
   __host__ __device__ static int smem_bytes(int G) { return kDecodeStages * stage_bytes(G) + 1024; }   // + alignment slack
   // INT4 pages (lserve_decode_int4): stage = K codes | V codes | K steps, offsets |
-  // V steps, offsets | q rows; the consumers dequantise their rows into a bf16
-  // staging area laid out like a bf16 stage (2 x kKVBytes after the ring)
+  // V steps, offsets | q rows (layouts in quant.cuh); the consumers build their
+  // tensor-core fragments from the code words directly
   static constexpr int kQ4Bytes = 64 * (D / 2);   // one page of codes
   static constexpr int kParKBytes = 2 * D * 4;    // fp32 step and offset per channel
   static constexpr int kParVBytes = 2 * 64 * 4;   // fp32 step and offset per token
   static constexpr int kQ4ParK = 2 * kQ4Bytes, kQ4ParV = kQ4ParK + kParKBytes, kQ4Q = kQ4ParV + kParVBytes;
   __host__ __device__ static int stage_bytes_q4(int G) { return ((kQ4Q + G * D * 2 + 1023) / 1024) * 1024; }
-  __host__ __device__ static int smem_bytes_q4(int G) { return kDecodeStages * stage_bytes_q4(G) + 2 * kKVBytes + 1024; }
+  __host__ __device__ static int smem_bytes_q4(int G) { return kDecodeStages * stage_bytes_q4(G) + 1024; }
 };
 
 // Ranges the T selected pages are cut into: at most R (the workspace's
@@ -225,21 +225,23 @@ __device__ __forceinline__ bool spin_until(F&& cond, uint64_t timeout_ns) {
   }
 }
 
-// Eight INT4 codes (one 32-bit word, channel e in bits 4e..4e+3) to eight bf16
-// values bf16(fma(code, s_e, lo_e)), as one 16-byte row chunk.  The code becomes
-// a float exactly through the bit pattern of 2^23 + code.
-__device__ __forceinline__ uint4 dequant8(uint32_t w, const float (&s)[8], const float (&lo)[8]) {
-  float v[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e)
-    v[e] = fmaf(__uint_as_float(0x4B000000u | ((w >> (4 * e)) & 15u)) - 8388608.f, s[e], lo[e]);
-  return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                    pack_bf16x2(v[6], v[7]));
-}
+// Two INT4 codes, nibbles k and k + 4 of w, as the bf16 pair (128 + code): the
+// codes become the low mantissa bits of 128 = 2^7, whose bf16 ulp is 1.
+__device__ __forceinline__ uint32_t q4_pair(uint32_t w, int k) { return ((w >> (4 * k)) & 0x000F000Fu) | 0x43004300u; }
+
 
 // Q4 = false: bf16 pages (tmK, tmV over [NP * Hkv * 64, d] bf16).  Q4 = true:
 // INT4 pages (tmK, tmV over [NP * Hkv * 64, d/2] bytes) with their steps and
-// offsets kpar, vpar (see quant.cuh); the math after dequantisation is the same.
+// offsets kpar, vpar (layouts in quant.cuh).  The steps fold into the other
+// operand, so the tensor cores multiply integer codes (exact in bf16, offset by
+// the 128 of q4_pair) and the offsets go into one fp32 term per head:
+//   q.k_t = sum_c (128 + code_tc) (s_c q_c) + sum_c (lo_c - 128 s_c) q_c
+//     with s q split into two bf16 parts (hi + lo, two MMAs), so the logits
+//     carry a rounding of about 2^-18 of each product;
+//   sum_t p_t v_t = sum_t (128 + code_tc) (s_t p_t) + sum_t (lo_t - 128 s_t) p_t
+//     with s p split the same way.
+// One bf16 rounding of s q or s p would scale with |x - lo| (or the step of an
+// outlier-wide group), not with |x|; the split keeps it near 2^-18.
 template <int D, bool Q4 = false>
 __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -261,8 +263,6 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
   __shared__ int s_abort;              // a bounded wait ran out or the plan was inconsistent
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int stage_bytes = Q4 ? Cfg::stage_bytes_q4(G) : Cfg::stage_bytes(G);
-  uint8_t* stage_k = smem + kDecodeStages * stage_bytes;   // Q4: dequantised rows, bf16-stage layout
-  uint8_t* stage_v = stage_k + Cfg::kKVBytes;
   const int q_bytes = G * D * 2;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
@@ -449,9 +449,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
     // heads, K = tokens), so the G <= 8 heads fill N exactly.  A lane holds
     // heads tc, tc + 1 of the tile.
     constexpr int KS = D / 16;
-    uint32_t qb[KS][2];                   // Q^T as the B operand (heads >= G are zero)
+    uint32_t qb[Q4 ? 1 : KS][2];          // Q^T as the B operand (heads >= G are zero)
+    float qf[Q4 ? D / 4 : 1];             // INT4: q of head qr at this lane's channels, key-chunk order
     float acc[D / 16][4];                 // O^T: m-tile mt = channels 16 mt .. 16 mt + 15
     float m_run[2], l_run[2];             // online softmax of heads tc, tc + 1
+    float vc_run[2];                      // INT4: sum_t (lo_t - 128 s_t) p_t, heads tc, tc + 1
     const int mi = lane >> 3, rr = lane & 7;
     const int qr = lane >> 2, tc = 2 * (lane & 3);
     for (int gp = 0;; ++gp) {
@@ -474,82 +476,134 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
       const bool page_ok = md.z >= 0, streaming = md.w & kSegStreaming;
       const int L = md.w >> 3;
       const uint8_t* stg = smem + st * stage_bytes;
-      const uint8_t* ks_base = Q4 ? stage_k : stg;
-      const uint8_t* vs_base = Q4 ? stage_v : stg + Cfg::kKVBytes;
+      const uint8_t* ks_base = stg;
+      const uint8_t* vs_base = stg + Cfg::kKVBytes;
       if (md.w & kSegStart) {
         const uint8_t* qs = stg + (Q4 ? Cfg::kQ4Q : 2 * Cfg::kKVBytes);   // [G][D] bf16, row-major
+        if constexpr (Q4) {
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {   // lane: head qr, channels 16 ks + tc, +1 and + 8, + 9
-          const int c0 = ks * 16 + tc;
-          qb[ks][0] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c0) * 2) : 0u;
-          qb[ks][1] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c0 + 8) * 2) : 0u;
+          for (int i = 0; i < D / 4; i += 2) {   // entries i, i + 1: channels 16 (i/4) + 8 ((i/2)%2) + tc, + 1
+            const int c = 16 * (i >> 2) + 8 * ((i >> 1) & 1) + tc;
+            const uint32_t w = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c) * 2) : 0u;
+            qf[i] = __uint_as_float(w << 16);
+            qf[i + 1] = __uint_as_float(w & 0xffff0000u);
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {   // lane: head qr, channels 16 ks + tc, +1 and + 8, + 9
+            const int c0 = ks * 16 + tc;
+            qb[ks][0] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c0) * 2) : 0u;
+            qb[ks][1] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c0 + 8) * 2) : 0u;
+          }
         }
 #pragma unroll
         for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
         m_run[0] = m_run[1] = kNegInf;
         l_run[0] = l_run[1] = 0.f;
+        vc_run[0] = vc_run[1] = 0.f;
       }
       const int t_warp = pidx * kPage + warp * 16;   // first token of this warp's slice
+
+      // ---- S^T = K Q^T (16 tokens x 8 heads) into two accumulators (alternate k-steps)
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t vf[Q4 ? 1 : D / 16][4];    // bf16: V^T fragments
+      uint32_t vw[Q4 ? D / 16 : 1];       // INT4: this lane's value code words (one per m-tile)
+      float2 vpt[2];                      // INT4: (s, lo) of tokens t_warp + qr, + 8
+      float kc_lane = 0.f;                // INT4: sum of (lo_c - 128 s_c) q_c over this lane's channels
       if constexpr (Q4) {
-        // ---- this warp's 16 rows of K and V, dequantised into the staging area
-        // (bf16-stage layout, 128-byte swizzle); then the stage goes back at once
-        constexpr int W8 = D / 8;   // 8-channel chunks (one code word) per row
-        const uint32_t* kw = reinterpret_cast<const uint32_t*>(stg);
-        const uint32_t* vw = reinterpret_cast<const uint32_t*>(stg + Cfg::kQ4Bytes);
-        const float* kp4 = reinterpret_cast<const float*>(stg + Cfg::kQ4ParK);   // s[D], lo[D]
-        const float* vp4 = reinterpret_cast<const float*>(stg + Cfg::kQ4ParV);   // s[64], lo[64]
-        __syncwarp();   // the previous page's fragment loads from these rows are done
-#pragma unroll 2
-        for (int idx = lane; idx < 16 * W8; idx += 32) {
-          const int r = warp * 16 + idx / W8, c8 = idx % W8;
-          float s8[8], l8[8];
+        // key rows qr, qr + 8 of the slice: chunk tc/2 (D/32 words each)
+        constexpr int WC = D / 32;
+        uint32_t kw0[WC], kw1[WC];
+        const uint8_t* kr0 = stg + (warp * 16 + qr) * (D / 2) + (lane & 3) * (D / 8);
+        const uint8_t* kr1 = kr0 + 8 * (D / 2);
+        if constexpr (WC % 4 == 0) {   // d = 128: 16-byte chunks
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            s8[e] = kp4[c8 * 8 + e];
-            l8[e] = kp4[D + c8 * 8 + e];
+          for (int x = 0; x < WC; x += 4) {
+            const uint4 a = *reinterpret_cast<const uint4*>(kr0 + 4 * x);
+            const uint4 b = *reinterpret_cast<const uint4*>(kr1 + 4 * x);
+            kw0[x] = a.x, kw0[x + 1] = a.y, kw0[x + 2] = a.z, kw0[x + 3] = a.w;
+            kw1[x] = b.x, kw1[x + 1] = b.y, kw1[x + 2] = b.z, kw1[x + 3] = b.w;
           }
-          const uint32_t off_b = (c8 >> 3) * Cfg::kBoxBytes + swz128(r, c8 & 7);
-          *reinterpret_cast<uint4*>(stage_k + off_b) = dequant8(kw[r * W8 + c8], s8, l8);
-          const float sv = vp4[r], lv = vp4[kPage + r];
+        } else {   // d = 64: 8-byte chunks
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            s8[e] = sv;
-            l8[e] = lv;
+          for (int x = 0; x < WC; x += 2) {
+            const uint2 a = *reinterpret_cast<const uint2*>(kr0 + 4 * x);
+            const uint2 b = *reinterpret_cast<const uint2*>(kr1 + 4 * x);
+            kw0[x] = a.x, kw0[x + 1] = a.y, kw1[x] = b.x, kw1[x + 1] = b.y;
           }
-          *reinterpret_cast<uint4*>(stage_v + off_b) = dequant8(vw[r * W8 + c8], s8, l8);
+        }
+        const uint8_t* vch = stg + Cfg::kQ4Bytes + (warp * 32 + lane) * (D / 4);
+#pragma unroll
+        for (int x = 0; x < D / 16; x += 4) {
+          const uint4 a = *reinterpret_cast<const uint4*>(vch + 4 * x);
+          vw[x] = a.x, vw[x + 1] = a.y, vw[x + 2] = a.z, vw[x + 3] = a.w;
+        }
+        const float2* vp2 = reinterpret_cast<const float2*>(stg + Cfg::kQ4ParV);
+        vpt[0] = vp2[warp * 16 + qr];
+        vpt[1] = vp2[warp * 16 + qr + 8];
+        const float* kps = reinterpret_cast<const float*>(stg + Cfg::kQ4ParK) + (lane & 3) * (D / 4);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          // B = s q at channels 16 ks + tc + {0, 1, 8, 9} (entries 4 ks .. 4 ks + 3), as bf16 hi + lo
+          const float4 s4 = *reinterpret_cast<const float4*>(kps + 4 * ks);
+          const float4 l4 = *reinterpret_cast<const float4*>(kps + D + 4 * ks);
+          const float* q4 = &qf[4 * ks];
+          kc_lane = fmaf(fmaf(-128.f, s4.x, l4.x), q4[0],
+                         fmaf(fmaf(-128.f, s4.y, l4.y), q4[1],
+                              fmaf(fmaf(-128.f, s4.z, l4.z), q4[2], fmaf(fmaf(-128.f, s4.w, l4.w), q4[3], kc_lane))));
+          const float x0 = q4[0] * s4.x, x1 = q4[1] * s4.y, x2 = q4[2] * s4.z, x3 = q4[3] * s4.w;
+          const uint32_t b0 = pack_bf16x2(x0, x1), b1 = pack_bf16x2(x2, x3);
+          const uint32_t c0 = pack_bf16x2(x0 - __uint_as_float(b0 << 16), x1 - __uint_as_float(b0 & 0xffff0000u));
+          const uint32_t c1 = pack_bf16x2(x2 - __uint_as_float(b1 << 16), x3 - __uint_as_float(b1 & 0xffff0000u));
+          // A = 128 + code of rows qr / qr + 8: pairs 2 ks (channels +0, +1) and 2 ks + 1 (+8, +9)
+          const int wi = ks >> 1, k0 = 2 * (ks & 1);
+          const uint32_t a[4] = {q4_pair(kw0[wi], k0), q4_pair(kw1[wi], k0), q4_pair(kw0[wi], k0 + 1),
+                                 q4_pair(kw1[wi], k0 + 1)};
+          if (ks & 1) {
+            mma_bf16_16816(sb, a, b0, b1);
+            mma_bf16_16816(sb, a, c0, c1);
+          } else {
+            mma_bf16_16816(sa, a, b0, b1);
+            mma_bf16_16816(sa, a, c0, c1);
+          }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[st]);   // codes, steps and q rows are no longer needed
-      }
-
-      // ---- this warp's K and V fragments into registers, then the stage goes back
-      // to the producer at once: the ring spends its time loading, not waiting for math
-      uint32_t kf[KS][4], vf[D / 16][4];
+        if (lane == 0) mbar_arrive(&empty_bar[st]);   // every read of this stage is done
+      } else {
+        // ---- this warp's K and V fragments into registers, then the stage goes back
+        // to the producer at once: the ring spends its time loading, not waiting for math
+        uint32_t kf[KS][4];
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {   // K as the A operand of S^T: rows = tokens, k = channels
-        const int box = ks >> 2, chunk = (ks & 3) * 2 + (lane >> 4);
-        const int row = warp * 16 + (mi & 1) * 8 + rr;
-        ldmatrix_x4(smem_u32(ks_base + box * Cfg::kBoxBytes + swz128(row, chunk)), kf[ks][0], kf[ks][1], kf[ks][2],
-                    kf[ks][3]);
-      }
+        for (int ks = 0; ks < KS; ++ks) {   // K as the A operand of S^T: rows = tokens, k = channels
+          const int box = ks >> 2, chunk = (ks & 3) * 2 + (lane >> 4);
+          const int row = warp * 16 + (mi & 1) * 8 + rr;
+          ldmatrix_x4(smem_u32(ks_base + box * Cfg::kBoxBytes + swz128(row, chunk)), kf[ks][0], kf[ks][1],
+                      kf[ks][2], kf[ks][3]);
+        }
 #pragma unroll
-      for (int mt = 0; mt < D / 16; ++mt) {   // V^T as the A operand of O^T: rows = channels, k = tokens
-        const int ch = mt * 16 + (mi & 1) * 8;   // channels of this lane's 8x8 source block
-        const int row = warp * 16 + (mi >> 1) * 8 + rr;
-        ldmatrix_x4_trans(smem_u32(vs_base + (ch >> 6) * Cfg::kBoxBytes + swz128(row, (ch & 63) >> 3)), vf[mt][0],
-                          vf[mt][1], vf[mt][2], vf[mt][3]);
-      }
-      __syncwarp();
-      if (!Q4 && lane == 0) mbar_arrive(&empty_bar[st]);   // release orders the shared-memory reads above
-
-      // ---- S^T = K Q^T: 16 tokens x 8 heads; alternate k-steps feed two accumulators
-      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int mt = 0; mt < D / 16; ++mt) {   // V^T as the A operand of O^T: rows = channels, k = tokens
+          const int ch = mt * 16 + (mi & 1) * 8;   // channels of this lane's 8x8 source block
+          const int row = warp * 16 + (mi >> 1) * 8 + rr;
+          ldmatrix_x4_trans(smem_u32(vs_base + (ch >> 6) * Cfg::kBoxBytes + swz128(row, (ch & 63) >> 3)),
+                            vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[st]);   // release orders the shared-memory reads above
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        if (ks & 1)
-          mma_bf16_16816(sb, kf[ks], qb[ks][0], qb[ks][1]);
-        else
-          mma_bf16_16816(sa, kf[ks], qb[ks][0], qb[ks][1]);
+        for (int ks = 0; ks < KS; ++ks) {
+          if (ks & 1)
+            mma_bf16_16816(sb, kf[ks], qb[ks][0], qb[ks][1]);
+          else
+            mma_bf16_16816(sa, kf[ks], qb[ks][0], qb[ks][1]);
+        }
+      }
+      // INT4: the offsets' term of heads tc, tc + 1 (sum over the four lanes of head qr first)
+      float kc[2] = {0.f, 0.f};
+      if constexpr (Q4) {
+        kc_lane += __shfl_xor_sync(0xffffffffu, kc_lane, 1);
+        kc_lane += __shfl_xor_sync(0xffffffffu, kc_lane, 2);
+        kc[0] = __shfl_sync(0xffffffffu, kc_lane, 4 * tc);
+        kc[1] = __shfl_sync(0xffffffffu, kc_lane, 4 * (tc + 1));
       }
       // ---- mask + online softmax.  Element e: token t_warp + qr + 8 (e >> 1), head tc + (e & 1)
       auto valid = [&](int t) -> bool {
@@ -558,7 +612,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
       const bool ok0 = valid(t_warp + qr), ok1 = valid(t_warp + qr + 8);
       float p[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) p[e] = ((e >> 1) ? ok1 : ok0) ? (sa[e] + sb[e]) * scale_log2 : kNegInf;
+      for (int e = 0; e < 4; ++e) p[e] = ((e >> 1) ? ok1 : ok0) ? (sa[e] + sb[e] + kc[e & 1]) * scale_log2 : kNegInf;
       // per-head max over the 16 tokens: the lanes with one lane % 4 hold one head pair
       float mh[2] = {fmaxf(p[0], p[2]), fmaxf(p[1], p[3])};
 #pragma unroll
@@ -587,6 +641,30 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
           acc[mt][3] *= corr[1];
         }
       }
+      if constexpr (Q4) {
+        // ---- P^T scaled by the value steps of its tokens, as bf16 hi + lo (masked
+        // tokens: 0, whatever the parameters of an unused row hold), and the
+        // offsets' term
+        float ps[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ps[e] = ((e >> 1) ? ok1 : ok0) ? p[e] * vpt[e >> 1].x : 0.f;
+        const uint32_t u0 = pack_bf16x2(ps[0], ps[1]), u1 = pack_bf16x2(ps[2], ps[3]);
+        const uint32_t w0 = pack_bf16x2(ps[0] - __uint_as_float(u0 << 16), ps[1] - __uint_as_float(u0 & 0xffff0000u));
+        const uint32_t w1 = pack_bf16x2(ps[2] - __uint_as_float(u1 << 16), ps[3] - __uint_as_float(u1 & 0xffff0000u));
+        const float o0 = ok0 ? fmaf(-128.f, vpt[0].x, vpt[0].y) : 0.f;   // lo - 128 s of token qr
+        const float o1 = ok1 ? fmaf(-128.f, vpt[1].x, vpt[1].y) : 0.f;   // ... of token qr + 8
+        vc_run[0] = vc_run[0] * corr[0] + fmaf(o0, p[0], o1 * p[2]);
+        vc_run[1] = vc_run[1] * corr[1] + fmaf(o0, p[1], o1 * p[3]);
+        const uint32_t pb0 = movmatrix_trans(u0), pb1 = movmatrix_trans(u1);   // tokens 0..7, 8..15
+        const uint32_t pl0 = movmatrix_trans(w0), pl1 = movmatrix_trans(w1);
+        // ---- O^T += (128 + code)^T (s P)^T: a_j of m-tile mt = nibbles j, j + 4 of word mt
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          const uint32_t a[4] = {q4_pair(vw[mt], 0), q4_pair(vw[mt], 1), q4_pair(vw[mt], 2), q4_pair(vw[mt], 3)};
+          mma_bf16_16816(acc[mt], a, pb0, pb1);
+          mma_bf16_16816(acc[mt], a, pl0, pl1);
+        }
+      } else {
       // ---- P^T as the B operand (k = tokens, n = heads): transpose the two 8x8 blocks
       const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p[0], p[1]));   // tokens 0..7
       const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p[2], p[3]));   // tokens 8..15
@@ -606,6 +684,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
         vf[mt][3] &= vm1;
         mma_bf16_16816(acc[mt], vf[mt], pb0, pb1);
       }
+      }
 
       // ---- end of a segment: this warp's partial, and the merge if it completes the unit
       if (md.w & kSegEnd) {
@@ -614,10 +693,15 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
         // (slot vr + u of every range of the unit is read by decode_merge_kernel)
         // l of heads tc, tc + 1: sum over the 8 lanes that share lane % 4
         float lh[2] = {l_run[0], l_run[1]};
+        float vh[2] = {vc_run[0], vc_run[1]};
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
           lh[0] += __shfl_xor_sync(0xffffffffu, lh[0], o);
           lh[1] += __shfl_xor_sync(0xffffffffu, lh[1], o);
+          if constexpr (Q4) {
+            vh[0] += __shfl_xor_sync(0xffffffffu, vh[0], o);
+            vh[1] += __shfl_xor_sync(0xffffffffu, vh[1], o);
+          }
         }
         const long pbase = (static_cast<long>(vr + u) * kDecodeWarps + warp) * G;   // this warp's partial
 #pragma unroll
@@ -627,10 +711,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
             const bool has = m_run[h2] != kNegInf && lh[h2] > 0.f;
             const float inv = has ? 1.f / lh[h2] : 0.f;
             float* po = part_o + (pbase + h) * D + qr;
+            const float add = Q4 ? vh[h2] : 0.f;   // INT4: the offsets' term
 #pragma unroll
             for (int mt = 0; mt < D / 16; ++mt) {
-              po[mt * 16] = acc[mt][h2] * inv;
-              po[mt * 16 + 8] = acc[mt][2 + h2] * inv;
+              po[mt * 16] = (acc[mt][h2] + add) * inv;
+              po[mt * 16 + 8] = (acc[mt][2 + h2] + add) * inv;
             }
             if (qr == 0) part_lse[pbase + h] = has ? m_run[h2] + __log2f(lh[h2]) : kNegInf;
           }
