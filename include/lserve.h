@@ -207,10 +207,10 @@ int32_t lserve_decode_max_selected(const lserve_decode_args* args);
 
 /* Bytes of workspace lserve_decode needs (page scores, selection, partition,
  * per-warp partials); lserve_decode_reuse needs the same, and may ask with
- * stats = NULL.  It depends on the current device's SM count (the
- * attention grid is one wave of SMs x 2 CTAs) or, when the environment
- * variable LSERVE_DECODE_GRID holds a positive integer, on that grid size;
- * ask again after changing either. */
+ * stats = NULL, and so does lserve_decode_int4.  It depends on the current
+ * device's SM count (the attention grid is one wave of SMs x 2 CTAs, x 3 for
+ * INT4 pages) or, when the environment variable LSERVE_DECODE_GRID holds a
+ * positive integer, on that grid size; ask again after changing either. */
 size_t lserve_decode_workspace_size(const lserve_decode_args* args);
 
 /*

@@ -52,12 +52,14 @@
 
 namespace lserve {
 
-constexpr int kDecodeStages = 3;
+constexpr int kDecodeStages = 3;     // bf16 pages: ring depth (three 34 KB stages at d = 128)
+constexpr int kDecodeStagesQ4 = 5;   // INT4 pages: its consumers hold a stage through the key loop
 constexpr int kDecodeWarps = 4;                           // consumer warps
 constexpr int kIssuerWarp = kDecodeWarps;                  // issues the TMA loads
 constexpr int kResolverWarp = kDecodeWarps + 1;            // claims ranges, resolves their pages
 constexpr int kDecodeThreads = (kDecodeWarps + 2) * 32;
-constexpr int kDecodeCtasPerSm = 2;
+constexpr int kDecodeCtasPerSm = 2;     // bf16 pages: the three-stage ring's shared memory admits two
+constexpr int kDecodeCtasPerSmQ4 = 3;   // INT4 pages: smaller stages; registers capped to admit three
 constexpr int kDecodeMaxG = 8;
 constexpr int kRangesPerCta = 4;   // ranges of the flat page list per attention CTA
 constexpr int kMetaRing = 64;      // resolved pages buffered ahead of the loads
@@ -84,7 +86,7 @@ struct DecodeCfg {
   static constexpr int kParVBytes = 2 * 64 * 4;   // fp32 step and offset per token
   static constexpr int kQ4ParK = 2 * kQ4Bytes, kQ4ParV = kQ4ParK + kParKBytes, kQ4Q = kQ4ParV + kParVBytes;
   __host__ __device__ static int stage_bytes_q4(int G) { return ((kQ4Q + G * D * 2 + 1023) / 1024) * 1024; }
-  __host__ __device__ static int smem_bytes_q4(int G) { return kDecodeStages * stage_bytes_q4(G) + 1024; }
+  __host__ __device__ static int smem_bytes_q4(int G) { return kDecodeStagesQ4 * stage_bytes_q4(G) + 1024; }
 };
 
 // Ranges the T selected pages are cut into: at most R (the workspace's
@@ -243,7 +245,7 @@ __device__ __forceinline__ uint32_t q4_pair(uint32_t w, int k) { return ((w >> (
 // One bf16 rounding of s q or s p would scale with |x - lo| (or the step of an
 // outlier-wide group), not with |x|; the split keeps it near 2^-18.
 template <int D, bool Q4 = false>
-__global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode_kernel(
+__global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) paged_decode_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const bf16* __restrict__ q, const int32_t* __restrict__ page_table, int maxP,
     const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind,
@@ -252,9 +254,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
     unsigned long long timeout_ns, int debug_stall, float* __restrict__ part_o, float* __restrict__ part_lse,
     const float* __restrict__ kpar = nullptr, const float* __restrict__ vpar = nullptr) {
   using Cfg = DecodeCfg<D>;
+  constexpr int NS = Q4 ? kDecodeStagesQ4 : kDecodeStages;   // ring depth
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kDecodeStages];    // stage loaded (issuer's expect_tx + bytes)
-  __shared__ __align__(8) uint64_t empty_bar[kDecodeStages];   // stage consumed (one arrive per consumer warp)
+  __shared__ __align__(8) uint64_t full_bar[NS];    // stage loaded (issuer's expect_tx + bytes)
+  __shared__ __align__(8) uint64_t empty_bar[NS];   // stage consumed (one arrive per consumer warp)
   __shared__ int4 s_meta[kMetaRing];   // {unit, logical page, physical page (-1: invalid), seq_len << 3 | flags}
   __shared__ int4 s_seg[kMetaRing];    // {range, first range of the unit, last range of the unit, -}
   __shared__ int s_resolved;           // pages whose metadata is in the ring
@@ -268,7 +271,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
   if (tid == 0) {
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
-    for (int s = 0; s < kDecodeStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], kDecodeWarps);
     }
@@ -350,7 +353,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
         // ring entries gp .. gp + cnt - 1 are free once page (entry - ring) is past the consumers
         bool room = true;
         if (lane == 0)
-          room = spin_until([&] { return *v_issued >= gp + cnt - kMetaRing + kDecodeStages || *v_abort; },
+          room = spin_until([&] { return *v_issued >= gp + cnt - kMetaRing + NS || *v_abort; },
                             timeout_ns) && !*v_abort;
         if (!__shfl_sync(0xffffffffu, room, 0)) {
           stopped = true;
@@ -410,8 +413,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
         }
         if (*v_resolved <= gp || *v_abort) break;   // no page gp: the ranges ran out
         __threadfence_block();
-        const int st = gp % kDecodeStages;
-        if (gp >= kDecodeStages && !mbar_wait_bounded(&empty_bar[st], ((gp / kDecodeStages) - 1) & 1, timeout_ns)) {
+        const int st = gp % NS;
+        if (gp >= NS && !mbar_wait_bounded(&empty_bar[st], ((gp / NS) - 1) & 1, timeout_ns)) {
           *v_abort = 1;
           break;
         }
@@ -450,7 +453,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
     // heads tc, tc + 1 of the tile.
     constexpr int KS = D / 16;
     uint32_t qb[Q4 ? 1 : KS][2];          // Q^T as the B operand (heads >= G are zero)
-    float qf[Q4 ? D / 4 : 1];             // INT4: q of head qr at this lane's channels, key-chunk order
+    uint32_t qp[Q4 ? D / 8 : 1];          // INT4: q of head qr at this lane's channels (bf16 pairs), key-chunk order
     float acc[D / 16][4];                 // O^T: m-tile mt = channels 16 mt .. 16 mt + 15
     float m_run[2], l_run[2];             // online softmax of heads tc, tc + 1
     float vc_run[2];                      // INT4: sum_t (lo_t - 128 s_t) p_t, heads tc, tc + 1
@@ -464,8 +467,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
         have = known && *v_resolved > gp && !*v_abort;
       }
       if (!__shfl_sync(0xffffffffu, have, 0)) break;
-      const int st = gp % kDecodeStages;
-      const bool landed = mbar_wait_bounded(&full_bar[st], (gp / kDecodeStages) & 1, timeout_ns);
+      const int st = gp % NS;
+      const bool landed = mbar_wait_bounded(&full_bar[st], (gp / NS) & 1, timeout_ns);
       if (__any_sync(0xffffffffu, !landed || *v_abort != 0)) {
         if (lane == 0) *v_abort = 1;
         break;
@@ -484,9 +487,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
 #pragma unroll
           for (int i = 0; i < D / 4; i += 2) {   // entries i, i + 1: channels 16 (i/4) + 8 ((i/2)%2) + tc, + 1
             const int c = 16 * (i >> 2) + 8 * ((i >> 1) & 1) + tc;
-            const uint32_t w = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c) * 2) : 0u;
-            qf[i] = __uint_as_float(w << 16);
-            qf[i + 1] = __uint_as_float(w & 0xffff0000u);
+            qp[i / 2] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c) * 2) : 0u;
           }
         } else {
 #pragma unroll
@@ -532,6 +533,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
             kw0[x] = a.x, kw0[x + 1] = a.y, kw1[x] = b.x, kw1[x + 1] = b.y;
           }
         }
+        // this lane's value code words and the steps / offsets of its two tokens
         const uint8_t* vch = stg + Cfg::kQ4Bytes + (warp * 32 + lane) * (D / 4);
 #pragma unroll
         for (int x = 0; x < D / 16; x += 4) {
@@ -547,7 +549,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
           // B = s q at channels 16 ks + tc + {0, 1, 8, 9} (entries 4 ks .. 4 ks + 3), as bf16 hi + lo
           const float4 s4 = *reinterpret_cast<const float4*>(kps + 4 * ks);
           const float4 l4 = *reinterpret_cast<const float4*>(kps + D + 4 * ks);
-          const float* q4 = &qf[4 * ks];
+          const float q4[4] = {__uint_as_float(qp[2 * ks] << 16), __uint_as_float(qp[2 * ks] & 0xffff0000u),
+                               __uint_as_float(qp[2 * ks + 1] << 16), __uint_as_float(qp[2 * ks + 1] & 0xffff0000u)};
           kc_lane = fmaf(fmaf(-128.f, s4.x, l4.x), q4[0],
                          fmaf(fmaf(-128.f, s4.y, l4.y), q4[1],
                               fmaf(fmaf(-128.f, s4.z, l4.z), q4[2], fmaf(fmaf(-128.f, s4.w, l4.w), q4[3], kc_lane))));
@@ -727,10 +730,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm) paged_decode
   __syncthreads();
   if (*v_abort && warp == kIssuerWarp && lane == 0) {
     // let every load this CTA issued land before the CTA (and its smem) goes away;
-    // the last kDecodeStages issued pages sit in distinct stages, earlier ones have landed
+    // the last NS issued pages sit in distinct stages, earlier ones have landed
     const int issued = *v_issued;
-    for (int gp = max(0, issued - kDecodeStages); gp < issued; ++gp)
-      mbar_wait_bounded(&full_bar[gp % kDecodeStages], (gp / kDecodeStages) & 1, kDrainTimeoutNs);
+    for (int gp = max(0, issued - NS); gp < issued; ++gp)
+      mbar_wait_bounded(&full_bar[gp % NS], (gp / NS) & 1, kDrainTimeoutNs);
   }
 }
 

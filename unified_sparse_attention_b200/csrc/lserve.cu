@@ -352,12 +352,13 @@ struct DecodePlan {
 
 // Attention CTAs for the current device: SMs x resident CTAs per SM, or the
 // value of LSERVE_DECODE_GRID (a positive integer) when that is set.
-int decode_grid() {
+// CTAs of the attention grid: one wave (SMs x resident CTAs of the variant)
+int decode_grid(bool q4) {
   if (const char* e = getenv("LSERVE_DECODE_GRID")) {
     const long v = strtol(e, nullptr, 10);
     if (v > 0 && v <= (1 << 20)) return static_cast<int>(v);
   }
-  return sm_count() * kDecodeCtasPerSm;
+  return sm_count() * (q4 ? kDecodeCtasPerSmQ4 : kDecodeCtasPerSm);
 }
 
 // Launch with programmatic stream serialisation: the kernel may start while its
@@ -410,13 +411,13 @@ lserve_status validate_decode(const lserve_decode_args* a, bool need_stats = tru
   return LSERVE_OK;
 }
 
-DecodePlan plan_decode(const lserve_decode_args* a, void* ws) {
+DecodePlan plan_decode(const lserve_decode_args* a, void* ws, bool q4 = false) {
   DecodePlan p{};
   p.G = a->Hq / a->Hkv;
   p.budget_pages = a->token_budget / kPage;
   const int dense_cap = std::min(p.budget_pages, a->maxP);
   p.kcap = std::max(1, std::max(dense_cap, std::min(streaming_page_bound(a->sink, a->local), a->maxP)));
-  p.P = decode_grid();
+  p.P = decode_grid(q4);
   p.R = kRangesPerCta * p.P;
 
   Carver c(ws);
@@ -653,9 +654,10 @@ int32_t lserve_decode_max_selected(const lserve_decode_args* args) {
 }
 
 size_t lserve_decode_workspace_size(const lserve_decode_args* args) {
-  // the size depends on the shapes only: a call with stats = NULL (lserve_decode_reuse) asks too
+  // the size depends on the shapes only: a call with stats = NULL (lserve_decode_reuse) asks too;
+  // it covers the INT4 step's plan as well (a wider attention grid, more ranges)
   if (validate_decode(args, /*need_stats=*/false) != LSERVE_OK) return 0;
-  return plan_decode(args, nullptr).bytes;
+  return std::max(plan_decode(args, nullptr).bytes, plan_decode(args, nullptr, /*q4=*/true).bytes);
 }
 
 lserve_status lserve_decode(const lserve_decode_args* args, void* out, float* lse, int32_t* sel_out,
@@ -735,10 +737,10 @@ lserve_status lserve_decode_int4(const lserve_decode_args* args, const float* kp
   if (!kpar || !vpar || !aligned16(kpar) || !aligned16(vpar))
     return fail(LSERVE_ERR_INVALID_ARG, "decode int4: kpar and vpar must be non-null and 16-byte aligned");
   if (!out || !aligned16(out)) return fail(LSERVE_ERR_INVALID_ARG, "decode: out must be non-null and 16-byte aligned");
-  const size_t need = plan_decode(args, nullptr).bytes;
+  const size_t need = plan_decode(args, nullptr, /*q4=*/true).bytes;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < need)
     return fail(LSERVE_ERR_WORKSPACE, "decode: workspace missing, misaligned or smaller than %zu bytes", need);
-  DecodePlan p = plan_decode(args, workspace);
+  DecodePlan p = plan_decode(args, workspace, /*q4=*/true);
   int32_t* sel = sel_out ? sel_out : p.sel;
   int32_t* seln = sel_n ? sel_n : p.sel_n;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
