@@ -232,3 +232,26 @@ def test_reuse_reports_a_page_index_outside_the_table():
     torch.cuda.synchronize()
     assert U.lserve_get_device_status() == 6   # LSERVE_ERR_DEVICE_BOUNDS
     assert U.lserve_get_device_status() == 0
+
+
+@pytest.mark.parametrize("G,d", [(1, 128), (4, 128), (2, 64)])
+def test_cross_mode_decode_equals_last_prefill_row(G, d):
+    """The two CUDA paths agree: decoding the last prefill query against the
+    prefill's own K/V (paged, pool rows outside the sequence NaN) with a budget
+    covering the context (dense heads) or the same sink / local (streaming
+    heads) gives the prefill's last output row."""
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2 * G, Hkv=2, d=d)
+    S, sink, local = 640, 64, 150
+    q, k, v = W.prefill_inputs(w, S=S)
+    dev = "cuda"
+    hk = torch.tensor([0, 1], dtype=torch.uint8, device=dev)
+    pre = U.lserve_prefill(q.to(dev), k.to(dev), v.to(dev), hk, sink, local)
+    pt = W.page_table(w, 1, S // 64, 16)
+    pc = W.scatter_to_pages(k, v, pt, 16)
+    kp, vp = pc.k_pages.to(dev), pc.v_pages.to(dev)
+    ptd, sl = pc.page_table.to(dev), pc.seq_lens.to(dev)
+    stats = U.lserve_update_page_stats(kp, ptd, sl, hk)
+    out = U.lserve_decode(q[:, S - 1].contiguous().to(dev), kp, vp, ptd, sl, stats, hk, sink, local, S)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+    assert_attn_close(f64(out[0]), f64(pre[0, S - 1]), "decode vs last prefill row")
