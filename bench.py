@@ -389,6 +389,10 @@ def main():
     # the same decode step over codes dequantised on chip
     kq, kpar, vq, vpar, stats4 = U.lserve_quantize_pages_int4(setup.kp, setup.vp, setup.pt, setup.sl, setup.hk_d)
 
+    def quantize_pool():
+        U.lserve_quantize_pages_int4(setup.kp, setup.vp, setup.pt, setup.sl, setup.hk_d, kq=kq, kpar=kpar, vq=vq,
+                                     vpar=vpar, stats=stats4)
+
     def decode_int4():
         U.lserve_decode_int4(setup.qd, kq, vq, kpar, vpar, setup.pt, setup.sl, stats4, setup.hk_d, wd.sink,
                              wd.local, wd.token_budget, out=out_d, workspace=ws_d)
@@ -411,6 +415,7 @@ def main():
     t_decode_flushed = time_loop(decode_only, args.steps, 2, stream, scratch)
     t_reuse = time_loop(decode_reuse, args.steps, args.warmup, stream, fl)
     t_int4 = time_loop(decode_int4, args.steps, args.warmup, stream, fl)
+    t_quant = time_loop(quantize_pool, 2, 1, stream)   # once per page in a server: off the step
     ms_legacy = None
     if not args.no_legacy:   # the mma.sync kernel on the same call, for comparison only
         os.environ["LSERVE_PREFILL_IMPL"] = "mma"
@@ -443,6 +448,12 @@ def main():
     ms_step, ms_prefill, us_decode, us_reuse, us_int4 = max_over_ranks(
         [ms_step, ms_prefill, us_decode, us_reuse, us_int4], dist, dev)
     int4_bytes = decode_bytes_int4(wd, setup.kind_d.tolist(), setup.k_sel, wd.d)
+    # quantiser: K and V of every held (page, head) read once; codes, steps/offsets and
+    # (dense heads) summaries written
+    held = sum((int(L) + 63) // 64 for L in setup.sl.tolist())   # pages the sequences hold
+    n_dense_d = sum(1 for x in setup.kind_d.tolist() if x == 0)
+    quant_bytes = held * (wd.Hkv * (2 * 64 * wd.d * 2 + 64 * wd.d + 2 * wd.d * 4 + 2 * 64 * 4)
+                          + n_dense_d * 4 * 2 * wd.d * 2)
     reuse_bytes = setup.dbytes["total"] - setup.dbytes["stats"]
 
     tflops_prefill = setup.prefill_flops / (ms_prefill * 1e-3) / 1e12
@@ -521,6 +532,9 @@ def main():
                         "GBps": int4_bytes["total"] / (us_int4 * 1e-6) / 1e9,
                         "frac_hbm": int4_bytes["total"] / (us_int4 * 1e-6) / 1e9 / pk["hbm"],
                         "speedup_vs_bf16": us_decode / us_int4,
+                        "quantize_pool_ms": float(np.median(t_quant)),
+                        "quantize_pool_bytes": quant_bytes,
+                        "quantize_GBps": quant_bytes / (float(np.median(t_quant)) * 1e-3) / 1e9,
                         "note": "decode step over INT4 pages (codes + fp32 steps/offsets, dequantised on chip); "
                                 "pool quantised once before timing"},
         "roofline": {"bound": "tensor", "kernel": "prefill attention", "achieved": tflops_attn,

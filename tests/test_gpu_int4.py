@@ -190,3 +190,41 @@ def test_int4_unattended_parameters_are_never_used():
                                 64, 100, 256)
     torch.cuda.synchronize()
     assert torch.equal(out2, r["out"])
+
+
+def test_quantiser_ties_and_near_ties():
+    """Groups built so that (x - lo) / s falls exactly on, or within float32
+    rounding of, a half-integer: the codes (round half to even on the IEEE
+    quotient) match the oracle bit for bit."""
+    d, S = 64, 128
+    k = torch.zeros(1, S, 2, d)
+    v = torch.zeros(1, S, 2, d)
+    t = torch.arange(64, dtype=torch.float32)
+    c = torch.arange(d, dtype=torch.float32)
+    # page 0: lo = 0, hi = 15, s = 1; values 0, 0.5, ..., 14.5 (exact ties at the odd halves)
+    k[0, :64, :, :] = ((t[:, None] + c[None, :]) % 30 * 0.5)[:, None, :]
+    k[0, 0, :, :], k[0, 1, :, :] = 0.0, 15.0
+    v[0, :64, :, :] = ((t[:, None] + c[None, :]) % 30 * 0.5)[:, None, :]
+    v[0, :64, :, 0], v[0, :64, :, 1] = 0.0, 15.0
+    # page 1: lo = -1.5, hi = 0, s = fl(0.1); values -1.5 + 0.05 j, rounded to bf16 (near ties)
+    k[0, 64:, :, :] = (-1.5 + 0.05 * ((t[:, None] * 7 + c[None, :]) % 31))[:, None, :]
+    k[0, 64, :, :], k[0, 65, :, :] = -1.5, 0.0
+    v[0, 64:, :, :] = (-1.5 + 0.05 * ((t[:, None] * 3 + c[None, :]) % 31))[:, None, :]
+    v[0, 64:, :, 0], v[0, 64:, :, 1] = -1.5, 0.0
+    k, v = k.to(torch.bfloat16), v.to(torch.bfloat16)
+    pt = torch.tensor([[1, 0]], dtype=torch.int32)
+    pc = W.scatter_to_pages(k, v, pt, 2)
+    kind = [0, 0]
+    g = quantize(pc, kind)
+    kq, kpar, vq, vpar, kdeq, _ = OQ.quantize_pages(f64(pc.k_pages), f64(pc.v_pages), pc.page_table.numpy(),
+                                                    pc.seq_lens.numpy())
+    np.testing.assert_array_equal(g["kq"].cpu().numpy(), kq)
+    np.testing.assert_array_equal(g["vq"].cpu().numpy(), vq.reshape(g["vq"].shape))
+    np.testing.assert_array_equal(g["kpar"].cpu().numpy(), kpar)
+    np.testing.assert_array_equal(g["vpar"].cpu().numpy(), vpar)
+    st = OQ.quantized_stats(kdeq, pc.page_table.numpy(), pc.seq_lens.numpy(), kind)
+    np.testing.assert_array_equal(f64(g["stats"]), st)
+    # the constructed groups do reach exact ties: some code is an even neighbour of x / s
+    codes = OQ.unpack_nibbles(kq[1, 0, 5], OQ.k_code_position(d))
+    x = f64(pc.k_pages)[1, 0, 5]
+    assert np.any((x % 1 == 0.5) & (codes % 2 == 0))
