@@ -92,3 +92,35 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 64, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         U.lserve_prefill(q, q[:, :, :1], q[:, :, :1], torch.zeros(1, dtype=torch.uint8), 0, 64)
+
+
+def test_int4_reuse_and_cra_validation():
+    """The next rows' entry points refuse bad arguments on the host, before any
+    launch: INT4 quantiser and decode, selection reuse, CRA."""
+    lib = U.load_library()
+    bad16 = ctypes.c_void_p((1 << 20) + 8)   # not 16-byte aligned
+    q = lib.lserve_quantize_pages_int4
+    #           B  Hkv  d  NP  k     v     table maxP lens first kind  kq    kpar  vq    vpar  stats stream
+    assert q(1, 2, 96, 4, FAKE, FAKE, FAKE, 4, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert q(1, 2, 64, 4, FAKE, FAKE, FAKE, 4, FAKE, -1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert q(1, 2, 64, 4, FAKE, FAKE, FAKE, 4, FAKE, 0, FAKE, None, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert q(1, 2, 64, 4, FAKE, FAKE, FAKE, 4, FAKE, 0, FAKE, bad16, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert q(0, 2, 64, 4, FAKE, FAKE, FAKE, 4, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+
+    d4 = lib.lserve_decode_int4
+    a = decode_args()
+    assert d4(ctypes.byref(a), None, FAKE, FAKE, None, None, None, FAKE, 1 << 30, None) == 1      # no kpar
+    assert d4(ctypes.byref(a), FAKE, bad16, FAKE, None, None, None, FAKE, 1 << 30, None) == 1     # misaligned vpar
+    assert d4(ctypes.byref(decode_args(d=96)), FAKE, FAKE, FAKE, None, None, None, FAKE, 1 << 30, None) == 2
+    assert d4(ctypes.byref(a), FAKE, FAKE, FAKE, None, None, None, None, 0, None) == 3           # no workspace
+    # one size query covers the bf16 and the INT4 plans
+    assert lib.lserve_decode_workspace_size(ctypes.byref(a)) > 0
+
+    r = lib.lserve_decode_reuse
+    a = decode_args(stats=0)   # reuse reads no summaries
+    assert r(ctypes.byref(a), None, FAKE, FAKE, None, None, None, FAKE, 1 << 30, None) == 1      # no sel_in
+    assert r(ctypes.byref(a), FAKE, FAKE, FAKE, None, None, None, None, 0, None) == 3            # no workspace
+
+    assert lib.lserve_cra_workspace_size(shape(S=1000)) == 0   # S not a multiple of 64
+    assert lib.lserve_cra_workspace_size(shape()) > 0
+    assert lib.lserve_cra(shape(d=96), FAKE, FAKE, FAKE, FAKE, 0, 64, None, None, FAKE, FAKE, 1 << 30, None) == 2
