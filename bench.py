@@ -52,7 +52,7 @@ TRAFFIC = {
                 "sha256": "54cd666b417c2fa7c423f9f076e7c3e5286e45e17d36d2ca046b15f1acc972e1"},
     "decode": {"bytes": 822210048,
                "sources": ["select.cuh", "decode.cuh", "page_stats.cuh", "common.cuh", "lserve.cu"],
-               "sha256": "7983cebf585940f6c6af6afe70f9028b46ad52ab14d2d49578ef196cae8d925d"},
+               "sha256": "14e72dc1520509444a40d2d2070759adca85691852e018fc85f9bbf84014044d"},
 }
 
 

@@ -13,7 +13,7 @@
 // n_u follows from the sequence lengths alone, so one extra block of the top-k
 // grid builds this plan (decode_partition) while the other blocks select.
 //
-// paged_decode_kernel: one wave of CTAs (SMs x 2) that claim ranges from a
+// paged_decode_kernel: one wave of CTAs (SMs x 2; x 3 for INT4 pages) that claim ranges from a
 // counter, so that SMs that run ahead take more.  Per CTA:
 //   * a resolver warp claims ranges and resolves their pages (unit, logical
 //     page, physical page, segment flags) into a shared-memory ring ahead of
@@ -37,6 +37,17 @@
 // list both r and u never decrease and one of them grows at every segment
 // boundary, so slots are distinct, and unit u's slots are the contiguous run
 // r_first(u) + u .. r_last(u) + u.  Slots <= Re + units - 1.
+//
+// INT4 pages (paged_decode_kernel<D, true>, lserve_decode_int4; blog post,
+// "LServe - Decode Phase" and Fig. 2: INT4 KV cuts the bytes of every page).
+// A stage holds the page's K and V codes (d/2 bytes a row, in the order of the
+// operand fragments, so a lane loads its share with one or two 16-byte reads),
+// the key steps/offsets per channel and value steps/offsets per token (fp32),
+// and the q rows at a segment start.  The integer codes go straight into the
+// MMAs; the steps are folded into the other operand (s q, s p, each as two bf16
+// parts) and the offsets into one fp32 term per head.  With 12 KB stages the
+// ring is 5 deep, and q kept as bf16 pairs under a 112-register cap admits 3
+// CTAs per SM (grid SMs x 3).  Bytes per selected page: 64 * d + 1.5 KB (d = 128).
 //
 // Bytes per selected page: 2 * 64 * d * 2 (K and V); the kernel is HBM-bound.
 // Tokens outside the attended set (past seq_len; outside the Lambda set of a
