@@ -120,6 +120,8 @@ def test_cra_is_one_without_dropping_and_matches_weight_sums():
     keep = A.kept_mask(np.arange(S), S, True, 5, 30, None)
     np.testing.assert_allclose(r[0, 1], (full * keep).sum(axis=1), atol=1e-12)
     np.testing.assert_allclose(r[0, 0], 1.0, atol=1e-12)
+    # CRA is the worst-kept row: the minimum of those brute-force sums
+    np.testing.assert_allclose(C.cra(q, k, v, kind, 5, 30)[0, 1], (full * keep).sum(axis=1).min(), atol=1e-12)
 
 
 def test_reuse_at_the_same_lengths_is_the_selection_step():

@@ -11,9 +11,12 @@ import pytest
 
 import test_oracle_attention as TA
 import test_oracle_decode as TD
+import test_oracle_quant as TQ
 import test_oracle_selection as TS
 from oracle import attention as A
+from oracle import cra as CR
 from oracle import decode as D
+from oracle import quant as Q
 from oracle import selection as Sel
 
 _kept = A.kept_mask
@@ -87,6 +90,34 @@ _stats = Sel.page_stats
 _token_set = D.token_set
 
 
+def cra_mean_not_min(q, k, v, head_kind, sink, local, block_mask=None, scale=None, rows=None):
+    return CR.retained_mass(q, k, v, head_kind, sink, local, block_mask, scale, rows).mean(axis=2)
+
+
+def retained_inverted(q, k, v, head_kind, sink, local, block_mask=None, scale=None, rows=None):
+    return 1.0 / _retained(q, k, v, head_kind, sink, local, block_mask, scale, rows)
+
+
+_retained = CR.retained_mass
+
+
+def codes_truncate(x, lo, s):
+    with np.errstate(divide="ignore", invalid="ignore"):
+        c = np.floor(((x - lo).astype(np.float32) / s).astype(np.float32))
+    c = np.where(s > 0, c, 0.0)
+    return np.clip(c, 0, 15).astype(np.uint8)
+
+
+def step_sixteen_levels(lo, hi):
+    return ((hi - lo) / np.float32(16.0)).astype(np.float32)
+
+
+def dequant_drops_offset(code, s, lo):
+    return (code.astype(np.float64) * s.astype(np.float64)).astype(np.float32)
+
+
+
+
 CASES = [
     ("window off by one", A, "kept_mask", kept_window_off_by_one,
      lambda: TA.test_streaming_equals_sdpa_with_lambda_mask(0, 64)),
@@ -106,6 +137,16 @@ CASES = [
      lambda: TD.test_full_budget_equals_dense_decode(None)),
     ("stats ignore sequence length", Sel, "page_stats", page_stats_ignores_length,
      TS.test_stats_closed_form_on_contiguous_keys),
+    ("CRA takes the mean", CR, "cra", cra_mean_not_min, TD.test_cra_is_one_without_dropping_and_matches_weight_sums),
+    ("retained mass inverted", CR, "retained_mass", retained_inverted,
+     TD.test_cra_is_one_without_dropping_and_matches_weight_sums),
+    ("INT4 codes truncated", Q, "_codes", codes_truncate, TQ.test_codes_range_extremes_monotone_and_error_bound),
+    ("INT4 step over 16 levels", Q, "_step", step_sixteen_levels,
+     TQ.test_codes_range_extremes_monotone_and_error_bound),
+    ("INT4 dequantisation drops the offset", Q, "dequant", dequant_drops_offset,
+     TQ.test_constant_group_dequantises_exactly),
+    ("INT4 summaries rounded to nearest", Q, "bf16_round_down", Q.bf16_round,
+     TQ.test_summaries_of_dequantised_keys_bound_them),
 ]
 
 
