@@ -321,7 +321,6 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--prefill-wl", default=PREFILL_WL, choices=sorted(W.WORKLOADS))
     ap.add_argument("--decode-wl", default=DECODE_WL, choices=sorted(W.WORKLOADS))
-    ap.add_argument("--no-legacy", action="store_true", help="skip timing the mma.sync prefill kernel")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -416,11 +415,6 @@ def main():
     t_reuse = time_loop(decode_reuse, args.steps, args.warmup, stream, fl)
     t_int4 = time_loop(decode_int4, args.steps, args.warmup, stream, fl)
     t_quant = time_loop(quantize_pool, 2, 1, stream)   # once per page in a server: off the step
-    ms_legacy = None
-    if not args.no_legacy:   # the mma.sync kernel on the same call, for comparison only
-        os.environ["LSERVE_PREFILL_IMPL"] = "mma"
-        ms_legacy = float(np.median(time_loop(prefill, max(2, args.steps // 2), 2, stream, fl)))
-        del os.environ["LSERVE_PREFILL_IMPL"]
 
     # the timed steps
     clocks = Clocks(local_rank)
@@ -517,7 +511,6 @@ def main():
                           f"per step") if big else "flushed between steps (write of 252 MB)",
                    "parallelism": f"replicas x{world}"},
         "prefill_ms": ms_prefill, "prefill_attention_ms": ms_attn, "tile_lists_ms": ms_tiles,
-        "prefill_mma_sync_ms": ms_legacy,
         "prefill_tflops": tflops_prefill, "kept_tile_tflop": setup.prefill_flops / 1e12,
         "decode_us_per_step": us_decode, "decode_GBps": gbps_decode, "decode_bytes": setup.dbytes,
         "decode_us_per_step_l2_flushed": float(np.median(t_decode_flushed)) * 1e3,
@@ -537,15 +530,16 @@ def main():
                         "quantize_GBps": quant_bytes / (float(np.median(t_quant)) * 1e-3) / 1e9,
                         "note": "decode step over INT4 pages (codes + fp32 steps/offsets, dequantised on chip); "
                                 "pool quantised once before timing"},
-        "roofline": {"bound": "tensor", "kernel": "prefill attention", "achieved": tflops_attn,
-                     "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tflops_attn / pk["bf16"],
+        "roofline": {"bound": "tensor", "kernel": "prefill attention", "achieved": tflops_prefill,
+                     "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tflops_prefill / pk["bf16"],
                      "traffic": traffic("prefill", wp.name == PREFILL_WL), "traffic_unit": "bytes per launch",
                      "algorithmic_bytes_note": "compulsory: q, k, v, mask read once, out and lse written once",
                      "peak_source": pk["source"] + " bf16 burst",
-                     "peak_sustained": pk["bf16_sust"], "frac_sustained": tflops_attn / pk["bf16_sust"],
+                     "peak_sustained": pk["bf16_sust"], "frac_sustained": tflops_prefill / pk["bf16_sust"],
                      "peak_note": "frac uses the burst peak; in loops this kernel runs at the 1 kW power cap "
                                   "(about 1.7 GHz, sw_power_cap), where the sustained cuBLAS figure applies",
-                     "achieved_note": "kept-tile FLOPs / (lserve_prefill - tile-list build) time"},
+                     "achieved_note": "kept-tile FLOPs / whole lserve_prefill time (the on-device tile-list "
+                                      "build included)"},
         "roofline_decode": {"bound": "hbm", "kernel": "decode step (score, top-k + plan, paged attention, merge)",
                             "achieved": gbps_decode, "peak": pk["hbm"], "unit": "GB/s",
                             "frac": gbps_decode / pk["hbm"],

@@ -257,12 +257,20 @@ lserve_status lserve_decode(const lserve_decode_args* args, void* out, float* ls
  * device that loads it, held until the process exits.  It calls no cudaMalloc,
  * cudaFree or any other allocating routine.
  *
- *   - The first call on a device looks up that array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
- *   - A batch whose scratch need (lserve_decode_workspace_size) exceeds
- *     LSERVE_NOALLOC_SCRATCH_BYTES is rejected with LSERVE_ERR_WORKSPACE and
- *     nothing is launched.
+ *   - The first call in each CUDA context of a device looks up that array's
+ *     device address (with that device current) and caches it; make that first
+ *     call before any stream capture.  After cudaDeviceReset the next call
+ *     looks it up again.
+ *   - The split partials of the attention grid grow with its width.  When a
+ *     full wave's would not fit in the array, the call narrows the grid to the
+ *     widest one whose scratch fits; the result is the same attention, merged
+ *     from fewer splits (equal to lserve_decode's within rounding; the page
+ *     selection is identical).  Only a batch whose scratch exceeds
+ *     LSERVE_NOALLOC_SCRATCH_BYTES even on a one-CTA grid (page scores and
+ *     selections of B * Hkv rows of maxP pages, mostly) is rejected, with
+ *     LSERVE_ERR_WORKSPACE, before anything is launched.
+ *     lserve_decode_workspace_size gives the need of lserve_decode's full-wave
+ *     grid, an upper bound of this call's.
  *   - All calls on a device share the one array and it keeps whatever the last
  *     call left in it (nothing in it needs to start at zero).  Calls whose
  *     kernels overlap on the GPU -- on different streams, or from different

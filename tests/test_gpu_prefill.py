@@ -18,16 +18,6 @@ pytestmark = pytest.mark.gpu
 U = pytest.importorskip("unified_sparse_attention_b200")
 
 
-@pytest.fixture(params=["tc", "mma"], autouse=True)
-def impl(request, monkeypatch):
-    """Run every case on the tcgen05 kernel (default) and on the mma.sync kernel."""
-    if request.param == "mma":
-        monkeypatch.setenv("LSERVE_PREFILL_IMPL", "mma")
-    else:
-        monkeypatch.delenv("LSERVE_PREFILL_IMPL", raising=False)
-    return request.param
-
-
 def run_case(w, S, kind, sink, local, mask_fill=None, B=None, seed_mask=True):
     dev = "cuda"
     q, k, v = W.prefill_inputs(w, S=S, B=B)
@@ -131,9 +121,10 @@ def test_repeated_calls_are_deterministic():
     assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("G,S", [(1, 960), (2, 512), (8, 384)])
+@pytest.mark.parametrize("G,S", [(1, 960), (2, 512), (3, 704), (5, 448), (8, 384)])
 def test_gqa_ratios_and_odd_tile_count(G, S):
-    """G = 1 pairs query tiles (odd tile count leaves a half pair); G = 8 splits heads."""
+    """Odd G (1, 3, 5) pairs query tiles of one head (an odd tile count leaves a
+    half pair); even G pairs two heads of one query tile."""
     w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2 * G, Hkv=2, d=128)
     run_case(w, S, [0, 1], 64, 150, mask_fill=0.5)
 

@@ -57,7 +57,6 @@ def test_decode_wait_limit_reports_timeout_and_context_survives(monkeypatch):
 
 
 def test_prefill_wait_limit_reports_timeout_and_context_survives(monkeypatch):
-    monkeypatch.delenv("LSERVE_PREFILL_IMPL", raising=False)   # the tcgen05 kernel
     w = W.WORKLOADS["tiny"]
     dev = "cuda"
     q, k, v = (t.to(dev) for t in W.prefill_inputs(w))

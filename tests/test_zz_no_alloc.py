@@ -63,6 +63,31 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls_in_a_row():
         assert_attn_close(f64(out), f64(ref), "noalloc vs workspace decode")
 
 
+def test_noalloc_narrows_its_grid_where_a_full_wave_would_not_fit():
+    """G = 8, d = 128: a full wave's split partials alone need more than the
+    array holds, so the call takes a narrower attention grid.  Same pages, same
+    attention within the decode tolerance, for a batch of one and of three."""
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=16, Hkv=2, d=128, dec_anchors=16)
+    for B, lens in ((1, [1500]), (3, [1500, 640, 64])):
+        args = case(w, B, 1500, lens, [0, 1], 512, 2)
+        q = args[0]
+        Hkv = args[1].shape[1]
+        kcap = U.lserve_decode_max_selected(B, 16, Hkv, 128, args[1].shape[0], args[3].shape[1],
+                                            args[7], args[8], args[9])
+        ref = torch.empty_like(q)
+        ref_sel = torch.empty(B, Hkv, kcap, dtype=torch.int32, device=q.device)
+        ref_n = torch.empty(B, Hkv, dtype=torch.int32, device=q.device)
+        U.lserve_decode(*args, out=ref, sel_out=ref_sel, sel_n=ref_n)
+        out = torch.full_like(q, float("nan"))
+        sel = torch.full((B, Hkv, kcap), -7, dtype=torch.int32, device=q.device)
+        sel_n = torch.full((B, Hkv), -7, dtype=torch.int32, device=q.device)
+        U.lserve_decode_noalloc(*args, out=out, sel_out=sel, sel_n=sel_n)
+        torch.cuda.synchronize()
+        assert U.lserve_get_device_status() == 0
+        assert torch.equal(sel, ref_sel) and torch.equal(sel_n, ref_n)
+        assert_attn_close(f64(out), f64(ref), "noalloc (narrowed grid) vs workspace decode")
+
+
 def test_noalloc_refuses_batches_larger_than_its_array():
     from unified_sparse_attention_b200 import binding as Bd
     lib = U.load_library()

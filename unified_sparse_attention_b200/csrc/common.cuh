@@ -193,21 +193,7 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x in [-126, 64): Cody-Waite split x = n + f with
-// n = round(x) taken from the low mantissa bits of x + 1.5*2^23, f in [-1/2, 1/2],
-// 2^f from a cubic fitted here by Remez iterations for minimax relative error
-// (7.5e-5 on [-1/2, 1/2]), and 2^n added into the exponent field.  Used for a
-// share of the softmax exponentials so that the MUFU unit is not the only
-// source of them; x = -inf is NOT supported (callers keep masked keys on ex2).
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// ---- packed fp32 pairs and bf16 exponentials (sm_100 PTX)
+// ---- packed fp32 pairs (sm_100 PTX)
 __device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -231,17 +217,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// (2^lo, 2^hi) as packed bf16 (lo in the low half).  The arguments are rounded
-// to bf16 with integer operations (add half an ulp of the 16 dropped bits, keep
-// the upper halves; -inf stays -inf), which keeps the conversion off the XU pipe
-// that the MUFU exponential itself occupies; one MUFU op evaluates both.
-__device__ __forceinline__ uint32_t exp2_bf16x2(float lo, float hi) {
-  const uint32_t t = __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-  uint32_t r;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(r) : "r"(t));
-  return r;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

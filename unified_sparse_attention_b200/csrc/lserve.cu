@@ -18,7 +18,6 @@
 #include "cra.cuh"
 #include "decode.cuh"
 #include "page_stats.cuh"
-#include "prefill_mma.cuh"
 #include "prefill_tc.cuh"
 #include "quant.cuh"
 #include "select.cuh"
@@ -236,31 +235,15 @@ lserve_status launch_tile_lists(const lserve_shape* s, const uint8_t* head_kind,
   return check_launch("tile lists");
 }
 
-template <int D>
-lserve_status launch_prefill_mma(const lserve_shape* s, const void* q, const void* k, const void* v,
-                                 const PrefillArgs& A, int n_rows, cudaStream_t st) {
-  CUtensorMap tq, tk, tv;
-  const uint64_t T = static_cast<uint64_t>(s->B) * s->S;
-  if (!make_map_3d(&tq, q, D, s->Hq, T) || !make_map_3d(&tk, k, D, s->Hkv, T) || !make_map_3d(&tv, v, D, s->Hkv, T))
-    return fail(LSERVE_ERR_CUDA, "prefill: cuTensorMapEncodeTiled failed");
-  ensure_smem(prefill_mma_kernel<D>, PrefillCfg<D>::kSmemBytes);
-  const long long grid = static_cast<long long>(n_rows) * A.G;
-  prefill_mma_kernel<D><<<static_cast<unsigned>(grid), kPrefillThreads, PrefillCfg<D>::kSmemBytes, st>>>(tq, tk, tv,
-                                                                                                      A);
-  return check_launch("prefill attention");
-}
-
-// tcgen05 path: work-item shape from the GQA ratio (see prefill_tc.cuh).
+// Work-item shape from the GQA ratio (see prefill_tc.cuh): an item is 128 query
+// rows that share one KV tile list.  Even G: two query heads of one query tile.
+// Odd G (1, 3, ...): one query head, two adjacent query tiles walking the union
+// of their lists.
 struct TcPlan {
-  int QG, HG, NM;
+  int QG, HG;
 };
 
-bool tc_plan(int G, TcPlan* p) {
-  if (G % 2 == 0) *p = {1, 2, 1};
-  else if (G == 1) *p = {2, 1, 1};
-  else return false;
-  return true;
-}
+TcPlan tc_plan(int G) { return G % 2 == 0 ? TcPlan{1, 2} : TcPlan{2, 1}; }
 
 template <int D>
 lserve_status launch_prefill_tc(const lserve_shape* s, const void* q, const void* k, const void* v,
@@ -297,11 +280,6 @@ lserve_status run_prefill(const lserve_shape* shape, const void* q, const void* 
 
 size_t round_up256(size_t b) { return (b + 255) / 256 * 256; }
 
-bool use_legacy_prefill() {
-  const char* e = getenv("LSERVE_PREFILL_IMPL");
-  return e && strcmp(e, "mma") == 0;
-}
-
 lserve_status run_prefill(const lserve_shape* shape, const void* q, const void* k, const void* v,
                           const uint8_t* head_kind, int sink, int local, const uint8_t* block_mask, void* out,
                           float* lse, void* workspace, cudaStream_t st) {
@@ -309,28 +287,20 @@ lserve_status run_prefill(const lserve_shape* shape, const void* q, const void* 
   const int G = shape->Hq / shape->Hkv;
   const int nQT = shape->S / kTile;
   const float scale = shape->scale > 0.f ? shape->scale : 1.f / std::sqrt(static_cast<float>(shape->d));
-  PrefillArgs A{w.offsets, w.cols, w.order, head_kind, static_cast<bf16*>(out), lse, G,
+  tc::PrefillArgs A{w.offsets, w.cols, w.order, head_kind, static_cast<bf16*>(out), lse, G,
                 shape->Hkv, nQT, shape->S, sink, local, scale * 1.4426950408889634f, wait_timeout_ns()};
-  TcPlan tp;
-  lserve_status s;
-  if (!use_legacy_prefill() && tc_plan(G, &tp)) {
-    // rows with a closed-form list (streaming heads; dense heads without a mask)
-    // get no CSR entries: the kernel computes their tiles
-    s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz, w.order, st,
-                          tp.QG, /*closed_form=*/true);
-    if (s != LSERVE_OK) return s;
-    const int nRow = (nQT + tp.QG - 1) / tp.QG;
-    const int n_rows = shape->B * shape->Hkv * nRow;
-    tc::TcArgs T{A, block_mask, tp.QG, tp.HG, nRow, G / tp.HG, n_rows * (G / tp.HG), w.work_counter,
-                 debug_stall_prefill()};
-    return shape->d == 128 ? launch_prefill_tc<128>(shape, q, k, v, T, n_rows, st)
-                           : launch_prefill_tc<64>(shape, q, k, v, T, n_rows, st);
-  }
-  s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz, w.order, st);
+  const TcPlan tp = tc_plan(G);
+  // rows with a closed-form list (streaming heads; dense heads without a mask)
+  // get no CSR entries: the kernel computes their tiles
+  lserve_status s = launch_tile_lists(shape, head_kind, sink, local, block_mask, w, w.offsets, w.cols, w.max_nnz,
+                                      w.order, st, tp.QG, /*closed_form=*/true);
   if (s != LSERVE_OK) return s;
-  const int n_rows = shape->B * shape->Hkv * nQT;
-  return shape->d == 128 ? launch_prefill_mma<128>(shape, q, k, v, A, n_rows, st)
-                         : launch_prefill_mma<64>(shape, q, k, v, A, n_rows, st);
+  const int nRow = (nQT + tp.QG - 1) / tp.QG;
+  const int n_rows = shape->B * shape->Hkv * nRow;
+  tc::TcArgs T{A, block_mask, tp.QG, tp.HG, nRow, G / tp.HG, n_rows * (G / tp.HG), w.work_counter,
+               debug_stall_prefill()};
+  return shape->d == 128 ? launch_prefill_tc<128>(shape, q, k, v, T, n_rows, st)
+                         : launch_prefill_tc<64>(shape, q, k, v, T, n_rows, st);
 }
 
 // ----------------------------------------------------------------- decode
@@ -411,13 +381,14 @@ lserve_status validate_decode(const lserve_decode_args* a, bool need_stats = tru
   return LSERVE_OK;
 }
 
-DecodePlan plan_decode(const lserve_decode_args* a, void* ws, bool q4 = false) {
+// grid > 0 sets the attention grid (CTAs) instead of one full wave.
+DecodePlan plan_decode(const lserve_decode_args* a, void* ws, bool q4 = false, int grid = 0) {
   DecodePlan p{};
   p.G = a->Hq / a->Hkv;
   p.budget_pages = a->token_budget / kPage;
   const int dense_cap = std::min(p.budget_pages, a->maxP);
   p.kcap = std::max(1, std::max(dense_cap, std::min(streaming_page_bound(a->sink, a->local), a->maxP)));
-  p.P = decode_grid(q4);
+  p.P = grid > 0 ? grid : decode_grid(q4);
   p.R = kRangesPerCta * p.P;
 
   Carver c(ws);
@@ -512,24 +483,51 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[LSERVE_NOALLOC_
 
 namespace {
 
-// Device address of g_noalloc_scratch on the current device.  Host code only
-// sees a host-side stand-in under that name, so the address must be asked for
-// once per device (with that device current) and cached.
+// The driver's cuCtxGetCurrent, found through the runtime (no link to libcuda).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  return fn;
+}
+
+// Device address of g_noalloc_scratch in the current context.  Host code only
+// sees a host-side stand-in under that name, so the address is asked for once
+// per (device, context), with that device current, and cached.  The context is
+// part of the key: after cudaDeviceReset the module is loaded again in a new
+// primary context and the array may sit elsewhere.
 lserve_status noalloc_scratch(void** out) {
   static std::mutex mu;
+  static CUcontext ctx_of[64] = {};
   static void* addr[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return fail(LSERVE_ERR_CUDA, "decode_noalloc: no usable current device");
+  auto get_ctx = ctx_get_current_fn();
+  CUcontext ctx = nullptr;   // null: no context bound to this thread yet
+  if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS)
+    return fail(LSERVE_ERR_CUDA, "decode_noalloc: cannot read the current CUDA context");
   std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(LSERVE_ERR_CUDA, "decode_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
-    addr[dev] = p;
+  if (ctx && addr[dev] && ctx_of[dev] == ctx) {
+    *out = addr[dev];
+    return LSERVE_OK;
   }
-  *out = addr[dev];
+  // the lookup binds the device's primary context to this thread when none was
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p)
+    return fail(LSERVE_ERR_CUDA, "decode_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+  if (!ctx && (get_ctx(&ctx) != CUDA_SUCCESS || !ctx))
+    return fail(LSERVE_ERR_CUDA, "decode_noalloc: no CUDA context after the symbol lookup");
+  addr[dev] = p;
+  ctx_of[dev] = ctx;
+  *out = p;
   return LSERVE_OK;
 }
 
@@ -682,18 +680,32 @@ lserve_status lserve_decode_noalloc(const lserve_decode_args* args, void* out, f
   lserve_status s = validate_decode(args);
   if (s != LSERVE_OK) return s;
   if (!out || !aligned16(out)) return fail(LSERVE_ERR_INVALID_ARG, "decode: out must be non-null and 16-byte aligned");
-  const size_t need = plan_decode(args, nullptr).bytes;
-  if (need > LSERVE_NOALLOC_SCRATCH_BYTES)
-    return fail(LSERVE_ERR_WORKSPACE,
-                "decode_noalloc: this batch needs %zu bytes of scratch but the built-in array holds %zu; "
-                "split the batch or call lserve_decode with a workspace",
-                need, static_cast<size_t>(LSERVE_NOALLOC_SCRATCH_BYTES));
+  // The split partials of the attention grid grow with its width (one full wave
+  // by default).  Where they would not fit, take the widest grid whose scratch
+  // does: the result is the same attention, split over fewer ranges.
+  const size_t cap = LSERVE_NOALLOC_SCRATCH_BYTES;
+  int grid = decode_grid(false);
+  if (plan_decode(args, nullptr, false, grid).bytes > cap) {
+    const size_t need1 = plan_decode(args, nullptr, false, 1).bytes;
+    if (need1 > cap)
+      return fail(LSERVE_ERR_WORKSPACE,
+                  "decode_noalloc: this batch needs %zu bytes of scratch even on a one-CTA grid but the built-in "
+                  "array holds %zu; split the batch or call lserve_decode with a workspace",
+                  need1, cap);
+    int lo = 1, hi = grid - 1;   // plan(lo) fits, plan(grid) does not; the need grows with the grid
+    while (lo < hi) {
+      const int mid = lo + (hi - lo + 1) / 2;
+      if (plan_decode(args, nullptr, false, mid).bytes <= cap) lo = mid;
+      else hi = mid - 1;
+    }
+    grid = lo;
+  }
   void* scratch = nullptr;
   s = noalloc_scratch(&scratch);
   if (s != LSERVE_OK) return s;
   // Every buffer carved here is fully written by the kernels before it is read,
   // so the previous call's leftovers need no clearing.
-  DecodePlan p = plan_decode(args, scratch);
+  DecodePlan p = plan_decode(args, scratch, false, grid);
   int32_t* sel = sel_out ? sel_out : p.sel;
   int32_t* seln = sel_n ? sel_n : p.sel_n;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -51,11 +51,23 @@
 #pragma once
 
 #include "common.cuh"
-#include "prefill_mma.cuh"   // PrefillArgs, tile_is_full
-#include "tile_lists.cuh"    // tile_keep
+#include "tile_lists.cuh"    // tile_keep, tile_is_full, row_runs
 
 namespace lserve {
 namespace tc {
+
+// Arguments shared by every work item of one prefill launch.
+struct PrefillArgs {
+  const int32_t* row_offsets;   // CSR of the block-masked rows (closed-form rows have none)
+  const uint16_t* cols;
+  const int32_t* order;         // work order: row of each position
+  const uint8_t* head_kind;
+  bf16* out;                    // null: only the LSE is written (the CRA passes)
+  float* lse;                   // nullable
+  int G, Hkv, nQT, S, sink, local;
+  float scale_log2;             // softmax scale times log2(e)
+  unsigned long long timeout_ns;
+};
 
 // ----------------------------------------------------------- tcgen05 wrappers
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {

@@ -86,6 +86,15 @@ __device__ __forceinline__ bool tile_keep(const TileListParams& P, bool streamin
   return mrow == nullptr || mrow[kt] != 0;
 }
 
+// Is every element of a kept tile (qt, kt) attended?  Then no element mask is
+// needed: a tile below the diagonal of a dense head, or one of a streaming head
+// that lies wholly inside the sink or wholly inside the window of every row of qt.
+__device__ __forceinline__ bool tile_is_full(bool streaming, int qt, int kt, int sink, int local) {
+  if (kt >= qt) return false;   // diagonal (or beyond): causal mask needed
+  if (!streaming) return true;
+  return kTile * kt + kTile <= sink || kTile * qt + (kTile - 1) - kTile * kt < local;
+}
+
 // Calls f(base, kt0, keep[4]) for kt = 0..(last query tile of the row) in
 // ascending order, 32 lanes x 4 tiles per step.  A row of qg query tiles keeps
 // the union of their tiles.
