@@ -30,89 +30,20 @@ The dequantised values stay float32: the decode step never forms them in bf16
 The page summaries are bf16, so the summaries of the dequantised keys round
 the minimum down and the maximum up: the bound stays a bound.
 
-Layouts (d channels, pages of 64 token rows; a byte holds two codes, the one
-with the even nibble index n in its low four bits; nibble n of a 32-bit word
-sits in byte n // 2 of the word, little-endian).  The order of the codes is a
-permutation chosen so that a decode lane's share of a page is a few contiguous
-words (see `k_code_position` and `v_code_position`):
-
-    kq     uint8 [NP, Hkv, 64, d/2]   row = token; codes in k_code_position order
-    vq     uint8 [NP, Hkv, 64 * d/2]  codes in v_code_position order
-    kpar   fp32  [NP, Hkv, 2, d]      [0] = s, [1] = lo, channels in k_param_order
-    vpar   fp32  [NP, Hkv, 64, 2]     (s, lo) per token
+Everything here is in the plain index order of the pages: codes [page, KV
+head, token, channel], key steps and offsets [page, KV head, channel], value
+steps and offsets [page, KV head, token].  How the library packs codes into
+bytes is a storage format, not part of the method; the tests unpack the
+library's bytes into this order before comparing.
 """
 from __future__ import annotations
+
+from typing import NamedTuple
 
 import numpy as np
 import torch
 
 from .selection import PAGE, n_pages, page_stats
-
-
-def k_code_position(d):
-    """Nibble position of channel c within a key row of d/2 bytes: an array P of
-    length d with P[c] = 2 * byte + (1 if high nibble).  A row is four chunks of
-    d/8 bytes; chunk t holds the channels 16 k + 8 h + 2 t + e (k < d/16,
-    h, e < 2).  Within chunk t, word w holds the eight nibbles n = j + 4 e of
-    the channel pairs r = 4 w + j (j < 4), pair r being channels
-    16 (r // 2) + 8 (r % 2) + 2 t + e.  d is a multiple of 32 (64 or 128)."""
-    if d % 32:
-        raise ValueError("the INT4 layouts need d to be a multiple of 32")
-    pos = np.empty(d, np.int64)
-    for t in range(4):
-        for r in range(d // 8):
-            w, j = divmod(r, 4)
-            for e in range(2):
-                c = 16 * (r // 2) + 8 * (r % 2) + 2 * t + e
-                n = j + 4 * e
-                byte = t * (d // 8) + 4 * w + n // 2
-                pos[c] = 2 * byte + (n % 2)
-    return pos
-
-
-def k_param_order(d):
-    """Channel held at each index of a kpar row: four chunks of d/4 entries;
-    entry i of chunk t is channel 16 (i // 4) + 8 ((i // 2) % 2) + 2 t + i % 2."""
-    return np.array([16 * (i // 4) + 8 * ((i // 2) % 2) + 2 * t + i % 2 for t in range(4) for i in range(d // 4)],
-                    np.int64)
-
-
-def v_code_position(d):
-    """Nibble position of (token u, channel c) within a page's d/2 * 64 value
-    bytes: an array P[64, d].  The page is four slices of 16 tokens; slice s is
-    32 chunks of d/4 bytes, chunk 4 g + t holding, in word m (m < d/16), the
-    nibbles n = j + 4 e with channel 16 m + g + 8 (j % 2) and token
-    16 s + 2 t + 8 (j // 2) + e.  d is a multiple of 16."""
-    if d % 16:
-        raise ValueError("the INT4 layouts need d to be a multiple of 16")
-    pos = np.empty((64, d), np.int64)
-    for sl in range(4):
-        for g in range(8):
-            for t in range(4):
-                chunk = (sl * 32 + 4 * g + t) * (d // 4)
-                for m in range(d // 16):
-                    for j in range(4):
-                        for e in range(2):
-                            c = 16 * m + g + 8 * (j % 2)
-                            u = 16 * sl + 2 * t + 8 * (j // 2) + e
-                            n = j + 4 * e
-                            pos[u, c] = 2 * (chunk + 4 * m + n // 2) + (n % 2)
-    return pos
-
-
-def pack_nibbles(codes, pos, nbytes):
-    """Place codes (any shape, values < 16) at nibble positions pos (same shape)."""
-    out = np.zeros(2 * nbytes, np.uint8)
-    out[pos.ravel()] = codes.ravel()
-    return (out[0::2] | (out[1::2] << 4)).astype(np.uint8)
-
-
-def unpack_nibbles(packed, pos):
-    """Inverse of pack_nibbles: the codes at nibble positions pos."""
-    nib = np.empty(2 * packed.size, np.uint8)
-    nib[0::2] = packed & 15
-    nib[1::2] = packed >> 4
-    return nib[pos]
 
 
 def bf16_round(x) -> np.ndarray:
@@ -161,17 +92,33 @@ def dequant(code, s, lo) -> np.ndarray:
     return exact.astype(np.float32)
 
 
-def quantize_pages(k_pages, v_pages, page_table, seq_lens):
-    """(kq, kpar, vq, vpar, kdeq, vdeq) for every page a sequence holds; pages no
-    sequence holds stay zero.  k_pages/v_pages: bf16 values [NP, Hkv, 64, d]."""
+class Int4Pages(NamedTuple):
+    """INT4 pages in plain index order (pages no sequence holds stay zero)."""
+    kcode: np.ndarray   # uint8 [NP, Hkv, 64, d]
+    kstep: np.ndarray   # float32 [NP, Hkv, d]
+    klo: np.ndarray     # float32 [NP, Hkv, d]
+    vcode: np.ndarray   # uint8 [NP, Hkv, 64, d]
+    vstep: np.ndarray   # float32 [NP, Hkv, 64]
+    vlo: np.ndarray     # float32 [NP, Hkv, 64]
+    kdeq: np.ndarray    # float32 [NP, Hkv, 64, d]
+    vdeq: np.ndarray    # float32 [NP, Hkv, 64, d]
+
+
+def quantize_pages(k_pages, v_pages, page_table, seq_lens) -> Int4Pages:
+    """Codes, steps, offsets and dequantised values of every page a sequence
+    holds.  k_pages/v_pages: bf16 values [NP, Hkv, 64, d].  Keys: one group per
+    (page, KV head, channel) over the page's valid tokens; values: one group per
+    (page, KV head, token) over the d channels.  Rows past a sequence's end keep
+    code 0 (and, for values, s = lo = 0)."""
     k = np.asarray(k_pages, dtype=np.float32)
     v = np.asarray(v_pages, dtype=np.float32)
     NP, Hkv, P, d = k.shape
-    kpos, vpos, korder = k_code_position(d), v_code_position(d), k_param_order(d)
-    kq = np.zeros((NP, Hkv, P, d // 2), np.uint8)
-    vq = np.zeros((NP, Hkv, P * d // 2), np.uint8)
-    kpar = np.zeros((NP, Hkv, 2, d), np.float32)
-    vpar = np.zeros((NP, Hkv, P, 2), np.float32)
+    kcode = np.zeros((NP, Hkv, P, d), np.uint8)
+    vcode = np.zeros((NP, Hkv, P, d), np.uint8)
+    kstep = np.zeros((NP, Hkv, d), np.float32)
+    klo = np.zeros((NP, Hkv, d), np.float32)
+    vstep = np.zeros((NP, Hkv, P), np.float32)
+    vlo = np.zeros((NP, Hkv, P), np.float32)
     kdeq = np.zeros_like(k)
     vdeq = np.zeros_like(v)
     for b in range(len(seq_lens)):
@@ -183,21 +130,16 @@ def quantize_pages(k_pages, v_pages, page_table, seq_lens):
                 kk = k[p, g, :nv, :]
                 lo, hi = kk.min(axis=0), kk.max(axis=0)
                 st = _step(lo, hi)
-                codes = np.zeros((P, d), np.uint8)
-                codes[:nv] = _codes(kk, lo[None, :], st[None, :])
-                for r in range(P):
-                    kq[p, g, r] = pack_nibbles(codes[r], kpos, d // 2)
-                kpar[p, g, 0], kpar[p, g, 1] = st[korder], lo[korder]
-                kdeq[p, g] = dequant(codes, st[None, :], lo[None, :])
+                kcode[p, g, :nv] = _codes(kk, lo[None, :], st[None, :])
+                kstep[p, g], klo[p, g] = st, lo
+                kdeq[p, g] = dequant(kcode[p, g], st[None, :], lo[None, :])
                 vv = v[p, g, :nv, :]
                 lo, hi = vv.min(axis=1), vv.max(axis=1)
                 st = _step(lo, hi)
-                codes = np.zeros((P, d), np.uint8)
-                codes[:nv] = _codes(vv, lo[:, None], st[:, None])
-                vq[p, g] = pack_nibbles(codes, vpos, P * d // 2)
-                vpar[p, g, :nv, 0], vpar[p, g, :nv, 1] = st, lo
-                vdeq[p, g] = dequant(codes, vpar[p, g, :, 0][:, None], vpar[p, g, :, 1][:, None])
-    return kq, kpar, vq, vpar, kdeq, vdeq
+                vcode[p, g, :nv] = _codes(vv, lo[:, None], st[:, None])
+                vstep[p, g, :nv], vlo[p, g, :nv] = st, lo
+                vdeq[p, g] = dequant(vcode[p, g], vstep[p, g][:, None], vlo[p, g][:, None])
+    return Int4Pages(kcode, kstep, klo, vcode, vstep, vlo, kdeq, vdeq)
 
 
 def quantized_stats(kdeq, page_table, seq_lens, head_kind):

@@ -4,7 +4,9 @@ pages) against the oracle, through the C ABI.
 The quantiser's codes, steps, offsets and page summaries are integer or float32
 decisions taken in float32 on both sides: bit-exact.  The decode step over INT4
 pages is compared with the oracle's decode on the dequantised pools (the
-oracle's own dequantisation), at the attention tolerances."""
+oracle's own dequantisation), at the attention tolerances.  The library's bytes
+are unpacked into the oracle's plain [token, channel] order first
+(tests/int4_format.py, the storage format declared in include/lserve.h)."""
 import dataclasses
 
 import numpy as np
@@ -16,6 +18,7 @@ from oracle import decode as OD
 from oracle import quant as OQ
 from oracle import selection as OS
 from parity import assert_attn_close, assert_lse_close, check_selection, f64
+import int4_format as F
 
 pytestmark = pytest.mark.gpu
 
@@ -36,19 +39,27 @@ def quantize(pc, kind, first_page=0, bufs=None):
     return dict(zip(("kq", "kpar", "vq", "vpar", "stats"), r))
 
 
+def assert_quantiser_equal(g, qp, d):
+    """The library's packed codes and parameters against the oracle's plain arrays, bit for bit."""
+    np.testing.assert_array_equal(F.unpack_keys(g["kq"].cpu().numpy(), d), qp.kcode)
+    np.testing.assert_array_equal(F.unpack_values(g["vq"].cpu().numpy(), d), qp.vcode)
+    ks, klo = F.unpack_key_params(g["kpar"].cpu().numpy())
+    np.testing.assert_array_equal(ks, qp.kstep)
+    np.testing.assert_array_equal(klo, qp.klo)
+    vs, vlo = F.unpack_value_params(g["vpar"].cpu().numpy())
+    np.testing.assert_array_equal(vs, qp.vstep)
+    np.testing.assert_array_equal(vlo, qp.vlo)
+
+
 @pytest.mark.parametrize("d,lens", [(128, [1000, 333, 65]), (64, [130, 1, 640])])
 def test_quantiser_bit_exact(d, lens):
     w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=4, Hkv=2, d=d)
     pc = W.decode_cache(w, B=len(lens), ctx=max(lens), seq_lens=lens)
     kind = [0, 1]
     g = quantize(pc, kind)
-    kq, kpar, vq, vpar, kdeq, _ = OQ.quantize_pages(f64(pc.k_pages), f64(pc.v_pages), pc.page_table.numpy(),
-                                                    pc.seq_lens.numpy())
-    np.testing.assert_array_equal(g["kq"].cpu().numpy(), kq)
-    np.testing.assert_array_equal(g["vq"].cpu().numpy(), vq.reshape(g["vq"].shape))
-    np.testing.assert_array_equal(g["kpar"].cpu().numpy(), kpar)
-    np.testing.assert_array_equal(g["vpar"].cpu().numpy(), vpar)
-    st = OQ.quantized_stats(kdeq, pc.page_table.numpy(), pc.seq_lens.numpy(), kind)
+    qp = OQ.quantize_pages(f64(pc.k_pages), f64(pc.v_pages), pc.page_table.numpy(), pc.seq_lens.numpy())
+    assert_quantiser_equal(g, qp, d)
+    st = OQ.quantized_stats(qp.kdeq, pc.page_table.numpy(), pc.seq_lens.numpy(), kind)
     np.testing.assert_array_equal(f64(g["stats"]), st)
 
 
@@ -86,7 +97,8 @@ def run_int4(w, B, ctx, budget, sink, local, lens=None, kind=None):
     torch.cuda.synchronize()
     assert U.lserve_get_device_status() == 0
     pt_np, L = pc.page_table.numpy(), pc.seq_lens.numpy()
-    _, _, _, _, kdeq, vdeq = OQ.quantize_pages(f64(pc.k_pages), f64(pc.v_pages), pt_np, L)
+    qp = OQ.quantize_pages(f64(pc.k_pages), f64(pc.v_pages), pt_np, L)
+    kdeq, vdeq = qp.kdeq, qp.vdeq
     st_ref = OQ.quantized_stats(kdeq, pt_np, L, kind)
     q64 = f64(q)
     sel_ref, _, scores = OS.select(q64, st_ref, pt_np, L, kind, budget, sink, local)
@@ -216,15 +228,11 @@ def test_quantiser_ties_and_near_ties():
     pc = W.scatter_to_pages(k, v, pt, 2)
     kind = [0, 0]
     g = quantize(pc, kind)
-    kq, kpar, vq, vpar, kdeq, _ = OQ.quantize_pages(f64(pc.k_pages), f64(pc.v_pages), pc.page_table.numpy(),
-                                                    pc.seq_lens.numpy())
-    np.testing.assert_array_equal(g["kq"].cpu().numpy(), kq)
-    np.testing.assert_array_equal(g["vq"].cpu().numpy(), vq.reshape(g["vq"].shape))
-    np.testing.assert_array_equal(g["kpar"].cpu().numpy(), kpar)
-    np.testing.assert_array_equal(g["vpar"].cpu().numpy(), vpar)
-    st = OQ.quantized_stats(kdeq, pc.page_table.numpy(), pc.seq_lens.numpy(), kind)
+    qp = OQ.quantize_pages(f64(pc.k_pages), f64(pc.v_pages), pc.page_table.numpy(), pc.seq_lens.numpy())
+    assert_quantiser_equal(g, qp, d)
+    st = OQ.quantized_stats(qp.kdeq, pc.page_table.numpy(), pc.seq_lens.numpy(), kind)
     np.testing.assert_array_equal(f64(g["stats"]), st)
     # the constructed groups do reach exact ties: some code is an even neighbour of x / s
-    codes = OQ.unpack_nibbles(kq[1, 0, 5], OQ.k_code_position(d))
+    codes = qp.kcode[1, 0, 5]
     x = f64(pc.k_pages)[1, 0, 5]
     assert np.any((x % 1 == 0.5) & (codes % 2 == 0))

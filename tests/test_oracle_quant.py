@@ -7,11 +7,19 @@
 * a group whose values are all equal dequantises exactly;
 * the directed bf16 roundings of the summaries are checked by hand and
   against torch's bf16 conversion (bracketing, one step apart at most);
-* the summaries of the dequantised keys bound every dequantised key.
+* the summaries of the dequantised keys bound every dequantised key;
+* the test-side unpacker of the library's byte format (tests/int4_format.py,
+  used by the GPU parity tests) hits the positions worked out by hand in
+  tests/golden/int4_layout.json and is a bijection.
 """
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
+
+import int4_format as F
 
 import workloads as W
 from oracle import quant as Q
@@ -30,44 +38,46 @@ def pool(seed=3, B=2, ctx=150, Hkv=2, d=64, lens=None):
     return pc.k_pages.float().numpy(), pc.v_pages.float().numpy(), pt.numpy(), lens
 
 
-def unpack_k(row_bytes, d):
-    return Q.unpack_nibbles(row_bytes, Q.k_code_position(d))
+def test_storage_format_positions_match_the_hand_worked_page():
+    """The test-side unpacker of the library's INT4 bytes (tests/int4_format.py)
+    against positions worked out by hand from include/lserve.h's prose."""
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "int4_layout.json")))
+    d = g["d"]
+    kp = F.key_nibble_positions(d)
+    for c, n in g["key_row"]["channel_to_nibble"].items():
+        assert kp[int(c)] == n, c
+    vp = F.value_nibble_positions(d)
+    for u, c, n in g["value_page"]["token_channel_to_nibble"]:
+        assert vp[u, c] == n, (u, c)
+    kc = F.key_param_channels(d)
+    for i, c in g["key_params"]["index_to_channel"].items():
+        assert kc[int(i)] == c, i
 
 
-def unpack_v(page_bytes, d):
-    return Q.unpack_nibbles(page_bytes, Q.v_code_position(d))
-
-
-def test_code_layouts_are_bijections():
-    """Every code of a key row / value page has its own nibble, and every
-    nibble holds one code; the parameter order lists each channel once."""
-    for d in (32, 64, 128):
-        kp = Q.k_code_position(d)
+def test_storage_format_is_a_bijection():
+    """Every code of a key row / value page has its own nibble and every nibble
+    holds one code; every channel's parameters sit at one index.  Unpacking
+    bytes built nibble by nibble recovers the codes."""
+    for d in (64, 128):
+        kp = F.key_nibble_positions(d)
         assert sorted(kp.tolist()) == list(range(d))
-        vp = Q.v_code_position(d)
+        vp = F.value_nibble_positions(d)
         assert sorted(vp.ravel().tolist()) == list(range(64 * d))
-        order = Q.k_param_order(d)
-        assert len(order) == d and sorted(order.tolist()) == list(range(d))
-        # round trip through the packed bytes
+        kc = F.key_param_channels(d)
+        assert sorted(kc.tolist()) == list(range(d))
         rng = np.random.default_rng(d)
         codes = rng.integers(0, 16, size=(64, d)).astype(np.uint8)
-        packed = Q.pack_nibbles(codes, vp, 32 * d)
-        np.testing.assert_array_equal(Q.unpack_nibbles(packed, vp), codes)
-        row = codes[0]
-        np.testing.assert_array_equal(Q.unpack_nibbles(Q.pack_nibbles(row, kp, d // 2), kp), row)
-    with pytest.raises(ValueError):
-        Q.k_code_position(16)
-
-
-def test_key_chunk_holds_the_lane_channels():
-    """Chunk t of a key row (d/8 bytes) holds exactly the channels 2t, 2t+1 of
-    every group of eight (the channels one lane of the decode step multiplies)."""
-    d = 128
-    kp = Q.k_code_position(d)
-    for t in range(4):
-        lo, hi = 2 * t * (d // 8), 2 * (t + 1) * (d // 8)
-        chans = sorted(int(c) for c in np.nonzero((kp >= lo) & (kp < hi))[0])
-        assert chans == sorted(c for c in range(d) if (c % 8) // 2 == t)
+        nib = np.zeros(64 * d, np.uint8)
+        nib[vp.ravel()] = codes.ravel()
+        packed = (nib[0::2] | (nib[1::2] << 4)).astype(np.uint8)
+        np.testing.assert_array_equal(F.unpack_values(packed, d), codes)
+        nib = np.zeros(d, np.uint8)
+        nib[kp] = codes[0]
+        np.testing.assert_array_equal(F.unpack_keys((nib[0::2] | (nib[1::2] << 4)).astype(np.uint8), d), codes[0])
+        par = rng.standard_normal((2, d)).astype(np.float32)
+        step, lo = F.unpack_key_params(par)
+        np.testing.assert_array_equal(step[kc], par[0])
+        np.testing.assert_array_equal(lo[kc], par[1])
 
 
 def test_bf16_directed_rounding_by_hand():
@@ -100,12 +110,13 @@ def test_bf16_directed_rounding_brackets_and_is_tight():
 
 def test_codes_range_extremes_monotone_and_error_bound():
     kp, vp, pt, L = pool(lens=[150, 97])
-    kq, kpar, vq, vpar, kdeq, vdeq = Q.quantize_pages(kp, vp, pt, L)
+    qp = Q.quantize_pages(kp, vp, pt, L)
+    kdeq, vdeq = qp.kdeq, qp.vdeq
     for b in range(2):
         for i in range(Sel.n_pages(L[b])):
             p, nv = pt[b, i], min(64, L[b] - 64 * i)
             for g in range(2):
-                kc = np.stack([unpack_k(kq[p, g, r], 2 * kq.shape[-1]) for r in range(64)])[:nv]
+                kc = qp.kcode[p, g, :nv]
                 x = kp[p, g, :nv]
                 assert kc.max() <= 15
                 for c in range(x.shape[1]):           # keys: per channel
@@ -114,27 +125,27 @@ def test_codes_range_extremes_monotone_and_error_bound():
                         assert kc[col.argmin(), c] == 0 and kc[col.argmax(), c] == 15
                     order = np.argsort(col, kind="stable")
                     assert np.all(np.diff(kc[order, c].astype(int)) >= 0)
-                step = np.empty_like(kpar[p, g, 0])
-                step[Q.k_param_order(step.size)] = kpar[p, g, 0]
+                step = qp.kstep[p, g]
                 err = np.abs(kdeq[p, g, :nv] - x)
                 # half a step, plus the float32 rounding of the fma
                 rnd = np.maximum(np.abs(x), np.abs(kdeq[p, g, :nv])) * 2 ** -22
                 assert np.all(err <= step[None, :] * 0.5 * (1 + 1e-5) + rnd + 1e-7)
-                vc = unpack_v(vq[p, g], kp.shape[-1])[:nv]
+                vc = qp.vcode[p, g, :nv]
                 y = vp[p, g, :nv]
                 for t in range(nv):                    # values: per token
                     if y[t].max() > y[t].min():
                         assert vc[t, y[t].argmin()] == 0 and vc[t, y[t].argmax()] == 15
                 err = np.abs(vdeq[p, g, :nv] - y)
                 rnd = np.maximum(np.abs(y), np.abs(vdeq[p, g, :nv])) * 2 ** -22
-                assert np.all(err <= vpar[p, g, :nv, 0, None] * 0.5 * (1 + 1e-5) + rnd + 1e-7)
+                assert np.all(err <= qp.vstep[p, g, :nv, None] * 0.5 * (1 + 1e-5) + rnd + 1e-7)
 
 
 def test_constant_group_dequantises_exactly():
     kp, vp, pt, L = pool()
     kp[:] = 1.5
     vp[:] = -0.25
-    _, _, _, _, kdeq, vdeq = Q.quantize_pages(kp, vp, pt, L)
+    qp = Q.quantize_pages(kp, vp, pt, L)
+    kdeq, vdeq = qp.kdeq, qp.vdeq
     for b in range(2):
         for i in range(Sel.n_pages(L[b])):
             p, nv = pt[b, i], min(64, L[b] - 64 * i)
@@ -144,7 +155,7 @@ def test_constant_group_dequantises_exactly():
 def test_summaries_of_dequantised_keys_bound_them():
     kp, vp, pt, L = pool(lens=[150, 70])
     kind = np.array([0, 1], np.uint8)
-    _, _, _, _, kdeq, _ = Q.quantize_pages(kp, vp, pt, L)
+    kdeq = Q.quantize_pages(kp, vp, pt, L).kdeq
     st = Q.quantized_stats(kdeq, pt, L, kind)
     for b in range(2):
         for t in range(L[b]):
