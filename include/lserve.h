@@ -76,6 +76,8 @@ typedef struct lserve_shape {
   int32_t Hkv;    /* KV heads; query head h reads KV head h / (Hq / Hkv)           */
   int32_t d;      /* head dim, 64 or 128                                           */
   float scale;    /* softmax scale; <= 0 selects 1/sqrt(d)                         */
+  int32_t lambda_tiles; /* 0: token-level Lambda support of streaming heads;
+                           1: tile-level (whole 64x64 tiles, see lserve_prefill) */
 } lserve_shape;
 
 /*
@@ -93,6 +95,10 @@ size_t lserve_prefill_workspace_size(const lserve_shape* shape);
  *   dense g      (head_kind[g] == 0):  { j <= i : block_mask[b,g,i/64,j/64] != 0 }
  *                                       (every j <= i when block_mask == NULL)
  *   streaming g  (head_kind[g] == 1):  { j <= i : j < sink  or  i - j < local }
+ *   streaming g, shape->lambda_tiles == 1 (the tile-level reading of the blog's
+ *                "no partial blocks", Fig. 1(b)): every causal key of every
+ *                64x64 tile that meets that support,
+ *                { j <= i : 64 (j/64) < sink  or  max(64 (i/64) - 64 (j/64) - 63, 0) < local }
  * out[b,i,h,:] = sum_j softmax_j(scale * q.k_j) v_j over the kept set; a row
  * whose kept set is empty gets out = 0 and lse = -inf.  A 64x64 tile with no
  * kept element is never read (whole-tile skipping, blog "LServe - Prefill
@@ -169,7 +175,7 @@ lserve_status lserve_update_page_stats(int32_t B, int32_t Hkv, int32_t d, int32_
  * every query row i, the share r_i of its causal softmax probability mass that
  * the sparse mask keeps, and CRA = the minimum of r_i over the rows -- the
  * worst-kept query, which a mask is judged by.  The mask is given exactly as to
- * lserve_prefill (head_kind, sink, local, block_mask).  Computed from two LSE-only
+ * lserve_prefill (head_kind, sink, local, block_mask, shape->lambda_tiles).  Computed from two LSE-only
  * passes of the prefill kernel (causal, and the sparse mask; no output written):
  * r_i = exp(lse_sparse(i) - lse_causal(i)); a row that keeps nothing retains 0.
  *

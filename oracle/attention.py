@@ -19,6 +19,17 @@ Readings where the pages are silent: the Lambda support is defined per token
 (the kernel keeps every 64x64 tile that meets it and masks inside boundary
 tiles); a block mask applies to dense heads only and is given per KV head; a
 row with an empty kept set yields o_i = 0 and lse_i = -inf.
+
+Tile-level Lambda (``lambda_tiles=True``): the same post's "no partial blocks"
+(each KV block is fully computed or fully skipped, Fig. 1(a)/(b)) read for the
+streaming heads too.  A streaming head then attends every causal key of every
+64x64 tile that meets the Lambda support:
+
+* streaming, tile level:  K(i) = { j <= i : 64 (j // 64) < sink  or
+                                   max(64 (i // 64) - 64 (j // 64) - 63, 0) < local }
+
+i.e. the tiles of ``tile_kept`` in full, with only the causal mask inside the
+diagonal tile.  Dense heads are unchanged.
 """
 from __future__ import annotations
 
@@ -28,14 +39,18 @@ TILE = 64
 
 
 def kept_mask(rows: np.ndarray, S: int, streaming: bool, sink: int, local: int,
-              tile_mask: np.ndarray | None) -> np.ndarray:
+              tile_mask: np.ndarray | None, lambda_tiles: bool = False) -> np.ndarray:
     """bool[len(rows), S]: element (r, j) is True iff key j is in K(rows[r]).
 
-    ``tile_mask`` is this (batch, KV head)'s uint8[S/64, S/64] block mask or None.
+    ``tile_mask`` is this (batch, KV head)'s uint8[S/64, S/64] block mask or None;
+    ``lambda_tiles`` selects the tile-level Lambda support of streaming heads.
     """
     i = np.asarray(rows, dtype=np.int64)[:, None]
     j = np.arange(S, dtype=np.int64)[None, :]
     causal = j <= i
+    if streaming and lambda_tiles:
+        qt, kt = i // TILE, j // TILE
+        return causal & ((TILE * kt < sink) | (np.maximum(TILE * qt - TILE * kt - (TILE - 1), 0) < local))
     if streaming:
         return causal & ((j < sink) | (i - j < local))
     if tile_mask is None:
@@ -44,7 +59,7 @@ def kept_mask(rows: np.ndarray, S: int, streaming: bool, sink: int, local: int,
 
 
 def masked_attention(q, k, v, head_kind, sink, local, block_mask=None, scale=None,
-                     rows=None, row_chunk=256, q_at_rows=False):
+                     rows=None, row_chunk=256, q_at_rows=False, lambda_tiles=False):
     """Exact masked attention in float64.
 
     q : [B, S, Hq, d]; k, v : [B, S, Hkv, d] (any float dtype, up-cast to f64)
@@ -53,6 +68,7 @@ def masked_attention(q, k, v, head_kind, sink, local, block_mask=None, scale=Non
     rows : optional 1-D array of query positions to evaluate (all when None);
            rows are independent, so a sampled row is an exact row.
     q_at_rows : q is given only at ``rows`` ([B, R, Hq, d]) instead of [B, S, Hq, d].
+    lambda_tiles : streaming heads use the tile-level Lambda support.
 
     Returns (out [B, R, Hq, d], lse [B, Hq, R]) with R = len(rows).
     """
@@ -77,7 +93,7 @@ def masked_attention(q, k, v, head_kind, sink, local, block_mask=None, scale=Non
             V = v[b, :, kvh, :]
             for c0 in range(0, R, row_chunk):
                 r = rows[c0:c0 + row_chunk]
-                keep = kept_mask(r, S, streaming, sink, local, tm)
+                keep = kept_mask(r, S, streaming, sink, local, tm, lambda_tiles)
                 qr = q[b, c0:c0 + len(r), h, :] if q_at_rows else q[b, r, h, :]
                 logits = scale * (qr @ K.T)
                 logits = np.where(keep, logits, -np.inf)
@@ -92,7 +108,8 @@ def masked_attention(q, k, v, head_kind, sink, local, block_mask=None, scale=Non
     return out, lse
 
 
-def attention_weights(q, k, head_kind, sink, local, block_mask=None, scale=None, b=0, h=0):
+def attention_weights(q, k, head_kind, sink, local, block_mask=None, scale=None, b=0, h=0,
+                      lambda_tiles=False):
     """float64[S, S] softmax weights of one (batch, query head); zero rows for empty K(i)."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -102,7 +119,7 @@ def attention_weights(q, k, head_kind, sink, local, block_mask=None, scale=None,
     streaming = bool(head_kind[kvh])
     scale = 1.0 / np.sqrt(d) if scale is None or scale <= 0 else float(scale)
     tm = None if (block_mask is None or streaming) else np.asarray(block_mask[b, kvh])
-    keep = kept_mask(np.arange(S), S, streaming, sink, local, tm)
+    keep = kept_mask(np.arange(S), S, streaming, sink, local, tm, lambda_tiles)
     logits = np.where(keep, scale * (q[b, :, h, :] @ k[b, :, kvh, :].T), -np.inf)
     m = logits.max(axis=1, keepdims=True)
     m = np.where(np.isfinite(m), m, 0.0)

@@ -18,14 +18,15 @@ import numpy as np
 from .attention import masked_attention
 
 
-def retained_mass(q, k, v, head_kind, sink, local, block_mask=None, scale=None, rows=None):
+def retained_mass(q, k, v, head_kind, sink, local, block_mask=None, scale=None, rows=None, lambda_tiles=False):
     """float64[B, Hq, R]: per query row the retained share of its causal softmax mass."""
     dense_kind = np.zeros(len(head_kind), dtype=np.uint8)
     _, lse_full = masked_attention(q, k, v, dense_kind, 0, 0, None, scale, rows)
-    _, lse_sparse = masked_attention(q, k, v, head_kind, sink, local, block_mask, scale, rows)
+    _, lse_sparse = masked_attention(q, k, v, head_kind, sink, local, block_mask, scale, rows,
+                                     lambda_tiles=lambda_tiles)
     return np.exp(lse_sparse - lse_full)
 
 
-def cra(q, k, v, head_kind, sink, local, block_mask=None, scale=None, rows=None):
+def cra(q, k, v, head_kind, sink, local, block_mask=None, scale=None, rows=None, lambda_tiles=False):
     """float64[B, Hq]: minimum over query rows of the retained mass."""
-    return retained_mass(q, k, v, head_kind, sink, local, block_mask, scale, rows).min(axis=2)
+    return retained_mass(q, k, v, head_kind, sink, local, block_mask, scale, rows, lambda_tiles).min(axis=2)

@@ -48,6 +48,8 @@ def test_prefill_validation():
     assert call(shape(Hq=3)) == 1
     assert call(shape(), q=None) == 1
     assert call(shape(), sink=-1) == 1
+    bad_flag = Bd.Shape(1, 1024, 4, 2, 64, 0.0, 2)                 # lambda_tiles is 0 or 1
+    assert call(ctypes.byref(bad_flag)) == 1
     assert call(shape(), q=ctypes.c_void_p((1 << 20) + 2)) == 1   # misaligned
     assert call(shape()) == 3                                      # no workspace
     need = lib.lserve_prefill_workspace_size(shape())

@@ -56,3 +56,21 @@ def test_cra_is_one_when_nothing_is_dropped():
     torch.cuda.synchronize()
     assert U.lserve_get_device_status() == 0
     assert torch.all(cra == 1.0)   # the two passes are the same computation
+
+
+def test_cra_tile_level_lambda():
+    """The CRA of the tile-level Lambda reading: it keeps a superset of the
+    token-level keys, so it retains at least as much."""
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=4, Hkv=2, d=64)
+    dev = "cuda"
+    q, k, v = W.prefill_inputs(w, S=768)
+    kind, sink, local = [1, 1], 30, 100
+    hk = torch.tensor(kind, dtype=torch.uint8, device=dev)
+    cra_t, ret_t = U.lserve_cra(q.to(dev), k.to(dev), v.to(dev), hk, sink, local, None, return_retained=True,
+                                lambda_tiles=True)
+    cra_e = U.lserve_cra(q.to(dev), k.to(dev), v.to(dev), hk, sink, local, None)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+    ref = OC.retained_mass(f64(q), f64(k), f64(v), kind, sink, local, lambda_tiles=True)
+    assert np.abs(f64(ret_t) - ref).max() <= TOL
+    assert np.all(f64(cra_t) >= f64(cra_e) - TOL)

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 U = pytest.importorskip("unified_sparse_attention_b200")
 
 
-def run_case(w, S, kind, sink, local, mask_fill=None, B=None, seed_mask=True):
+def run_case(w, S, kind, sink, local, mask_fill=None, B=None, seed_mask=True, lambda_tiles=False):
     dev = "cuda"
     q, k, v = W.prefill_inputs(w, S=S, B=B)
     hk = torch.tensor(kind, dtype=torch.uint8)
@@ -27,11 +27,11 @@ def run_case(w, S, kind, sink, local, mask_fill=None, B=None, seed_mask=True):
         ww = dataclasses.replace(w, mask_columns=2, mask_band=2)
         bm = W.block_mask(ww, S=S, fill=mask_fill, B=q.shape[0])
     out, lse = U.lserve_prefill(q.to(dev), k.to(dev), v.to(dev), hk.to(dev), sink, local,
-                                None if bm is None else bm.to(dev), return_lse=True)
+                                None if bm is None else bm.to(dev), return_lse=True, lambda_tiles=lambda_tiles)
     torch.cuda.synchronize()
     assert U.lserve_get_device_status() == 0
     ref, ref_lse = OA.masked_attention(f64(q), f64(k), f64(v), kind, sink, local,
-                                       None if bm is None else bm.numpy())
+                                       None if bm is None else bm.numpy(), lambda_tiles=lambda_tiles)
     assert_attn_close(f64(out), ref, "prefill out")
     assert_lse_close(f64(lse), ref_lse, "prefill lse")
     return q, k, v, hk, bm, out
@@ -144,3 +144,27 @@ def test_streaming_tile_runs_edges(G, sink, local):
     unmasked dense heads against the oracle's token-level kept sets."""
     w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2 * G, Hkv=2, d=64)
     run_case(w, 576, [1, 0], sink, local)
+
+
+@pytest.mark.parametrize("G", [1, 4])
+@pytest.mark.parametrize("sink,local", [(64, 256), (0, 65), (70, 130), (1, 0), (0, 4096)])
+def test_tile_level_lambda(G, sink, local):
+    """Tile-level Lambda (every causal key of every tile that meets the support):
+    against the oracle's tile-level kept sets, next to a block-masked dense head."""
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2 * G, Hkv=2, d=128)
+    run_case(w, 704, [1, 0], sink, local, mask_fill=0.4, lambda_tiles=True)
+
+
+def test_tile_level_lambda_differs_from_token_level_only_at_the_edges():
+    """With sink and window on tile boundaries plus one (local = 65) the two
+    readings differ; with sink = 64 and a window covering whole tiles in both
+    (local >= S) they are the same computation."""
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=4, Hkv=2, d=64)
+    q, k, v = (t.cuda() for t in W.prefill_inputs(w, S=512))
+    hk = torch.tensor([1, 1], dtype=torch.uint8, device="cuda")
+    a = U.lserve_prefill(q, k, v, hk, 64, 65)
+    b = U.lserve_prefill(q, k, v, hk, 64, 65, lambda_tiles=True)
+    assert not torch.equal(a, b)
+    a = U.lserve_prefill(q, k, v, hk, 64, 4096)
+    b = U.lserve_prefill(q, k, v, hk, 64, 4096, lambda_tiles=True)
+    assert torch.equal(a, b)

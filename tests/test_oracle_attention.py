@@ -250,3 +250,55 @@ def test_q_at_rows_matches_full_q():
     o2, lse2 = A.masked_attention(q[:, rows], k, v, kind, 5, 20, rows=rows, q_at_rows=True, row_chunk=2)
     np.testing.assert_allclose(o, o2, atol=1e-14, rtol=0)
     np.testing.assert_allclose(lse, lse2, atol=1e-14, rtol=0)
+
+
+# ---------------------------------------------------------------- tile-level Lambda
+
+def brute_tile_lambda(S, sink, local):
+    """Pure-Python: a tile is kept iff some causal pair inside it meets the token-level
+    Lambda support; K(i) is then every causal key of the kept tiles of row i's tile."""
+    n = S // 64
+    kept = [[False] * n for _ in range(n)]
+    for qt in range(n):
+        for kt in range(qt + 1):
+            kept[qt][kt] = any(j <= i and (j < sink or i - j < local)
+                               for i in range(64 * qt, 64 * qt + 64) for j in range(64 * kt, 64 * kt + 64))
+    m = np.zeros((S, S), bool)
+    for i in range(S):
+        for j in range(i + 1):
+            m[i, j] = kept[i // 64][j // 64]
+    return m
+
+
+@pytest.mark.parametrize("sink,local", [(64, 256), (0, 1), (1, 0), (70, 130), (0, 65), (130, 0)])
+def test_tile_level_lambda_brute_force(sink, local):
+    S = 320
+    got = A.kept_mask(np.arange(S), S, True, sink, local, None, lambda_tiles=True)
+    np.testing.assert_array_equal(got, brute_tile_lambda(S, sink, local))
+    # a superset of the token-level support, equal to it when every boundary is tile-aligned
+    tok = A.kept_mask(np.arange(S), S, True, sink, local, None)
+    assert np.all(got[tok])
+
+
+def test_tile_level_lambda_hand_count():
+    g = GOLD["tile_lambda_pairs"]
+    m = A.kept_mask(np.arange(g["S"]), g["S"], True, g["sink"], g["local"], None, lambda_tiles=True)
+    assert int(m.sum()) == g["kept_pairs"]
+
+
+def test_tile_level_lambda_equals_sdpa_with_its_mask():
+    q, k, v = rand_qkv(1, 256, 4, 2, 16, seed=31)
+    kind, sink, local = [1, 0], 30, 70
+    out, _ = A.masked_attention(q, k, v, kind, sink, local, lambda_tiles=True)
+    m = brute_tile_lambda(256, sink, local)
+    mask = np.where(m, 0.0, -np.inf)[None, None]
+    ref_s = sdpa(q[:, :, :2], k[:, :, :1], v[:, :, :1], mask=mask)   # query heads 0, 1 read KV head 0 (streaming)
+    np.testing.assert_allclose(out[:, :, :2], ref_s, atol=1e-12)
+    ref_d = sdpa(q[:, :, 2:], k[:, :, 1:], v[:, :, 1:], causal=True)   # the dense head is unchanged
+    np.testing.assert_allclose(out[:, :, 2:], ref_d, atol=1e-12)
+
+
+def test_tile_level_lambda_covering_sequence_equals_dense():
+    q, k, v = rand_qkv(1, 192, 2, 1, 8, seed=32)
+    out, _ = A.masked_attention(q, k, v, [1], 192, 0, lambda_tiles=True)
+    np.testing.assert_allclose(out, sdpa(q, k, v, causal=True), atol=1e-12)

@@ -24,28 +24,37 @@ _bounds = Sel.logical_bounds
 _masked = A.masked_attention
 
 
-def kept_window_off_by_one(rows, S, streaming, sink, local, tm):
+def kept_window_off_by_one(rows, S, streaming, sink, local, tm, lambda_tiles=False):
     i = np.asarray(rows)[:, None]
     j = np.arange(S)[None, :]
     if streaming:
         return (j <= i) & ((j < sink) | (i - j <= local))
-    return _kept(rows, S, streaming, sink, local, tm)
+    return _kept(rows, S, streaming, sink, local, tm, lambda_tiles)
 
 
-def kept_sink_inclusive(rows, S, streaming, sink, local, tm):
+def kept_sink_inclusive(rows, S, streaming, sink, local, tm, lambda_tiles=False):
     i = np.asarray(rows)[:, None]
     j = np.arange(S)[None, :]
     if streaming:
         return (j <= i) & ((j <= sink) | (i - j < local))
-    return _kept(rows, S, streaming, sink, local, tm)
+    return _kept(rows, S, streaming, sink, local, tm, lambda_tiles)
 
 
-def kept_mask_transposed(rows, S, streaming, sink, local, tm):
+def kept_mask_transposed(rows, S, streaming, sink, local, tm, lambda_tiles=False):
     i = np.asarray(rows)[:, None]
     j = np.arange(S)[None, :]
     if not streaming and tm is not None:
         return (j <= i) & (np.asarray(tm)[j // 64, i // 64] != 0)
-    return _kept(rows, S, streaming, sink, local, tm)
+    return _kept(rows, S, streaming, sink, local, tm, lambda_tiles)
+
+
+def kept_tile_lambda_drops_causal(rows, S, streaming, sink, local, tm, lambda_tiles=False):
+    i = np.asarray(rows)[:, None]
+    j = np.arange(S)[None, :]
+    if streaming and lambda_tiles:   # whole kept tiles, the diagonal one included past the query
+        qt, kt = i // 64, j // 64
+        return (kt <= qt) & ((64 * kt < sink) | (np.maximum(64 * qt - 64 * kt - 63, 0) < local))
+    return _kept(rows, S, streaming, sink, local, tm, lambda_tiles)
 
 
 def bounds_kmax_only(q, stats, page_table, seq_len, b, h, G):
@@ -90,12 +99,12 @@ _stats = Sel.page_stats
 _token_set = D.token_set
 
 
-def cra_mean_not_min(q, k, v, head_kind, sink, local, block_mask=None, scale=None, rows=None):
-    return CR.retained_mass(q, k, v, head_kind, sink, local, block_mask, scale, rows).mean(axis=2)
+def cra_mean_not_min(q, k, v, head_kind, sink, local, block_mask=None, scale=None, rows=None, lambda_tiles=False):
+    return CR.retained_mass(q, k, v, head_kind, sink, local, block_mask, scale, rows, lambda_tiles).mean(axis=2)
 
 
-def retained_inverted(q, k, v, head_kind, sink, local, block_mask=None, scale=None, rows=None):
-    return 1.0 / _retained(q, k, v, head_kind, sink, local, block_mask, scale, rows)
+def retained_inverted(q, k, v, head_kind, sink, local, block_mask=None, scale=None, rows=None, lambda_tiles=False):
+    return 1.0 / _retained(q, k, v, head_kind, sink, local, block_mask, scale, rows, lambda_tiles)
 
 
 _retained = CR.retained_mass
@@ -125,6 +134,8 @@ CASES = [
      lambda: TA.test_streaming_equals_sdpa_with_lambda_mask(3, 1)),
     ("block mask transposed", A, "kept_mask", kept_mask_transposed,
      TA.test_block_mask_equals_sdpa_with_expanded_mask),
+    ("tile-level Lambda drops the causal mask", A, "kept_mask", kept_tile_lambda_drops_causal,
+     lambda: TA.test_tile_level_lambda_brute_force(64, 256)),
     ("no softmax scale", A, "masked_attention", masked_no_scale,
      lambda: TA.test_all_tiles_kept_equals_dense_causal(2)),
     ("bound drops kmin", Sel, "logical_bounds", bounds_kmax_only,

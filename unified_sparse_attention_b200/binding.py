@@ -57,7 +57,8 @@ class LServeError(RuntimeError):
 
 class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("S", ctypes.c_int32), ("Hq", ctypes.c_int32),
-                ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("scale", ctypes.c_float)]
+                ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("lambda_tiles", ctypes.c_int32)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -159,18 +160,20 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.
 
 # ---------------------------------------------------------------- prefill
 
-def _shape(q, k, scale):
+def _shape(q, k, scale, lambda_tiles=False):
     B, S, Hq, d = q.shape
-    return Shape(B, S, Hq, k.shape[2], d, float(scale))
+    return Shape(B, S, Hq, k.shape[2], d, float(scale), 1 if lambda_tiles else 0)
 
 
 def lserve_prefill_workspace_size(B: int, S: int, Hq: int, Hkv: int, d: int) -> int:
-    return int(load_library().lserve_prefill_workspace_size(ctypes.byref(Shape(B, S, Hq, Hkv, d, 0.0))))
+    return int(load_library().lserve_prefill_workspace_size(ctypes.byref(Shape(B, S, Hq, Hkv, d, 0.0, 0))))
 
 
 def lserve_prefill(q, k, v, head_kind, sink: int, local: int, block_mask=None, out=None, lse=None,
-                   scale: float = 0.0, workspace=None, stream=None, return_lse: bool = False):
-    """Block-sparse causal prefill; see include/lserve.h.  Returns out (and lse)."""
+                   scale: float = 0.0, workspace=None, stream=None, return_lse: bool = False,
+                   lambda_tiles: bool = False):
+    """Block-sparse causal prefill; see include/lserve.h.  Returns out (and lse).
+    lambda_tiles: streaming heads keep whole tiles of the Lambda support."""
     lib = load_library()
     _dev(q, "q", torch.bfloat16)
     B, S, Hq, d = q.shape
@@ -185,7 +188,7 @@ def lserve_prefill(q, k, v, head_kind, sink: int, local: int, block_mask=None, o
         lse = torch.empty(B, Hq, S, dtype=torch.float32, device=q.device)
     if lse is not None:
         _dev(lse, "lse", torch.float32, (B, Hq, S))
-    shape = _shape(q, k, scale)
+    shape = _shape(q, k, scale, lambda_tiles)
     need = int(lib.lserve_prefill_workspace_size(ctypes.byref(shape)))
     ws = _workspace(need, q.device, workspace)
     _check(lib.lserve_prefill(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(head_kind), int(sink),
@@ -195,11 +198,11 @@ def lserve_prefill(q, k, v, head_kind, sink: int, local: int, block_mask=None, o
 
 
 def lserve_cra_workspace_size(B: int, S: int, Hq: int, Hkv: int, d: int) -> int:
-    return int(load_library().lserve_cra_workspace_size(ctypes.byref(Shape(B, S, Hq, Hkv, d, 0.0))))
+    return int(load_library().lserve_cra_workspace_size(ctypes.byref(Shape(B, S, Hq, Hkv, d, 0.0, 0))))
 
 
 def lserve_cra(q, k, v, head_kind, sink: int, local: int, block_mask=None, scale: float = 0.0,
-               return_retained: bool = False, workspace=None, stream=None):
+               return_retained: bool = False, workspace=None, stream=None, lambda_tiles: bool = False):
     """Cumulative residual attention of a sparse prefill mask; see include/lserve.h.
     Returns cra fp32[B, Hq] (and the per-row retained mass fp32[B, Hq, S])."""
     lib = load_library()
@@ -213,7 +216,7 @@ def lserve_cra(q, k, v, head_kind, sink: int, local: int, block_mask=None, scale
         _dev(block_mask, "block_mask", torch.uint8, (B, Hkv, S // PAGE, S // PAGE))
     cra = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
     retained = torch.empty(B, Hq, S, dtype=torch.float32, device=q.device) if return_retained else None
-    shape = _shape(q, k, scale)
+    shape = _shape(q, k, scale, lambda_tiles)
     need = int(lib.lserve_cra_workspace_size(ctypes.byref(shape)))
     ws = _workspace(need, q.device, workspace)
     _check(lib.lserve_cra(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(head_kind), int(sink), int(local),
@@ -233,7 +236,7 @@ def lserve_prefill_tile_lists(B, S, Hq, Hkv, d, head_kind, sink, local, block_ma
     max_nnz = R * (n + 1) // 2
     offsets = torch.empty(R + 1, dtype=torch.int32, device=dev)
     cols = torch.empty(max(max_nnz, 1), dtype=torch.int16, device=dev)
-    shape = Shape(B, S, Hq, Hkv, d, 0.0)
+    shape = Shape(B, S, Hq, Hkv, d, 0.0, 0)
     ws = _workspace(lib.lserve_prefill_workspace_size(ctypes.byref(shape)), dev, None)
     _check(lib.lserve_prefill_tile_lists(ctypes.byref(shape), _ptr(head_kind), int(sink), int(local),
                                          _ptr(block_mask), _ptr(offsets), _ptr(cols), max_nnz, _ptr(ws),

@@ -211,6 +211,8 @@ lserve_status validate_prefill(const lserve_shape* s, int sink, int local) {
   if (static_cast<long long>(s->B) * s->S > (1ll << 31) - 1)
     return fail(LSERVE_ERR_UNSUPPORTED, "prefill: B*S too large");
   if (sink < 0 || local < 0) return fail(LSERVE_ERR_INVALID_ARG, "prefill: sink/local must be >= 0");
+  if (s->lambda_tiles != 0 && s->lambda_tiles != 1)
+    return fail(LSERVE_ERR_INVALID_ARG, "prefill: lambda_tiles must be 0 or 1");
   const long long R = static_cast<long long>(s->B) * s->Hkv * (s->S / kTile);
   if (R * (s->S / kTile + 1) / 2 > (1ll << 31) - 1) return fail(LSERVE_ERR_UNSUPPORTED, "prefill: too many tiles");
   return LSERVE_OK;
@@ -288,7 +290,8 @@ lserve_status run_prefill(const lserve_shape* shape, const void* q, const void* 
   const int nQT = shape->S / kTile;
   const float scale = shape->scale > 0.f ? shape->scale : 1.f / std::sqrt(static_cast<float>(shape->d));
   tc::PrefillArgs A{w.offsets, w.cols, w.order, head_kind, static_cast<bf16*>(out), lse, G,
-                shape->Hkv, nQT, shape->S, sink, local, scale * 1.4426950408889634f, wait_timeout_ns()};
+                shape->Hkv, nQT, shape->S, sink, local, scale * 1.4426950408889634f, wait_timeout_ns(),
+                shape->lambda_tiles ? 1 : 0};
   const TcPlan tp = tc_plan(G);
   // rows with a closed-form list (streaming heads; dense heads without a mask)
   // get no CSR entries: the kernel computes their tiles

@@ -67,6 +67,7 @@ struct PrefillArgs {
   int G, Hkv, nQT, S, sink, local;
   float scale_log2;             // softmax scale times log2(e)
   unsigned long long timeout_ns;
+  int lambda_tiles;             // streaming heads keep whole tiles (no element mask at the Lambda edges)
 };
 
 // ----------------------------------------------------------- tcgen05 wrappers
@@ -581,12 +582,14 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
                                 : nullptr;
       float m_run = kNegInf, l_run = 0.f;
       // keep mask of this row over one 64-key tile (bit c <-> key 64 kt + c)
+      // (with tile-level Lambda a kept tile of a streaming head is masked like a dense one: causally only)
+      const bool lam_edges = streaming && !A.lambda_tiles;
       auto tile_mask = [&](int kt) -> uint64_t {
         if (!rb_valid || !(T.QG == 1 || tile_keep(tp, streaming, mrow, qt, kt))) return 0ull;
-        if (tile_is_full(streaming, qt, kt, A.sink, A.local)) return ~0ull;
+        if (tile_is_full(lam_edges, qt, kt, A.sink, A.local)) return ~0ull;
         const int d0 = i - kt * kTile;   // offset of the query position inside the tile
         uint64_t k = bits_upto(d0);
-        if (streaming) k &= bits_below(A.sink - kt * kTile) | bits_from(d0 - A.local + 1);
+        if (lam_edges) k &= bits_below(A.sink - kt * kTile) | bits_from(d0 - A.local + 1);
         return k;
       };
       // raw scores of one 64-key half, masked keys set to -inf
