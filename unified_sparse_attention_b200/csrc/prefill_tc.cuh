@@ -323,6 +323,9 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   // two-slot ring; q_empty frees the Q buffer (all S MMAs of an item done), o_free
   // frees the O accumulators (both warpgroups have read them in the epilogue)
   __shared__ __align__(8) uint64_t item_full[2], item_empty[2], q_empty, o_free, mma_drain;
+  // ml_full[ii & 1]: both softmax warpgroups have published their (m, l) of item ii
+  // (a bounded wait, unlike a named barrier, so that no protocol slip can hang a CTA)
+  __shared__ __align__(8) uint64_t ml_full[2];
   __shared__ int s_item[2];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
@@ -353,6 +356,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       mbar_init(&o_done[x], 1);
       mbar_init(&item_full[x], 1);
       mbar_init(&item_empty[x], kItemReaders);
+      mbar_init(&ml_full[x], 256);
     }
     mbar_init(&q_empty, 1);
     mbar_init(&o_free, 256);
@@ -493,6 +497,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       auto issue_s = [&](int p) {   // S[p&1] = Q [K_a; K_b]^T
         const int gt = gk + p, st = gt % kKStages, x = p & 1;
         wait_or_abort(&k_full[st], (gt / kKStages) & 1, &s_abort, tmo);
+        __syncwarp();   // converged for elect.sync / tcgen05
         fence_after_sync();
 #pragma unroll
         for (int k4 = 0; k4 < D / 16; k4 += 4) {
@@ -520,6 +525,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         // PV(0) overwrites O[0] (and PV(1) O[1]): the previous item's epilogue must
         // have read both accumulators
         if (p == 0 && ii > 0) wait_or_abort(&o_free, (ii - 1) & 1, &s_abort, tmo);
+        __syncwarp();
         fence_after_sync();
 #pragma unroll
         for (int k4 = 0; k4 < 8; k4 += 4) {
@@ -622,6 +628,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         const uint64_t keep0 = tile_mask(kt0);
         const uint64_t keep1 = (2 * p + 1 < n) ? tile_mask(kt1) : 0ull;
         wait_or_abort(&s_full[x], (cs_own + j) & 1, &s_abort, tmo);
+        __syncwarp();   // converged for the warp-collective tcgen05 loads
         fence_after_sync();
         uint32_t v[64];
         uint32_t pk0[32], pk1[32];
@@ -676,7 +683,11 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         }
         float rsum = 0.f;
         bool ok = false;
-        if (m_run != kNegInf) {   // steady state: one pass against the current reference
+        // steady state: one pass against the current reference.  The branch is taken
+        // by the whole warp or not at all (the pass holds warp-collective TMEM loads
+        // and votes): a warp with any row still without a reference takes the exact
+        // row max below instead.
+        if (__all_sync(0xffffffffu, m_run != kNegInf)) {
           rsum = exp_pass(m_run);
           // every weight is at most the row sum: none near the fp32/bf16 limit (catches inf/NaN too)
           ok = !__any_sync(0xffffffffu, !(rsum <= 1099511627776.f));   // 2^40
@@ -717,6 +728,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         if (j > 0) {
           wait_or_abort(&o_done[x], (cs_own + j - 1) & 1, &s_abort, tmo);
           ++seen;
+          __syncwarp();
           fence_after_sync();
           if (__any_sync(0xffffffffu, f != 1.f)) {
   #pragma unroll 1
@@ -743,10 +755,14 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       }
       s_ml[ii & 1][x][0][row] = m_run;
       s_ml[ii & 1][x][1][row] = l_run;
-      // the other warpgroup observed its stream's last P.V before this barrier; the
-      // fences order that observation before this warpgroup's reads of O[x^1]
+      // the other warpgroup observed its stream's last P.V before it arrived; the
+      // fences order that observation before this warpgroup's reads of O[x^1].  The
+      // next phase of ml_full[ii & 1] (item ii + 2) needs this thread's arrival, so
+      // the parity wait is unambiguous.
       fence_before_sync();
-      asm volatile("bar.sync 1, 256;" ::: "memory");
+      mbar_arrive(&ml_full[ii & 1]);
+      wait_or_abort(&ml_full[ii & 1], (ii >> 1) & 1, &s_abort, tmo);
+      __syncwarp();   // converged for the warp-collective tcgen05 loads below
       fence_after_sync();
       const float m_o = s_ml[ii & 1][x ^ 1][0][row], l_o = s_ml[ii & 1][x ^ 1][1][row];
       const int nx_o = (np > (x ^ 1)) ? (np - (x ^ 1) + 1) >> 1 : 0;
