@@ -240,6 +240,102 @@ def time_loop(fn, steps, warmup, stream, scratch=None, events_per_step=1):
     return [s.elapsed_time(e) for s, e in zip(starts, ends)]
 
 
+# ------------------------------------------------------------ other configs
+
+def prefill_config(U, wl, dev, stream, steps, pk, fill=None, lambda_tiles=False, tensors=None):
+    """One prefill workload: median ms per call, kept-tile TFLOP/s and fraction of the bf16 peak."""
+    w = W.WORKLOADS[wl]
+    q, k, v = tensors if tensors is not None else W.prefill_inputs(w, device=dev)
+    bm = W.block_mask(w, device=dev, fill=fill) if (fill is not None or w.mask_fill is not None) else None
+    kind = W.head_kind(w)
+    hk = kind.to(dev)
+    tiles = kept_tile_counts(w, bm, kind.tolist())
+    flops = sum(tiles) * (w.Hq // w.Hkv) * 4 * 64 * 64 * w.d
+    out = torch.empty_like(q)
+    ws = torch.empty(U.lserve_prefill_workspace_size(w.B, w.S, w.Hq, w.Hkv, w.d), dtype=torch.uint8, device=dev)
+    fn = lambda: U.lserve_prefill(q, k, v, hk, w.sink, w.local, bm, out=out, workspace=ws, lambda_tiles=lambda_tiles)
+    ms = float(np.median(time_loop(fn, steps, 3, stream)))
+    n = w.S // 64
+    dense = [t for t, x in zip(tiles, kind.tolist()) if x == 0]
+    density = sum(dense) / max(1, len(dense) * n * (n + 1) // 2 * w.B)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"prefill_ms": ms, "kept_tile_tflop": flops / 1e12, "tflops": tf, "frac_bf16_peak": tf / pk["bf16"],
+            "dense_tile_density": density}
+
+
+def decode_config(U, wl, dev, stream, steps, pk, scratch):
+    """One decode workload: median µs per step (selection re-run), GB/s on the algorithmic bytes, fraction
+    of HBM, and the same step with L2 flushed before it."""
+    w = W.WORKLOADS[wl]
+    kind = W.head_kind(w)
+    pc = W.decode_cache(w, device=dev)
+    pt, sl, hk = pc.page_table.to(dev), pc.seq_lens.to(dev), kind.to(dev)
+    stats = U.lserve_update_page_stats(pc.k_pages, pt, sl, hk)
+    qd = W.decode_query(w, device=dev)
+    args = (qd, pc.k_pages, pc.v_pages, pt, sl, stats, hk, w.sink, w.local, w.token_budget)
+    ws = torch.empty(U.lserve_decode_workspace_size(*args), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(qd)
+    fn = lambda: U.lserve_decode(*args, out=out, workspace=ws)
+    us = float(np.median(time_loop(fn, steps, 3, stream))) * 1e3
+    us_fl = float(np.median(time_loop(fn, steps, 2, stream, scratch))) * 1e3
+    k_sel = min(w.token_budget // 64, (w.ctx + 63) // 64)
+    db = decode_bytes(w, kind.tolist(), k_sel, w.d)
+    gbs = db["total"] / (us * 1e-6) / 1e9
+    del pc, stats
+    return {"decode_us_per_step": us, "decode_bytes": db["total"], "GBps": gbs, "frac_hbm": gbs / pk["hbm"],
+            "decode_us_per_step_l2_flushed": us_fl,
+            "frac_hbm_l2_flushed": db["total"] / (us_fl * 1e-6) / 1e9 / pk["hbm"]}
+
+
+def other_configs(U, setup, dev, stream, steps, pk, scratch):
+    """The other workloads of the problem statement, measured in the same run (own inputs)."""
+    n = max(3, steps // 2)
+    res = {}
+    c1 = prefill_config(U, "llama3_8b_32k", dev, stream, n, pk)
+    c1.update(decode_config(U, "llama3_8b_32k", dev, stream, n, pk, scratch))
+    c1["note"] = "B1 S32768 Hq32/Hkv8: 4 dense (unmasked) + 4 streaming KV heads; decode 1 sequence, budget 4096 " \
+                 "(latency-bound: 13 MB per step)"
+    res["llama3_8b_32k"] = c1
+    res["llama3_8b_decode_b16_64k"] = decode_config(U, "llama3_8b_decode_b16_64k", dev, stream, n, pk, scratch)
+    res["llama3_8b_decode_b16_64k"]["note"] = "B16 ctx 65536 Hq32/Hkv8, 64 outlier-channel anchors, budget 4096"
+    torch.cuda.empty_cache()
+    c4 = prefill_config(U, "llama2_7b_mha", dev, stream, n, pk)
+    c4["note"] = "B1 S65536 Hq=Hkv=32: 16 dense (unmasked) + 16 streaming KV heads"
+    res["llama2_7b_mha_prefill_64k"] = c4
+    torch.cuda.empty_cache()
+    lit = prefill_config(U, "llama3_8b_prefill_128k_vslash_literal", dev, stream, n, pk,
+                         tensors=(setup.q, setup.k, setup.v))
+    lit["note"] = "the 128K recipe with the literal 5 % random fill (reading A)"
+    res["llama3_8b_prefill_128k_vslash_literal"] = lit
+    # tile-level Lambda on the default 128K workload: streaming heads keep whole tiles
+    lt = prefill_config(U, setup.prefill_wl, dev, stream, n, pk, tensors=(setup.q, setup.k, setup.v),
+                        lambda_tiles=True)
+    res["lambda_tiles_128k"] = {"prefill_ms": lt["prefill_ms"], "tflops": lt["tflops"],
+                                "note": "the default 128K prefill with tile-level Lambda on its streaming heads "
+                                        "(compare prefill_ms of the main line)"}
+    # vertical-slash mask construction from sampled queries on the 128K q/k
+    wp = setup.wp
+    stride, tau = 16, 0.95
+    ws = torch.empty(U.lserve_vslash_workspace_size(wp.B, wp.S, wp.Hq, wp.Hkv, wp.d, stride), dtype=torch.uint8,
+                     device=dev)
+    bm_out = torch.empty(wp.B, wp.Hkv, wp.S // 64, wp.S // 64, dtype=torch.uint8, device=dev)
+    fn = lambda: U.lserve_build_vslash_mask(setup.q, setup.k, setup.hk_p, stride, tau, block_mask=bm_out,
+                                            workspace=ws)
+    ms = float(np.median(time_loop(fn, n, 2, stream)))
+    _, cra, ncol, nsla = fn()
+    torch.cuda.synchronize()
+    nt = wp.S // 64
+    dense = [g for g in range(wp.Hkv) if setup.kind_p[g] == 0]
+    causal = torch.tril(torch.ones(nt, nt, dtype=torch.bool, device=dev))
+    dens = float(np.mean([float((bm_out[0, g].bool() & causal).sum()) / float(causal.sum()) for g in dense]))
+    res["vslash_mask_128k"] = {"ms": ms, "sample_stride": stride, "tau": tau, "dense_tile_density": dens,
+                               "sampled_cra_min": float(cra[0, dense].min()),
+                               "columns": [int(ncol[0, g]) for g in dense], "slashes": [int(nsla[0, g]) for g in dense],
+                               "note": "lserve_build_vslash_mask on the 128K q/k: last row of every 16th query tile "
+                                       "sampled, greedy columns/slashes until the sampled CRA reaches tau"}
+    return res
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 def oracle_prefill_sample(setup, seconds=10.0, seed=0):
@@ -319,6 +415,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true", help="skip the other workloads' fields")
     ap.add_argument("--prefill-wl", default=PREFILL_WL, choices=sorted(W.WORKLOADS))
     ap.add_argument("--decode-wl", default=DECODE_WL, choices=sorted(W.WORKLOADS))
     args = ap.parse_args()
@@ -415,6 +512,7 @@ def main():
     t_reuse = time_loop(decode_reuse, args.steps, args.warmup, stream, fl)
     t_int4 = time_loop(decode_int4, args.steps, args.warmup, stream, fl)
     t_quant = time_loop(quantize_pool, 2, 1, stream)   # once per page in a server: off the step
+    extra = None if args.no_other_configs else other_configs(U, setup, dev, stream, args.steps, pk, scratch)
 
     # the timed steps
     clocks = Clocks(local_rank)
@@ -545,6 +643,7 @@ def main():
                             "frac": gbps_decode / pk["hbm"],
                             "traffic": traffic("decode", wd.name == DECODE_WL), "traffic_unit": "bytes per step",
                             "algorithmic_bytes": setup.dbytes["total"], "peak_source": pk["source"]},
+        "other_configs": extra,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "e2e": e2e,

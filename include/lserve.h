@@ -169,6 +169,52 @@ lserve_status lserve_update_page_stats(int32_t B, int32_t Hkv, int32_t d, int32_
                                        void* stats, void* stream);
 
 /*
+ * lserve_build_vslash_mask -- a vertical-slash block mask for the dense heads,
+ * built from sampled queries.
+ *
+ * LServe + SampleAttention blog post, "SampleAttention - Column Pattern" and
+ * "Slash Pattern" (Fig. 3), with "CRA - The Accuracy Proxy" (Fig. 4): column
+ * and slash candidates are added until the worst-kept query keeps a share tau
+ * of its causal softmax mass.  The post leaves the estimator to its paper; this
+ * library's reading, at the 64 x 64 tile grain of lserve_prefill:
+ *   sampled queries  the last row of query tiles nQT-1, nQT-1-stride, ... (>= 0),
+ *                    each for the Hq/Hkv query heads of the KV head
+ *   tile masses      r[s,h,kt] = that row's causal softmax weights (exact, over
+ *                    all keys <= the row) summed over the keys of tile kt
+ *   candidates       column kt (tiles (qt, kt), qt >= kt), score sum_{s,h} r[s,h,kt];
+ *                    slash delta (tiles (qt, qt - delta)), score sum_{s,h} r[s,h,qt(s)-delta]
+ *   greedy           the diagonal slash (delta = 0) first, always; then by score,
+ *                    descending (equal scores: columns first, then the lower
+ *                    index); stop as soon as min over (s, h) of the retained mass
+ *                    (r summed over the row's covered tiles) is >= tau
+ *   mask             block_mask[b,g,qt,kt] = 1 for kt <= qt covered by a taken
+ *                    column or slash, else 0
+ * Streaming heads get an all-zero mask (lserve_prefill ignores it for them),
+ * cra 0 and no candidates.  The mask is ready to pass to lserve_prefill and
+ * lserve_cra.
+ *
+ *   q, k           bf16 [B, S, Hq, d], [B, S, Hkv, d]; S a multiple of 64, d in {64, 128}
+ *   head_kind      uint8 [Hkv]                   (device)
+ *   sample_stride  >= 1; (S/64 - 1)/stride + 1 rows sampled per (sequence, KV head);
+ *                  rows x Hq/Hkv at most 16384, Hq/Hkv at most 8, S/64 at most 8192
+ *   tau            in [0, 1]
+ *   block_mask     uint8 [B, Hkv, S/64, S/64]     (written)
+ *   cra            fp32 [B, Hkv] or NULL: the sampled rows' minimum retained mass
+ *   n_columns, n_slashes  int32 [B, Hkv] or NULL: candidates taken (the diagonal counts as a slash)
+ *   workspace      >= lserve_vslash_workspace_size(shape, stride) bytes, 256-byte
+ *                  aligned (the tile masses: B*Hkv*rows*Hq/Hkv*S/64 floats)
+ * Errors: LSERVE_ERR_INVALID_ARG (shape, stride < 1, tau outside [0, 1], null or
+ * misaligned pointers), LSERVE_ERR_UNSUPPORTED (d, S, Hq/Hkv or sample count past
+ * the limits above), LSERVE_ERR_WORKSPACE.  Asynchronous on the stream.
+ */
+size_t lserve_vslash_workspace_size(const lserve_shape* shape, int32_t sample_stride);
+lserve_status lserve_build_vslash_mask(const lserve_shape* shape, const void* q, const void* k,
+                                       const uint8_t* head_kind, int32_t sample_stride, float tau,
+                                       uint8_t* block_mask, float* cra, int32_t* n_columns,
+                                       int32_t* n_slashes, void* workspace, size_t ws_bytes,
+                                       void* stream);
+
+/*
  * lserve_cra -- cumulative residual attention of a sparse prefill mask.
  *
  * LServe + SampleAttention blog post, "CRA - The Accuracy Proxy", Fig. 4: for

@@ -126,3 +126,18 @@ def test_int4_reuse_and_cra_validation():
     assert lib.lserve_cra_workspace_size(shape(S=1000)) == 0   # S not a multiple of 64
     assert lib.lserve_cra_workspace_size(shape()) > 0
     assert lib.lserve_cra(shape(d=96), FAKE, FAKE, FAKE, FAKE, 0, 64, None, None, FAKE, FAKE, 1 << 30, None) == 2
+
+
+def test_vslash_validation():
+    lib = U.load_library()
+    assert lib.lserve_vslash_workspace_size(shape(), 1) > 0
+    assert lib.lserve_vslash_workspace_size(shape(), 0) == 0
+    call = lambda shp, stride=1, tau=0.9, ws=None, wsb=0: lib.lserve_build_vslash_mask(
+        shp, FAKE, FAKE, FAKE, stride, tau, FAKE, None, None, None, ws, wsb, None)
+    assert call(shape(), stride=0) == 1
+    assert call(shape(), tau=1.5) == 1
+    assert call(shape(), tau=float("nan")) == 1
+    assert call(shape(Hq=18, Hkv=2)) == 2          # Hq/Hkv = 9 > 8
+    assert call(shape(d=96)) == 2
+    assert call(shape()) == 3                      # no workspace
+    assert "vslash" in U.lserve_last_error_string()

@@ -18,6 +18,8 @@ from oracle import cra as CR
 from oracle import decode as D
 from oracle import quant as Q
 from oracle import selection as Sel
+from oracle import vslash as VS
+import test_oracle_vslash as TV
 
 _kept = A.kept_mask
 _bounds = Sel.logical_bounds
@@ -55,6 +57,15 @@ def kept_tile_lambda_drops_causal(rows, S, streaming, sink, local, tm, lambda_ti
         qt, kt = i // 64, j // 64
         return (kt <= qt) & ((64 * kt < sink) | (np.maximum(64 * qt - 64 * kt - 63, 0) < local))
     return _kept(rows, S, streaming, sink, local, tm, lambda_tiles)
+
+
+def vslash_covered_wrong_side(kind, idx, qt, kt):
+    return kt <= qt and ((kind == "column" and kt == idx) or (kind == "slash" and kt - qt == idx))
+
+
+def vslash_order_no_forced_diagonal(tiles, r):
+    order = _vs_order(tiles, r)
+    return sorted(order, key=lambda c: (-c[2], 0 if c[0] == "column" else 1, c[1]))
 
 
 def bounds_kmax_only(q, stats, page_table, seq_len, b, h, G):
@@ -108,6 +119,7 @@ def retained_inverted(q, k, v, head_kind, sink, local, block_mask=None, scale=No
 
 
 _retained = CR.retained_mass
+_vs_order = VS.candidate_order
 
 
 def codes_truncate(x, lo, s):
@@ -151,6 +163,10 @@ CASES = [
     ("CRA takes the mean", CR, "cra", cra_mean_not_min, TD.test_cra_is_one_without_dropping_and_matches_weight_sums),
     ("retained mass inverted", CR, "retained_mass", retained_inverted,
      TD.test_cra_is_one_without_dropping_and_matches_weight_sums),
+    ("vslash slash offset from the wrong side", VS, "covered", vslash_covered_wrong_side,
+     TV.test_hand_example_order_and_cra),
+    ("vslash diagonal not forced first", VS, "candidate_order", vslash_order_no_forced_diagonal,
+     TV.test_hand_example_order_and_cra),
     ("INT4 codes truncated", Q, "_codes", codes_truncate, TQ.test_codes_range_extremes_monotone_and_error_bound),
     ("INT4 step over 16 levels", Q, "_step", step_sixteen_levels,
      TQ.test_codes_range_extremes_monotone_and_error_bound),

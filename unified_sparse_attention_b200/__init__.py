@@ -21,6 +21,8 @@ from .binding import (  # noqa: F401
     lserve_quantize_pages_int4,
     lserve_cra,
     lserve_cra_workspace_size,
+    lserve_build_vslash_mask,
+    lserve_vslash_workspace_size,
     lserve_decode_workspace_size,
     lserve_get_device_status,
     lserve_last_error_string,

@@ -35,6 +35,8 @@ EXPORTED_SYMBOLS = (
     "lserve_prefill_tile_lists",
     "lserve_cra_workspace_size",
     "lserve_cra",
+    "lserve_vslash_workspace_size",
+    "lserve_build_vslash_mask",
     "lserve_update_page_stats",
     "lserve_decode_max_selected",
     "lserve_decode_workspace_size",
@@ -93,6 +95,9 @@ def load_library():
         "lserve_prefill": (i32, [ctypes.POINTER(Shape), vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
         "lserve_cra_workspace_size": (sz, [ctypes.POINTER(Shape)]),
         "lserve_cra": (i32, [ctypes.POINTER(Shape), vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
+        "lserve_vslash_workspace_size": (sz, [ctypes.POINTER(Shape), i32]),
+        "lserve_build_vslash_mask": (i32, [ctypes.POINTER(Shape), vp, vp, vp, i32, ctypes.c_float, vp, vp, vp, vp,
+                                           vp, sz, vp]),
         "lserve_prefill_tile_lists": (i32, [ctypes.POINTER(Shape), vp, i32, i32, vp, vp, vp, ctypes.c_int64,
                                             vp, sz, vp]),
         "lserve_update_page_stats": (i32, [i32, i32, i32, i32, vp, vp, i32, vp, i32, vp, vp, vp]),
@@ -222,6 +227,37 @@ def lserve_cra(q, k, v, head_kind, sink: int, local: int, block_mask=None, scale
     _check(lib.lserve_cra(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(head_kind), int(sink), int(local),
                           _ptr(block_mask), _ptr(retained), _ptr(cra), _ptr(ws), ws.numel(), _stream(stream)))
     return (cra, retained) if return_retained else cra
+
+
+def lserve_vslash_workspace_size(B: int, S: int, Hq: int, Hkv: int, d: int, sample_stride: int) -> int:
+    return int(load_library().lserve_vslash_workspace_size(ctypes.byref(Shape(B, S, Hq, Hkv, d, 0.0, 0)),
+                                                           int(sample_stride)))
+
+
+def lserve_build_vslash_mask(q, k, head_kind, sample_stride: int, tau: float, scale: float = 0.0, block_mask=None,
+                             workspace=None, stream=None):
+    """Vertical-slash block mask of the dense heads from sampled queries; see include/lserve.h.
+    Returns (block_mask uint8[B, Hkv, S/64, S/64], cra fp32[B, Hkv], n_columns, n_slashes int32[B, Hkv])."""
+    lib = load_library()
+    _dev(q, "q", torch.bfloat16)
+    B, S, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _dev(k, "k", torch.bfloat16, (B, S, Hkv, d))
+    _dev(head_kind, "head_kind", torch.uint8, (Hkv,))
+    n = S // PAGE
+    dev = q.device
+    block_mask = torch.empty(B, Hkv, n, n, dtype=torch.uint8, device=dev) if block_mask is None else \
+        _dev(block_mask, "block_mask", torch.uint8, (B, Hkv, n, n))
+    cra = torch.empty(B, Hkv, dtype=torch.float32, device=dev)
+    ncol = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+    nsla = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+    shape = _shape(q, k, scale)
+    need = int(lib.lserve_vslash_workspace_size(ctypes.byref(shape), int(sample_stride)))
+    ws = _workspace(max(need, 1), dev, workspace)
+    _check(lib.lserve_build_vslash_mask(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(head_kind), int(sample_stride),
+                                        float(tau), _ptr(block_mask), _ptr(cra), _ptr(ncol), _ptr(nsla), _ptr(ws),
+                                        ws.numel(), _stream(stream)))
+    return block_mask, cra, ncol, nsla
 
 
 def lserve_prefill_tile_lists(B, S, Hq, Hkv, d, head_kind, sink, local, block_mask=None, stream=None):

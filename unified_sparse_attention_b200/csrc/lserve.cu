@@ -22,6 +22,7 @@
 #include "quant.cuh"
 #include "select.cuh"
 #include "tile_lists.cuh"
+#include "vslash.cuh"
 
 using namespace lserve;
 
@@ -475,6 +476,28 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
   return check_launch("decode");
 }
 
+// ------------------------------------------------------- vertical-slash masks
+lserve_status validate_vslash(const lserve_shape* s, int stride, float tau) {
+  if (!shape_valid(s)) return fail(LSERVE_ERR_INVALID_ARG, "vslash: invalid shape");
+  if (s->d != 64 && s->d != 128) return fail(LSERVE_ERR_UNSUPPORTED, "vslash: head dim %d not in {64,128}", s->d);
+  if (s->S % kTile) return fail(LSERVE_ERR_UNSUPPORTED, "vslash: S=%d is not a multiple of 64", s->S);
+  if (stride < 1) return fail(LSERVE_ERR_INVALID_ARG, "vslash: sample stride must be >= 1");
+  if (!(tau >= 0.f && tau <= 1.f)) return fail(LSERVE_ERR_INVALID_ARG, "vslash: tau must lie in [0, 1]");
+  const int nQT = s->S / kTile, G = s->Hq / s->Hkv;
+  if (G > kVsMaxG) return fail(LSERVE_ERR_UNSUPPORTED, "vslash: Hq/Hkv=%d above %d", G, kVsMaxG);
+  if (nQT > kVsMaxTiles) return fail(LSERVE_ERR_UNSUPPORTED, "vslash: S=%d above %d tiles", s->S, kVsMaxTiles);
+  if (static_cast<long long>(vs_rows(nQT, stride)) * G > kVsMaxEntries)
+    return fail(LSERVE_ERR_UNSUPPORTED, "vslash: %d sampled rows x %d heads above %d; raise the stride",
+                vs_rows(nQT, stride), G, kVsMaxEntries);
+  if (static_cast<long long>(s->B) * s->Hkv > 65535) return fail(LSERVE_ERR_UNSUPPORTED, "vslash: B*Hkv too large");
+  return LSERVE_OK;
+}
+
+size_t vslash_ws_bytes(const lserve_shape* s, int stride) {
+  const long long nQT = s->S / kTile, G = s->Hq / s->Hkv;
+  return static_cast<size_t>(s->B) * s->Hkv * vs_rows(static_cast<int>(nQT), stride) * G * nQT * sizeof(float) + 256;
+}
+
 }  // namespace
 
 // ------------------------------------------------- decode without a workspace
@@ -582,6 +605,45 @@ lserve_status lserve_prefill(const lserve_shape* shape, const void* q, const voi
                 lserve_prefill_workspace_size(shape));
   s = run_prefill(shape, q, k, v, head_kind, sink, local, block_mask, out, lse, workspace,
                   static_cast<cudaStream_t>(stream));
+  return s == LSERVE_OK ? ok() : s;
+}
+
+size_t lserve_vslash_workspace_size(const lserve_shape* shape, int32_t sample_stride) {
+  if (validate_vslash(shape, sample_stride, 0.f) != LSERVE_OK) return 0;
+  return vslash_ws_bytes(shape, sample_stride);
+}
+
+lserve_status lserve_build_vslash_mask(const lserve_shape* shape, const void* q, const void* k,
+                                       const uint8_t* head_kind, int32_t sample_stride, float tau,
+                                       uint8_t* block_mask, float* cra, int32_t* n_columns, int32_t* n_slashes,
+                                       void* workspace, size_t ws_bytes, void* stream) {
+  lserve_status s = validate_vslash(shape, sample_stride, tau);
+  if (s != LSERVE_OK) return s;
+  if (!q || !k || !head_kind || !block_mask) return fail(LSERVE_ERR_INVALID_ARG, "vslash: null tensor pointer");
+  if (!aligned16(q) || !aligned16(k)) return fail(LSERVE_ERR_INVALID_ARG, "vslash: q/k must be 16-byte aligned");
+  const size_t need = vslash_ws_bytes(shape, sample_stride);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < need)
+    return fail(LSERVE_ERR_WORKSPACE, "vslash: workspace missing, misaligned or smaller than %zu bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int nQT = shape->S / kTile, G = shape->Hq / shape->Hkv, n_rows = vs_rows(nQT, sample_stride);
+  const float scale = shape->scale > 0.f ? shape->scale : 1.f / std::sqrt(static_cast<float>(shape->d));
+  float* r = static_cast<float*>(workspace);
+  const dim3 grid_m(n_rows, shape->B * shape->Hkv);
+  if (shape->d == 128)
+    vslash_mass_kernel<128><<<grid_m, kVsThreads, 0, st>>>(static_cast<const bf16*>(q), static_cast<const bf16*>(k),
+                                                          head_kind, shape->S, shape->Hkv, G, nQT, sample_stride,
+                                                          n_rows, scale * 1.4426950408889634f, r);
+  else
+    vslash_mass_kernel<64><<<grid_m, kVsThreads, 0, st>>>(static_cast<const bf16*>(q), static_cast<const bf16*>(k),
+                                                         head_kind, shape->S, shape->Hkv, G, nQT, sample_stride,
+                                                         n_rows, scale * 1.4426950408889634f, r);
+  s = check_launch("vslash tile masses");
+  if (s != LSERVE_OK) return s;
+  const size_t smem = vs_greedy_smem(n_rows * G, nQT);
+  ensure_smem(vslash_greedy_kernel, static_cast<int>(vs_greedy_smem(kVsMaxEntries, kVsMaxTiles)));
+  vslash_greedy_kernel<<<shape->B * shape->Hkv, kVsGreedyThreads, smem, st>>>(
+      r, head_kind, shape->Hkv, G, nQT, sample_stride, n_rows, tau, block_mask, cra, n_columns, n_slashes);
+  s = check_launch("vslash greedy");
   return s == LSERVE_OK ? ok() : s;
 }
 
