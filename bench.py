@@ -48,7 +48,7 @@ L2_BYTES = 126 * 1024 * 1024
 # the kernel sources hash as they did when the counters were taken.
 TRAFFIC = {
     "prefill": {"bytes": 3535284992,
-                "sources": ["prefill_tc.cuh", "prefill_mma.cuh", "tile_lists.cuh", "common.cuh", "lserve.cu"],
+                "sources": ["prefill_tc.cuh", "tile_lists.cuh", "common.cuh", "lserve.cu"],
                 "sha256": "54cd666b417c2fa7c423f9f076e7c3e5286e45e17d36d2ca046b15f1acc972e1"},
     "decode": {"bytes": 822210048,
                "sources": ["select.cuh", "decode.cuh", "page_stats.cuh", "common.cuh", "lserve.cu"],
@@ -64,7 +64,10 @@ def traffic(key, workload_is_default):
         return None
     h = hashlib.sha256()
     for f in t["sources"]:
-        with open(os.path.join(ROOT, "unified_sparse_attention_b200", "csrc", f), "rb") as fh:
+        path = os.path.join(ROOT, "unified_sparse_attention_b200", "csrc", f)
+        if not os.path.exists(path):
+            return None
+        with open(path, "rb") as fh:
             h.update(fh.read())
     return t["bytes"] if h.hexdigest() == t["sha256"] else None
 
@@ -287,53 +290,76 @@ def decode_config(U, wl, dev, stream, steps, pk, scratch):
             "frac_hbm_l2_flushed": db["total"] / (us_fl * 1e-6) / 1e9 / pk["hbm"]}
 
 
-def other_configs(U, setup, dev, stream, steps, pk, scratch):
-    """The other workloads of the problem statement, measured in the same run (own inputs)."""
+def other_configs(U, setup, dev, stream, steps, pk, scratch, names):
+    """The other workloads of the problem statement, and the next rows' features, measured in the same
+    run (own inputs).  `names`: the entries to run (all by default)."""
     n = max(3, steps // 2)
     res = {}
-    c1 = prefill_config(U, "llama3_8b_32k", dev, stream, n, pk)
-    c1.update(decode_config(U, "llama3_8b_32k", dev, stream, n, pk, scratch))
-    c1["note"] = "B1 S32768 Hq32/Hkv8: 4 dense (unmasked) + 4 streaming KV heads; decode 1 sequence, budget 4096 " \
-                 "(latency-bound: 13 MB per step)"
-    res["llama3_8b_32k"] = c1
-    res["llama3_8b_decode_b16_64k"] = decode_config(U, "llama3_8b_decode_b16_64k", dev, stream, n, pk, scratch)
-    res["llama3_8b_decode_b16_64k"]["note"] = "B16 ctx 65536 Hq32/Hkv8, 64 outlier-channel anchors, budget 4096"
-    torch.cuda.empty_cache()
-    c4 = prefill_config(U, "llama2_7b_mha", dev, stream, n, pk)
-    c4["note"] = "B1 S65536 Hq=Hkv=32: 16 dense (unmasked) + 16 streaming KV heads"
-    res["llama2_7b_mha_prefill_64k"] = c4
-    torch.cuda.empty_cache()
-    lit = prefill_config(U, "llama3_8b_prefill_128k_vslash_literal", dev, stream, n, pk,
-                         tensors=(setup.q, setup.k, setup.v))
-    lit["note"] = "the 128K recipe with the literal 5 % random fill (reading A)"
-    res["llama3_8b_prefill_128k_vslash_literal"] = lit
-    # tile-level Lambda on the default 128K workload: streaming heads keep whole tiles
-    lt = prefill_config(U, setup.prefill_wl, dev, stream, n, pk, tensors=(setup.q, setup.k, setup.v),
-                        lambda_tiles=True)
-    res["lambda_tiles_128k"] = {"prefill_ms": lt["prefill_ms"], "tflops": lt["tflops"],
-                                "note": "the default 128K prefill with tile-level Lambda on its streaming heads "
-                                        "(compare prefill_ms of the main line)"}
-    # vertical-slash mask construction from sampled queries on the 128K q/k
     wp = setup.wp
-    stride, tau = 16, 0.95
-    ws = torch.empty(U.lserve_vslash_workspace_size(wp.B, wp.S, wp.Hq, wp.Hkv, wp.d, stride), dtype=torch.uint8,
-                     device=dev)
-    bm_out = torch.empty(wp.B, wp.Hkv, wp.S // 64, wp.S // 64, dtype=torch.uint8, device=dev)
-    fn = lambda: U.lserve_build_vslash_mask(setup.q, setup.k, setup.hk_p, stride, tau, block_mask=bm_out,
-                                            workspace=ws)
-    ms = float(np.median(time_loop(fn, n, 2, stream)))
-    _, cra, ncol, nsla = fn()
-    torch.cuda.synchronize()
-    nt = wp.S // 64
-    dense = [g for g in range(wp.Hkv) if setup.kind_p[g] == 0]
-    causal = torch.tril(torch.ones(nt, nt, dtype=torch.bool, device=dev))
-    dens = float(np.mean([float((bm_out[0, g].bool() & causal).sum()) / float(causal.sum()) for g in dense]))
-    res["vslash_mask_128k"] = {"ms": ms, "sample_stride": stride, "tau": tau, "dense_tile_density": dens,
-                               "sampled_cra_min": float(cra[0, dense].min()),
-                               "columns": [int(ncol[0, g]) for g in dense], "slashes": [int(nsla[0, g]) for g in dense],
-                               "note": "lserve_build_vslash_mask on the 128K q/k: last row of every 16th query tile "
-                                       "sampled, greedy columns/slashes until the sampled CRA reaches tau"}
+    if "llama3_8b_32k" in names:
+        c1 = prefill_config(U, "llama3_8b_32k", dev, stream, n, pk)
+        c1.update(decode_config(U, "llama3_8b_32k", dev, stream, n, pk, scratch))
+        c1["note"] = "B1 S32768 Hq32/Hkv8: 4 dense (unmasked) + 4 streaming KV heads; decode 1 sequence, " \
+                     "budget 4096 (latency-bound: 13 MB per step)"
+        res["llama3_8b_32k"] = c1
+    if "llama3_8b_decode_b16_64k" in names:
+        res["llama3_8b_decode_b16_64k"] = decode_config(U, "llama3_8b_decode_b16_64k", dev, stream, n, pk, scratch)
+        res["llama3_8b_decode_b16_64k"]["note"] = "B16 ctx 65536 Hq32/Hkv8, 64 outlier-channel anchors, budget 4096"
+        torch.cuda.empty_cache()
+    if "llama2_7b_mha_prefill_64k" in names:
+        c4 = prefill_config(U, "llama2_7b_mha", dev, stream, n, pk)
+        c4["note"] = "B1 S65536 Hq=Hkv=32: 16 dense (unmasked) + 16 streaming KV heads"
+        res["llama2_7b_mha_prefill_64k"] = c4
+        torch.cuda.empty_cache()
+    if "literal" in names and wp.name == "llama3_8b_prefill_128k_vslash":
+        lit = prefill_config(U, "llama3_8b_prefill_128k_vslash_literal", dev, stream, n, pk,
+                             tensors=(setup.q, setup.k, setup.v))
+        lit["note"] = "the 128K recipe with the literal 5 % random fill (reading A)"
+        res["llama3_8b_prefill_128k_vslash_literal"] = lit
+    if "lambda_tiles" in names:
+        # tile-level Lambda on the prefill workload: streaming heads keep whole tiles
+        lt = prefill_config(U, wp.name, dev, stream, n, pk, tensors=(setup.q, setup.k, setup.v), lambda_tiles=True)
+        res["lambda_tiles"] = {"workload": wp.name, "prefill_ms": lt["prefill_ms"], "tflops": lt["tflops"],
+                               "note": "the prefill workload with tile-level Lambda on its streaming heads "
+                                       "(compare prefill_ms of the main line)"}
+    if "cra" in names:
+        # CRA report of the prefill workload's mask: a causal and a sparse LSE-only pass, then the reduction
+        fn = lambda: U.lserve_cra(setup.q, setup.k, setup.v, setup.hk_p, wp.sink, wp.local, setup.bm)
+        ms = float(np.median(time_loop(fn, max(2, n // 2), 2, stream)))
+        cra = fn()
+        torch.cuda.synchronize()
+        G = wp.Hq // wp.Hkv
+        dense_q = [h for h in range(wp.Hq) if setup.kind_p[h // G] == 0]
+        res["cra"] = {"workload": wp.name, "ms": ms, "cra_min_dense_heads": float(cra[0, dense_q].min()),
+                      "cra_min_streaming_heads": float(cra[0, [h for h in range(wp.Hq) if h not in dense_q]].min()),
+                      "note": "lserve_cra: one causal and one sparse LSE-only prefill pass and the reduction"}
+    if "vslash" in names:
+        # vertical-slash mask construction from sampled queries on the prefill workload's q/k
+        stride, tau = 16, 0.95
+        ws = torch.empty(U.lserve_vslash_workspace_size(wp.B, wp.S, wp.Hq, wp.Hkv, wp.d, stride), dtype=torch.uint8,
+                         device=dev)
+        bm_out = torch.empty(wp.B, wp.Hkv, wp.S // 64, wp.S // 64, dtype=torch.uint8, device=dev)
+        fn = lambda: U.lserve_build_vslash_mask(setup.q, setup.k, setup.hk_p, stride, tau, block_mask=bm_out,
+                                                workspace=ws)
+        ms = float(np.median(time_loop(fn, n, 2, stream)))
+        _, cra, ncol, nsla = fn()
+        torch.cuda.synchronize()
+        nt = wp.S // 64
+        dense = [g for g in range(wp.Hkv) if setup.kind_p[g] == 0]
+        causal = torch.tril(torch.ones(nt, nt, dtype=torch.bool, device=dev))
+        dens = float(np.mean([float((bm_out[0, g].bool() & causal).sum()) / float(causal.sum()) for g in dense]))
+        res["vslash_mask"] = {"workload": wp.name, "ms": ms, "sample_stride": stride, "tau": tau,
+                              "dense_tile_density": dens, "sampled_cra_min": float(cra[0, dense].min()),
+                              "columns": [int(ncol[0, g]) for g in dense],
+                              "slashes": [int(nsla[0, g]) for g in dense],
+                              "note": "lserve_build_vslash_mask: last row of every 16th query tile sampled, greedy "
+                                      "columns/slashes until the sampled CRA reaches tau (N(0,1) keys give near-"
+                                      "uniform attention, so little can be dropped)"}
     return res
+
+
+OTHER_CONFIGS = ("llama3_8b_32k", "llama3_8b_decode_b16_64k", "llama2_7b_mha_prefill_64k", "literal",
+                 "lambda_tiles", "cra", "vslash")
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -415,7 +441,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-other-configs", action="store_true", help="skip the other workloads' fields")
+    ap.add_argument("--other-configs", default="all",
+                    help="comma list of the other workloads / features to measure (all, none, or names from "
+                         "OTHER_CONFIGS)")
     ap.add_argument("--prefill-wl", default=PREFILL_WL, choices=sorted(W.WORKLOADS))
     ap.add_argument("--decode-wl", default=DECODE_WL, choices=sorted(W.WORKLOADS))
     args = ap.parse_args()
@@ -512,7 +540,9 @@ def main():
     t_reuse = time_loop(decode_reuse, args.steps, args.warmup, stream, fl)
     t_int4 = time_loop(decode_int4, args.steps, args.warmup, stream, fl)
     t_quant = time_loop(quantize_pool, 2, 1, stream)   # once per page in a server: off the step
-    extra = None if args.no_other_configs else other_configs(U, setup, dev, stream, args.steps, pk, scratch)
+    names = OTHER_CONFIGS if args.other_configs == "all" else \
+        tuple(x for x in args.other_configs.split(",") if x and x != "none")
+    extra = other_configs(U, setup, dev, stream, args.steps, pk, scratch, names) if names else None
 
     # the timed steps
     clocks = Clocks(local_rank)

@@ -679,7 +679,10 @@ lserve_status lserve_cra(const lserve_shape* shape, const void* q, const void* k
   if (s != LSERVE_OK) return s;
   s = run_prefill(shape, q, k, v, head_kind, sink, local, block_mask, nullptr, lse_sparse, workspace, st);
   if (s != LSERVE_OK) return s;
-  cra_reduce_kernel<<<shape->B * shape->Hq, kCraThreads, 0, st>>>(lse_sparse, lse_full, shape->S, retained, cra);
+  if (cudaMemsetAsync(cra, 0x7f, sizeof(float) * shape->B * shape->Hq, st) != cudaSuccess)
+    return fail(LSERVE_ERR_CUDA, "cra: memset failed");
+  const dim3 grid_r(shape->B * shape->Hq, (shape->S + kCraChunk - 1) / kCraChunk);
+  cra_reduce_kernel<<<grid_r, kCraThreads, 0, st>>>(lse_sparse, lse_full, shape->S, retained, cra);
   s = check_launch("cra reduction");
   return s == LSERVE_OK ? ok() : s;
 }

@@ -103,6 +103,10 @@ WORKLOADS = {
 # Half-length version of the long prefill (same recipe), sized for profiler captures.
 WORKLOADS["llama3_8b_prefill_64k_vslash"] = dataclasses.replace(
     WORKLOADS["llama3_8b_prefill_128k_vslash"], name="llama3_8b_prefill_64k_vslash", S=65536)
+# The MHA decode at 4 x 64K (a quarter of the context), sized for profiler captures of the
+# G = 1 scoring path: 4.3 GB of pool, 134 MB of summaries (more than L2 holds).
+WORKLOADS["llama2_7b_mha_decode_b4_64k"] = dataclasses.replace(
+    WORKLOADS["llama2_7b_mha"], name="llama2_7b_mha_decode_b4_64k", ctx=65536, pool_pages=4096)
 # The literal reading of the long-prefill mask (5 % random fill, ~6.5 % density).
 WORKLOADS["llama3_8b_prefill_128k_vslash_literal"] = dataclasses.replace(
     WORKLOADS["llama3_8b_prefill_128k_vslash"],
