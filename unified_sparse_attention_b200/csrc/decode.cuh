@@ -13,12 +13,17 @@
 // n_u follows from the sequence lengths alone, so one extra block of the top-k
 // grid builds this plan (decode_partition) while the other blocks select.
 //
-// paged_decode_kernel: one wave of CTAs (SMs x 2; x 3 for INT4 pages) that claim ranges from a
+// The top-k blocks also write the flat list itself, pre-resolved: entry f holds
+// (unit, logical page, physical page, sequence length and flags), so that the
+// attention kernel reads one 16-byte entry per page instead of chasing the
+// plan, the selection and the page table.
+//
+// paged_decode_kernel: one wave of CTAs (SMs x 2) that claim ranges from a
 // counter, so that SMs that run ahead take more.  Per CTA:
-//   * a resolver warp claims ranges and resolves their pages (unit, logical
-//     page, physical page, segment flags) into a shared-memory ring ahead of
-//     the loads; a range that crosses unit boundaries is cut into segments,
-//     one per unit;
+//   * a resolver warp claims ranges (the next claim in flight while one is
+//     copied) and copies their entries of the flat list into a shared-memory
+//     ring ahead of the loads, adding the range's own start and end; a range
+//     that crosses unit boundaries is cut into segments, one per unit;
 //   * an issuer warp streams each page's K and V (64 x d bf16 each, contiguous
 //     in the pool) through a 3-stage ring with TMA (128-byte swizzle), and the
 //     group's G query rows with a bulk copy at a segment start (full and empty
@@ -41,13 +46,17 @@
 // INT4 pages (paged_decode_kernel<D, true>, lserve_decode_int4; blog post,
 // "LServe - Decode Phase" and Fig. 2: INT4 KV cuts the bytes of every page).
 // A stage holds the page's K and V codes (d/2 bytes a row, in the order of the
-// operand fragments, so a lane loads its share with one or two 16-byte reads),
-// the key steps/offsets per channel and value steps/offsets per token (fp32),
-// and the q rows at a segment start.  The integer codes go straight into the
-// MMAs; the steps are folded into the other operand (s q, s p, each as two bf16
-// parts) and the offsets into one fp32 term per head.  With 12 KB stages the
-// ring is 5 deep, and q kept as bf16 pairs under a 112-register cap admits 3
-// CTAs per SM (grid SMs x 3).  Bytes per selected page: 64 * d + 1.5 KB (d = 128).
+// operand fragments, so a lane loads its share with 16-byte reads), the key
+// steps/offsets per channel, the value steps/offsets per token (fp32) and the
+// unit's q rows.  Each consumer warp takes whole pages (four 16-token tiles),
+// so a page's step fold and softmax reductions are done once.  The codes go
+// into fp16 MMAs as 1024 + code or 1024 + 16 code (one mask per code pair, the
+// nibble lying in the mantissa of 1024, whose ulp is 1), the steps fold into
+// the other operand (s q as fp16 hi + lo; s p as fp16), and the offsets into
+// one fp32 term per head; the 1024 terms are taken out by MMAs of a constant
+// 1024 operand with the same fp16 operands, so they cancel exactly.  Eight
+// 12 KB stages, two CTAs per SM.  Bytes per selected page: 64 * d + 1.5 KB
+// (d = 128).
 //
 // Bytes per selected page: 2 * 64 * d * 2 (K and V); the kernel is HBM-bound.
 // Tokens outside the attended set (past seq_len; outside the Lambda set of a
@@ -64,13 +73,13 @@
 namespace lserve {
 
 constexpr int kDecodeStages = 3;     // bf16 pages: ring depth (three 34 KB stages at d = 128)
-constexpr int kDecodeStagesQ4 = 5;   // INT4 pages: its consumers hold a stage through the key loop
+constexpr int kDecodeStagesQ4 = 8;   // INT4 pages: two pages in flight per consumer warp
 constexpr int kDecodeWarps = 4;                           // consumer warps
 constexpr int kIssuerWarp = kDecodeWarps;                  // issues the TMA loads
 constexpr int kResolverWarp = kDecodeWarps + 1;            // claims ranges, resolves their pages
 constexpr int kDecodeThreads = (kDecodeWarps + 2) * 32;
 constexpr int kDecodeCtasPerSm = 2;     // bf16 pages: the three-stage ring's shared memory admits two
-constexpr int kDecodeCtasPerSmQ4 = 3;   // INT4 pages: smaller stages; registers capped to admit three
+constexpr int kDecodeCtasPerSmQ4 = 2;   // INT4 pages: registers admit two
 constexpr int kDecodeMaxG = 8;
 constexpr int kRangesPerCta = 4;   // ranges of the flat page list per attention CTA
 constexpr int kMetaRing = 64;      // resolved pages buffered ahead of the loads
@@ -124,20 +133,27 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// Pages selected for unit u: known from the sequence length alone
+// (unit_selected(), the count topk_unit() writes), or a kept selection's size.
+__device__ __forceinline__ int unit_count(int u, const int32_t* __restrict__ seq_lens,
+                                          const uint8_t* __restrict__ head_kind, int Hkv, int maxP, int budget_pages,
+                                          int sink, int local, int kcap, const int32_t* sel_n_in) {
+  const bool dense = head_kind[u % Hkv] == LSERVE_HEAD_DENSE;
+  return (dense && sel_n_in) ? min(max(sel_n_in[u], 0), kcap)
+                             : unit_selected(seq_lens[u / Hkv], maxP, dense, budget_pages, sink, local, kcap);
+}
+
 // The plan of the attention grid, by one block (any multiple of 32 threads).
-// The selection sizes are known from the sequence lengths alone
-// (unit_selected(), the counts the top-k blocks write), so this runs beside
-// the top-k blocks instead of after them.  off[u] = pages selected before unit
-// u, off[units] = T; with Re = ranges_in_use(R, T) ranges sharing the pages,
-// range_unit[r] = unit holding flat position floor(r T / Re) for r < Re; the
-// range counter zeroed for the attention kernel.  Units with nothing selected
-// get their output here: out = 0, lse = -inf.
+// The selection sizes are known before the selection (unit_count()), so this
+// runs beside the top-k blocks instead of after them.  off[u] = pages selected
+// before unit u, off[units] = T; the range counter zeroed for the attention
+// kernel.  Units with nothing selected get their output here: out = 0,
+// lse = -inf.
 __device__ __forceinline__ void decode_partition(const int32_t* __restrict__ seq_lens,
                                                  const uint8_t* __restrict__ head_kind, int Hkv, int maxP,
-                                                 int budget_pages, int sink, int local, int units, int kcap, int R,
-                                                 int G, int D, int32_t* off, int32_t* range_unit,
-                                                 int32_t* range_counter, bf16* out, float* lse_out,
-                                                 const int32_t* sel_n_in) {
+                                                 int budget_pages, int sink, int local, int units, int kcap,
+                                                 int G, int D, int32_t* off, int32_t* range_counter, bf16* out,
+                                                 float* lse_out, const int32_t* sel_n_in) {
   __shared__ int s_warp[32];
   __shared__ int s_carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x, nw = nt >> 5;
@@ -145,12 +161,9 @@ __device__ __forceinline__ void decode_partition(const int32_t* __restrict__ seq
   __syncthreads();
   for (int base = 0; base < units; base += nt) {
     const int u = base + tid;
-    int v = 0;
-    if (u < units) {
-      const bool dense = head_kind[u % Hkv] == LSERVE_HEAD_DENSE;
-      v = (dense && sel_n_in) ? min(max(sel_n_in[u], 0), kcap)   // a kept selection's size
-                              : unit_selected(seq_lens[u / Hkv], maxP, dense, budget_pages, sink, local, kcap);
-    }
+    const int v = u < units ? unit_count(u, seq_lens, head_kind, Hkv, maxP, budget_pages, sink, local, kcap,
+                                         sel_n_in)
+                            : 0;
     int x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -181,43 +194,66 @@ __device__ __forceinline__ void decode_partition(const int32_t* __restrict__ seq
     *range_counter = 0;
   }
   __syncthreads();   // off[] of this block is visible to the block from here on
-  const long long Re = ranges_in_use(R, T);   // every range below Re gets >= 1 page
   for (int u = tid; u < units; u += nt) {
-    const long long a = off[u], e = off[u + 1];
-    if (e == a) {   // nothing selected: out = 0, lse = -inf
+    if (off[u + 1] == off[u]) {   // nothing selected: out = 0, lse = -inf
       for (int idx = 0; idx < G * D; idx += 8)
         *reinterpret_cast<uint4*>(out + static_cast<long>(u) * G * D + idx) = make_uint4(0u, 0u, 0u, 0u);
       if (lse_out)
         for (int h = 0; h < G; ++h) lse_out[static_cast<long>(u) * G + h] = kNegInf;
-      continue;
     }
-    // ranges whose share starts inside [a, e): ceil(a Re / T) .. ceil(e Re / T) - 1
-    const int r0 = static_cast<int>((a * Re + T - 1) / T);
-    const int r1 = static_cast<int>((e * Re + T - 1) / T) - 1;
-    for (int r = r0; r <= r1; ++r) range_unit[r] = u;
   }
 }
 
 // Selection step: blocks 0 .. units-1 select the pages of one unit each
 // (topk_unit; with a kept selection sel_in / sel_n_in the dense units copy
-// their rows instead); block `units` lays out the attention grid's work
-// (decode_partition), which does not depend on the selected pages.
+// their rows instead) and write the unit's entries of the flat list; block
+// `units` lays out the attention grid's work (decode_partition), which does not
+// depend on the selected pages.
 __global__ void __launch_bounds__(kTopkThreads, 2) topk_pages_kernel(
     const float* scores, int maxP, const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind,
-    int Hkv, int budget_pages, int sink, int local, int32_t* sel, int32_t* sel_n, int kcap, int units, int R, int G,
-    int D, int32_t* off, int32_t* range_unit, int32_t* range_counter, bf16* out, float* lse_out,
-    const int32_t* sel_in, const int32_t* sel_n_in) {
-  const int unit = blockIdx.x;
-  // sequence length and head kind are inputs of the step, not results of the scoring grid
+    const int32_t* __restrict__ page_table, int num_pages, int Hkv, int budget_pages, int sink, int local,
+    int32_t* sel, int32_t* sel_n, int kcap, int units, int G, int D, int32_t* off, int4* flat,
+    int32_t* range_counter, bf16* out, float* lse_out, const int32_t* sel_in, const int32_t* sel_n_in) {
+  __shared__ int s_part[kTopkThreads / 32];
+  const int unit = blockIdx.x, tid = threadIdx.x;
+  // sequence length, head kind and the unit's place in the flat list are inputs
+  // of the step, not results of the scoring grid: computed before the wait
   const int L = unit < units ? seq_lens[unit / Hkv] : 0;
   const bool dense = unit < units && head_kind[unit % Hkv] == LSERVE_HEAD_DENSE;
+  int start = 0;
+  if (unit < units) {
+    int part = 0;
+    for (int v = tid; v < unit; v += blockDim.x)
+      part += unit_count(v, seq_lens, head_kind, Hkv, maxP, budget_pages, sink, local, kcap, sel_n_in);
+    part = __reduce_add_sync(0xffffffffu, part);
+    if ((tid & 31) == 0) s_part[tid >> 5] = part;
+    __syncthreads();
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) start += s_part[w];
+  }
   pdl_wait();
   pdl_launch_dependents();   // the attention grid may get resident; it waits for this grid
-  if (unit < units)
-    topk_unit(scores, unit, maxP, L, dense, budget_pages, sink, local, sel, sel_n, kcap, sel_in, sel_n_in);
-  else
-    decode_partition(seq_lens, head_kind, Hkv, maxP, budget_pages, sink, local, units, kcap, R, G, D, off,
-                     range_unit, range_counter, out, lse_out, sel_n_in);
+  if (unit < units) {
+    const int m = topk_unit(scores, unit, maxP, L, dense, budget_pages, sink, local, sel, sel_n, kcap, sel_in,
+                            sel_n_in);
+    __syncthreads();   // the unit's selection row, written by every thread, is complete
+    const int32_t* row = sel + static_cast<long>(unit) * kcap;
+    const int b = unit / Hkv;
+    const int flags = dense ? 0 : kSegStreaming;
+    for (int j = tid; j < m; j += blockDim.x) {
+      const int pidx = row[j];
+      int phys = -1;
+      if (pidx >= 0 && pidx < maxP) {
+        const int p = page_table[static_cast<long>(b) * maxP + pidx];
+        if (p >= 0 && p < num_pages) phys = p;
+      }
+      if (phys < 0) report(LSERVE_ERR_DEVICE_BOUNDS);
+      flat[start + j] = make_int4(unit, pidx, phys,
+                                  (max(L, 0) << 3) | flags | (j == 0 ? kSegStart : 0) | (j == m - 1 ? kSegEnd : 0));
+    }
+  } else {
+    decode_partition(seq_lens, head_kind, Hkv, maxP, budget_pages, sink, local, units, kcap, G, D, off,
+                     range_counter, out, lse_out, sel_n_in);
+  }
 }
 
 // Spin (with short sleeps) until cond() holds; false (and LSERVE_ERR_DEVICE_TIMEOUT
@@ -238,43 +274,68 @@ __device__ __forceinline__ bool spin_until(F&& cond, uint64_t timeout_ns) {
   }
 }
 
-// Two INT4 codes, nibbles k and k + 4 of w, as the bf16 pair (128 + code): the
-// codes become the low mantissa bits of 128 = 2^7, whose bf16 ulp is 1.
-__device__ __forceinline__ uint32_t q4_pair(uint32_t w, int k) { return ((w >> (4 * k)) & 0x000F000Fu) | 0x43004300u; }
+// fp16 operands from INT4 code words.  Code pair j of a word sits in nibbles j
+// and j + 4 (bits 4j..4j+3 of each half-word); q4h_lo gives the pair in
+// nibbles 0, 4 as 1024 + code and q4h_hi the pair in nibbles 1, 5 as
+// 1024 + 16 code (fp16 1024 is 0x6400; its ulp is 1); the word shifted right
+// by 8 gives pairs 2 and 3 the same way.
+constexpr uint32_t kF16x2_1024 = 0x64006400u;
+__device__ __forceinline__ uint32_t q4h_lo(uint32_t w) { return (w & 0x000F000Fu) | kF16x2_1024; }
+__device__ __forceinline__ uint32_t q4h_hi(uint32_t w) { return (w & 0x00F000F0u) | kF16x2_1024; }
 
+// fp16 pair {low half a, high half b}, rounded to nearest even
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(b), "f"(a));
+  return d;
+}
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
+  float a, b;
+  asm("{\n.reg .f16 l, h;\nmov.b32 {l, h}, %2;\ncvt.f32.f16 %0, l;\ncvt.f32.f16 %1, h;\n}" : "=f"(a), "=f"(b) : "r"(v));
+  return make_float2(a, b);
+}
+// x = hi + lo with hi, lo fp16 pairs (about 22 significant bits together)
+__device__ __forceinline__ void split_f16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_f16x2(a, b);
+  const float2 h = unpack_f16x2(hi);
+  lo = pack_f16x2(a - h.x, b - h.y);
+}
+// D = A(16x16, row) * B(16x8, col) + D, fp16 inputs, fp32 accumulators (no side
+// effects, so that the compiler may interleave independent chains)
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 
 // Q4 = false: bf16 pages (tmK, tmV over [NP * Hkv * 64, d] bf16).  Q4 = true:
 // INT4 pages (tmK, tmV over [NP * Hkv * 64, d/2] bytes) with their steps and
 // offsets kpar, vpar (layouts in quant.cuh).  The steps fold into the other
-// operand, so the tensor cores multiply integer codes (exact in bf16, offset by
-// the 128 of q4_pair) and the offsets go into one fp32 term per head:
-//   q.k_t = sum_c (128 + code_tc) (s_c q_c) + sum_c (lo_c - 128 s_c) q_c
-//     with s q split into two bf16 parts (hi + lo, two MMAs), so the logits
-//     carry a rounding of about 2^-18 of each product;
-//   sum_t p_t v_t = sum_t (128 + code_tc) (s_t p_t) + sum_t (lo_t - 128 s_t) p_t
-//     with s p split the same way.
-// One bf16 rounding of s q or s p would scale with |x - lo| (or the step of an
-// outlier-wide group), not with |x|; the split keeps it near 2^-18.
+// operand, so the tensor cores multiply integer codes (exact in fp16, offset by
+// 1024, with the multiplier m = 1 or 16 of their nibble position):
+//   q.k_t = sum_c (1024 + m_c code_tc) (s_c q_c / m_c) + sum_c lo_c q_c - 1024 sum_c (s_c q_c / m_c)
+//     with s q / m as two fp16 parts (hi + lo, two MMAs);
+//   sum_t p_t v_tc = ((sum_t (1024 + m_c code_tc) (s_t p_t)) - 1024 sum_t (s_t p_t)) / m_c + sum_t lo_t p_t
+//     with s p as one fp16 part (its rounding, 2^-11, is finer than the bf16 P of bf16 pages).
 template <int D, bool Q4 = false>
-__global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) paged_decode_kernel(
+__global__ void __launch_bounds__(kDecodeThreads, 2) paged_decode_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-    const bf16* __restrict__ q, const int32_t* __restrict__ page_table, int maxP,
-    const int32_t* __restrict__ seq_lens, const uint8_t* __restrict__ head_kind,
-    const int32_t* sel, const int32_t* off, const int32_t* range_unit, int32_t* range_counter, int R,
-    int kcap, int units, int Hkv, int G, int num_pages, int sink, int local, float scale_log2,
+    const bf16* __restrict__ q, const int4* flat, const int32_t* off, int32_t* range_counter, int R,
+    int kcap, int units, int Hkv, int G, int sink, int local, float scale_log2,
     unsigned long long timeout_ns, int debug_stall, float* __restrict__ part_o, float* __restrict__ part_lse,
     const float* __restrict__ kpar = nullptr, const float* __restrict__ vpar = nullptr) {
   using Cfg = DecodeCfg<D>;
   constexpr int NS = Q4 ? kDecodeStagesQ4 : kDecodeStages;   // ring depth
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[NS];    // stage loaded (issuer's expect_tx + bytes)
-  __shared__ __align__(8) uint64_t empty_bar[NS];   // stage consumed (one arrive per consumer warp)
+  __shared__ __align__(8) uint64_t empty_bar[NS];   // stage consumed (bf16: one arrive per consumer warp; INT4: one)
   __shared__ int4 s_meta[kMetaRing];   // {unit, logical page, physical page (-1: invalid), seq_len << 3 | flags}
-  __shared__ int4 s_seg[kMetaRing];    // {range, first range of the unit, last range of the unit, -}
+  __shared__ int s_range[kMetaRing];   // range of each ring entry (its partial slot is range + unit)
   __shared__ int s_resolved;           // pages whose metadata is in the ring
   __shared__ int s_total;              // pages this CTA processes (INT_MAX until the ranges run out)
   __shared__ int s_issued;             // pages whose loads were issued
   __shared__ int s_abort;              // a bounded wait ran out or the plan was inconsistent
+  __shared__ int s_seen[kDecodeWarps]; // INT4: pages whose metadata each consumer warp has read
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int stage_bytes = Q4 ? Cfg::stage_bytes_q4(G) : Cfg::stage_bytes(G);
   const int q_bytes = G * D * 2;
@@ -284,19 +345,21 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) pa
     prefetch_tensormap(&tmV);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], kDecodeWarps);
+      mbar_init(&empty_bar[s], Q4 ? 1 : kDecodeWarps);   // INT4: one warp consumes a page
     }
     fence_barrier_init();
     s_resolved = 0;
     s_total = INT_MAX;
     s_issued = 0;
     s_abort = 0;
+    for (int w = 0; w < kDecodeWarps; ++w) s_seen[w] = 0;
   }
   __syncthreads();
   volatile int* v_resolved = &s_resolved;
   volatile int* v_total = &s_total;
   volatile int* v_issued = &s_issued;
   volatile int* v_abort = &s_abort;
+  volatile int* v_seen = s_seen;
   // off / range_unit / the selection come from the previous kernels, which may
   // still be running: they are read only after this wait, with L2 loads through
   // pointers that are not restrict-qualified (no load of them can move above it).
@@ -312,98 +375,55 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) pa
     // failure-detection test: publish nothing, so that every other wait of the
     // CTA runs out (nothing is issued, so nothing is in flight when it leaves)
   } else if (warp == kResolverWarp) {
-    // ---- claim ranges one after another and resolve their pages into the ring.
-    // Window: unit wu + l (lane l) ends at flat position wend (INT_MAX past the
-    // last unit); the window is shifted so that it always starts at the unit of
-    // the next page to resolve.
-    int gp = 0;   // pages resolved
-    bool ok = true, stopped = false;   // !ok: inconsistent plan; stopped: the CTA is giving up
+    // ---- claim ranges and copy their entries of the flat list into the ring,
+    // adding each range's own start and end to the unit's; the next claim is in
+    // flight while a range is copied, and a batch's entries are loaded before
+    // the wait for room in the ring
+    int gp = 0;   // pages in the ring so far
+    bool ok = true, stopped = false;   // !ok: inconsistent entry; stopped: the CTA is giving up
+    int r_next = 0;
+    if (lane == 0) r_next = atomicAdd(range_counter, 1);
     while (ok && !stopped) {
-      int r = 0;
-      if (lane == 0) r = atomicAdd(range_counter, 1);
-      r = __shfl_sync(0xffffffffu, r, 0);
+      const int r = __shfl_sync(0xffffffffu, r_next, 0);
       if (r >= Re) break;
+      if (lane == 0) r_next = atomicAdd(range_counter, 1);
       const int lo = static_cast<int>(r * T / Re), hi = static_cast<int>((r + 1) * T / Re);
-      int wu = __ldcg(range_unit + r);
-      if (wu < 0 || wu >= units) {
-        ok = false;
-        break;
-      }
-      int wstart = __ldcg(off + wu);
-      int wend = wu + lane < units ? __ldcg(off + wu + lane + 1) : INT_MAX;
-      int f0 = lo;
-      while (f0 < hi && ok && !stopped) {
-        // shift the window to the unit of f0
-        int k0 = 0;
-#pragma unroll 8
-        for (int l = 0; l < 32; ++l) k0 += __shfl_sync(0xffffffffu, wend, l) <= f0;
-        if (k0 > 0) {
-          wu += k0;
-          if (wu >= units) {
-            ok = false;
-            break;
-          }
-          wstart = __ldcg(off + wu);
-          wend = wu + lane < units ? __ldcg(off + wu + lane + 1) : INT_MAX;
-          continue;
-        }
-        if (wstart > f0) {
-          ok = false;
-          break;
-        }
-        // page f of this lane lies in unit wu + k (k < 32 inside the window)
-        const int f = f0 + lane;
-        int k = 0;
-#pragma unroll 8
-        for (int l = 0; l < 32; ++l) k += __shfl_sync(0xffffffffu, wend, l) <= f;
-        const int kk = min(k, 31);
-        const int end_k = __shfl_sync(0xffffffffu, wend, kk);
-        const int prev_end = __shfl_sync(0xffffffffu, wend, max(kk - 1, 0));
-        const bool act = f < hi && k < 32;   // a prefix of the lanes
-        const int cnt = __popc(__ballot_sync(0xffffffffu, act));
-        // ring entries gp .. gp + cnt - 1 are free once page (entry - ring) is past the consumers
+      for (int f0 = lo; f0 < hi; f0 += 32) {
+        const int f = f0 + lane, cnt = min(32, hi - f0);
+        int4 e = make_int4(-1, 0, -1, 0);
+        if (f < hi) e = __ldcg(flat + f);
         bool room = true;
         if (lane == 0)
-          room = spin_until([&] { return *v_issued >= gp + cnt - kMetaRing + NS || *v_abort; },
-                            timeout_ns) && !*v_abort;
+          room = spin_until(
+                     [&] {
+                       if (*v_abort) return true;
+                       const int need = gp + cnt - kMetaRing;   // entries of pages below it are reused
+                       if (*v_issued < need + NS) return false;
+                       if constexpr (Q4) {   // INT4 consumers read every page's entry, their own or not
+                         for (int w = 0; w < kDecodeWarps; ++w)
+                           if (v_seen[w] < need) return false;
+                       }
+                       return true;
+                     },
+                     timeout_ns) && !*v_abort;
         if (!__shfl_sync(0xffffffffu, room, 0)) {
           stopped = true;
           break;
         }
-        bool bad = false;
-        if (act) {
-          const int u = wu + k;
-          const int start = k == 0 ? wstart : prev_end;
-          const int j = f - start, n_u = end_k - start;
-          bad = j < 0 || j >= n_u || n_u > kcap;
-          int pidx = -1, phys = -1, flags = 0, L = 0;
-          int c_first = 0, c_last = -1;
-          if (!bad) {
-            const int b = u / Hkv, g = u % Hkv;
-            pidx = __ldcg(sel + static_cast<long>(u) * kcap + j);
-            if (pidx >= 0 && pidx < maxP) {
-              const int p = page_table[static_cast<long>(b) * maxP + pidx];
-              if (p >= 0 && p < num_pages) phys = p;
-            }
-            if (phys < 0) report(LSERVE_ERR_DEVICE_BOUNDS);
-            L = seq_lens[b];
-            flags = ((j == 0 || f == lo) ? kSegStart : 0) | ((j == n_u - 1 || f == hi - 1) ? kSegEnd : 0) |
-                    (head_kind[g] != LSERVE_HEAD_DENSE ? kSegStreaming : 0);
-            c_first = flat_owner(start, T, Re);
-            c_last = flat_owner(start + n_u - 1, T, Re);
-          }
-          const int e = (gp + lane) % kMetaRing;
-          s_meta[e] = make_int4(u, pidx, phys, (max(L, 0) << 3) | flags);
-          s_seg[e] = make_int4(r, c_first, c_last, 0);
-        }
+        const bool bad = f < hi && (e.x < 0 || e.x >= units);
         if (__any_sync(0xffffffffu, bad)) {
           ok = false;
           break;
         }
+        if (f < hi) {
+          e.w |= (f == lo ? kSegStart : 0) | (f == hi - 1 ? kSegEnd : 0);
+          const int slot = (gp + lane) % kMetaRing;
+          s_meta[slot] = e;
+          s_range[slot] = r;
+        }
         __syncwarp();
         __threadfence_block();
         gp += cnt;
-        f0 += cnt;
         if (lane == 0) *v_resolved = gp;
       }
     }
@@ -433,7 +453,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) pa
         const int g = md.x % Hkv;
         const int p = md.z >= 0 ? md.z : 0;   // an invalid page loads page 0; all its tokens are masked
         uint8_t* kdst = smem + st * stage_bytes;
-        const bool with_q = md.w & kSegStart;
+        const bool with_q = Q4 || (md.w & kSegStart);   // INT4: every page carries q (its warp folds it)
         const int row = (p * Hkv + g) * kPage;
         if constexpr (Q4) {
           mbar_arrive_expect_tx(&full_bar[st], Cfg::kQ4Q + (with_q ? q_bytes : 0));
@@ -457,17 +477,272 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) pa
       }
     }
     __syncwarp();
+  } else if constexpr (Q4) {
+    // ---- INT4 consumers: warp w takes the pages gp = w (mod 4) whole (four
+    // 16-token tiles), so that a page's step fold, softmax reductions and
+    // offsets' terms are computed once per page and its four tiles give the
+    // tensor-core chains independent work.  Every warp reads every page's
+    // metadata, keeps its own online softmax per segment and writes one partial
+    // per segment (an empty one where it took no page of the segment).
+    // Transposed fp16 tiles as for bf16 pages: S^T = K Q^T (M = 16 tokens, N =
+    // 8 heads), O^T += V^T P^T (M = 16 channels, N = heads, K = 16 tokens); a
+    // lane holds heads tc, tc + 1.
+    constexpr int KS = D / 16;
+    constexpr int WC = D / 32;   // key code words of one row in a lane's chunk
+    const uint32_t kA1024[4] = {kF16x2_1024, kF16x2_1024, kF16x2_1024, kF16x2_1024};
+    const int qr = lane >> 2, tq = lane & 3, tc = 2 * tq;
+    float acc[D / 16][4];   // O^T: rows 16 mt + qr (code multiplier 1) and 16 mt + qr + 8 (multiplier 16)
+    float voff[4];          // 1024 sum_t (s_t p_t): the codes' offset in every row of acc
+    float m_run[2], l_run[2], vl_run[2];   // heads tc, tc + 1; vl = sum_t lo_t p_t (lane-partial)
+    auto reset = [&]() {
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      voff[0] = voff[1] = voff[2] = voff[3] = 0.f;
+      m_run[0] = m_run[1] = kNegInf;
+      l_run[0] = l_run[1] = 0.f;
+      vl_run[0] = vl_run[1] = 0.f;
+    };
+    reset();
+    for (int gp = 0;; ++gp) {
+      bool have = false;
+      if (lane == 0) {
+        const bool known = spin_until([&] { return *v_resolved > gp || *v_total <= gp || *v_abort; }, timeout_ns);
+        if (!known) *v_abort = 1;
+        have = known && *v_resolved > gp && !*v_abort;
+      }
+      if (!__shfl_sync(0xffffffffu, have, 0)) break;
+      const int4 md = s_meta[gp % kMetaRing];
+      const int vr = s_range[gp % kMetaRing];
+      __syncwarp();
+      __threadfence_block();
+      if (lane == 0) v_seen[warp] = gp + 1;   // the resolver may reuse this ring entry from here on
+      if (md.w & kSegStart) reset();
+      if (gp % kDecodeWarps == warp) {
+        const int st = gp % NS;
+        const bool landed = mbar_wait_bounded(&full_bar[st], (gp / NS) & 1, timeout_ns);
+        if (__any_sync(0xffffffffu, !landed || *v_abort != 0)) {
+          if (lane == 0) *v_abort = 1;
+          break;
+        }
+        const int pidx = md.y;
+        const bool page_ok = md.z >= 0, streaming = md.w & kSegStreaming;
+        const int L = md.w >> 3;
+        const uint8_t* stg = smem + st * stage_bytes;
+        const uint8_t* qs = stg + Cfg::kQ4Q;   // q rows of the unit, [G][D] bf16
+        // ---- fold the key steps into q: B = s q of head qr at channels 16 ks + tc + {0, 1}
+        // (b0) and + {8, 9} (b1, divided by 16: those codes carry the multiplier 16), each
+        // as an fp16 pair hi + lo; kl = sum of lo_c q_c over this lane's channels
+        uint32_t bh[KS][2], bl[KS][2];
+        float kl = 0.f;
+        {
+          const float* kps = reinterpret_cast<const float*>(stg + Cfg::kQ4ParK) + tq * (D / 4);
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const float4 s4 = *reinterpret_cast<const float4*>(kps + 4 * ks);
+            const float4 l4 = *reinterpret_cast<const float4*>(kps + D + 4 * ks);
+            const int c = 16 * ks + tc;
+            uint32_t qa = 0u, qb = 0u;
+            if (qr < G) {
+              qa = *reinterpret_cast<const uint32_t*>(qs + (qr * D + c) * 2);
+              qb = *reinterpret_cast<const uint32_t*>(qs + (qr * D + c + 8) * 2);
+            }
+            const float q0 = bf16_lo(qa), q1 = bf16_hi(qa), q2 = bf16_lo(qb), q3 = bf16_hi(qb);
+            kl = fmaf(l4.x, q0, fmaf(l4.y, q1, fmaf(l4.z, q2, fmaf(l4.w, q3, kl))));
+            split_f16x2(s4.x * q0, s4.y * q1, bh[ks][0], bl[ks][0]);
+            split_f16x2((s4.z * 0.0625f) * q2, (s4.w * 0.0625f) * q3, bh[ks][1], bl[ks][1]);
+          }
+        }
+        // the codes' offset: 1024 sum_c B (hi + lo) of heads tc, tc + 1, by the tensor
+        // cores from the same operands, so that it cancels the MMAs' own term exactly
+        float ko[4] = {0.f, 0.f, 0.f, 0.f}, kol[4] = {0.f, 0.f, 0.f, 0.f};   // two chains: hi and lo parts
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          mma_f16_16816(ko, kA1024, bh[ks][0], bh[ks][1]);
+          mma_f16_16816(kol, kA1024, bl[ks][0], bl[ks][1]);
+        }
+        ko[0] += kol[0];
+        ko[1] += kol[1];
+        kl += __shfl_xor_sync(0xffffffffu, kl, 1);
+        kl += __shfl_xor_sync(0xffffffffu, kl, 2);
+        const float kc[2] = {__shfl_sync(0xffffffffu, kl, 4 * tc) - ko[0],
+                             __shfl_sync(0xffffffffu, kl, 4 * (tc + 1)) - ko[1]};
+        // ---- S^T of the four tiles: A = 1024 + code (channels + 0, + 1) or 1024 + 16 code
+        // (+ 8, + 9) of key rows 16 t + qr, + 8
+        float sacc[4][4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) sacc[t][0] = sacc[t][1] = sacc[t][2] = sacc[t][3] = 0.f;
+        // word wi of a row's chunk holds the code pairs of k-steps 2 wi (nibbles 0, 1, 4, 5)
+        // and 2 wi + 1 (nibbles 2, 3, 6, 7); two tiles at a time, 16-byte reads
+#pragma unroll
+        for (int t0 = 0; t0 < 4; t0 += 2) {
+          uint32_t kw[2][2][WC];
+#pragma unroll
+          for (int tt = 0; tt < 2; ++tt) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const uint8_t* kr = stg + (16 * (t0 + tt) + qr + 8 * r) * (D / 2) + tq * (D / 8);
+              if constexpr (WC % 4 == 0) {
+#pragma unroll
+                for (int x = 0; x < WC; x += 4) {
+                  const uint4 v = *reinterpret_cast<const uint4*>(kr + 4 * x);
+                  kw[tt][r][x] = v.x, kw[tt][r][x + 1] = v.y, kw[tt][r][x + 2] = v.z, kw[tt][r][x + 3] = v.w;
+                }
+              } else {
+#pragma unroll
+                for (int x = 0; x < WC; x += 2) {
+                  const uint2 v = *reinterpret_cast<const uint2*>(kr + 4 * x);
+                  kw[tt][r][x] = v.x, kw[tt][r][x + 1] = v.y;
+                }
+              }
+            }
+          }
+          float sl[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};   // lo parts: chains of their own
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+              const uint32_t w0 = (ks & 1) ? kw[tt][0][ks >> 1] >> 8 : kw[tt][0][ks >> 1];
+              const uint32_t w1 = (ks & 1) ? kw[tt][1][ks >> 1] >> 8 : kw[tt][1][ks >> 1];
+              const uint32_t a[4] = {q4h_lo(w0), q4h_lo(w1), q4h_hi(w0), q4h_hi(w1)};
+              mma_f16_16816(sacc[t0 + tt], a, bh[ks][0], bh[ks][1]);
+              mma_f16_16816(sl[tt], a, bl[ks][0], bl[ks][1]);
+            }
+          }
+#pragma unroll
+          for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[t0 + tt][e] += sl[tt][e];
+        }
+        // ---- mask + online softmax over the page.  Element (t, e): token 16 t + qr + 8 (e >> 1),
+        // head tc + (e & 1)
+        const int tok0 = pidx * kPage + qr;
+        bool ok[4][2];
+        float p[4][4];
+        float mh[2] = {kNegInf, kNegInf};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int tk = tok0 + 16 * t + 8 * r;
+            ok[t][r] = page_ok && tk < L && (!streaming || tk < sink || tk >= L - local);
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            p[t][e] = ok[t][e >> 1] ? (sacc[t][e] + kc[e & 1]) * scale_log2 : kNegInf;
+            mh[e & 1] = fmaxf(mh[e & 1], p[t][e]);
+          }
+        }
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          mh[0] = fmaxf(mh[0], __shfl_xor_sync(0xffffffffu, mh[0], o));
+          mh[1] = fmaxf(mh[1], __shfl_xor_sync(0xffffffffu, mh[1], o));
+        }
+        float corr[2], m_use[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float m_new = fmaxf(m_run[h], mh[h]);
+          m_use[h] = m_new == kNegInf ? 0.f : m_new;
+          corr[h] = fast_exp2(m_run[h] - m_use[h]);
+          m_run[h] = m_new;
+        }
+        if (__any_sync(0xffffffffu, corr[0] != 1.f || corr[1] != 1.f)) {
+#pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt) {
+            acc[mt][0] *= corr[0];
+            acc[mt][1] *= corr[1];
+            acc[mt][2] *= corr[0];
+            acc[mt][3] *= corr[1];
+          }
+          voff[0] *= corr[0];
+          voff[1] *= corr[1];
+          voff[2] *= corr[0];
+          voff[3] *= corr[1];
+        }
+        // ---- per tile: P^T scaled by the value steps of its tokens (masked tokens: 0,
+        // whatever the parameters of an unused row hold), as fp16, and the value offsets'
+        // term; then O^T += (1024 + m code)^T (s P)^T and the offset 1024 sum_t (s P)^T
+        const float2* vp2 = reinterpret_cast<const float2*>(stg + Cfg::kQ4ParV);
+        float ls[2] = {0.f, 0.f}, vs[2] = {0.f, 0.f};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          float sp[4];
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const float2 par = vp2[16 * t + qr + 8 * r];   // (s, lo) of the token
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float pe = fast_exp2(p[t][2 * r + h] - m_use[h]);
+              ls[h] += pe;
+              sp[2 * r + h] = ok[t][r] ? pe * par.x : 0.f;
+              vs[h] = ok[t][r] ? fmaf(pe, par.y, vs[h]) : vs[h];
+            }
+          }
+          const uint32_t pb0 = movmatrix_trans(pack_f16x2(sp[0], sp[1]));   // tokens 0..7 of the tile
+          const uint32_t pb1 = movmatrix_trans(pack_f16x2(sp[2], sp[3]));   // tokens 8..15
+          uint32_t vw[D / 16];
+          const uint8_t* vch = stg + Cfg::kQ4Bytes + (t * 32 + lane) * (D / 4);
+#pragma unroll
+          for (int x = 0; x < D / 16; x += 4) {
+            const uint4 v = *reinterpret_cast<const uint4*>(vch + 4 * x);
+            vw[x] = v.x, vw[x + 1] = v.y, vw[x + 2] = v.z, vw[x + 3] = v.w;
+          }
+#pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt) {
+            const uint32_t w8 = vw[mt] >> 8;
+            const uint32_t a[4] = {q4h_lo(vw[mt]), q4h_hi(vw[mt]), q4h_lo(w8), q4h_hi(w8)};
+            mma_f16_16816(acc[mt], a, pb0, pb1);
+          }
+          mma_f16_16816(voff, kA1024, pb0, pb1);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          l_run[h] = l_run[h] * corr[h] + ls[h];
+          vl_run[h] = vl_run[h] * corr[h] + vs[h];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[st]);   // every read of this stage is done
+      }
+      // ---- end of a segment: this warp's partial (empty if it took none of its pages)
+      if (md.w & kSegEnd) {
+        const int u = md.x;
+        const bool slots_ok = vr >= 0 && vr < Re;   // slot vr + u < Re + units
+        float lh[2] = {l_run[0], l_run[1]};
+        float vh[2] = {vl_run[0], vl_run[1]};
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          lh[0] += __shfl_xor_sync(0xffffffffu, lh[0], o);
+          lh[1] += __shfl_xor_sync(0xffffffffu, lh[1], o);
+          vh[0] += __shfl_xor_sync(0xffffffffu, vh[0], o);
+          vh[1] += __shfl_xor_sync(0xffffffffu, vh[1], o);
+        }
+        const long pbase = (static_cast<long>(vr + u) * kDecodeWarps + warp) * G;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int h = tc + h2;
+          if (h < G && slots_ok) {
+            const bool has = m_run[h2] != kNegInf && lh[h2] > 0.f;
+            const float inv = has ? 1.f / lh[h2] : 0.f;
+            float* po = part_o + (pbase + h) * D + qr;
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+              po[mt * 16] = (acc[mt][h2] - voff[h2] + vh[h2]) * inv;
+              po[mt * 16 + 8] = fmaf(acc[mt][2 + h2] - voff[2 + h2], 0.0625f, vh[h2]) * inv;
+            }
+            if (qr == 0) part_lse[pbase + h] = has ? m_run[h2] + __log2f(lh[h2]) : kNegInf;
+          }
+        }
+        if (!slots_ok && lane == 0) report(LSERVE_ERR_DEVICE_BOUNDS);
+      }
+    }
   } else {
     // ---- consumers.  Transposed tiles: S^T = K Q^T (M = the warp's 16 tokens,
     // N = 8 query heads, K = channels) and O^T += V^T P^T (M = channels, N =
     // heads, K = tokens), so the G <= 8 heads fill N exactly.  A lane holds
     // heads tc, tc + 1 of the tile.
     constexpr int KS = D / 16;
-    uint32_t qb[Q4 ? 1 : KS][2];          // Q^T as the B operand (heads >= G are zero)
-    uint32_t qp[Q4 ? D / 8 : 1];          // INT4: q of head qr at this lane's channels (bf16 pairs), key-chunk order
+    uint32_t qb[KS][2];                   // Q^T as the B operand (heads >= G are zero)
     float acc[D / 16][4];                 // O^T: m-tile mt = channels 16 mt .. 16 mt + 15
     float m_run[2], l_run[2];             // online softmax of heads tc, tc + 1
-    float vc_run[2];                      // INT4: sum_t (lo_t - 128 s_t) p_t, heads tc, tc + 1
     const int mi = lane >> 3, rr = lane & 7;
     const int qr = lane >> 2, tc = 2 * (lane & 3);
     for (int gp = 0;; ++gp) {
@@ -485,7 +760,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) pa
         break;
       }
       const int4 md = s_meta[gp % kMetaRing];
-      const int4 sg = s_seg[gp % kMetaRing];
+      const int vr = s_range[gp % kMetaRing];
       const int u = md.x, pidx = md.y;
       const bool page_ok = md.z >= 0, streaming = md.w & kSegStreaming;
       const int L = md.w >> 3;
@@ -493,97 +768,24 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) pa
       const uint8_t* ks_base = stg;
       const uint8_t* vs_base = stg + Cfg::kKVBytes;
       if (md.w & kSegStart) {
-        const uint8_t* qs = stg + (Q4 ? Cfg::kQ4Q : 2 * Cfg::kKVBytes);   // [G][D] bf16, row-major
-        if constexpr (Q4) {
+        const uint8_t* qs = stg + 2 * Cfg::kKVBytes;   // [G][D] bf16, row-major
 #pragma unroll
-          for (int i = 0; i < D / 4; i += 2) {   // entries i, i + 1: channels 16 (i/4) + 8 ((i/2)%2) + tc, + 1
-            const int c = 16 * (i >> 2) + 8 * ((i >> 1) & 1) + tc;
-            qp[i / 2] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c) * 2) : 0u;
-          }
-        } else {
-#pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {   // lane: head qr, channels 16 ks + tc, +1 and + 8, + 9
-            const int c0 = ks * 16 + tc;
-            qb[ks][0] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c0) * 2) : 0u;
-            qb[ks][1] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c0 + 8) * 2) : 0u;
-          }
+        for (int ks = 0; ks < KS; ++ks) {   // lane: head qr, channels 16 ks + tc, +1 and + 8, + 9
+          const int c0 = ks * 16 + tc;
+          qb[ks][0] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c0) * 2) : 0u;
+          qb[ks][1] = qr < G ? *reinterpret_cast<const uint32_t*>(qs + (qr * D + c0 + 8) * 2) : 0u;
         }
 #pragma unroll
         for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
         m_run[0] = m_run[1] = kNegInf;
         l_run[0] = l_run[1] = 0.f;
-        vc_run[0] = vc_run[1] = 0.f;
       }
       const int t_warp = pidx * kPage + warp * 16;   // first token of this warp's slice
 
       // ---- S^T = K Q^T (16 tokens x 8 heads) into two accumulators (alternate k-steps)
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t vf[Q4 ? 1 : D / 16][4];    // bf16: V^T fragments
-      uint32_t vw[Q4 ? D / 16 : 1];       // INT4: this lane's value code words (one per m-tile)
-      float2 vpt[2];                      // INT4: (s, lo) of tokens t_warp + qr, + 8
-      float kc_lane = 0.f;                // INT4: sum of (lo_c - 128 s_c) q_c over this lane's channels
-      if constexpr (Q4) {
-        // key rows qr, qr + 8 of the slice: chunk tc/2 (D/32 words each)
-        constexpr int WC = D / 32;
-        uint32_t kw0[WC], kw1[WC];
-        const uint8_t* kr0 = stg + (warp * 16 + qr) * (D / 2) + (lane & 3) * (D / 8);
-        const uint8_t* kr1 = kr0 + 8 * (D / 2);
-        if constexpr (WC % 4 == 0) {   // d = 128: 16-byte chunks
-#pragma unroll
-          for (int x = 0; x < WC; x += 4) {
-            const uint4 a = *reinterpret_cast<const uint4*>(kr0 + 4 * x);
-            const uint4 b = *reinterpret_cast<const uint4*>(kr1 + 4 * x);
-            kw0[x] = a.x, kw0[x + 1] = a.y, kw0[x + 2] = a.z, kw0[x + 3] = a.w;
-            kw1[x] = b.x, kw1[x + 1] = b.y, kw1[x + 2] = b.z, kw1[x + 3] = b.w;
-          }
-        } else {   // d = 64: 8-byte chunks
-#pragma unroll
-          for (int x = 0; x < WC; x += 2) {
-            const uint2 a = *reinterpret_cast<const uint2*>(kr0 + 4 * x);
-            const uint2 b = *reinterpret_cast<const uint2*>(kr1 + 4 * x);
-            kw0[x] = a.x, kw0[x + 1] = a.y, kw1[x] = b.x, kw1[x + 1] = b.y;
-          }
-        }
-        // this lane's value code words and the steps / offsets of its two tokens
-        const uint8_t* vch = stg + Cfg::kQ4Bytes + (warp * 32 + lane) * (D / 4);
-#pragma unroll
-        for (int x = 0; x < D / 16; x += 4) {
-          const uint4 a = *reinterpret_cast<const uint4*>(vch + 4 * x);
-          vw[x] = a.x, vw[x + 1] = a.y, vw[x + 2] = a.z, vw[x + 3] = a.w;
-        }
-        const float2* vp2 = reinterpret_cast<const float2*>(stg + Cfg::kQ4ParV);
-        vpt[0] = vp2[warp * 16 + qr];
-        vpt[1] = vp2[warp * 16 + qr + 8];
-        const float* kps = reinterpret_cast<const float*>(stg + Cfg::kQ4ParK) + (lane & 3) * (D / 4);
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          // B = s q at channels 16 ks + tc + {0, 1, 8, 9} (entries 4 ks .. 4 ks + 3), as bf16 hi + lo
-          const float4 s4 = *reinterpret_cast<const float4*>(kps + 4 * ks);
-          const float4 l4 = *reinterpret_cast<const float4*>(kps + D + 4 * ks);
-          const float q4[4] = {__uint_as_float(qp[2 * ks] << 16), __uint_as_float(qp[2 * ks] & 0xffff0000u),
-                               __uint_as_float(qp[2 * ks + 1] << 16), __uint_as_float(qp[2 * ks + 1] & 0xffff0000u)};
-          kc_lane = fmaf(fmaf(-128.f, s4.x, l4.x), q4[0],
-                         fmaf(fmaf(-128.f, s4.y, l4.y), q4[1],
-                              fmaf(fmaf(-128.f, s4.z, l4.z), q4[2], fmaf(fmaf(-128.f, s4.w, l4.w), q4[3], kc_lane))));
-          const float x0 = q4[0] * s4.x, x1 = q4[1] * s4.y, x2 = q4[2] * s4.z, x3 = q4[3] * s4.w;
-          const uint32_t b0 = pack_bf16x2(x0, x1), b1 = pack_bf16x2(x2, x3);
-          const uint32_t c0 = pack_bf16x2(x0 - __uint_as_float(b0 << 16), x1 - __uint_as_float(b0 & 0xffff0000u));
-          const uint32_t c1 = pack_bf16x2(x2 - __uint_as_float(b1 << 16), x3 - __uint_as_float(b1 & 0xffff0000u));
-          // A = 128 + code of rows qr / qr + 8: pairs 2 ks (channels +0, +1) and 2 ks + 1 (+8, +9)
-          const int wi = ks >> 1, k0 = 2 * (ks & 1);
-          const uint32_t a[4] = {q4_pair(kw0[wi], k0), q4_pair(kw1[wi], k0), q4_pair(kw0[wi], k0 + 1),
-                                 q4_pair(kw1[wi], k0 + 1)};
-          if (ks & 1) {
-            mma_bf16_16816(sb, a, b0, b1);
-            mma_bf16_16816(sb, a, c0, c1);
-          } else {
-            mma_bf16_16816(sa, a, b0, b1);
-            mma_bf16_16816(sa, a, c0, c1);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[st]);   // every read of this stage is done
-      } else {
+      uint32_t vf[D / 16][4];             // V^T fragments
+      {
         // ---- this warp's K and V fragments into registers, then the stage goes back
         // to the producer at once: the ring spends its time loading, not waiting for math
         uint32_t kf[KS][4];
@@ -611,14 +813,6 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) pa
             mma_bf16_16816(sa, kf[ks], qb[ks][0], qb[ks][1]);
         }
       }
-      // INT4: the offsets' term of heads tc, tc + 1 (sum over the four lanes of head qr first)
-      float kc[2] = {0.f, 0.f};
-      if constexpr (Q4) {
-        kc_lane += __shfl_xor_sync(0xffffffffu, kc_lane, 1);
-        kc_lane += __shfl_xor_sync(0xffffffffu, kc_lane, 2);
-        kc[0] = __shfl_sync(0xffffffffu, kc_lane, 4 * tc);
-        kc[1] = __shfl_sync(0xffffffffu, kc_lane, 4 * (tc + 1));
-      }
       // ---- mask + online softmax.  Element e: token t_warp + qr + 8 (e >> 1), head tc + (e & 1)
       auto valid = [&](int t) -> bool {
         return page_ok && t < L && (!streaming || t < sink || t >= L - local);
@@ -626,7 +820,7 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) pa
       const bool ok0 = valid(t_warp + qr), ok1 = valid(t_warp + qr + 8);
       float p[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) p[e] = ((e >> 1) ? ok1 : ok0) ? (sa[e] + sb[e] + kc[e & 1]) * scale_log2 : kNegInf;
+      for (int e = 0; e < 4; ++e) p[e] = ((e >> 1) ? ok1 : ok0) ? (sa[e] + sb[e]) * scale_log2 : kNegInf;
       // per-head max over the 16 tokens: the lanes with one lane % 4 hold one head pair
       float mh[2] = {fmaxf(p[0], p[2]), fmaxf(p[1], p[3])};
 #pragma unroll
@@ -655,30 +849,6 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) pa
           acc[mt][3] *= corr[1];
         }
       }
-      if constexpr (Q4) {
-        // ---- P^T scaled by the value steps of its tokens, as bf16 hi + lo (masked
-        // tokens: 0, whatever the parameters of an unused row hold), and the
-        // offsets' term
-        float ps[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) ps[e] = ((e >> 1) ? ok1 : ok0) ? p[e] * vpt[e >> 1].x : 0.f;
-        const uint32_t u0 = pack_bf16x2(ps[0], ps[1]), u1 = pack_bf16x2(ps[2], ps[3]);
-        const uint32_t w0 = pack_bf16x2(ps[0] - __uint_as_float(u0 << 16), ps[1] - __uint_as_float(u0 & 0xffff0000u));
-        const uint32_t w1 = pack_bf16x2(ps[2] - __uint_as_float(u1 << 16), ps[3] - __uint_as_float(u1 & 0xffff0000u));
-        const float o0 = ok0 ? fmaf(-128.f, vpt[0].x, vpt[0].y) : 0.f;   // lo - 128 s of token qr
-        const float o1 = ok1 ? fmaf(-128.f, vpt[1].x, vpt[1].y) : 0.f;   // ... of token qr + 8
-        vc_run[0] = vc_run[0] * corr[0] + fmaf(o0, p[0], o1 * p[2]);
-        vc_run[1] = vc_run[1] * corr[1] + fmaf(o0, p[1], o1 * p[3]);
-        const uint32_t pb0 = movmatrix_trans(u0), pb1 = movmatrix_trans(u1);   // tokens 0..7, 8..15
-        const uint32_t pl0 = movmatrix_trans(w0), pl1 = movmatrix_trans(w1);
-        // ---- O^T += (128 + code)^T (s P)^T: a_j of m-tile mt = nibbles j, j + 4 of word mt
-#pragma unroll
-        for (int mt = 0; mt < D / 16; ++mt) {
-          const uint32_t a[4] = {q4_pair(vw[mt], 0), q4_pair(vw[mt], 1), q4_pair(vw[mt], 2), q4_pair(vw[mt], 3)};
-          mma_bf16_16816(acc[mt], a, pb0, pb1);
-          mma_bf16_16816(acc[mt], a, pl0, pl1);
-        }
-      } else {
       // ---- P^T as the B operand (k = tokens, n = heads): transpose the two 8x8 blocks
       const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p[0], p[1]));   // tokens 0..7
       const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p[2], p[3]));   // tokens 8..15
@@ -698,24 +868,17 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) pa
         vf[mt][3] &= vm1;
         mma_bf16_16816(acc[mt], vf[mt], pb0, pb1);
       }
-      }
 
       // ---- end of a segment: this warp's partial, and the merge if it completes the unit
       if (md.w & kSegEnd) {
-        const int vr = sg.x, c_first = sg.y, c_last = sg.z;   // this range; the unit's first and last range
-        const bool slots_ok = c_first >= 0 && c_first <= vr && vr <= c_last && c_last < Re;
+        const bool slots_ok = vr >= 0 && vr < Re;   // slot vr + u < Re + units
         // (slot vr + u of every range of the unit is read by decode_merge_kernel)
         // l of heads tc, tc + 1: sum over the 8 lanes that share lane % 4
         float lh[2] = {l_run[0], l_run[1]};
-        float vh[2] = {vc_run[0], vc_run[1]};
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
           lh[0] += __shfl_xor_sync(0xffffffffu, lh[0], o);
           lh[1] += __shfl_xor_sync(0xffffffffu, lh[1], o);
-          if constexpr (Q4) {
-            vh[0] += __shfl_xor_sync(0xffffffffu, vh[0], o);
-            vh[1] += __shfl_xor_sync(0xffffffffu, vh[1], o);
-          }
         }
         const long pbase = (static_cast<long>(vr + u) * kDecodeWarps + warp) * G;   // this warp's partial
 #pragma unroll
@@ -725,11 +888,10 @@ __global__ void __launch_bounds__(kDecodeThreads) __maxnreg__(Q4 ? 112 : 168) pa
             const bool has = m_run[h2] != kNegInf && lh[h2] > 0.f;
             const float inv = has ? 1.f / lh[h2] : 0.f;
             float* po = part_o + (pbase + h) * D + qr;
-            const float add = Q4 ? vh[h2] : 0.f;   // INT4: the offsets' term
 #pragma unroll
             for (int mt = 0; mt < D / 16; ++mt) {
-              po[mt * 16] = (acc[mt][h2] + add) * inv;
-              po[mt * 16 + 8] = (acc[mt][2 + h2] + add) * inv;
+              po[mt * 16] = acc[mt][h2] * inv;
+              po[mt * 16 + 8] = acc[mt][2 + h2] * inv;
             }
             if (qr == 0) part_lse[pbase + h] = has ? m_run[h2] + __log2f(lh[h2]) : kNegInf;
           }

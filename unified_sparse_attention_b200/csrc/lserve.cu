@@ -316,7 +316,7 @@ struct DecodePlan {
   int32_t* sel;
   int32_t* sel_n;
   int32_t* off;          // [units + 1] flat offsets of the units' selections
-  int32_t* range_unit;   // [R] unit holding the first page of each range
+  int4* flat;            // [units * kcap] pre-resolved flat page list (first off[units] entries used)
   int32_t* range_counter;   // next range to claim (zeroed by the partition step)
   float* part_o;         // [R + units][4 warps][G][d]
   float* part_lse;       // [R + units][4 warps][G]
@@ -401,7 +401,7 @@ DecodePlan plan_decode(const lserve_decode_args* a, void* ws, bool q4 = false, i
   p.sel = c.take<int32_t>(units * p.kcap);
   p.sel_n = c.take<int32_t>(units);
   p.off = c.take<int32_t>(units + 1);
-  p.range_unit = c.take<int32_t>(p.R);
+  p.flat = c.take<int4>(units * p.kcap);
   p.range_counter = c.take<int32_t>(1);
   p.part_o = c.take<float>((p.R + units) * kDecodeWarps * p.G * a->d);
   p.part_lse = c.take<float>((p.R + units) * kDecodeWarps * p.G);
@@ -447,9 +447,9 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
   const int units = a->B * a->Hkv;
   // one block per unit selects its pages; one more lays out the attention grid's work
   if (launch_pdl(sel_in == nullptr, topk_pages_kernel, dim3(units + 1), dim3(kTopkThreads), topk_smem, st,
-                 static_cast<const float*>(p.scores), a->maxP, a->seq_lens, a->head_kind, a->Hkv, p.budget_pages,
-                 a->sink, a->local, sel, sel_n, p.kcap, units, p.R, p.G, D, p.off, p.range_unit, p.range_counter,
-                 static_cast<bf16*>(out), lse, sel_in, sel_n_in) != cudaSuccess)
+                 static_cast<const float*>(p.scores), a->maxP, a->seq_lens, a->head_kind, a->page_table,
+                 a->num_pages, a->Hkv, p.budget_pages, a->sink, a->local, sel, sel_n, p.kcap, units, p.G, D, p.off,
+                 p.flat, p.range_counter, static_cast<bf16*>(out), lse, sel_in, sel_n_in) != cudaSuccess)
     return check_launch("decode top-k");
   // kpar set: INT4 pages (codes of d/2 bytes a row, steps and offsets in kpar, vpar)
   const bool q4 = kpar != nullptr;
@@ -463,10 +463,9 @@ lserve_status launch_decode_d(const lserve_decode_args* a, const DecodePlan& p, 
   const int smem = q4 ? DecodeCfg<D>::smem_bytes_q4(p.G) : DecodeCfg<D>::smem_bytes(p.G);
   const float scale = a->scale > 0.f ? a->scale : 1.f / std::sqrt(static_cast<float>(D));
   if (launch_pdl(true, kern, dim3(p.P), dim3(kDecodeThreads), smem, st, tk,
-                 tv, static_cast<const bf16*>(a->q), a->page_table, a->maxP, a->seq_lens, a->head_kind,
-                 static_cast<const int32_t*>(sel), static_cast<const int32_t*>(p.off),
-                 static_cast<const int32_t*>(p.range_unit), p.range_counter, p.R, p.kcap, units, a->Hkv, p.G,
-                 a->num_pages, a->sink, a->local, scale * 1.4426950408889634f, wait_timeout_ns(),
+                 tv, static_cast<const bf16*>(a->q), static_cast<const int4*>(p.flat),
+                 static_cast<const int32_t*>(p.off), p.range_counter, p.R, p.kcap, units, a->Hkv, p.G,
+                 a->sink, a->local, scale * 1.4426950408889634f, wait_timeout_ns(),
                  debug_stall_decode(), p.part_o, p.part_lse, kpar, vpar) != cudaSuccess)
     return check_launch("decode attention");
   if (launch_pdl(true, decode_merge_kernel, dim3(units), dim3(kMergeThreads), 0, st, static_cast<const int32_t*>(p.off),

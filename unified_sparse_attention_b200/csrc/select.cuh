@@ -376,7 +376,8 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned lo
 // share, a pass costs two barriers (the histogram of the next pass is cleared
 // while this one fills), and the search ends once the k-th key's bin is
 // taken whole; one scan of (above, equal) counts places the output.
-__device__ __forceinline__ void topk_unit(const float* scores, int unit, int maxP, int L, bool dense,
+// Returns the number of pages selected (the same value in every thread).
+__device__ __forceinline__ int topk_unit(const float* scores, int unit, int maxP, int L, bool dense,
                                           int budget_pages, int sink, int local, int32_t* sel, int32_t* sel_n,
                                           int kcap, const int32_t* sel_in = nullptr,
                                           const int32_t* sel_n_in = nullptr) {
@@ -408,7 +409,7 @@ __device__ __forceinline__ void topk_unit(const float* scores, int unit, int max
       row[j] = v;
     }
     if (tid == 0 && sel_n) sel_n[unit] = cnt;
-    return;
+    return cnt;
   }
 
   if (sel_in) {   // a selection kept from an earlier step: its row as it stands
@@ -416,13 +417,13 @@ __device__ __forceinline__ void topk_unit(const float* scores, int unit, int max
     const int32_t* src = sel_in + static_cast<long>(unit) * kcap;
     for (int j = tid; j < kcap; j += nt) row[j] = j < m ? src[j] : -1;
     if (tid == 0 && sel_n) sel_n[unit] = m;
-    return;
+    return m;
   }
   const int k = min(budget_pages, n);
   if (k >= n) {
     for (int j = tid; j < kcap; j += nt) row[j] = j < n ? j : -1;
     if (tid == 0 && sel_n) sel_n[unit] = n;
-    return;
+    return n;
   }
   const float* srow = scores + static_cast<long>(unit) * maxP;
   const bool cached = n <= kTopkSmemKeys;
@@ -544,6 +545,7 @@ __device__ __forceinline__ void topk_unit(const float* scores, int unit, int max
   }
   for (int j = k + tid; j < kcap; j += nt) row[j] = -1;
   if (tid == 0 && sel_n) sel_n[unit] = k;
+  return k;
 }
 
 }  // namespace lserve
