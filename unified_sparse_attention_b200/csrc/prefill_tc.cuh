@@ -681,34 +681,36 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           m_run += rebase;
           rebase = 0.f;
         }
+        // steady state: one pass against the current reference.  A warp with any row
+        // still without a reference (the stream's first step), or whose pass shows a row
+        // sum past 2^40 (a weight near the fp32/bf16 limit; inf/NaN too), takes the exact
+        // row max and passes again.  Both decisions are warp votes, so the branches (which
+        // hold warp-collective TMEM loads) are taken by the whole warp or not at all; one
+        // copy of the pass serves both attempts.
+        bool exact = !__all_sync(0xffffffffu, m_run != kNegInf);
         float rsum = 0.f;
-        bool ok = false;
-        // steady state: one pass against the current reference.  The branch is taken
-        // by the whole warp or not at all (the pass holds warp-collective TMEM loads
-        // and votes): a warp with any row still without a reference takes the exact
-        // row max below instead.
-        if (__all_sync(0xffffffffu, m_run != kNegInf)) {
-          rsum = exp_pass(m_run);
-          // every weight is at most the row sum: none near the fp32/bf16 limit (catches inf/NaN too)
-          ok = !__any_sync(0xffffffffu, !(rsum <= 1099511627776.f));   // 2^40
-        }
-        if (!ok) {                // first step of the stream, or a jump: exact row max first
-          float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
   #pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            load_half(half, half ? keep1 : keep0, v);
+        while (true) {
+          if (exact) {
+            float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+  #pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+              load_half(half, half ? keep1 : keep0, v);
   #pragma unroll
-            for (int c = 0; c < 64; c += 8) {
+              for (int c = 0; c < 64; c += 8) {
   #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                mx[e] = max3(mx[e], __uint_as_float(v[c + 2 * e]), __uint_as_float(v[c + 2 * e + 1]));
+                for (int e = 0; e < 4; ++e)
+                  mx[e] = max3(mx[e], __uint_as_float(v[c + 2 * e]), __uint_as_float(v[c + 2 * e + 1]));
+              }
             }
+            const float mloc = max3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;
+            const float m_new = fmaxf(m_run, mloc);
+            if (m_run != kNegInf && m_new != m_run) f *= fast_exp2(m_run - m_new);
+            m_run = m_new;
           }
-          const float mloc = max3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;
-          const float m_new = fmaxf(m_run, mloc);
-          if (m_run != kNegInf && m_new != m_run) f *= fast_exp2(m_run - m_new);
-          m_run = m_new;
           rsum = exp_pass(m_run);
+          if (exact || !__any_sync(0xffffffffu, !(rsum <= 1099511627776.f))) break;   // 2^40
+          exact = true;
         }
         // weights well above the reference (row sum beyond 2^12): move the reference to the
         // largest argument at this stream's next step (O must first absorb this step); the
