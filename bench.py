@@ -41,18 +41,18 @@ DECODE_WL = "llama2_7b_mha"
 L2_BYTES = 126 * 1024 * 1024
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) from a one-pass ncu
-# capture of this script's default workloads (launch list under profiles/):
-# per launch of the prefill attention kernel, and per decode step (stats
-# refresh, scoring, top-k + plan, paged attention, merge).  Reported only while
-# the kernel sources hash as they did when the counters were taken.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) from one-pass ncu
+# captures of single kernels of this script's default workloads (profiles/
+# launch_list__bench_default.md): per launch of the prefill attention kernel, and
+# per decode step (scoring, top-k + plan, paged attention, merge).  Reported only
+# while the kernel sources hash as they did when the counters were taken.
 TRAFFIC = {
-    "prefill": {"bytes": 3535284992,
+    "prefill": {"bytes": 3558144256,
                 "sources": ["prefill_tc.cuh", "tile_lists.cuh", "common.cuh", "lserve.cu"],
-                "sha256": "54cd666b417c2fa7c423f9f076e7c3e5286e45e17d36d2ca046b15f1acc972e1"},
-    "decode": {"bytes": 822210048,
+                "sha256": "db1d900ec13bbc74095b150f7c539d81d0bc70b8cbfcf75fde595f91bf6c3f62"},
+    "decode": {"bytes": 821670656,
                "sources": ["select.cuh", "decode.cuh", "page_stats.cuh", "common.cuh", "lserve.cu"],
-               "sha256": "14e72dc1520509444a40d2d2070759adca85691852e018fc85f9bbf84014044d"},
+               "sha256": "492ddd0cb25fec76ba89bc2797b2921ce745fdd7f76ecebd6a15525e0d923f34"},
 }
 
 
