@@ -222,12 +222,17 @@ def max_over_ranks(vals, dist=None, device="cpu"):
 
 
 def flush_l2(buf):
-    buf.add_(1.0)
+    """Flush L2 between timed steps: write 2 x L2 of one half of `buf`, then read 2 x L2 of the
+    other half, so that the written half's dirty lines are written back here, before the step,
+    instead of inside it (that write-back alone is ~126 MB, about 19 µs of HBM time)."""
+    n = buf.numel() // 2
+    buf[:n].add_(1.0)
+    buf[n:].sum()
 
 
 def time_loop(fn, steps, warmup, stream, scratch=None, events_per_step=1):
     """Warm up, then time `steps` calls with CUDA events on `stream`; with `scratch`,
-    L2 is flushed (by writing it) between calls."""
+    L2 is flushed (flush_l2) between calls, outside the events."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
@@ -548,8 +553,9 @@ def main():
 
     # Every step reads far more than L2 holds (prefill: q, k, v; decode: page
     # summaries + selected pages), so the timed loops do not flush L2 between
-    # steps; the decode step is also timed with a flush (a 252 MB write) for reference.
-    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    # steps; the decode step is also timed with a flush (a 252 MB write, then a 252 MB read that
+    # takes the written lines' write-back out of the step) for reference.
+    scratch = torch.zeros(4 * L2_BYTES // 4, dtype=torch.float32, device=dev)   # 2 x L2 written + 2 x L2 read
     prefill_in_bytes = sum(t.numel() * t.element_size() for t in (setup.q, setup.k, setup.v))
     big = prefill_in_bytes > L2_BYTES and setup.dbytes["total"] > L2_BYTES
     fl = None if big else scratch   # smaller (profiling) workloads are flushed instead
@@ -670,7 +676,7 @@ def main():
                                f"Hkv{wd.Hkv} d{wd.d}, budget {wd.token_budget})",
                    "l2": (f"no flush: inputs larger than L2 ({L2_BYTES / 2**20:.0f} MiB) -- prefill reads "
                           f"{prefill_in_bytes / 1e9:.2f} GB of q/k/v, decode {setup.dbytes['total'] / 1e6:.0f} MB "
-                          f"per step") if big else "flushed between steps (write of 252 MB)",
+                          f"per step") if big else "flushed between steps (a 252 MB write, then a 252 MB read)",
                    "parallelism": f"replicas x{world}"},
         "prefill_ms": ms_prefill, "prefill_attention_ms": ms_attn, "tile_lists_ms": ms_tiles,
         "prefill_tflops": tflops_prefill, "kept_tile_tflop": setup.prefill_flops / 1e12,

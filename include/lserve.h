@@ -383,10 +383,10 @@ lserve_status lserve_quantize_pages_int4(int32_t B, int32_t Hkv, int32_t d, int3
  * same selection and attention as lserve_decode, with every K and V row read
  * as INT4 codes: keys s_c code + lo_c, values s_t code + lo_t (the values
  * lserve_quantize_pages_int4 defines).  The steps are folded into the other
- * operand (the tensor cores multiply the integer codes by s q and s p, each
- * carried as the sum of two bf16 parts, so about 2^-18 of each product is
- * lost) and the offsets into one fp32 term per head; no dequantised value is
- * ever rounded to bf16.  args->k_pages / args->v_pages point at
+ * operand: the tensor cores multiply the integer codes, exact in fp16, by s q
+ * (carried as the sum of two fp16 parts, so about 2^-22 of each product is
+ * lost) and by s p (one fp16 part, 2^-11).  The offsets go into one fp32 term
+ * per head; no dequantised value is ever rounded to a 16-bit format.  args->k_pages / args->v_pages point at
  * the code pools kq / vq and args->stats at the summaries that
  * lserve_quantize_pages_int4 wrote (so the bound holds for the dequantised keys).
  *
