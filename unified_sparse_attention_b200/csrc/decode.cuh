@@ -20,7 +20,8 @@
 //
 // paged_decode_kernel: one wave of CTAs (SMs x 2) that claim ranges from a
 // counter, so that SMs that run ahead take more.  Per CTA:
-//   * a resolver warp claims ranges (the next claim in flight while one is
+//   * a resolver warp claims ranges (CTA c's first is range c, later ones come
+//     from the counter; the next claim in flight while one is
 //     copied) and copies their entries of the flat list into a shared-memory
 //     ring ahead of the loads, adding the range's own start and end; a range
 //     that crosses unit boundaries is cut into segments, one per unit;
@@ -381,12 +382,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) paged_decode_kernel(
     // the wait for room in the ring
     int gp = 0;   // pages in the ring so far
     bool ok = true, stopped = false;   // !ok: inconsistent entry; stopped: the CTA is giving up
-    int r_next = 0;
-    if (lane == 0) r_next = atomicAdd(range_counter, 1);
+    // the first range is this CTA's own (range blockIdx.x), so the first pages need no
+    // atomic round trip; later ranges come from the counter, above the grid's own ones
+    int r_next = blockIdx.x;
     while (ok && !stopped) {
       const int r = __shfl_sync(0xffffffffu, r_next, 0);
       if (r >= Re) break;
-      if (lane == 0) r_next = atomicAdd(range_counter, 1);
+      if (lane == 0) r_next = static_cast<int>(gridDim.x) + atomicAdd(range_counter, 1);
       const int lo = static_cast<int>(r * T / Re), hi = static_cast<int>((r + 1) * T / Re);
       for (int f0 = lo; f0 < hi; f0 += 32) {
         const int f = f0 + lane, cnt = min(32, hi - f0);
