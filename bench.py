@@ -50,9 +50,9 @@ TRAFFIC = {
     "prefill": {"bytes": 3558144256,
                 "sources": ["prefill_tc.cuh", "tile_lists.cuh", "common.cuh", "lserve.cu"],
                 "sha256": "db1d900ec13bbc74095b150f7c539d81d0bc70b8cbfcf75fde595f91bf6c3f62"},
-    "decode": {"bytes": 821670656,
+    "decode": {"bytes": 821830656,
                "sources": ["select.cuh", "decode.cuh", "page_stats.cuh", "common.cuh", "lserve.cu"],
-               "sha256": "492ddd0cb25fec76ba89bc2797b2921ce745fdd7f76ecebd6a15525e0d923f34"},
+               "sha256": "a1b7174ba0090e62612adbda45af0d5ead5aeed1f79253701a7b50c90c7592d0"},
 }
 
 
