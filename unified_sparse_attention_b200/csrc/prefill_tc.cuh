@@ -539,7 +539,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           mma_ts4(tmem + C::kColO + 128 * x, at[0], at[1], at[2], at[3], bd[0], bd[1], bd[2], bd[3], kIdPV,
                   (p >= 2 || k4 > 0) ? 1u : 0u);
         }
-        commit(&o_done[x]);
+        if (p + 2 >= np) commit(&o_done[x]);   // the stream's last P.V of the item (the epilogue waits)
         commit(&v_empty[st]);
         if (p + 2 < np) issue_s(p + 2);
       }
@@ -569,6 +569,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     const float sc = A.scale_log2;
     TileListParams tp{0, A.Hkv, A.nQT, A.sink, A.local, nullptr, nullptr};
     int cs_own = 0;   // steps of this stream over the previous items (barrier phases)
+    int n_last = 0;   // items in which this stream had steps (phases of o_done[x])
     for (int ii = 0;; ++ii) {
       const int slot = ii & 1;
       if (!wait_or_abort(&item_full[slot], (ii >> 1) & 1, &s_abort, tmo)) break;
@@ -609,7 +610,6 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
             if (!((keep >> c) & 1ull)) v[c] = 0xff800000u;   // -inf: exp2 gives exactly 0
         }
       };
-      int seen = 0;   // completions of o_done[x] observed by this warpgroup
 
       float rebase = 0.f;   // shift of the reference max decided at this stream's previous step
       // tile indices of this stream's next step, loaded one step ahead (hides the load latency)
@@ -725,23 +725,18 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         tmem_st32(t_s, pk0);        // P[x] over S[x] columns 0..63 (S is no longer needed)
         tmem_st32(t_s + 32, pk1);
         l_run = l_run * f + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-        // O[x] holds this stream's steps < p; PV(p-2) completed before S(p) was issued,
-        // observe it (in order) before touching O[x]
-        if (j > 0) {
-          wait_or_abort(&o_done[x], (cs_own + j - 1) & 1, &s_abort, tmo);
-          ++seen;
-          __syncwarp();
-          fence_after_sync();
-          if (__any_sync(0xffffffffu, f != 1.f)) {
+        // O[x] holds this stream's steps < p, the latest being PV(p-2), and it is complete:
+        // S(p) was issued after it, and the commit behind s_full tracks every earlier MMA of
+        // the issuing thread.  PV(p) needs this step's P, so O[x] may be rescaled here.
+        if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
   #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t ov[32];
-              tmem_ld32(t_o + c0, ov);
-              tmem_wait_ld();
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld32(t_o + c0, ov);
+            tmem_wait_ld();
   #pragma unroll
-              for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * f);
-              tmem_st32(t_o + c0, ov);
-            }
+            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * f);
+            tmem_st32(t_o + c0, ov);
           }
         }
         tmem_wait_st();
@@ -751,8 +746,9 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       // a pending shift is never needed for the result: (m, l, O) stay consistent
       // ---- epilogue: merge the two streams (log-sum-exp), each warpgroup stores half of O
       const int nx = (np > x) ? (np - x + 1) >> 1 : 0;   // steps of this stream
-      if (nx > 0) {
-        wait_or_abort(&o_done[x], (cs_own + nx - 1) & 1, &s_abort, tmo);   // PV of its last step
+      if (nx > 0) {   // o_done[x] completes once per item in which this stream has steps
+        wait_or_abort(&o_done[x], n_last & 1, &s_abort, tmo);   // PV of its last step
+        ++n_last;
         fence_after_sync();
       }
       s_ml[ii & 1][x][0][row] = m_run;
@@ -809,7 +805,6 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           A.lse[(static_cast<long>(b) * Hq + h) * A.S + i] =
               has ? (m_all + __log2f(l_tot)) * 0.6931471805599453f : kNegInf;
       }
-      (void)seen;
       // both accumulators have been read: the MMA warp may let the next item's PV(0)
       // overwrite them
       fence_before_sync();
