@@ -56,7 +56,7 @@ typedef enum lserve_status {
   LSERVE_ERR_WORKSPACE = 3,       /* workspace pointer null/misaligned or too small       */
   LSERVE_ERR_CUDA = 4,            /* a CUDA runtime call or kernel launch failed          */
   LSERVE_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait ran out (device status)      */
-  LSERVE_ERR_DEVICE_BOUNDS = 6    /* a kernel met an out-of-range index (device status)   */
+  LSERVE_ERR_DEVICE_BOUNDS = 6    /* an out-of-range index, or an INT4 operand past fp16 (device status) */
 } lserve_status;
 
 #define LSERVE_PAGE 64            /* tokens per physical KV page                          */
@@ -386,16 +386,20 @@ lserve_status lserve_quantize_pages_int4(int32_t B, int32_t Hkv, int32_t d, int3
  * operand: the tensor cores multiply the integer codes, exact in fp16, by s q
  * (carried as the sum of two fp16 parts, so about 2^-22 of each product is
  * lost) and by s p (one fp16 part, 2^-11).  The offsets go into one fp32 term
- * per head; no dequantised value is ever rounded to a 16-bit format.  args->k_pages / args->v_pages point at
- * the code pools kq / vq and args->stats at the summaries that
- * lserve_quantize_pages_int4 wrote (so the bound holds for the dequantised keys).
+ * per head; no dequantised value is ever rounded to a 16-bit format.  Range:
+ * each |s_c q_c| and |s_t| must stay within the fp16 range (65504); a page
+ * whose key steps times q exceed it is reported as LSERVE_ERR_DEVICE_BOUNDS by
+ * lserve_get_device_status (its output is then not meaningful).
+ * args->k_pages / args->v_pages point at the code pools kq / vq and args->stats
+ * at the summaries that lserve_quantize_pages_int4 wrote (so the bound holds for
+ * the dequantised keys).
  *
  *   kpar   fp32 [num_pages, Hkv, 2, d], 16-byte aligned (read)
  *   vpar   fp32 [num_pages, Hkv, 64, 2], 16-byte aligned (read)
  *   out, lse, sel_out, sel_n, workspace: as lserve_decode (the same
  *   lserve_decode_workspace_size).
- * Errors: LSERVE_ERR_INVALID_ARG for a null or misaligned kpar / vpar, and
- * every error lserve_decode returns.
+ * Errors: LSERVE_ERR_INVALID_ARG for a null or misaligned kpar / vpar, every
+ * error lserve_decode returns, and the device-reported range error above.
  */
 lserve_status lserve_decode_int4(const lserve_decode_args* args, const float* kpar,
                                  const float* vpar, void* out, float* lse, int32_t* sel_out,

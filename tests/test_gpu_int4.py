@@ -236,3 +236,30 @@ def test_quantiser_ties_and_near_ties():
     codes = qp.kcode[1, 0, 5]
     x = f64(pc.k_pages)[1, 0, 5]
     assert np.any((x % 1 == 0.5) & (codes % 2 == 0))
+
+
+def test_int4_decode_reports_operands_past_fp16():
+    """The folded operands are fp16: a key channel whose step times q leaves the fp16 range
+    (|s q| > 65504) must be reported (LSERVE_ERR_DEVICE_BOUNDS), not turned into a silent
+    non-finite output; the same call on ordinary keys reports nothing."""
+    w = dataclasses.replace(W.WORKLOADS["tiny"], Hq=2, Hkv=2, d=128)
+    dev = "cuda"
+    pc = W.decode_cache(w, B=1, ctx=300)
+    kind = [0, 1]
+    q = W.decode_query(w, B=1).to(dev)
+    pt, sl = pc.page_table.to(dev), pc.seq_lens.to(dev)
+    hk = torch.tensor(kind, dtype=torch.uint8, device=dev)
+    g = quantize(pc, kind)
+    U.lserve_decode_int4(q, g["kq"], g["vq"], g["kpar"], g["vpar"], pt, sl, g["stats"], hk, 64, 64, 256)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 0
+    # channel 5 of every key scaled so that its per-page step is ~1e5 (finite in bf16)
+    big = pc.k_pages.clone()
+    big[:, :, :, 5] = big[:, :, :, 5] * 3.0e5
+    pc_big = dataclasses.replace(pc, k_pages=big)
+    gb = quantize(pc_big, kind)
+    qb = q.clone()
+    qb[:, :, 5] = 1.0   # so that |s q| is the step itself, far past 65504
+    U.lserve_decode_int4(qb, gb["kq"], gb["vq"], gb["kpar"], gb["vpar"], pt, sl, gb["stats"], hk, 64, 64, 256)
+    torch.cuda.synchronize()
+    assert U.lserve_get_device_status() == 6   # LSERVE_ERR_DEVICE_BOUNDS

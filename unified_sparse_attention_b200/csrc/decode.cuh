@@ -717,6 +717,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) paged_decode_kernel(
           vh[0] += __shfl_xor_sync(0xffffffffu, vh[0], o);
           vh[1] += __shfl_xor_sync(0xffffffffu, vh[1], o);
         }
+        // an operand past the fp16 range (|s q| or |s p| > 65504) leaves a non-finite value
+        // in the sums or the accumulators (masked tokens never contribute): reported here,
+        // once per segment, not silent
+        {
+          float probe = (lh[0] + lh[1]) + (vh[0] + vh[1]) + (voff[0] + voff[1]);
+#pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt) probe += (acc[mt][0] + acc[mt][1]) + (acc[mt][2] + acc[mt][3]);
+          if (!(fabsf(probe) <= 3.0e38f)) report(LSERVE_ERR_DEVICE_BOUNDS);
+        }
         const long pbase = (static_cast<long>(vr + u) * kDecodeWarps + warp) * G;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
