@@ -50,9 +50,9 @@ TRAFFIC = {
     "prefill": {"bytes": 3557373952,
                 "sources": ["prefill_tc.cuh", "tile_lists.cuh", "common.cuh", "lserve.cu"],
                 "sha256": "b1d09e7c5320b552d3dda4c598978867feea33e13a7a3528e44f196e30b8b3be"},
-    "decode": {"bytes": 821830656,
+    "decode": {"bytes": 822332160,
                "sources": ["select.cuh", "decode.cuh", "page_stats.cuh", "common.cuh", "lserve.cu"],
-               "sha256": "a1b7174ba0090e62612adbda45af0d5ead5aeed1f79253701a7b50c90c7592d0"},
+               "sha256": "ba77db93b18250ae5d80398b0ab70475c9f9a38669d88b33c9488a8871020c8b"},
 }
 
 
