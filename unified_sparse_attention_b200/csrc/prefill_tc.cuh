@@ -517,7 +517,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       wait_or_abort(&q_full, nq & 1, &s_abort, tmo);
       ++nq;
       issue_s(0);
-      if (np > 1) issue_s(1);
+      if (np > 1) {
+        // stream 1 starts one exponential phase behind stream 0: S(1) goes out once P(0)
+        // is ready, so that the two streams' exponentials alternate instead of sharing
+        // the unit (the in-order issue that follows keeps them apart)
+        wait_or_abort(&p_full[0], cs[0] & 1, &s_abort, tmo);
+        issue_s(1);
+      }
       for (int p = 0; p < np; ++p) {
         const int gu = gv + p, st = gu % kVStages, x = p & 1;
         wait_or_abort(&v_full[st], (gu / kVStages) & 1, &s_abort, tmo);
