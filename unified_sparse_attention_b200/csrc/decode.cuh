@@ -536,8 +536,38 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) paged_decode_kernel(
         // as an fp16 pair hi + lo; kl = sum of lo_c q_c over this lane's channels
         uint32_t bh[KS][2], bl[KS][2];
         float kl = 0.f;
-        {
-          const float* kps = reinterpret_cast<const float*>(stg + Cfg::kQ4ParK) + tq * (D / 4);
+        const float* kps = reinterpret_cast<const float*>(stg + Cfg::kQ4ParK) + tq * (D / 4);
+        if (G == 1) {
+          // one head: only the lanes qr = 0 hold a non-zero B, so lane (qr, tq) folds
+          // k-step qr alone and those lanes take every k-step's pair from lane 4 ks + tq
+          uint32_t h0 = 0u, h1 = 0u, l0 = 0u, l1 = 0u;
+          if (qr < KS) {
+            const float4 s4 = *reinterpret_cast<const float4*>(kps + 4 * qr);
+            const float4 l4 = *reinterpret_cast<const float4*>(kps + D + 4 * qr);
+            const int c = 16 * qr + tc;
+            const uint32_t qa = *reinterpret_cast<const uint32_t*>(qs + c * 2);
+            const uint32_t qb = *reinterpret_cast<const uint32_t*>(qs + (c + 8) * 2);
+            const float q0 = bf16_lo(qa), q1 = bf16_hi(qa), q2 = bf16_lo(qb), q3 = bf16_hi(qb);
+            kl = fmaf(l4.x, q0, fmaf(l4.y, q1, fmaf(l4.z, q2, l4.w * q3)));
+            split_f16x2(s4.x * q0, s4.y * q1, h0, l0);
+            split_f16x2((s4.z * 0.0625f) * q2, (s4.w * 0.0625f) * q3, h1, l1);
+          }
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const int src = 4 * ks + tq;
+            const uint32_t x0 = __shfl_sync(0xffffffffu, h0, src), x1 = __shfl_sync(0xffffffffu, h1, src);
+            const uint32_t y0 = __shfl_sync(0xffffffffu, l0, src), y1 = __shfl_sync(0xffffffffu, l1, src);
+            bh[ks][0] = qr == 0 ? x0 : 0u;
+            bh[ks][1] = qr == 0 ? x1 : 0u;
+            bl[ks][0] = qr == 0 ? y0 : 0u;
+            bl[ks][1] = qr == 0 ? y1 : 0u;
+          }
+          // the head's lo_c q_c over every k-step, left on its own lanes (summed over tq below)
+          kl += __shfl_xor_sync(0xffffffffu, kl, 4);
+          kl += __shfl_xor_sync(0xffffffffu, kl, 8);
+          kl += __shfl_xor_sync(0xffffffffu, kl, 16);
+          if (qr != 0) kl = 0.f;
+        } else {
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
             const float4 s4 = *reinterpret_cast<const float4*>(kps + 4 * ks);
