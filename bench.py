@@ -50,9 +50,9 @@ TRAFFIC = {
     "prefill": {"bytes": 3580308224,
                 "sources": ["prefill_tc.cuh", "tile_lists.cuh", "common.cuh", "lserve.cu"],
                 "sha256": "ef6557d1c5dc32360d988c00841410d9348e121b19022ecef1c67280a53e08bf"},
-    "decode": {"bytes": 821980160,
+    "decode": {"bytes": 821729792,
                "sources": ["select.cuh", "decode.cuh", "page_stats.cuh", "common.cuh", "lserve.cu"],
-               "sha256": "ede8ab2c3ae1c159bae6b0f37c4e156c45b759736df217e6bdea583acdc183d9"},
+               "sha256": "315f552b689e827de55a67f81fcaf23efebac042beee7f01196f3b306ed86eba"},
 }
 
 

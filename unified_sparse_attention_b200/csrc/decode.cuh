@@ -295,6 +295,12 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
   asm("{\n.reg .f16 l, h;\nmov.b32 {l, h}, %2;\ncvt.f32.f16 %0, l;\ncvt.f32.f16 %1, h;\n}" : "=f"(a), "=f"(b) : "r"(v));
   return make_float2(a, b);
 }
+// A compile-time int passed to a generic lambda.
+template <int N>
+struct IntConst {
+  static constexpr int value = N;
+};
+
 // x = hi + lo with hi, lo fp16 pairs (about 22 significant bits together)
 __device__ __forceinline__ void split_f16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
   hi = pack_f16x2(a, b);
@@ -537,36 +543,52 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) paged_decode_kernel(
         uint32_t bh[KS][2], bl[KS][2];
         float kl = 0.f;
         const float* kps = reinterpret_cast<const float*>(stg + Cfg::kQ4ParK) + tq * (D / 4);
-        if (G == 1) {
-          // one head: only the lanes qr = 0 hold a non-zero B, so lane (qr, tq) folds
-          // k-step qr alone and those lanes take every k-step's pair from lane 4 ks + tq
-          uint32_t h0 = 0u, h1 = 0u, l0 = 0u, l1 = 0u;
-          if (qr < KS) {
-            const float4 s4 = *reinterpret_cast<const float4*>(kps + 4 * qr);
-            const float4 l4 = *reinterpret_cast<const float4*>(kps + D + 4 * qr);
-            const int c = 16 * qr + tc;
-            const uint32_t qa = *reinterpret_cast<const uint32_t*>(qs + c * 2);
-            const uint32_t qb = *reinterpret_cast<const uint32_t*>(qs + (c + 8) * 2);
-            const float q0 = bf16_lo(qa), q1 = bf16_hi(qa), q2 = bf16_lo(qb), q3 = bf16_hi(qb);
-            kl = fmaf(l4.x, q0, fmaf(l4.y, q1, fmaf(l4.z, q2, l4.w * q3)));
-            split_f16x2(s4.x * q0, s4.y * q1, h0, l0);
-            split_f16x2((s4.z * 0.0625f) * q2, (s4.w * 0.0625f) * q3, h1, l1);
+        // G = 1, 2, 4: only the lanes qr < G hold a non-zero B, so every lane group
+        // qr = h + G r folds k-steps j R + r (R = 8 / G) of head h, and the head's
+        // lanes take k-step ks from lane 4 (qr + G (ks % R)) + tq, slot ks / R
+        auto fold_spread = [&](auto g_const) {
+          constexpr int GG = decltype(g_const)::value, R = 8 / GG, NJ = (KS + R - 1) / R;
+          const int h = qr % GG, r = qr / GG;
+          uint32_t fh[NJ][2], fl[NJ][2];
+#pragma unroll
+          for (int j = 0; j < NJ; ++j) {
+            const int ks = j * R + r;
+            fh[j][0] = fh[j][1] = fl[j][0] = fl[j][1] = 0u;
+            if (ks < KS) {
+              const float4 s4 = *reinterpret_cast<const float4*>(kps + 4 * ks);
+              const float4 l4 = *reinterpret_cast<const float4*>(kps + D + 4 * ks);
+              const int c = 16 * ks + tc;
+              const uint32_t qa = *reinterpret_cast<const uint32_t*>(qs + (h * D + c) * 2);
+              const uint32_t qb = *reinterpret_cast<const uint32_t*>(qs + (h * D + c + 8) * 2);
+              const float q0 = bf16_lo(qa), q1 = bf16_hi(qa), q2 = bf16_lo(qb), q3 = bf16_hi(qb);
+              kl = fmaf(l4.x, q0, fmaf(l4.y, q1, fmaf(l4.z, q2, fmaf(l4.w, q3, kl))));
+              split_f16x2(s4.x * q0, s4.y * q1, fh[j][0], fl[j][0]);
+              split_f16x2((s4.z * 0.0625f) * q2, (s4.w * 0.0625f) * q3, fh[j][1], fl[j][1]);
+            }
           }
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
-            const int src = 4 * ks + tq;
-            const uint32_t x0 = __shfl_sync(0xffffffffu, h0, src), x1 = __shfl_sync(0xffffffffu, h1, src);
-            const uint32_t y0 = __shfl_sync(0xffffffffu, l0, src), y1 = __shfl_sync(0xffffffffu, l1, src);
-            bh[ks][0] = qr == 0 ? x0 : 0u;
-            bh[ks][1] = qr == 0 ? x1 : 0u;
-            bl[ks][0] = qr == 0 ? y0 : 0u;
-            bl[ks][1] = qr == 0 ? y1 : 0u;
+            const int src = 4 * (h + GG * (ks % R)) + tq;
+            const uint32_t x0 = __shfl_sync(0xffffffffu, fh[ks / R][0], src);
+            const uint32_t x1 = __shfl_sync(0xffffffffu, fh[ks / R][1], src);
+            const uint32_t y0 = __shfl_sync(0xffffffffu, fl[ks / R][0], src);
+            const uint32_t y1 = __shfl_sync(0xffffffffu, fl[ks / R][1], src);
+            bh[ks][0] = qr < GG ? x0 : 0u;
+            bh[ks][1] = qr < GG ? x1 : 0u;
+            bl[ks][0] = qr < GG ? y0 : 0u;
+            bl[ks][1] = qr < GG ? y1 : 0u;
           }
-          // the head's lo_c q_c over every k-step, left on its own lanes (summed over tq below)
-          kl += __shfl_xor_sync(0xffffffffu, kl, 4);
-          kl += __shfl_xor_sync(0xffffffffu, kl, 8);
-          kl += __shfl_xor_sync(0xffffffffu, kl, 16);
-          if (qr != 0) kl = 0.f;
+          // head h's lo_c q_c over every k-step, left on its own lanes (summed over tq below)
+#pragma unroll
+          for (int o = 4 * GG; o < 32; o <<= 1) kl += __shfl_xor_sync(0xffffffffu, kl, o);
+          if (qr >= GG) kl = 0.f;
+        };
+        if (G == 1) {
+          fold_spread(IntConst<1>{});
+        } else if (G == 2) {
+          fold_spread(IntConst<2>{});
+        } else if (G == 4) {
+          fold_spread(IntConst<4>{});
         } else {
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
