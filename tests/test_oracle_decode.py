@@ -6,7 +6,8 @@
   equals the last prefill row (dense head: full budget; streaming head: the same
   sink/local);
 * an explicit selection equals SDPA with the corresponding token mask;
-* CRA equals 1 when nothing is dropped and matches brute-force weight sums.
+* CRA equals 1 when nothing is dropped and matches brute-force weight sums;
+* the paged gather against a per-token walk of the page table.
 """
 import math
 
@@ -156,3 +157,21 @@ def test_reuse_after_appending_tokens_matches_sdpa_with_the_kept_pages():
             m = dense_mask if kvh == 0 else stream_mask
             ref = sdpa_one(q[b, h], k[b, m, kvh], v[b, m, kvh])
             np.testing.assert_allclose(out[b, h], ref, atol=1e-12)
+
+
+def test_gather_tokens_against_a_per_token_walk_of_the_page_table():
+    """Token t of sequence b lives at slot t mod PAGE of physical page page_table[b, t // PAGE]."""
+    rng = np.random.default_rng(7)
+    B, maxP, Hkv, d = 2, 5, 3, 4
+    P = B * maxP
+    pool = rng.standard_normal((P, Hkv, D.PAGE, d)).astype(np.float32)
+    pt = rng.permutation(P).reshape(B, maxP)
+    for b in range(B):
+        for kvh in range(Hkv):
+            toks = np.array([0, 1, D.PAGE - 1, D.PAGE, 2 * D.PAGE + 3, maxP * D.PAGE - 1])
+            got = D.gather_tokens(pool, pt, b, kvh, toks)
+            assert got.dtype == np.float64 and got.shape == (len(toks), d)
+            for n, t in enumerate(toks):
+                page, slot = divmod(int(t), D.PAGE)
+                np.testing.assert_array_equal(got[n], pool[pt[b][page]][kvh][slot])
+    assert D.gather_tokens(pool, pt, 0, 0, np.array([], dtype=np.int64)).shape == (0, d)

@@ -8,7 +8,8 @@
 * the greedy against pure-Python brute force on random tiny inputs: the taken
   prefix is the shortest whose minimum retained mass (recounted tile by tile)
   reaches tau, and the mask holds exactly the tiles its candidates cover;
-* tau = 1 keeps every causal tile; tau = 0 keeps only the diagonal.
+* tau = 1 keeps every causal tile; tau = 0 keeps only the diagonal;
+* the sampled query tiles against their closed form.
 """
 import json
 import os
@@ -107,3 +108,19 @@ def test_tau_extremes():
     assert not m1[0, 1].any()                     # streaming head: no mask
     m0, _, nc, ns = V.build_vslash_mask(q, k, kind, 1, 0.0)
     assert np.array_equal(m0[0, 0], np.eye(4, dtype=np.uint8)) and nc[0, 0] == 0 and ns[0, 0] == 1
+
+
+@pytest.mark.parametrize("nQT,stride", [(1, 1), (7, 1), (7, 2), (7, 3), (8, 3), (5, 5), (4, 9), (64, 16)])
+def test_sampled_tiles_closed_form(nQT, stride):
+    """The last query tile is always sampled, then every stride-th tile below it."""
+    t = V.sampled_tiles(nQT, stride)
+    assert t[-1] == nQT - 1 and t[0] >= 0 and t[0] < stride
+    assert len(t) == (nQT - 1) // stride + 1
+    assert np.all(np.diff(t) == stride)
+    if stride == 1:
+        np.testing.assert_array_equal(t, np.arange(nQT))
+
+
+def test_sampled_tiles_rejects_a_stride_below_one():
+    with pytest.raises(ValueError):
+        V.sampled_tiles(4, 0)
